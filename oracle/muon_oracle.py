@@ -1,0 +1,302 @@
+"""Float64 reference implementation of one Muon step (test infrastructure only).
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
+``bench.py`` may import this module. It shares no code with the CUDA path.
+
+Sources (web pages; cited by title and section):
+
+* "About Muon: Why Not Adam" -- the authority on the arithmetic.
+  - section "The whole thing, in about forty lines": the step order
+    (momentum lerp, Nesterov lerp, bf16 cast, Frobenius normalisation with
+    eps = 1e-7, short-side transpose, the quintic loop, cast back, scale,
+    decoupled weight decay, write), default hyper-parameters and the
+    Moonlight scale used by that program.
+  - section "The lemma that makes it possible": an odd polynomial in X and
+    X^T X acts on the singular values only.
+  - section "The iteration does not converge, and that is deliberate":
+    (a, b, c) = (3.4445, -4.7750, 2.0315) and the scalar facts used as pins.
+  - section "How Do We Turn It Into a Real Optimizer?": the Jordan and
+    Moonlight multipliers, (m, n) = (fan-out, fan-in) = p.shape.
+  - section "The spectral ball gives UV^T": Bernstein's multiplier
+    sqrt(fan-out / fan-in).
+* "Por qué AdamW para entrenar modelos de lenguaje, y qué está cambiando",
+  section "Momentum: recordar el paso anterior": Muon uses the Nesterov form.
+* "The Optimizer Wars: How Muon Is Replacing Adam in Frontier AI Training",
+  section "What is Muon? Momentum orthogonalized by Newton-Schulz": five
+  quintic iterations in bf16 with the same coefficients.
+
+Readings where the pages are silent or disagree (each also listed in the
+design notes):
+
+* Momentum is the exponential moving average ``m' = beta*m + (1-beta)*g``
+  (the only program on the pages uses the lerp form), and the Nesterov blend
+  uses the *updated* buffer: ``u = g + beta*(m' - g)``.
+* Nesterov defaults to on; a flag turns it off (``u = m'``).
+* The norm is taken of the float64 ``u``; eps = 1e-7 is added to the norm,
+  not to its square.
+* The short-side transpose is strict: only m > n is transposed.
+* No bf16 rounding in the exact mode. ``emulate_bf16=True`` rounds X, A, B
+  (round-to-nearest-even) at the points where the GPU rounds: the cast of
+  u, and every Gram / polynomial / combine output. Diagnostic only.
+* ``ns_steps = 0`` returns the normalised matrix.
+"""
+
+from __future__ import annotations
+
+import numpy as np
+
+# (a, b, c): "About Muon: Why Not Adam", section "The iteration does not
+# converge, and that is deliberate"; the same triple in "The Optimizer Wars",
+# section "What is Muon? Momentum orthogonalized by Newton-Schulz".
+DEFAULT_COEFFS = (3.4445, -4.7750, 2.0315)
+
+# Added to ||G||_F before dividing: "About Muon: Why Not Adam", section
+# "The whole thing, in about forty lines".
+EPS = 1e-7
+
+SCALE_MOONLIGHT = 0   # 0.2 * sqrt(max(m, n))
+SCALE_JORDAN = 1      # sqrt(max(1, m / n))
+SCALE_BERNSTEIN = 2   # sqrt(m / n)  (fan-out / fan-in)
+SCALE_NONE = 3        # 1
+
+
+# ---------------------------------------------------------------------------
+# bf16 rounding (used only by the emulating diagnostic mode)
+# ---------------------------------------------------------------------------
+
+def bf16_round(x: np.ndarray) -> np.ndarray:
+    """Round float64 values to the nearest bf16 value (ties to even).
+
+    bf16 keeps 8 significant bits (1 implicit + 7 stored) and float32's
+    exponent range. Rounding is done directly on the float64 bit pattern
+    (52 stored mantissa bits, of which the top 7 are kept), so there is no
+    double rounding through float32. Values stay float64.
+    """
+    x = np.asarray(x, dtype=np.float64)
+    bits = x.view(np.uint64).copy()
+    drop = np.uint64(52 - 7)
+    lsb = (bits >> drop) & np.uint64(1)
+    bias = (np.uint64(1) << (drop - np.uint64(1))) - np.uint64(1) + lsb
+    finite = np.isfinite(x)
+    rounded = (bits + bias) & ~((np.uint64(1) << drop) - np.uint64(1))
+    out = np.where(finite, rounded, bits).view(np.float64)
+    return out
+
+
+# ---------------------------------------------------------------------------
+# Scalar polynomial ("About Muon: Why Not Adam", sections "The lemma that
+# makes it possible" and "The iteration does not converge, and that is
+# deliberate")
+# ---------------------------------------------------------------------------
+
+def ns_poly(s, coeffs=DEFAULT_COEFFS):
+    """The odd quintic p(s) = a s + b s^3 + c s^5 applied to scalars."""
+    a, b, c = coeffs
+    s = np.asarray(s, dtype=np.float64)
+    return a * s + b * s ** 3 + c * s ** 5
+
+
+def ns_poly_iterate(s, steps=5, coeffs=DEFAULT_COEFFS):
+    """p composed with itself ``steps`` times."""
+    s = np.asarray(s, dtype=np.float64)
+    for _ in range(steps):
+        s = ns_poly(s, coeffs)
+    return s
+
+
+# ---------------------------------------------------------------------------
+# Matrix Newton-Schulz
+# ---------------------------------------------------------------------------
+
+def _ns_iterations(X, steps, coeffs, emulate_bf16):
+    """Run the quintic iteration on a short-side-first matrix X (s x l).
+
+    Each step forms the Gram A = X X^T, the polynomial B = bA + cA^2 and the
+    combine X <- aX + BX. This equals aX + bX(X^T X) + cX(X^T X)^2 because
+    (X X^T)^k X = X (X^T X)^k ("About Muon: Why Not Adam", section "The lemma
+    that makes it possible").
+    """
+    a, b, c = coeffs
+    rnd = bf16_round if emulate_bf16 else (lambda v: v)
+    for _ in range(steps):
+        A = rnd(X @ X.T)
+        B = rnd(b * A + c * (A @ A))
+        X = rnd(a * X + B @ X)
+    return X
+
+
+def newton_schulz(G, steps=5, coeffs=DEFAULT_COEFFS, eps=EPS,
+                  emulate_bf16=False):
+    """Approximate orthogonal polar factor of G (float64).
+
+    "About Muon: Why Not Adam", section "The whole thing, in about forty
+    lines": normalise by the Frobenius norm plus eps so every singular value
+    lies in (0, 1], work on the short side (transpose when rows > columns),
+    iterate the quintic ``steps`` times, undo the transpose.
+
+    With ``emulate_bf16`` the input is rounded to bf16 before normalising and
+    the normalisation factor is applied exactly where the GPU applies it
+    (inside the first Gram and first combine); otherwise no rounding happens.
+    """
+    G = np.asarray(G, dtype=np.float64)
+    if G.ndim != 2:
+        raise ValueError("Newton-Schulz is defined for 2D matrices only")
+    transposed = G.shape[0] > G.shape[1]
+    if not emulate_bf16:
+        X = G / (np.linalg.norm(G) + eps)
+        if transposed:
+            X = X.T
+        X = _ns_iterations(X, steps, coeffs, False)
+        return X.T if transposed else X
+
+    # bf16-emulating diagnostic: Y = bf16(G); alpha = 1/(||G|| + eps) is
+    # folded into the first Gram (alpha^2) and the first combine (alpha).
+    alpha = 1.0 / (np.linalg.norm(G) + eps)
+    Y = bf16_round(G)
+    if transposed:
+        Y = Y.T
+    a, b, c = coeffs
+    if steps == 0:
+        X = alpha * Y
+    else:
+        A = bf16_round(alpha * alpha * (Y @ Y.T))
+        B = bf16_round(b * A + c * (A @ A))
+        X = bf16_round(alpha * (a * Y + B @ Y))
+        X = _ns_iterations(X, steps - 1, coeffs, True)
+    return X.T if transposed else X
+
+
+def ns_only(X, steps=5, coeffs=DEFAULT_COEFFS):
+    """The Newton-Schulz phases alone on an already-scaled X (no norm).
+
+    Used for the NS-only sweep workload, whose inputs are generated with
+    singular values already in [1e-4, 1]. Same orientation rule as
+    ``newton_schulz``.
+    """
+    X = np.asarray(X, dtype=np.float64)
+    transposed = X.shape[0] > X.shape[1]
+    if transposed:
+        X = X.T
+    X = _ns_iterations(X, steps, coeffs, False)
+    return X.T if transposed else X
+
+
+# ---------------------------------------------------------------------------
+# Momentum and Nesterov ("About Muon: Why Not Adam", section "The whole
+# thing, in about forty lines"; Nesterov: "Por qué AdamW ...", section
+# "Momentum: recordar el paso anterior")
+# ---------------------------------------------------------------------------
+
+def momentum_update(m, g, beta):
+    """m' = m + (1 - beta)(g - m) = beta*m + (1 - beta)*g (in float64)."""
+    m = np.asarray(m, dtype=np.float64)
+    g = np.asarray(g, dtype=np.float64)
+    return beta * m + (1.0 - beta) * g
+
+
+def nesterov_blend(g, m_new, beta, nesterov=True):
+    """u = g + beta*(m' - g) with Nesterov, else u = m'."""
+    g = np.asarray(g, dtype=np.float64)
+    m_new = np.asarray(m_new, dtype=np.float64)
+    if not nesterov:
+        return m_new.copy()
+    return g + beta * (m_new - g)
+
+
+# ---------------------------------------------------------------------------
+# Update scale and apply
+# ---------------------------------------------------------------------------
+
+def update_scale(m, n, mode=SCALE_MOONLIGHT, extra_scale=1.0):
+    """Shape multiplier for the orthogonalised update, (m, n) = p.shape.
+
+    * Moonlight 0.2*sqrt(max(m, n)) -- "About Muon: Why Not Adam", sections
+      "Scaling answers Problem 1" and "How Do We Turn It Into a Real
+      Optimizer?"; it is the multiplier of the program in "The whole thing,
+      in about forty lines".
+    * Jordan sqrt(max(1, m/n)) -- same page, "How Do We Turn It Into a Real
+      Optimizer?".
+    * Bernstein sqrt(fan-out / fan-in) = sqrt(m/n) -- same page, "The
+      spectral ball gives UV^T".
+    * None: 1.
+    ``extra_scale`` multiplies the result (the "extra scale factor" knob of
+    the Megatron configuration in "Why Muon Works").
+    """
+    m = float(m)
+    n = float(n)
+    if mode == SCALE_MOONLIGHT:
+        s = 0.2 * np.sqrt(max(m, n))
+    elif mode == SCALE_JORDAN:
+        s = np.sqrt(max(1.0, m / n))
+    elif mode == SCALE_BERNSTEIN:
+        s = np.sqrt(m / n)
+    elif mode == SCALE_NONE:
+        s = 1.0
+    else:
+        raise ValueError(f"unknown scale mode {mode}")
+    return s * float(extra_scale)
+
+
+def apply_update(p, O, lr, wd, scale):
+    """p' = p*(1 - lr*wd) - lr*scale*O (decoupled weight decay, then the step).
+
+    Both terms use the old p ("About Muon: Why Not Adam", section "The whole
+    thing, in about forty lines").
+    """
+    p = np.asarray(p, dtype=np.float64)
+    O = np.asarray(O, dtype=np.float64)
+    return p * (1.0 - lr * wd) - lr * scale * O
+
+
+# ---------------------------------------------------------------------------
+# Whole step
+# ---------------------------------------------------------------------------
+
+def muon_step_matrix(p, g, m, *, lr, beta=0.95, nesterov=True, wd=0.1,
+                     ns_steps=5, coeffs=DEFAULT_COEFFS,
+                     scale_mode=SCALE_MOONLIGHT, extra_scale=1.0,
+                     emulate_bf16=False):
+    """One Muon step on one matrix. Returns (p', m', O, ||u||_F).
+
+    Order: momentum, Nesterov blend, Newton-Schulz (normalise, orient,
+    iterate, orient back), scale, decoupled weight decay, write.
+    """
+    p = np.asarray(p, dtype=np.float64)
+    if p.ndim != 2:
+        raise ValueError("Muon applies to 2D weight matrices only")
+    m_new = momentum_update(m, g, beta)
+    u = nesterov_blend(g, m_new, beta, nesterov)
+    nu = float(np.linalg.norm(u))
+    O = newton_schulz(u, ns_steps, coeffs, EPS, emulate_bf16)
+    scale = update_scale(p.shape[0], p.shape[1], scale_mode, extra_scale)
+    p_new = apply_update(p, O, lr, wd, scale)
+    return p_new, m_new, O, nu
+
+
+def muon_step(params, grads, momenta, *, lr, beta=0.95, nesterov=True,
+              wd=0.1, ns_steps=5, coeffs=DEFAULT_COEFFS,
+              scale_mode=SCALE_MOONLIGHT, extra_scale=1.0,
+              emulate_bf16=False):
+    """One Muon step over a list of matrices, one at a time.
+
+    A ``None`` gradient skips its matrix (parameter and momentum unchanged).
+    Returns lists (params', momenta', O, norms); O and norm are None for
+    skipped matrices.
+    """
+    out_p, out_m, out_o, out_n = [], [], [], []
+    for p, g, m in zip(params, grads, momenta):
+        if g is None:
+            out_p.append(np.asarray(p, dtype=np.float64).copy())
+            out_m.append(np.asarray(m, dtype=np.float64).copy())
+            out_o.append(None)
+            out_n.append(None)
+            continue
+        r = muon_step_matrix(p, g, m, lr=lr, beta=beta, nesterov=nesterov,
+                             wd=wd, ns_steps=ns_steps, coeffs=coeffs,
+                             scale_mode=scale_mode, extra_scale=extra_scale,
+                             emulate_bf16=emulate_bf16)
+        out_p.append(r[0])
+        out_m.append(r[1])
+        out_o.append(r[2])
+        out_n.append(r[3])
+    return out_p, out_m, out_o, out_n

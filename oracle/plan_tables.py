@@ -1,0 +1,118 @@
+"""Independent restatement of the integer plan tables (test infrastructure only).
+
+Only ``tests/`` may import this module. The C++ plan builder in the CUDA
+library produces the same tables; a test compares the two bit for bit.
+
+The rules restated here:
+
+Orientation ("About Muon: Why Not Adam", section "The whole thing, in about
+forty lines"): a matrix with m > n (rows > columns) is "tall" and the
+iteration runs on its transpose; s = min(m, n), l = max(m, n). Square
+matrices are not transposed.
+
+Storage. Every bf16 (or, in the fp32 debug mode, fp32) matrix in the
+workspace is row-major with a leading dimension rounded up to a multiple of
+8 elements, so each row starts on a 16-byte boundary (the alignment the
+bulk-tensor copy engine requires):
+  * X ping-pong buffers X0, X1: m rows, ldx = round_up(n, 8).
+  * Gram A and polynomial B: s rows, lds = round_up(s, 8).
+The workspace begins with one float64 sum-of-squares accumulator per
+matrix, then an int32 error word, 4 bytes of padding and a uint64
+non-finite counter, padded to 1024 bytes; then all X0 regions, all X1
+regions, all A regions, all B regions, each region aligned to 1024 bytes.
+
+Tiles. Output tiles are BM = 128 rows by BN = 256 columns.
+  * Gram and polynomial (both symmetric s x s): tile (ti, tj) is listed iff
+    tj >= ti // 2, i.e. its 256-wide column block is on or right of the
+    256-block diagonal. Off-diagonal tiles are also written transposed, so
+    each entry is produced once.
+  * Combine (output in the original m x n layout): every tile of the
+    ceil(m/128) x ceil(n/256) grid. For wide matrices (m <= n) the column
+    block is the outer loop, for tall ones the row block.
+  Each phase's list is ordered by the matrix's reduction length K
+  (descending; Gram: K = l, polynomial and combine: K = s), ties by matrix
+  index, then by the per-matrix order above. A tile entry is
+  (matrix, ti, tj).
+
+Elementwise chunks. The fused momentum and apply kernels give each thread
+block CHUNK = 8192 consecutive elements of one matrix; chunk_prefix[i] is
+the number of chunks of matrices 0..i-1.
+"""
+
+from __future__ import annotations
+
+BM = 128
+BN = 256
+CHUNK = 8192
+ALIGN = 1024
+
+
+def round_up(x: int, k: int) -> int:
+    return (x + k - 1) // k * k
+
+
+def ceil_div(x: int, k: int) -> int:
+    return (x + k - 1) // k
+
+
+def matrix_geometry(m: int, n: int):
+    """(tall, s, l, ldx, lds) for an m x n matrix."""
+    tall = m > n
+    s = min(m, n)
+    l = max(m, n)
+    return tall, s, l, round_up(n, 8), round_up(s, 8)
+
+
+def workspace_layout(shapes, elem_bytes: int = 2):
+    """Byte offsets (X0, X1, A, B) per matrix and the total workspace size."""
+    count = len(shapes)
+    head = round_up(8 * count + 16, ALIGN)
+    off = head
+    regions = [[0, 0, 0, 0] for _ in range(count)]
+    for which in range(4):
+        for i, (m, n) in enumerate(shapes):
+            _, s, _, ldx, lds = matrix_geometry(m, n)
+            nbytes = (m * ldx if which < 2 else s * lds) * elem_bytes
+            regions[i][which] = off
+            off = round_up(off + nbytes, ALIGN)
+    return regions, off
+
+
+def _sym_tiles(s: int):
+    out = []
+    for ti in range(ceil_div(s, BM)):
+        for tj in range(ti // 2, ceil_div(s, BN)):
+            out.append((ti, tj))
+    return out
+
+
+def _comb_tiles(m: int, n: int):
+    rows, cols = ceil_div(m, BM), ceil_div(n, BN)
+    if m <= n:   # wide: column block outer
+        return [(ti, tj) for tj in range(cols) for ti in range(rows)]
+    return [(ti, tj) for ti in range(rows) for tj in range(cols)]
+
+
+def tile_lists(shapes):
+    """(gram, poly, comb) lists of (matrix, ti, tj)."""
+    gram, poly, comb = [], [], []
+    geo = [matrix_geometry(m, n) for (m, n) in shapes]
+
+    def order(klen):
+        return sorted(range(len(shapes)), key=lambda i: (-klen(i), i))
+
+    for i in order(lambda i: geo[i][2]):
+        gram += [(i, ti, tj) for ti, tj in _sym_tiles(geo[i][1])]
+    for i in order(lambda i: geo[i][1]):
+        poly += [(i, ti, tj) for ti, tj in _sym_tiles(geo[i][1])]
+    for i in order(lambda i: geo[i][1]):
+        m, n = shapes[i]
+        comb += [(i, ti, tj) for ti, tj in _comb_tiles(m, n)]
+    return gram, poly, comb
+
+
+def chunk_prefix(shapes):
+    out = [0]
+    for (m, n) in shapes:
+        out.append(out[-1] + ceil_div(m * n, CHUNK))
+    return out

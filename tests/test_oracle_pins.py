@@ -1,0 +1,372 @@
+"""Pins for the float64 oracle: printed values, closed forms, invariants.
+
+Every check here ties the oracle to something other than itself: numbers
+printed on the pages (``tests/golden``), the SVD closed form of the
+odd-polynomial lemma, the textbook convergent iterations, hand-unrolled
+recurrences and library routines (numpy SVD, torch bf16 conversion).
+"""
+
+import json
+import os
+
+import numpy as np
+import pytest
+
+from oracle import muon_oracle as O
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden", "ns_scalar_facts.json")
+
+
+def _golden():
+    with open(GOLDEN) as f:
+        return json.load(f)
+
+
+def _close_printed(x, entry_value, digits):
+    # The page prints rounded or truncated decimals (0.5545 appears as
+    # 0.554), so allow one unit of the last printed digit.
+    return abs(x - entry_value) <= 10.0 ** (-digits) + 1e-12
+
+
+def _haar(rng, n, k):
+    """n x k matrix with orthonormal columns (QR of a Gaussian, sign fixed)."""
+    q, r = np.linalg.qr(rng.standard_normal((n, k)))
+    return q * np.sign(np.diag(r))
+
+
+def _diag_ns(d, steps=5, coeffs=O.DEFAULT_COEFFS):
+    """The oracle's matrix Newton-Schulz on diag(d): returns the diagonal."""
+    out = O.newton_schulz(np.diag(d), steps, coeffs)
+    return np.diag(out)
+
+
+# ---------------------------------------------------------------------------
+# Printed scalar facts ("About Muon: Why Not Adam", section "The iteration
+# does not converge, and that is deliberate"), checked through the oracle's
+# matrix iteration wherever possible.
+# ---------------------------------------------------------------------------
+
+def test_golden_coefficients_match_oracle_default():
+    g = _golden()
+    assert tuple(g["coeffs"]) == O.DEFAULT_COEFFS
+
+
+def test_one_step_on_unit_matrix_gives_printed_p_of_1():
+    g = _golden()["p_at_1"]
+    # A 1x1 matrix normalises to 1/(1 + eps); one matrix step gives p(1).
+    out = O.newton_schulz(np.array([[5.0]]), steps=1)[0, 0]
+    assert _close_printed(out, g["value"], g["digits"])
+
+
+def test_five_steps_on_small_singular_values_match_printed():
+    g = _golden()
+    # diag(d) with ||d|| = 1: the normalised singular values are d itself
+    # (up to eps = 1e-7), so the output diagonal is p^5(d).
+    small = np.array([1e-3, 1e-4])
+    d = np.concatenate([[np.sqrt(1.0 - np.sum(small ** 2))], small])
+    out = _diag_ns(d)
+    e3, e4 = g["five_steps_from_1e-3"], g["five_steps_from_1e-4"]
+    assert _close_printed(out[1], e3["value"], e3["digits"])
+    assert _close_printed(out[2], e4["value"], e4["digits"])
+
+
+def test_fixed_points_and_slopes_match_printed():
+    g = _golden()
+    a, b, c = O.DEFAULT_COEFFS
+    # p(s) = s  <=>  c s^4 + b s^2 + (a - 1) = 0  (s != 0): a quadratic in s^2.
+    disc = b * b - 4 * c * (a - 1)
+    roots = sorted(np.sqrt([(-b - np.sqrt(disc)) / (2 * c), (-b + np.sqrt(disc)) / (2 * c)]))
+    fp = g["fixed_points"]
+    for r, v in zip(roots, fp["value"]):
+        assert _close_printed(r, v, fp["digits"])
+    # The oracle's matrix iteration leaves the fixed point inside (0, 1]
+    # where it is: diag(r, sqrt(1 - r^2)) has unit norm, so one matrix step
+    # maps the normalised singular value r to p(r) = r.
+    r = roots[0]
+    d = np.array([r, np.sqrt(1.0 - r * r)])
+    assert abs(_diag_ns(d, steps=1)[0] - r) < 1e-6
+    # Slope by central difference of the oracle's scalar map.
+    sl = g["slope_at_fixed_points"]
+    for r, v in zip(roots, sl["value"]):
+        h = 1e-6
+        slope = (O.ns_poly(r + h) - O.ns_poly(r - h)) / (2 * h)
+        assert _close_printed(slope, v, sl["digits"])
+    sz = g["slope_at_zero"]
+    assert _close_printed((O.ns_poly(1e-7) - O.ns_poly(-1e-7)) / 2e-7, sz["value"], sz["digits"])
+
+
+def test_maximum_on_unit_interval_matches_printed():
+    g = _golden()
+    s = np.linspace(0.0, 1.0, 2_000_001)
+    v = O.ns_poly(s)
+    mx, am = g["max_on_unit_interval"], g["argmax_on_unit_interval"]
+    assert _close_printed(v.max(), mx["value"], mx["digits"])
+    assert _close_printed(s[v.argmax()], am["value"], am["digits"])
+
+
+def test_iterates_settle_in_printed_band():
+    g = _golden()["cycle_band"]
+    s = np.linspace(1e-3, 1.0, 2001)
+    s = O.ns_poly_iterate(s, steps=200)
+    lo, hi = np.inf, -np.inf
+    for _ in range(200):
+        s = O.ns_poly(s)
+        lo, hi = min(lo, s.min()), max(hi, s.max())
+    assert _close_printed(lo, g["value"][0], g["digits"])
+    assert _close_printed(hi, g["value"][1], g["digits"])
+
+
+# ---------------------------------------------------------------------------
+# Odd-polynomial lemma: NS(G) = U diag(f(sigma / (||G|| + eps))) V^T
+# ("About Muon: Why Not Adam", section "The lemma that makes it possible").
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("shape", [(3, 5), (8, 8), (16, 4), (33, 17), (1, 7), (7, 1), (40, 64)])
+@pytest.mark.parametrize("steps", [0, 1, 5])
+def test_ns_equals_svd_closed_form(shape, steps):
+    rng = np.random.default_rng(hash(shape) % 2 ** 32 + steps)
+    G = rng.standard_normal(shape)
+    U, sig, Vt = np.linalg.svd(G, full_matrices=False)
+    x = sig / (np.linalg.norm(G) + O.EPS)
+    a, b, c = O.DEFAULT_COEFFS
+    for _ in range(steps):          # scalar map, written independently here
+        x = a * x + b * x ** 3 + c * x ** 5
+    expect = (U * x) @ Vt
+    got = O.newton_schulz(G, steps)
+    assert np.max(np.abs(got - expect)) < 1e-12
+
+
+@pytest.mark.parametrize("shape", [(12, 20), (20, 12), (16, 16)])
+def test_singular_vectors_preserved(shape):
+    rng = np.random.default_rng(7)
+    G = rng.standard_normal(shape)
+    U, sig, Vt = np.linalg.svd(G, full_matrices=False)
+    D = U.T @ O.newton_schulz(G) @ Vt.T
+    off = D - np.diag(np.diag(D))
+    assert np.max(np.abs(off)) < 1e-12
+    assert np.all(np.diag(D) > 0)
+
+
+def test_rank_one_closed_form():
+    rng = np.random.default_rng(3)
+    x, y = rng.standard_normal(9), rng.standard_normal(13)
+    G = 2.5 * np.outer(x, y)
+    f1 = O.ns_poly_iterate(np.linalg.norm(G) / (np.linalg.norm(G) + O.EPS))
+    expect = f1 * np.outer(x, y) / (np.linalg.norm(x) * np.linalg.norm(y))
+    assert np.max(np.abs(O.newton_schulz(G) - expect)) < 1e-12
+
+
+def test_scaled_orthogonal_closed_form():
+    rng = np.random.default_rng(4)
+    n = 24
+    Q = _haar(rng, n, n)
+    G = 3.0 * Q
+    # ||G||_F = 3 sqrt(n): every normalised singular value is 3/(3 sqrt(n)+eps).
+    f = O.ns_poly_iterate(3.0 / (3.0 * np.sqrt(n) + O.EPS))
+    assert np.max(np.abs(O.newton_schulz(G) - f * Q)) < 1e-12
+
+
+def test_diagonal_signs():
+    d = np.array([0.5, -0.3, 0.2, -0.01])
+    out = _diag_ns(d)
+    assert np.all(np.sign(out) == np.sign(d))
+    full = O.newton_schulz(np.diag(d))
+    assert np.max(np.abs(full - np.diag(np.diag(full)))) == 0.0
+
+
+# ---------------------------------------------------------------------------
+# Textbook convergent members of the family reduce NS to the polar factor
+# ("About Muon: Why Not Adam", section "The iteration does not converge, and
+# that is deliberate"): cubic 1.5x - 0.5x^3 and quintic (15/8, -10/8, 3/8).
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("coeffs,steps", [((1.5, -0.5, 0.0), 60), ((15 / 8, -10 / 8, 3 / 8), 40)])
+@pytest.mark.parametrize("shape", [(10, 16), (16, 10), (12, 12)])
+def test_convergent_coefficients_give_polar_factor(coeffs, steps, shape):
+    rng = np.random.default_rng(11)
+    m, n = shape
+    k = min(m, n)
+    U, V = _haar(rng, m, k), _haar(rng, n, k)
+    sig = np.linspace(1.0, 0.2, k)        # well conditioned
+    G = (U * sig) @ V.T
+    polar = U @ V.T
+    got = O.newton_schulz(G, steps, coeffs)
+    assert np.max(np.abs(got - polar)) < 1e-10
+    # LMO optimality ("The spectral ball gives UV^T"): <G, UV^T> = sum sigma.
+    assert abs(np.sum(G * got) - sig.sum()) < 1e-9
+    # ||UV^T||_F^2 = min(m, n) ("Scaling answers Problem 1").
+    assert abs(np.sum(got ** 2) - k) < 1e-9
+
+
+# ---------------------------------------------------------------------------
+# Invariances
+# ---------------------------------------------------------------------------
+
+def test_transpose_invariance():
+    rng = np.random.default_rng(5)
+    G = rng.standard_normal((9, 21))
+    assert np.max(np.abs(O.newton_schulz(G.T) - O.newton_schulz(G).T)) < 1e-13
+
+
+def test_scale_invariance_up_to_eps():
+    # LMO(alpha G) = LMO(G) ("How Do We Turn It Into a Real Optimizer?").
+    rng = np.random.default_rng(6)
+    G = rng.standard_normal((9, 21))
+    assert np.max(np.abs(O.newton_schulz(1e3 * G) - O.newton_schulz(G))) < 1e-6
+
+
+def test_square_is_not_transposed_but_agrees():
+    rng = np.random.default_rng(8)
+    G = rng.standard_normal((15, 15))
+    X = G / (np.linalg.norm(G) + O.EPS)
+    alt = O.newton_schulz(X.T * (np.linalg.norm(G) + O.EPS)).T
+    assert np.max(np.abs(O.newton_schulz(G) - alt)) < 1e-12
+
+
+def test_zero_gradient_gives_zero_update():
+    out = O.newton_schulz(np.zeros((4, 6)))
+    assert np.all(out == 0.0)
+
+
+def test_ns_only_matches_normalised_path():
+    rng = np.random.default_rng(9)
+    G = rng.standard_normal((6, 10))
+    X = G / (np.linalg.norm(G) + O.EPS)
+    assert np.max(np.abs(O.ns_only(X) - O.newton_schulz(G))) < 1e-14
+
+
+# ---------------------------------------------------------------------------
+# Momentum and Nesterov: hand-unrolled three-step recurrence from zero.
+# ---------------------------------------------------------------------------
+
+def test_momentum_nesterov_unrolled():
+    rng = np.random.default_rng(10)
+    beta = 0.95
+    g1, g2, g3 = (rng.standard_normal((3, 4)) for _ in range(3))
+    m = np.zeros((3, 4))
+    m = O.momentum_update(m, g1, beta)
+    u1 = O.nesterov_blend(g1, m, beta)
+    assert np.allclose(m, (1 - beta) * g1, rtol=0, atol=1e-15)
+    assert np.allclose(u1, (1 - beta ** 2) * g1, rtol=0, atol=1e-15)
+    m = O.momentum_update(m, g2, beta)
+    m2 = beta * (1 - beta) * g1 + (1 - beta) * g2
+    assert np.allclose(m, m2, rtol=0, atol=1e-15)
+    u2 = O.nesterov_blend(g2, m, beta)
+    assert np.allclose(u2, (1 - beta) * g2 + beta * m2, rtol=0, atol=1e-15)
+    m = O.momentum_update(m, g3, beta)
+    m3 = beta ** 2 * (1 - beta) * g1 + beta * (1 - beta) * g2 + (1 - beta) * g3
+    assert np.allclose(m, m3, rtol=0, atol=1e-15)
+    u3 = O.nesterov_blend(g3, m, beta)
+    assert np.allclose(u3, (1 - beta) * g3 + beta * m3, rtol=0, atol=1e-15)
+    # Nesterov off: the update direction is the buffer itself.
+    assert np.array_equal(O.nesterov_blend(g3, m, beta, nesterov=False), m)
+
+
+def test_nesterov_off_beta_zero_is_plain_gradient():
+    rng = np.random.default_rng(12)
+    g = rng.standard_normal((5, 5))
+    m = O.momentum_update(rng.standard_normal((5, 5)), g, 0.0)
+    assert np.array_equal(O.nesterov_blend(g, m, 0.0, nesterov=False), g)
+
+
+# ---------------------------------------------------------------------------
+# Scale and apply
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("shape", [(64, 256), (256, 64), (128, 128)])
+def test_moonlight_scale_gives_entry_rms_point_two(shape):
+    # "Scaling answers Problem 1": 0.2 sqrt(max(m, n)) makes the entry RMS of
+    # the scaled polar factor 0.2.
+    rng = np.random.default_rng(13)
+    m, n = shape
+    k = min(m, n)
+    polar = _haar(rng, m, k) @ _haar(rng, n, k).T
+    lr = 1e-3
+    p = rng.standard_normal(shape)
+    scale = O.update_scale(m, n, O.SCALE_MOONLIGHT)
+    dp = O.apply_update(p, polar, lr, 0.0, scale) - p
+    rms = np.sqrt(np.mean(dp ** 2)) / lr
+    assert abs(rms - 0.2) < 1e-12
+
+
+def test_jordan_and_bernstein_scales():
+    # "How Do We Turn It Into a Real Optimizer?": Jordan = Bernstein when
+    # m >= n, Jordan = 1 when the layer shrinks (m < n).
+    assert O.update_scale(64, 256, O.SCALE_JORDAN) == 1.0
+    assert O.update_scale(256, 64, O.SCALE_JORDAN) == O.update_scale(256, 64, O.SCALE_BERNSTEIN) == 2.0
+    # "The spectral ball gives UV^T": Bernstein's prefactor on a square layer is 1.
+    assert O.update_scale(300, 300, O.SCALE_BERNSTEIN) == 1.0
+    assert O.update_scale(300, 300, O.SCALE_MOONLIGHT) == pytest.approx(0.2 * np.sqrt(300), rel=1e-15)
+    assert O.update_scale(5, 7, O.SCALE_NONE, 2.5) == 2.5
+
+
+def test_weight_decay_alone():
+    p = np.array([[1.0, -2.0], [3.0, 4.0]])
+    out = O.apply_update(p, np.zeros_like(p), lr=0.1, wd=0.5, scale=3.0)
+    assert np.allclose(out, p * 0.95, rtol=0, atol=1e-15)
+
+
+def test_muon_step_skips_none_and_checks_2d():
+    rng = np.random.default_rng(14)
+    p = [rng.standard_normal((4, 6)), rng.standard_normal((6, 4))]
+    m = [np.zeros((4, 6)), np.ones((6, 4))]
+    g = [rng.standard_normal((4, 6)), None]
+    P, M, Os, N = O.muon_step(p, g, m, lr=0.1)
+    assert np.array_equal(P[1], p[1]) and np.array_equal(M[1], m[1])
+    assert Os[1] is None and N[1] is None
+    assert N[0] == pytest.approx(np.linalg.norm(O.nesterov_blend(g[0], M[0], 0.95)))
+    with pytest.raises(ValueError):
+        O.muon_step_matrix(np.zeros(3), np.zeros(3), np.zeros(3), lr=0.1)
+
+
+def test_full_step_against_composed_closed_form():
+    # p' = p(1 - lr wd) - lr*scale*U f^5(sigma_u/(||u||+eps)) V^T with u the
+    # Nesterov blend of the hand-unrolled first step, u = (1 - beta^2) g.
+    rng = np.random.default_rng(15)
+    p, g = rng.standard_normal((6, 9)), rng.standard_normal((6, 9))
+    beta, lr, wd = 0.9, 0.02, 0.1
+    u = (1 - beta ** 2) * g
+    U, sig, Vt = np.linalg.svd(u, full_matrices=False)
+    x = sig / (np.linalg.norm(u) + O.EPS)
+    a, b, c = O.DEFAULT_COEFFS
+    for _ in range(5):
+        x = a * x + b * x ** 3 + c * x ** 5
+    expect = p * (1 - lr * wd) - lr * 0.2 * np.sqrt(9) * ((U * x) @ Vt)
+    got, _, _, _ = O.muon_step_matrix(p, g, np.zeros_like(p), lr=lr, beta=beta, wd=wd)
+    assert np.max(np.abs(got - expect)) < 1e-13
+
+
+# ---------------------------------------------------------------------------
+# bf16 rounding (diagnostic mode) against torch's float32 -> bfloat16 cast.
+# ---------------------------------------------------------------------------
+
+def test_bf16_round_matches_torch_on_float32_values():
+    torch = pytest.importorskip("torch")
+    rng = np.random.default_rng(16)
+    x = np.concatenate([
+        rng.standard_normal(20000) * 10.0 ** rng.integers(-20, 20, 20000),
+        # ties and near-ties around 1
+        1.0 + np.arange(-64, 64) * 2.0 ** -9,
+        np.array([0.0, -0.0, 1.0, -1.0, 3.0e38, np.inf, -np.inf]),
+    ]).astype(np.float32)
+    ref = torch.from_numpy(x).to(torch.bfloat16).to(torch.float64).numpy()
+    got = O.bf16_round(x.astype(np.float64))
+    assert np.array_equal(got, ref)
+
+
+def test_bf16_ties_to_even():
+    one = 1.0
+    ulp = 2.0 ** -7
+    assert O.bf16_round(np.array([one + ulp / 2]))[0] == one          # tie -> even
+    assert O.bf16_round(np.array([one + 3 * ulp / 2]))[0] == one + 2 * ulp
+    assert O.bf16_round(np.array([one + ulp / 2 + 1e-12]))[0] == one + ulp
+
+
+def test_emulated_bf16_close_to_exact():
+    rng = np.random.default_rng(17)
+    m, n = 48, 80
+    G = (_haar(rng, m, m) * np.linspace(1, 0.05, m)) @ _haar(rng, n, m).T
+    exact = O.newton_schulz(G)
+    emu = O.newton_schulz(G, emulate_bf16=True)
+    rel = np.linalg.norm(emu - exact) / np.linalg.norm(exact)
+    assert 1e-5 < rel < 2e-2
