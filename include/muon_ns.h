@@ -1,0 +1,248 @@
+/*
+ * muon_ns.h -- C ABI of the B200 (sm_100a) Muon optimizer step.
+ *
+ * One Muon step on a set of 2D weight matrices, entirely in hand-written
+ * CUDA kernels:
+ *   1. momentum m' = beta*m + (1-beta)*g, Nesterov blend u = g + beta*(m'-g),
+ *      per-matrix sum of squares of u and the bf16 cast of u (one kernel);
+ *   2. the quintic Newton-Schulz iteration on the short side,
+ *      A = X X^T, B = bA + cA^2, X <- aX + BX, with X = u / (||u||_F + 1e-7)
+ *      (tensor-core GEMMs, one launch per phase for all matrices);
+ *   3. p' = p*(1 - lr*wd) - lr*scale(m, n)*O (one kernel).
+ *
+ * Sources (web pages, cited by title and section):
+ *   "About Muon: Why Not Adam": "The whole thing, in about forty lines"
+ *     (step order, eps, transpose rule, lerp forms, defaults, Moonlight
+ *     scale); "The lemma that makes it possible"; "The iteration does not
+ *     converge, and that is deliberate" (coefficients); "How Do We Turn It
+ *     Into a Real Optimizer?" (Jordan and Moonlight multipliers,
+ *     (m, n) = (fan-out, fan-in) = p.shape); "The spectral ball gives UV^T"
+ *     (Bernstein multiplier).
+ *   "Por que AdamW para entrenar modelos de lenguaje, y que esta cambiando",
+ *     "Momentum: recordar el paso anterior" (Muon uses Nesterov).
+ *   "The Optimizer Wars: How Muon Is Replacing Adam in Frontier AI
+ *     Training", "What is Muon? Momentum orthogonalized by Newton-Schulz"
+ *     (five quintic steps in bf16 on tensor cores).
+ *   "Why Muon Works", section 6 configuration block (scale mode, extra
+ *     scale factor, number of NS steps, Nesterov flag).
+ *
+ * Conventions for every entry point:
+ *   - Return value: a muon_status code; MUON_OK (0) on success. No C++
+ *     exception crosses this boundary. muon_last_error() returns a
+ *     thread-local description of the last failure on the calling thread.
+ *   - "Device pointer" means memory of the handle's device; "host array"
+ *     means an ordinary host array read during the call only.
+ *   - Matrices are row-major m x n with (m, n) = (fan-out, fan-in), i.e. the
+ *     PyTorch layout of a weight p of shape (m, n). The shape table is a
+ *     host int32 array shapes[count][3] = {m, n, flags}; m, n >= 1;
+ *     flags bit 0 (MUON_FLAG_GRAD_BF16) says the gradient is bf16 (else
+ *     fp32). Other flag bits must be zero.
+ *   - Parameters and momenta are fp32, densely packed (row stride n).
+ *     Gradients are fp32 or bf16 per the flag, densely packed. Every
+ *     caller pointer must be 16-byte aligned; params, grads and momenta of
+ *     one matrix must not overlap.
+ *   - "X layout": a bf16 (fp32 in the fp32 debug mode) row-major m x ldx
+ *     buffer with ldx = round_up(n, 8); columns n..ldx-1 are ignored on
+ *     input and left unspecified on output.
+ *   - Work is enqueued on `stream` (a cudaStream_t; NULL = legacy default
+ *     stream) and runs asynchronously; the call does not wait for the GPU
+ *     unless documented. The caller keeps every buffer alive until the
+ *     stream has reached the end of the enqueued work.
+ *   - The handle is not thread-safe: one thread at a time per handle.
+ */
+#ifndef MUON_NS_H
+#define MUON_NS_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Status codes. */
+enum muon_status {
+  MUON_OK = 0,
+  MUON_ERR_INVALID_ARG = 1, /* bad shape, count, pointer, alignment, flag   */
+  MUON_ERR_CUDA = 2,        /* a CUDA runtime/driver call failed           */
+  MUON_ERR_OOM = 3,         /* workspace above the configured cap, or a
+                               device allocation failed                     */
+  MUON_ERR_TIMEOUT = 4,     /* a bounded device-side wait expired; the
+                               kernel stopped early and results are invalid */
+  MUON_ERR_NONFINITE = 5,   /* reported by muon_get_status only            */
+  MUON_ERR_NO_DEVICE = 6,   /* no usable CUDA device                       */
+  MUON_ERR_UNSUPPORTED = 7  /* device is not sm_100                        */
+};
+
+/* Update-scale families, (m, n) = (fan-out, fan-in). */
+enum muon_scale_mode {
+  MUON_SCALE_MOONLIGHT = 0, /* 0.2*sqrt(max(m,n)): "About Muon: Why Not
+                               Adam", "How Do We Turn It Into a Real
+                               Optimizer?" and the program in "The whole
+                               thing, in about forty lines"               */
+  MUON_SCALE_JORDAN = 1,    /* sqrt(max(1, m/n)): same section            */
+  MUON_SCALE_BERNSTEIN = 2, /* sqrt(m/n) = sqrt(fan-out/fan-in):
+                               "The spectral ball gives UV^T"             */
+  MUON_SCALE_NONE = 3       /* 1                                          */
+};
+
+/* Newton-Schulz arithmetic. */
+enum muon_ns_precision {
+  MUON_NS_BF16 = 0, /* bf16 operands, fp32 tensor-core accumulation,
+                       one round-to-nearest-even per GEMM output (default) */
+  MUON_NS_FP32 = 1  /* debug: fp32 operands and FFMA accumulation          */
+};
+
+#define MUON_FLAG_GRAD_BF16 1
+
+typedef struct muon_config {
+  int scale_mode;             /* enum muon_scale_mode; default MOONLIGHT    */
+  float extra_scale;          /* multiplies the scale; default 1.0
+                                 ("Why Muon Works", configuration block)   */
+  int ns_precision;           /* enum muon_ns_precision; default BF16      */
+  int check_nonfinite;        /* 1: count non-finite u entries; read back
+                                 with muon_get_status. Default 0           */
+  int num_sms;                /* persistent-grid width; 0 = all SMs        */
+  size_t workspace_cap_bytes; /* 0 = no cap                                */
+  double wait_timeout_s;      /* limit of every device-side wait; a wait
+                                 that runs out sets the error word and the
+                                 kernel returns. Default 2.0 seconds       */
+} muon_config;
+
+typedef struct muon_handle muon_handle;
+
+/* Fill *cfg with the defaults listed above. Returns MUON_ERR_INVALID_ARG if
+ * cfg is NULL. Needs no GPU. */
+int muon_config_init(muon_config* cfg);
+
+/* Create a handle on CUDA device `device`. cfg may be NULL (defaults).
+ * Allocates nothing large: the workspace is allocated on the first step of
+ * a given shape table and reused while the table is unchanged. Fails with
+ * MUON_ERR_NO_DEVICE / MUON_ERR_UNSUPPORTED when the device is missing or
+ * not sm_100. *out is set only on success. */
+int muon_init(int device, const muon_config* cfg, muon_handle** out);
+
+/* Wait for the handle's work, free its workspace and the handle.
+ * NULL is accepted and ignored. */
+int muon_destroy(muon_handle* h);
+
+/* One Muon step over `count` matrices ("About Muon: Why Not Adam", "The
+ * whole thing, in about forty lines").
+ *   params[i]  : device pointer, fp32 m x n, updated in place.
+ *   grads[i]   : device pointer, fp32 or bf16 m x n (shapes flag); NULL
+ *                skips matrix i entirely (its param and momentum are left
+ *                unchanged), like a parameter without a gradient.
+ *   momenta[i] : device pointer, fp32 m x n, updated in place; the caller
+ *                zero-initialises it before the first step.
+ *   params, grads, momenta are HOST arrays of `count` device pointers.
+ *   shapes     : host int32[count][3], see the conventions above.
+ *   lr, beta, wd : learning rate, momentum (0 <= beta < 1), decoupled
+ *                weight decay (p is multiplied by 1 - lr*wd).
+ *   nesterov   : 1 = u = g + beta*(m' - g); 0 = u = m'.
+ *   ns_steps   : number of quintic iterations, 0..64 (0 returns the
+ *                normalised u).
+ *   coeffs     : host float[3] = (a, b, c); NULL = (3.4445, -4.7750, 2.0315).
+ *   stream     : cudaStream_t.
+ * Scale mode, extra scale and precision come from the handle's config.
+ * The first call for a shape table builds the plan and the workspace
+ * (device allocation and a host-to-device copy of the tables; do it before
+ * any stream capture); later calls with the same shape table and pointers
+ * only enqueue kernels and are safe to capture in a CUDA graph. */
+int muon_step(muon_handle* h, float* const* params, const void* const* grads,
+              float* const* momenta, const int32_t* shapes, int count,
+              float lr, float beta, int nesterov, float wd, int ns_steps,
+              const float* coeffs, void* stream);
+
+/* Same step with every tensor in HOST memory (pinned memory gives
+ * asynchronous copies): the library copies params, grads and momenta to
+ * its own device staging area, runs muon_step there and copies params and
+ * momenta back, all on `stream`. The host buffers must stay valid and
+ * untouched until the stream completes. Staging is allocated on first use
+ * per shape table and counts against the workspace cap. */
+int muon_step_host(muon_handle* h, float* const* params,
+                   const void* const* grads, float* const* momenta,
+                   const int32_t* shapes, int count, float lr, float beta,
+                   int nesterov, float wd, int ns_steps, const float* coeffs,
+                   void* stream);
+
+/* ---- Stage entry points (each a row of the step; used by the tests and
+ *      the NS-only sweep). Same validation and conventions. ---- */
+
+/* Stage 1 (momentum, Nesterov, norm, cast). For each matrix with a
+ * non-NULL grad: momenta[i] <- beta*m + (1-beta)*g (in place);
+ * u = nesterov ? g + beta*(m' - g) : m'; y[i] <- cast(u) in X layout
+ * (bf16 round-to-nearest-even, or fp32 in the fp32 mode);
+ * sumsq[i] <- sum of u^2 (fp64, device array of count doubles, overwritten;
+ * left unchanged for skipped matrices). */
+int muon_momentum_norm(muon_handle* h, const void* const* grads,
+                       float* const* momenta, void* const* y, double* sumsq,
+                       const int32_t* shapes, int count, float beta,
+                       int nesterov, void* stream);
+
+/* Stage 2 (Newton-Schulz). For each matrix: X0 = x_in[i] * alpha with
+ * alpha = 1/(sqrt(sumsq[i]) + 1e-7) when sumsq (device array) is non-NULL,
+ * else alpha = 1; if m > n the iteration runs on the transpose (through
+ * operand layout, no transposed copy); ns_steps iterations with `coeffs`;
+ * result in x_out[i]. x_in and x_out are device pointers in X layout and
+ * must not overlap; x_in is not modified. ns_steps = 0 copies alpha*x_in
+ * (rounded to the storage type) to x_out. */
+int muon_newton_schulz(muon_handle* h, const void* const* x_in,
+                       void* const* x_out, const double* sumsq,
+                       const int32_t* shapes, int count, int ns_steps,
+                       const float* coeffs, void* stream);
+
+/* Stage 3 (apply). params[i] <- params[i]*(1 - lr*wd) - lr*scale*o_scale*O
+ * with O = o[i] (X layout, upcast exactly to fp32), scale from the handle's
+ * scale mode and extra scale, o_scale = 1/(sqrt(sumsq[i]) + 1e-7) when
+ * sumsq (device array) is non-NULL, else 1. A NULL o[i] skips matrix i. */
+int muon_apply(muon_handle* h, float* const* params, const void* const* o,
+               const double* sumsq, const int32_t* shapes, int count,
+               float lr, float wd, void* stream);
+
+/* ---- Plan, workspace and status ---- */
+
+/* Integer plan tables for a shape table, computed on the host (needs no
+ * GPU). Any output pointer may be NULL.
+ *   ws_bytes      : total workspace bytes for `ns_precision`.
+ *   region_offsets: int64[count][4], byte offsets of X0, X1, A, B.
+ *   ntiles        : int32[3], tile counts of the Gram, polynomial and
+ *                   combine phases.
+ *   tiles         : int32[ntiles[0]+ntiles[1]+ntiles[2]][3] =
+ *                   {matrix, row tile, column tile} for the three phases,
+ *                   one after the other.
+ *   chunk_prefix  : int64[count+1], elementwise chunks before matrix i.
+ * Call once with tiles = NULL to learn ntiles. */
+int muon_plan_query(const int32_t* shapes, int count, int ns_precision,
+                    int64_t* ws_bytes, int64_t* region_offsets,
+                    int32_t* ntiles, int32_t* tiles, int64_t* chunk_prefix);
+
+/* Workspace bytes the handle would allocate for this shape table
+ * (excluding muon_step_host staging). */
+int muon_workspace_size(muon_handle* h, const int32_t* shapes, int count,
+                        size_t* bytes);
+
+/* Device base address and size of the current workspace (for inspection by
+ * tests; the layout is given by muon_plan_query). */
+int muon_workspace_ptr(muon_handle* h, void** base, size_t* bytes);
+
+/* Wait for `stream`, then report the device error word (0 = none, else the
+ * code of the first expired wait) and the non-finite count, and clear both.
+ * Returns MUON_ERR_TIMEOUT if the error word was set, MUON_ERR_NONFINITE if
+ * only the counter was non-zero, else MUON_OK. Either output may be NULL. */
+int muon_get_status(muon_handle* h, void* stream, int32_t* error_word,
+                    uint64_t* nonfinite_count);
+
+/* Number of kernels the last muon_step / stage call enqueued. */
+int muon_last_launch_count(muon_handle* h, int32_t* launches);
+
+/* Thread-local text of the last error ("" if none). Never NULL. */
+const char* muon_last_error(void);
+
+/* Library version string. */
+const char* muon_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MUON_NS_H */

@@ -1,0 +1,283 @@
+"""Muon optimizer step for sets of 2D weight matrices on B200 (sm_100a).
+
+A thin Python binding over the C ABI in ``include/muon_ns.h``: it only turns
+torch tensors into device pointers, shape tables and the current CUDA
+stream. Every stage of the step runs in the library's CUDA kernels; there is
+no Python or CPU fallback.
+
+    import torch, muon_newton_schulz_03_b200 as muon
+    opt = muon.Muon(device=0)                     # Moonlight scale, bf16 NS
+    opt.step(params, grads, momenta, lr=2e-4)     # lists of 2D CUDA tensors
+
+Readings of the method (see the C header): momentum EMA with the Nesterov
+blend, u / (||u||_F + 1e-7), five quintic Newton-Schulz steps with
+(3.4445, -4.7750, 2.0315) on the short side, scale * lr update with decoupled
+weight decay ("About Muon: Why Not Adam", "The whole thing, in about forty
+lines").
+"""
+
+from __future__ import annotations
+
+import ctypes
+
+from ._lib import EXPORTED, MuonConfig, MuonError, check, lib_path, load
+
+__all__ = ["Muon", "MuonError", "plan_query", "x_layout", "round_up", "SCALE_MODES", "DEFAULT_COEFFS",
+           "EXPORTED", "lib_path", "load"]
+
+DEFAULT_COEFFS = (3.4445, -4.7750, 2.0315)
+SCALE_MODES = {"moonlight": 0, "jordan": 1, "bernstein": 2, "none": 3}
+PRECISIONS = {"bf16": 0, "fp32": 1}
+FLAG_GRAD_BF16 = 1
+
+
+def round_up(x: int, k: int) -> int:
+    return (x + k - 1) // k * k
+
+
+def _ptr_array(ptrs):
+    arr = (ctypes.c_void_p * len(ptrs))()
+    for i, p in enumerate(ptrs):
+        arr[i] = p
+    return arr
+
+
+def _shapes_array(shapes):
+    arr = (ctypes.c_int32 * (3 * len(shapes)))()
+    for i, (m, n, f) in enumerate(shapes):
+        arr[3 * i], arr[3 * i + 1], arr[3 * i + 2] = m, n, f
+    return arr
+
+
+def _coeffs(coeffs):
+    if coeffs is None:
+        return None
+    c = (ctypes.c_float * 3)(*[float(v) for v in coeffs])
+    return c
+
+
+def _stream_handle(stream):
+    import torch
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _ptr(t):
+    return None if t is None else t.data_ptr()
+
+
+def _check_2d(t, what, dtypes, device=None, contiguous=True):
+    import torch
+    if t.dim() != 2:
+        raise ValueError(f"{what} must be 2D (Muon applies to 2D weight matrices), got shape {tuple(t.shape)}")
+    if t.dtype not in dtypes:
+        raise TypeError(f"{what} must have dtype in {dtypes}, got {t.dtype}")
+    if contiguous and not t.is_contiguous():
+        raise ValueError(f"{what} must be contiguous")
+    if device is not None and t.device != device:
+        raise ValueError(f"{what} must be on {device}, got {t.device}")
+    return torch
+
+
+def x_layout(m: int, n: int, dtype, device):
+    """An empty X-layout buffer: row-major m x round_up(n, 8)."""
+    import torch
+    return torch.empty((m, round_up(n, 8)), dtype=dtype, device=device)
+
+
+def plan_query(shapes, ns_precision: str = "bf16"):
+    """Integer plan tables of a shape table (list of (m, n) or (m, n, flags)).
+
+    Returns dict(ws_bytes, region_offsets [count][4], tiles (gram, poly,
+    comb lists of (mat, ti, tj)), chunk_prefix). Needs no GPU.
+    """
+    lib = load()
+    sh = [(int(s[0]), int(s[1]), int(s[2]) if len(s) > 2 else 0) for s in shapes]
+    count = len(sh)
+    arr = _shapes_array(sh)
+    prec = PRECISIONS[ns_precision]
+    nt = (ctypes.c_int32 * 3)()
+    ws = ctypes.c_int64()
+    check(lib.muon_plan_query(arr, count, prec, ctypes.byref(ws), None, nt, None, None))
+    total = nt[0] + nt[1] + nt[2]
+    offs = (ctypes.c_int64 * (4 * count))()
+    tiles = (ctypes.c_int32 * (3 * max(total, 1)))()
+    pref = (ctypes.c_int64 * (count + 1))()
+    check(lib.muon_plan_query(arr, count, prec, ctypes.byref(ws), offs, nt, tiles, pref))
+    tl = [(tiles[3 * k], tiles[3 * k + 1], tiles[3 * k + 2]) for k in range(total)]
+    return {
+        "ws_bytes": ws.value,
+        "region_offsets": [list(offs[4 * i:4 * i + 4]) for i in range(count)],
+        "tiles": (tl[:nt[0]], tl[nt[0]:nt[0] + nt[1]], tl[nt[0] + nt[1]:]),
+        "chunk_prefix": list(pref),
+    }
+
+
+class Muon:
+    """A handle of the Muon library on one CUDA device."""
+
+    def __init__(self, device: int = 0, scale_mode: str = "moonlight", extra_scale: float = 1.0,
+                 ns_precision: str = "bf16", check_nonfinite: bool = False, num_sms: int = 0,
+                 workspace_cap_bytes: int = 0, wait_timeout_s: float = 2.0):
+        self._lib = load()
+        cfg = MuonConfig()
+        check(self._lib.muon_config_init(ctypes.byref(cfg)))
+        cfg.scale_mode = SCALE_MODES[scale_mode]
+        cfg.extra_scale = float(extra_scale)
+        cfg.ns_precision = PRECISIONS[ns_precision]
+        cfg.check_nonfinite = int(bool(check_nonfinite))
+        cfg.num_sms = int(num_sms)
+        cfg.workspace_cap_bytes = int(workspace_cap_bytes)
+        cfg.wait_timeout_s = float(wait_timeout_s)
+        h = ctypes.c_void_p()
+        check(self._lib.muon_init(int(device), ctypes.byref(cfg), ctypes.byref(h)))
+        self._h = h
+        self.device = device
+        self.ns_precision = ns_precision
+        self.x_dtype = None
+
+    # -- lifetime -----------------------------------------------------------
+    def close(self):
+        if getattr(self, "_h", None):
+            self._lib.muon_destroy(self._h)
+            self._h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    def __enter__(self):
+        return self
+
+    def __exit__(self, *exc):
+        self.close()
+
+    def _xdtype(self):
+        import torch
+        return torch.float32 if self.ns_precision == "fp32" else torch.bfloat16
+
+    # -- full step ----------------------------------------------------------
+    def step(self, params, grads, momenta, lr, beta=0.95, nesterov=True, wd=0.1, ns_steps=5, coeffs=None,
+             stream=None):
+        """One Muon step, in place on params and momenta (lists of CUDA tensors).
+
+        A ``None`` gradient skips its matrix.
+        """
+        import torch
+        shapes, pp, gp, mp = [], [], [], []
+        for i, (p, g, m) in enumerate(zip(params, grads, momenta, strict=True)):
+            _check_2d(p, f"params[{i}]", (torch.float32,))
+            _check_2d(m, f"momenta[{i}]", (torch.float32,), p.device)
+            flag = 0
+            if g is not None:
+                _check_2d(g, f"grads[{i}]", (torch.float32, torch.bfloat16), p.device)
+                if g.shape != p.shape:
+                    raise ValueError(f"grads[{i}] shape {tuple(g.shape)} != params shape {tuple(p.shape)}")
+                flag = FLAG_GRAD_BF16 if g.dtype == torch.bfloat16 else 0
+            if m.shape != p.shape:
+                raise ValueError(f"momenta[{i}] shape {tuple(m.shape)} != params shape {tuple(p.shape)}")
+            shapes.append((p.shape[0], p.shape[1], flag))
+            pp.append(p.data_ptr()); gp.append(_ptr(g)); mp.append(m.data_ptr())
+        check(self._lib.muon_step(self._h, _ptr_array(pp), _ptr_array(gp), _ptr_array(mp), _shapes_array(shapes),
+                                  len(shapes), float(lr), float(beta), int(bool(nesterov)), float(wd),
+                                  int(ns_steps), _coeffs(coeffs), _stream_handle(stream)))
+
+    def step_host(self, params, grads, momenta, lr, beta=0.95, nesterov=True, wd=0.1, ns_steps=5,
+                  coeffs=None, stream=None):
+        """The same step with every tensor in host memory (pinned for async copies).
+
+        The copies and the kernels are enqueued on ``stream``; synchronise it
+        before reading params / momenta.
+        """
+        import torch
+        shapes, pp, gp, mp = [], [], [], []
+        for i, (p, g, m) in enumerate(zip(params, grads, momenta, strict=True)):
+            _check_2d(p, f"params[{i}]", (torch.float32,))
+            _check_2d(m, f"momenta[{i}]", (torch.float32,))
+            flag = 0
+            if g is not None:
+                _check_2d(g, f"grads[{i}]", (torch.float32, torch.bfloat16))
+                flag = FLAG_GRAD_BF16 if g.dtype == torch.bfloat16 else 0
+            for t, what in ((p, "params"), (m, "momenta"), (g, "grads")):
+                if t is not None and t.device.type != "cpu":
+                    raise ValueError(f"{what}[{i}] must be in host memory for step_host")
+            shapes.append((p.shape[0], p.shape[1], flag))
+            pp.append(p.data_ptr()); gp.append(_ptr(g)); mp.append(m.data_ptr())
+        check(self._lib.muon_step_host(self._h, _ptr_array(pp), _ptr_array(gp), _ptr_array(mp),
+                                       _shapes_array(shapes), len(shapes), float(lr), float(beta),
+                                       int(bool(nesterov)), float(wd), int(ns_steps), _coeffs(coeffs),
+                                       _stream_handle(stream)))
+
+    # -- stages -------------------------------------------------------------
+    def momentum_norm(self, grads, momenta, ys, sumsq, beta=0.95, nesterov=True, stream=None):
+        """Stage 1: momentum in place, y = cast(u) in X layout, sumsq[i] = sum u^2."""
+        import torch
+        shapes = []
+        for i, (g, m, y) in enumerate(zip(grads, momenta, ys, strict=True)):
+            _check_2d(m, f"momenta[{i}]", (torch.float32,))
+            if g is not None:
+                _check_2d(g, f"grads[{i}]", (torch.float32, torch.bfloat16), m.device)
+            self._check_x(y, m.shape, f"y[{i}]")
+            shapes.append((m.shape[0], m.shape[1],
+                           FLAG_GRAD_BF16 if (g is not None and g.dtype == torch.bfloat16) else 0))
+        if sumsq.dtype != torch.float64 or sumsq.numel() < len(shapes) or not sumsq.is_contiguous():
+            raise ValueError("sumsq must be a contiguous float64 tensor with one entry per matrix")
+        check(self._lib.muon_momentum_norm(self._h, _ptr_array([_ptr(g) for g in grads]),
+                                           _ptr_array([m.data_ptr() for m in momenta]),
+                                           _ptr_array([y.data_ptr() for y in ys]), sumsq.data_ptr(),
+                                           _shapes_array(shapes), len(shapes), float(beta), int(bool(nesterov)),
+                                           _stream_handle(stream)))
+
+    def newton_schulz(self, x_in, x_out, shapes, sumsq=None, ns_steps=5, coeffs=None, stream=None):
+        """Stage 2 on X-layout buffers; shapes is a list of (m, n)."""
+        sh = [(int(m), int(n), 0) for (m, n) in shapes]
+        for i, ((m, n, _), xi, xo) in enumerate(zip(sh, x_in, x_out, strict=True)):
+            self._check_x(xi, (m, n), f"x_in[{i}]")
+            self._check_x(xo, (m, n), f"x_out[{i}]")
+        check(self._lib.muon_newton_schulz(self._h, _ptr_array([x.data_ptr() for x in x_in]),
+                                           _ptr_array([x.data_ptr() for x in x_out]),
+                                           None if sumsq is None else sumsq.data_ptr(), _shapes_array(sh),
+                                           len(sh), int(ns_steps), _coeffs(coeffs), _stream_handle(stream)))
+
+    def apply(self, params, os_, lr, wd, sumsq=None, stream=None):
+        """Stage 3: params <- params (1 - lr wd) - lr scale o_scale O."""
+        import torch
+        shapes = []
+        for i, (p, o) in enumerate(zip(params, os_, strict=True)):
+            _check_2d(p, f"params[{i}]", (torch.float32,))
+            if o is not None:
+                self._check_x(o, p.shape, f"o[{i}]")
+            shapes.append((p.shape[0], p.shape[1], 0))
+        check(self._lib.muon_apply(self._h, _ptr_array([p.data_ptr() for p in params]),
+                                   _ptr_array([_ptr(o) for o in os_]),
+                                   None if sumsq is None else sumsq.data_ptr(), _shapes_array(shapes),
+                                   len(shapes), float(lr), float(wd), _stream_handle(stream)))
+
+    def _check_x(self, x, shape, what):
+        m, n = int(shape[0]), int(shape[1])
+        if x.dtype != self._xdtype():
+            raise TypeError(f"{what} must be {self._xdtype()} in {self.ns_precision} mode")
+        if tuple(x.shape) != (m, round_up(n, 8)) or not x.is_contiguous():
+            raise ValueError(f"{what} must be a contiguous X-layout buffer of shape ({m}, {round_up(n, 8)})")
+
+    # -- inspection ---------------------------------------------------------
+    def status(self, stream=None):
+        """(code, error_word, nonfinite_count); waits for the stream."""
+        ew = ctypes.c_int32()
+        nf = ctypes.c_uint64()
+        code = self._lib.muon_get_status(self._h, _stream_handle(stream), ctypes.byref(ew), ctypes.byref(nf))
+        return code, ew.value, nf.value
+
+    def workspace(self):
+        base = ctypes.c_void_p()
+        size = ctypes.c_size_t()
+        check(self._lib.muon_workspace_ptr(self._h, ctypes.byref(base), ctypes.byref(size)))
+        return base.value or 0, size.value
+
+    def last_launch_count(self) -> int:
+        n = ctypes.c_int32()
+        check(self._lib.muon_last_launch_count(self._h, ctypes.byref(n)))
+        return n.value

@@ -1,0 +1,70 @@
+// Host-side launch interfaces of the CUDA kernels (internal to the library).
+#pragma once
+
+#include <cstdint>
+#include <cuda_runtime.h>
+
+#include "common.cuh"
+
+namespace muon {
+
+// Grouped elementwise launch: one block per chunk of kElemChunk elements.
+struct ElemLaunch {
+  const MatPlan* plans;     // device
+  const MatBind* binds;     // device
+  const long long* prefix;  // device, count + 1 entries
+  int count;
+  long long nblocks;        // prefix[count]
+};
+
+cudaError_t launch_momentum_norm(const ElemLaunch& L, int ysel, float beta, int nesterov, double* sumsq,
+                                 DevStatus* status, int check_nonfinite, bool fp32_out, cudaStream_t st);
+cudaError_t launch_apply(const ElemLaunch& L, int osel, float lr, float wd, int scale_mode, float extra_scale,
+                         const double* sumsq, bool fp32_in, cudaStream_t st);
+cudaError_t launch_scale_copy(const ElemLaunch& L, int isel, int osel, const double* sumsq, bool fp32,
+                              cudaStream_t st);
+
+// Newton-Schulz phases.
+enum NsPhase : int { PHASE_GRAM = 0, PHASE_POLY = 1, PHASE_COMB = 2 };
+
+// Tensor maps of one matrix (bf16 path). Each CUtensorMap is 128 bytes and
+// must be 64-byte aligned in global memory.
+struct alignas(64) TmapBlob {
+  unsigned char bytes[128];
+};
+// Index of each map inside a matrix's block of kMapsPerMat maps.
+// X-buffer maps come in triples (K-major 128-row box, K-major 256-row box,
+// MN-major 64x64 box): X0 at 0, X1 at 3. A caller input buffer has its own
+// triple per matrix in a separate table.
+enum MapIdx : int {
+  MAP_X0 = 0, MAP_X1 = 3,
+  MAP_K128 = 0, MAP_K256 = 1, MAP_MN = 2,   // offsets inside a triple
+  MAP_A_K128 = 6, MAP_A_K256 = 7,
+  MAP_B_K128 = 8, MAP_B_K256 = 9,
+  kMapsPerMat = 10,
+  kInMapsPerMat = 3
+};
+
+struct NsLaunch {
+  const MatPlan* plans;      // device
+  const MatBind* binds;      // device
+  const TmapBlob* maps;      // device, kMapsPerMat per matrix (workspace)
+  const TmapBlob* in_maps;   // device, kInMapsPerMat per matrix (caller input) or NULL
+  const int4* tiles;         // device tile list of the phase
+  int ntiles;
+  const double* sumsq;       // device or NULL
+  DevStatus* status;         // device
+  int grid;                  // persistent CTAs
+  unsigned long long timeout_ns;
+};
+
+cudaError_t launch_ns_phase_bf16(const NsLaunch& L, int phase, int src_sel, int dst_sel, int first, float a,
+                                 float b, float c, cudaStream_t st);
+
+// fp32 debug Newton-Schulz: one launch per matrix and phase.
+cudaError_t launch_ns_phase_fp32(const MatPlan& mp_host, int mat, int phase, const float* src, float* dst,
+                                 const double* sumsq, int first, float a, float b, float c, cudaStream_t st);
+
+int ns_bf16_smem_bytes();
+
+}  // namespace muon

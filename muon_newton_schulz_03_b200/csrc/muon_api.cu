@@ -1,0 +1,782 @@
+// C ABI of the Muon step (declared in include/muon_ns.h).
+//
+// Host responsibilities only: argument validation, the plan (cached per
+// shape table), the workspace, tensor maps for the bulk-tensor loads, the
+// device copies of the per-call pointer tables (cached by content), and the
+// ordered enqueue of the kernels on the caller's stream. All arithmetic of
+// the step runs in the kernels of elementwise.cu, ns_tcgen05.cu and
+// ns_fp32.cu.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cmath>
+#include <cstdio>
+#include <cstring>
+#include <list>
+#include <memory>
+#include <string>
+#include <vector>
+
+#include "../../include/muon_ns.h"
+#include "common.cuh"
+#include "kernels.h"
+#include "plan.h"
+
+using namespace muon;
+
+namespace {
+
+thread_local std::string g_last_error;
+
+int fail(int code, const std::string& msg) {
+  g_last_error = msg;
+  return code;
+}
+
+#define MUON_CUDA_TRY(expr)                                                                 \
+  do {                                                                                      \
+    cudaError_t _e = (expr);                                                                \
+    if (_e != cudaSuccess)                                                                  \
+      return fail(_e == cudaErrorMemoryAllocation ? MUON_ERR_OOM : MUON_ERR_CUDA,           \
+                  std::string(#expr) + ": " + cudaGetErrorString(_e));                     \
+  } while (0)
+
+// Restores the caller's current device on scope exit.
+struct DeviceGuard {
+  int prev = -1;
+  bool ok = false;
+  explicit DeviceGuard(int dev) {
+    if (cudaGetDevice(&prev) != cudaSuccess) prev = -1;
+    ok = cudaSetDevice(dev) == cudaSuccess;
+  }
+  ~DeviceGuard() {
+    if (prev >= 0) cudaSetDevice(prev);
+  }
+};
+
+// Device copy of a host byte blob, uploaded once and kept while in the cache.
+struct DevBlob {
+  std::vector<unsigned char> key;
+  void* dptr = nullptr;
+};
+
+class BlobCache {
+ public:
+  ~BlobCache() { clear(); }
+  // Returns the device copy of `bytes`, uploading it (synchronously) on a miss.
+  int get(const void* bytes, size_t n, void** out) {
+    const unsigned char* b = static_cast<const unsigned char*>(bytes);
+    for (auto it = entries_.begin(); it != entries_.end(); ++it) {
+      if (it->key.size() == n && std::memcmp(it->key.data(), b, n) == 0) {
+        entries_.splice(entries_.begin(), entries_, it);
+        *out = entries_.front().dptr;
+        return MUON_OK;
+      }
+    }
+    if (entries_.size() >= kMax) {
+      // The evicted table may still be read by queued work: wait for it.
+      MUON_CUDA_TRY(cudaDeviceSynchronize());
+      cudaFree(entries_.back().dptr);
+      entries_.pop_back();
+    }
+    DevBlob e;
+    e.key.assign(b, b + n);
+    MUON_CUDA_TRY(cudaMalloc(&e.dptr, std::max<size_t>(n, 16)));
+    cudaError_t err = cudaMemcpy(e.dptr, b, n, cudaMemcpyHostToDevice);
+    if (err != cudaSuccess) {
+      cudaFree(e.dptr);
+      return fail(MUON_ERR_CUDA, std::string("table upload: ") + cudaGetErrorString(err));
+    }
+    entries_.push_front(std::move(e));
+    *out = entries_.front().dptr;
+    return MUON_OK;
+  }
+  void clear() {
+    for (auto& e : entries_) cudaFree(e.dptr);
+    entries_.clear();
+  }
+
+ private:
+  static constexpr size_t kMax = 8;
+  std::list<DevBlob> entries_;
+};
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn get_encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static bool tried = false;
+  if (!tried) {
+    tried = true;
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+
+// 2D bf16 row-major tensor (rows x cols, leading dimension ld elements),
+// 128-byte swizzle, box of box_cols (inner) x box_rows.
+int encode_map(TmapBlob* out, const void* base, int rows, int cols, int ld, int box_cols, int box_rows) {
+  static_assert(sizeof(CUtensorMap) == sizeof(TmapBlob), "tensor map size");
+  EncodeTiledFn enc = get_encode_fn();
+  if (!enc) return fail(MUON_ERR_CUDA, "cuTensorMapEncodeTiled is not available");
+  cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)ld * 2};
+  cuuint32_t box[2] = {(cuuint32_t)box_cols, (cuuint32_t)box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = enc(reinterpret_cast<CUtensorMap*>(out), CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base),
+                   dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(MUON_ERR_CUDA, "cuTensorMapEncodeTiled failed: " + std::to_string((int)r));
+  return MUON_OK;
+}
+
+// Maps of one X-layout buffer (m x n, ld): K-major 128- and 256-row boxes and
+// the 64 x 64 M/N-major box.
+int encode_x_triple(TmapBlob* out3, const void* base, const MatPlan& mp) {
+  int rc;
+  if ((rc = encode_map(out3 + MAP_K128, base, mp.m, mp.n, mp.ldx, 64, 128))) return rc;
+  if ((rc = encode_map(out3 + MAP_K256, base, mp.m, mp.n, mp.ldx, 64, 256))) return rc;
+  if ((rc = encode_map(out3 + MAP_MN, base, mp.m, mp.n, mp.ldx, 64, 64))) return rc;
+  return MUON_OK;
+}
+
+}  // namespace
+
+// ---------------------------------------------------------------------------
+// Handle
+// ---------------------------------------------------------------------------
+
+struct DevPlan {
+  HostPlan hp;
+  std::vector<int32_t> key;          // (m, n) per matrix
+  void* ws = nullptr;
+  size_t ws_size = 0;
+  void* tables = nullptr;            // MatPlan[count] | prefix | tiles x3 | maps
+  MatPlan* d_mats = nullptr;
+  long long* d_prefix = nullptr;
+  int4* d_tiles[3] = {nullptr, nullptr, nullptr};
+  TmapBlob* d_maps = nullptr;
+  std::vector<MatPlan> mats;         // host copy with workspace pointers
+  void* staging = nullptr;           // muon_step_host buffers
+  size_t staging_size = 0;
+  std::vector<int64_t> staging_off;  // count * 3: param, grad, momentum
+};
+
+struct muon_handle {
+  int device = 0;
+  muon_config cfg{};
+  int num_sms = 0;
+  DevStatus* status = nullptr;
+  std::unique_ptr<DevPlan> plan;
+  BlobCache binds;
+  BlobCache in_maps;
+  int last_launches = 0;
+};
+
+namespace {
+
+void free_plan(DevPlan* p) {
+  if (!p) return;
+  cudaFree(p->ws);
+  cudaFree(p->tables);
+  cudaFree(p->staging);
+}
+
+int64_t align_up(int64_t x, int64_t a) { return (x + a - 1) / a * a; }
+
+// Builds (or reuses) the plan, workspace, device tables and tensor maps for
+// this shape table.
+int ensure_plan(muon_handle* h, const int32_t* shapes, int count) {
+  std::vector<int32_t> key((size_t)count * 2);
+  for (int i = 0; i < count; ++i) {
+    key[2 * i] = shapes[3 * i];
+    key[2 * i + 1] = shapes[3 * i + 1];
+  }
+  if (h->plan && h->plan->key == key) return MUON_OK;
+
+  auto np = std::make_unique<DevPlan>();
+  std::string why;
+  if (!build_plan(shapes, count, h->cfg.ns_precision, np->hp, why)) return fail(MUON_ERR_INVALID_ARG, why);
+  np->key = key;
+  const HostPlan& hp = np->hp;
+  if (h->cfg.workspace_cap_bytes && (size_t)hp.ws_bytes > h->cfg.workspace_cap_bytes)
+    return fail(MUON_ERR_OOM, "workspace of " + std::to_string(hp.ws_bytes) + " bytes exceeds the cap of " +
+                                  std::to_string(h->cfg.workspace_cap_bytes));
+
+  // Drop the previous plan first (queued work may still use it).
+  if (h->plan) {
+    MUON_CUDA_TRY(cudaDeviceSynchronize());
+    h->binds.clear();
+    h->in_maps.clear();
+    free_plan(h->plan.get());
+    h->plan.reset();
+  }
+
+  cudaError_t e = cudaMalloc(&np->ws, (size_t)hp.ws_bytes);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return fail(MUON_ERR_OOM, "workspace allocation of " + std::to_string(hp.ws_bytes) + " bytes failed");
+  }
+  np->ws_size = (size_t)hp.ws_bytes;
+
+  char* ws = static_cast<char*>(np->ws);
+  np->mats = hp.mats;
+  for (int i = 0; i < count; ++i) {
+    MatPlan& mp = np->mats[i];
+    mp.x0 = ws + hp.region_off[(size_t)i * 4 + 0];
+    mp.x1 = ws + hp.region_off[(size_t)i * 4 + 1];
+    mp.a = ws + hp.region_off[(size_t)i * 4 + 2];
+    mp.b = ws + hp.region_off[(size_t)i * 4 + 3];
+  }
+
+  // Device tables, one allocation.
+  const bool bf16 = h->cfg.ns_precision == MUON_NS_BF16;
+  int64_t off = 0;
+  const int64_t o_mats = off;  off = align_up(off + (int64_t)sizeof(MatPlan) * count, 256);
+  const int64_t o_pref = off;  off = align_up(off + (int64_t)sizeof(long long) * (count + 1), 256);
+  int64_t o_tiles[3];
+  for (int p = 0; p < 3; ++p) {
+    o_tiles[p] = off;
+    off = align_up(off + (int64_t)sizeof(int4) * std::max<size_t>(hp.tiles[p].size(), 1), 256);
+  }
+  const int64_t o_maps = off;
+  if (bf16) off = align_up(off + (int64_t)sizeof(TmapBlob) * kMapsPerMat * count, 256);
+  std::vector<unsigned char> host((size_t)off, 0);
+  std::memcpy(host.data() + o_mats, np->mats.data(), sizeof(MatPlan) * count);
+  std::memcpy(host.data() + o_pref, hp.prefix.data(), sizeof(long long) * (count + 1));
+  for (int p = 0; p < 3; ++p) {
+    int4* t = reinterpret_cast<int4*>(host.data() + o_tiles[p]);
+    for (size_t k = 0; k < hp.tiles[p].size(); ++k)
+      t[k] = make_int4(hp.tiles[p][k].mat, hp.tiles[p][k].ti, hp.tiles[p][k].tj, 0);
+  }
+  if (bf16) {
+    TmapBlob* maps = reinterpret_cast<TmapBlob*>(host.data() + o_maps);
+    for (int i = 0; i < count; ++i) {
+      const MatPlan& mp = np->mats[i];
+      TmapBlob* mm = maps + (size_t)i * kMapsPerMat;
+      int rc;
+      if ((rc = encode_x_triple(mm + MAP_X0, mp.x0, mp))) { free_plan(np.get()); return rc; }
+      if ((rc = encode_x_triple(mm + MAP_X1, mp.x1, mp))) { free_plan(np.get()); return rc; }
+      if ((rc = encode_map(mm + MAP_A_K128, mp.a, mp.s, mp.s, mp.lds, 64, 128))) { free_plan(np.get()); return rc; }
+      if ((rc = encode_map(mm + MAP_A_K256, mp.a, mp.s, mp.s, mp.lds, 64, 256))) { free_plan(np.get()); return rc; }
+      if ((rc = encode_map(mm + MAP_B_K128, mp.b, mp.s, mp.s, mp.lds, 64, 128))) { free_plan(np.get()); return rc; }
+      if ((rc = encode_map(mm + MAP_B_K256, mp.b, mp.s, mp.s, mp.lds, 64, 256))) { free_plan(np.get()); return rc; }
+    }
+  }
+  e = cudaMalloc(&np->tables, (size_t)off);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    free_plan(np.get());
+    return fail(MUON_ERR_OOM, "plan table allocation failed");
+  }
+  e = cudaMemcpy(np->tables, host.data(), (size_t)off, cudaMemcpyHostToDevice);
+  if (e != cudaSuccess) {
+    free_plan(np.get());
+    return fail(MUON_ERR_CUDA, std::string("plan table upload: ") + cudaGetErrorString(e));
+  }
+  char* tb = static_cast<char*>(np->tables);
+  np->d_mats = reinterpret_cast<MatPlan*>(tb + o_mats);
+  np->d_prefix = reinterpret_cast<long long*>(tb + o_pref);
+  for (int p = 0; p < 3; ++p) np->d_tiles[p] = reinterpret_cast<int4*>(tb + o_tiles[p]);
+  np->d_maps = bf16 ? reinterpret_cast<TmapBlob*>(tb + o_maps) : nullptr;
+  h->plan = std::move(np);
+  return MUON_OK;
+}
+
+int check_ptr(const void* p, const char* what, int i) {
+  if (p == nullptr) return fail(MUON_ERR_INVALID_ARG, std::string(what) + "[" + std::to_string(i) + "] is NULL");
+  if (reinterpret_cast<uintptr_t>(p) % 16 != 0)
+    return fail(MUON_ERR_INVALID_ARG, std::string(what) + "[" + std::to_string(i) + "] is not 16-byte aligned");
+  return MUON_OK;
+}
+
+bool overlaps(const void* a, size_t na, const void* b, size_t nb) {
+  const uintptr_t x = reinterpret_cast<uintptr_t>(a), y = reinterpret_cast<uintptr_t>(b);
+  return x < y + nb && y < x + na;
+}
+
+int check_common(muon_handle* h, const int32_t* shapes, int count) {
+  if (h == nullptr) return fail(MUON_ERR_INVALID_ARG, "handle is NULL");
+  if (shapes == nullptr) return fail(MUON_ERR_INVALID_ARG, "shapes is NULL");
+  if (count < 1) return fail(MUON_ERR_INVALID_ARG, "count must be >= 1");
+  for (int i = 0; i < count; ++i) {
+    const int m = shapes[3 * i], n = shapes[3 * i + 1], fl = shapes[3 * i + 2];
+    if (m < 1 || n < 1 || m > kMaxDim || n > kMaxDim)
+      return fail(MUON_ERR_INVALID_ARG, "matrix " + std::to_string(i) + ": bad shape " + std::to_string(m) + " x " +
+                                            std::to_string(n));
+    if (fl & ~1) return fail(MUON_ERR_INVALID_ARG, "matrix " + std::to_string(i) + ": unknown flag bits");
+  }
+  return MUON_OK;
+}
+
+int check_coeffs(const float* coeffs, int ns_steps, float* abc) {
+  if (ns_steps < 0 || ns_steps > 64) return fail(MUON_ERR_INVALID_ARG, "ns_steps must be in [0, 64]");
+  const float def[3] = {3.4445f, -4.7750f, 2.0315f};
+  const float* c = coeffs ? coeffs : def;
+  for (int k = 0; k < 3; ++k) {
+    if (!std::isfinite(c[k])) return fail(MUON_ERR_INVALID_ARG, "coefficients must be finite");
+    abc[k] = c[k];
+  }
+  return MUON_OK;
+}
+
+ElemLaunch elem_launch(const DevPlan& P, const MatBind* d_binds) {
+  ElemLaunch L;
+  L.plans = P.d_mats;
+  L.binds = d_binds;
+  L.prefix = P.d_prefix;
+  L.count = P.hp.count;
+  L.nblocks = P.hp.prefix[P.hp.count];
+  return L;
+}
+
+// Enqueue `ns_steps` Newton-Schulz iterations. The input of step 1 is
+// `first_src`; intermediate results alternate X1, X0, X1, ...; the result of
+// the last step goes to `last_dst` (or stays in the ping-pong buffers when
+// last_dst < 0). *result receives the selector of the result buffer.
+int enqueue_ns(muon_handle* h, const MatBind* d_binds, const std::vector<MatBind>& hbinds,
+               const TmapBlob* d_in_maps, const double* sumsq, int ns_steps, const float* abc, int first_src,
+               int last_dst, cudaStream_t st, int* launches, int* result) {
+  DevPlan& P = *h->plan;
+  const HostPlan& hp = P.hp;
+  const bool bf16 = h->cfg.ns_precision == MUON_NS_BF16;
+  int src = first_src;
+  for (int t = 1; t <= ns_steps; ++t) {
+    const int dst = (t == ns_steps && last_dst >= 0) ? last_dst : (t % 2 == 1 ? BUF_X1 : BUF_X0);
+    const int first = t == 1 ? 1 : 0;
+    if (bf16) {
+      NsLaunch L;
+      L.plans = P.d_mats;
+      L.binds = d_binds;
+      L.maps = P.d_maps;
+      L.in_maps = d_in_maps;
+      L.sumsq = sumsq;
+      L.status = h->status;
+      L.grid = h->num_sms;
+      L.timeout_ns = (unsigned long long)(h->cfg.wait_timeout_s * 1e9);
+      for (int ph = 0; ph < 3; ++ph) {
+        L.tiles = P.d_tiles[ph];
+        L.ntiles = (int)hp.tiles[ph].size();
+        MUON_CUDA_TRY(launch_ns_phase_bf16(L, ph, src, dst, first, abc[0], abc[1], abc[2], st));
+        ++*launches;
+      }
+    } else {
+      for (int i = 0; i < hp.count; ++i) {
+        if (!hbinds[i].active) continue;
+        const MatPlan& mp = P.mats[i];
+        const float* s_ptr = static_cast<const float*>(sel_buf(mp, hbinds[i], src));
+        float* d_ptr = static_cast<float*>(const_cast<void*>(sel_buf(mp, hbinds[i], dst)));
+        MUON_CUDA_TRY(launch_ns_phase_fp32(mp, i, PHASE_GRAM, s_ptr, d_ptr, sumsq, first, abc[0], abc[1], abc[2], st));
+        MUON_CUDA_TRY(launch_ns_phase_fp32(mp, i, PHASE_POLY, s_ptr, d_ptr, sumsq, first, abc[0], abc[1], abc[2], st));
+        MUON_CUDA_TRY(launch_ns_phase_fp32(mp, i, PHASE_COMB, s_ptr, d_ptr, sumsq, first, abc[0], abc[1], abc[2], st));
+        *launches += 3;
+      }
+    }
+    src = dst;
+  }
+  *result = src;
+  return MUON_OK;
+}
+
+// Validation of a full step's pointers: alignment and per-matrix overlap.
+int check_step_ptrs(float* const* params, const void* const* grads, float* const* momenta, const int32_t* shapes,
+                    int count) {
+  if (!params || !grads || !momenta) return fail(MUON_ERR_INVALID_ARG, "params, grads and momenta arrays are required");
+  int rc;
+  for (int i = 0; i < count; ++i) {
+    const size_t numel = (size_t)shapes[3 * i] * (size_t)shapes[3 * i + 1];
+    const size_t gbytes = numel * ((shapes[3 * i + 2] & 1) ? 2 : 4);
+    if ((rc = check_ptr(params[i], "params", i))) return rc;
+    if ((rc = check_ptr(momenta[i], "momenta", i))) return rc;
+    if (grads[i] && (rc = check_ptr(grads[i], "grads", i))) return rc;
+    if (overlaps(params[i], numel * 4, momenta[i], numel * 4) ||
+        (grads[i] && (overlaps(params[i], numel * 4, grads[i], gbytes) ||
+                      overlaps(momenta[i], numel * 4, grads[i], gbytes))))
+      return fail(MUON_ERR_INVALID_ARG, "matrix " + std::to_string(i) + ": params, grads and momenta overlap");
+  }
+  return MUON_OK;
+}
+
+int check_scalars(float lr, float beta, float wd) {
+  if (!std::isfinite(lr) || !std::isfinite(wd)) return fail(MUON_ERR_INVALID_ARG, "lr and wd must be finite");
+  if (!(beta >= 0.0f && beta < 1.0f)) return fail(MUON_ERR_INVALID_ARG, "beta must be in [0, 1)");
+  return MUON_OK;
+}
+
+int step_impl(muon_handle* h, float* const* params, const void* const* grads, float* const* momenta,
+              const int32_t* shapes, int count, float lr, float beta, int nesterov, float wd, int ns_steps,
+              const float* abc, cudaStream_t st) {
+  int rc;
+  if ((rc = ensure_plan(h, shapes, count))) return rc;
+  DevPlan& P = *h->plan;
+  std::vector<MatBind> hb((size_t)count);
+  for (int i = 0; i < count; ++i) {
+    MatBind& b = hb[i];
+    std::memset(&b, 0, sizeof(b));
+    b.p = params[i];
+    b.g = grads[i];
+    b.mom = momenta[i];
+    b.flags = shapes[3 * i + 2];
+    b.active = grads[i] != nullptr;
+  }
+  void* d_binds = nullptr;
+  if ((rc = h->binds.get(hb.data(), sizeof(MatBind) * count, &d_binds))) return rc;
+  const MatBind* db = static_cast<const MatBind*>(d_binds);
+  double* sumsq = static_cast<double*>(P.ws);
+  const bool fp32 = h->cfg.ns_precision == MUON_NS_FP32;
+  int launches = 0;
+  MUON_CUDA_TRY(cudaMemsetAsync(sumsq, 0, sizeof(double) * count, st));
+  const ElemLaunch EL = elem_launch(P, db);
+  MUON_CUDA_TRY(launch_momentum_norm(EL, BUF_X0, beta, nesterov ? 1 : 0, sumsq, h->status, h->cfg.check_nonfinite,
+                                     fp32, st));
+  ++launches;
+  int res = BUF_X0;
+  if ((rc = enqueue_ns(h, db, hb, nullptr, sumsq, ns_steps, abc, BUF_X0, -1, st, &launches, &res))) return rc;
+  MUON_CUDA_TRY(launch_apply(EL, res, lr, wd, h->cfg.scale_mode, h->cfg.extra_scale, ns_steps == 0 ? sumsq : nullptr,
+                             fp32, st));
+  ++launches;
+  h->last_launches = launches;
+  return MUON_OK;
+}
+
+}  // namespace
+
+// ---------------------------------------------------------------------------
+// Exported entry points
+// ---------------------------------------------------------------------------
+
+extern "C" {
+
+const char* muon_last_error(void) { return g_last_error.c_str(); }
+
+const char* muon_version(void) { return "muon_ns 0.1.0 (sm_100a)"; }
+
+int muon_config_init(muon_config* cfg) {
+  if (!cfg) return fail(MUON_ERR_INVALID_ARG, "cfg is NULL");
+  cfg->scale_mode = MUON_SCALE_MOONLIGHT;
+  cfg->extra_scale = 1.0f;
+  cfg->ns_precision = MUON_NS_BF16;
+  cfg->check_nonfinite = 0;
+  cfg->num_sms = 0;
+  cfg->workspace_cap_bytes = 0;
+  cfg->wait_timeout_s = 2.0;
+  return MUON_OK;
+}
+
+int muon_init(int device, const muon_config* cfg, muon_handle** out) {
+  g_last_error.clear();
+  if (!out) return fail(MUON_ERR_INVALID_ARG, "out is NULL");
+  muon_config c;
+  if (cfg) c = *cfg; else muon_config_init(&c);
+  if (c.scale_mode < 0 || c.scale_mode > 3) return fail(MUON_ERR_INVALID_ARG, "unknown scale_mode");
+  if (c.ns_precision != 0 && c.ns_precision != 1) return fail(MUON_ERR_INVALID_ARG, "unknown ns_precision");
+  if (!std::isfinite(c.extra_scale)) return fail(MUON_ERR_INVALID_ARG, "extra_scale must be finite");
+  if (!(c.wait_timeout_s > 0.0 && c.wait_timeout_s <= 600.0))
+    return fail(MUON_ERR_INVALID_ARG, "wait_timeout_s must be in (0, 600]");
+  if (c.num_sms < 0) return fail(MUON_ERR_INVALID_ARG, "num_sms must be >= 0");
+  int ndev = 0;
+  if (cudaGetDeviceCount(&ndev) != cudaSuccess || ndev == 0) {
+    cudaGetLastError();
+    return fail(MUON_ERR_NO_DEVICE, "no CUDA device");
+  }
+  if (device < 0 || device >= ndev) return fail(MUON_ERR_INVALID_ARG, "device index out of range");
+  cudaDeviceProp prop;
+  MUON_CUDA_TRY(cudaGetDeviceProperties(&prop, device));
+  if (prop.major != 10 || prop.minor != 0)
+    return fail(MUON_ERR_UNSUPPORTED, std::string("device is sm_") + std::to_string(prop.major) +
+                                          std::to_string(prop.minor) + "; this library is built for sm_100a");
+  DeviceGuard g(device);
+  if (!g.ok) return fail(MUON_ERR_CUDA, "cudaSetDevice failed");
+  auto h = std::make_unique<muon_handle>();
+  h->device = device;
+  h->cfg = c;
+  h->num_sms = c.num_sms > 0 ? std::min(c.num_sms, prop.multiProcessorCount) : prop.multiProcessorCount;
+  MUON_CUDA_TRY(cudaMalloc(&h->status, sizeof(DevStatus)));
+  MUON_CUDA_TRY(cudaMemset(h->status, 0, sizeof(DevStatus)));
+  *out = h.release();
+  return MUON_OK;
+}
+
+int muon_destroy(muon_handle* h) {
+  if (!h) return MUON_OK;
+  {
+    DeviceGuard g(h->device);
+    cudaDeviceSynchronize();
+    h->binds.clear();
+    h->in_maps.clear();
+    if (h->plan) free_plan(h->plan.get());
+    cudaFree(h->status);
+  }
+  delete h;
+  return MUON_OK;
+}
+
+int muon_step(muon_handle* h, float* const* params, const void* const* grads, float* const* momenta,
+              const int32_t* shapes, int count, float lr, float beta, int nesterov, float wd, int ns_steps,
+              const float* coeffs, void* stream) {
+  g_last_error.clear();
+  int rc;
+  if ((rc = check_common(h, shapes, count))) return rc;
+  if ((rc = check_step_ptrs(params, grads, momenta, shapes, count))) return rc;
+  if ((rc = check_scalars(lr, beta, wd))) return rc;
+  float abc[3];
+  if ((rc = check_coeffs(coeffs, ns_steps, abc))) return rc;
+  DeviceGuard g(h->device);
+  if (!g.ok) return fail(MUON_ERR_CUDA, "cudaSetDevice failed");
+  return step_impl(h, params, grads, momenta, shapes, count, lr, beta, nesterov, wd, ns_steps, abc,
+                   static_cast<cudaStream_t>(stream));
+}
+
+int muon_step_host(muon_handle* h, float* const* params, const void* const* grads, float* const* momenta,
+                   const int32_t* shapes, int count, float lr, float beta, int nesterov, float wd, int ns_steps,
+                   const float* coeffs, void* stream) {
+  g_last_error.clear();
+  int rc;
+  if ((rc = check_common(h, shapes, count))) return rc;
+  if (!params || !grads || !momenta) return fail(MUON_ERR_INVALID_ARG, "params, grads and momenta arrays are required");
+  for (int i = 0; i < count; ++i)
+    if (!params[i] || !momenta[i]) return fail(MUON_ERR_INVALID_ARG, "host params and momenta must be non-NULL");
+  if ((rc = check_scalars(lr, beta, wd))) return rc;
+  float abc[3];
+  if ((rc = check_coeffs(coeffs, ns_steps, abc))) return rc;
+  DeviceGuard g(h->device);
+  if (!g.ok) return fail(MUON_ERR_CUDA, "cudaSetDevice failed");
+  if ((rc = ensure_plan(h, shapes, count))) return rc;
+  DevPlan& P = *h->plan;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (!P.staging) {
+    P.staging_off.assign((size_t)count * 3, 0);
+    int64_t off = 0;
+    for (int i = 0; i < count; ++i) {
+      const int64_t numel = P.mats[i].numel;
+      for (int k = 0; k < 3; ++k) {
+        P.staging_off[(size_t)i * 3 + k] = off;
+        off = align_up(off + numel * 4, 256);
+      }
+    }
+    if (h->cfg.workspace_cap_bytes && (size_t)(off + P.hp.ws_bytes) > h->cfg.workspace_cap_bytes)
+      return fail(MUON_ERR_OOM, "staging plus workspace exceed the cap");
+    cudaError_t e = cudaMalloc(&P.staging, (size_t)off);
+    if (e != cudaSuccess) {
+      cudaGetLastError();
+      P.staging = nullptr;
+      return fail(MUON_ERR_OOM, "staging allocation of " + std::to_string(off) + " bytes failed");
+    }
+    P.staging_size = (size_t)off;
+  }
+  std::vector<float*> dp(count), dm(count);
+  std::vector<const void*> dg(count);
+  char* sb = static_cast<char*>(P.staging);
+  for (int i = 0; i < count; ++i) {
+    const size_t numel = (size_t)P.mats[i].numel;
+    const size_t gbytes = numel * ((shapes[3 * i + 2] & 1) ? 2 : 4);
+    dp[i] = reinterpret_cast<float*>(sb + P.staging_off[(size_t)i * 3 + 0]);
+    dg[i] = grads[i] ? sb + P.staging_off[(size_t)i * 3 + 1] : nullptr;
+    dm[i] = reinterpret_cast<float*>(sb + P.staging_off[(size_t)i * 3 + 2]);
+    MUON_CUDA_TRY(cudaMemcpyAsync(dp[i], params[i], numel * 4, cudaMemcpyHostToDevice, st));
+    MUON_CUDA_TRY(cudaMemcpyAsync(dm[i], momenta[i], numel * 4, cudaMemcpyHostToDevice, st));
+    if (grads[i]) MUON_CUDA_TRY(cudaMemcpyAsync(const_cast<void*>(dg[i]), grads[i], gbytes, cudaMemcpyHostToDevice, st));
+  }
+  if ((rc = step_impl(h, dp.data(), dg.data(), dm.data(), shapes, count, lr, beta, nesterov, wd, ns_steps, abc, st)))
+    return rc;
+  for (int i = 0; i < count; ++i) {
+    if (!grads[i]) continue;
+    const size_t numel = (size_t)P.mats[i].numel;
+    MUON_CUDA_TRY(cudaMemcpyAsync(params[i], dp[i], numel * 4, cudaMemcpyDeviceToHost, st));
+    MUON_CUDA_TRY(cudaMemcpyAsync(momenta[i], dm[i], numel * 4, cudaMemcpyDeviceToHost, st));
+  }
+  return MUON_OK;
+}
+
+int muon_momentum_norm(muon_handle* h, const void* const* grads, float* const* momenta, void* const* y,
+                       double* sumsq, const int32_t* shapes, int count, float beta, int nesterov, void* stream) {
+  g_last_error.clear();
+  int rc;
+  if ((rc = check_common(h, shapes, count))) return rc;
+  if (!grads || !momenta || !y || !sumsq) return fail(MUON_ERR_INVALID_ARG, "grads, momenta, y and sumsq are required");
+  if (reinterpret_cast<uintptr_t>(sumsq) % 8) return fail(MUON_ERR_INVALID_ARG, "sumsq must be 8-byte aligned");
+  if (!(beta >= 0.0f && beta < 1.0f)) return fail(MUON_ERR_INVALID_ARG, "beta must be in [0, 1)");
+  for (int i = 0; i < count; ++i) {
+    if (!grads[i]) continue;
+    if ((rc = check_ptr(grads[i], "grads", i)) || (rc = check_ptr(momenta[i], "momenta", i)) ||
+        (rc = check_ptr(y[i], "y", i)))
+      return rc;
+  }
+  DeviceGuard g(h->device);
+  if (!g.ok) return fail(MUON_ERR_CUDA, "cudaSetDevice failed");
+  if ((rc = ensure_plan(h, shapes, count))) return rc;
+  DevPlan& P = *h->plan;
+  std::vector<MatBind> hb((size_t)count);
+  for (int i = 0; i < count; ++i) {
+    std::memset(&hb[i], 0, sizeof(MatBind));
+    hb[i].g = grads[i];
+    hb[i].mom = momenta[i];
+    hb[i].xout = y[i];
+    hb[i].flags = shapes[3 * i + 2];
+    hb[i].active = grads[i] != nullptr;
+  }
+  void* d_binds = nullptr;
+  if ((rc = h->binds.get(hb.data(), sizeof(MatBind) * count, &d_binds))) return rc;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  MUON_CUDA_TRY(cudaMemsetAsync(sumsq, 0, sizeof(double) * count, st));
+  MUON_CUDA_TRY(launch_momentum_norm(elem_launch(P, static_cast<const MatBind*>(d_binds)), BUF_OUT, beta,
+                                     nesterov ? 1 : 0, sumsq, h->status, h->cfg.check_nonfinite,
+                                     h->cfg.ns_precision == MUON_NS_FP32, st));
+  h->last_launches = 1;
+  return MUON_OK;
+}
+
+int muon_newton_schulz(muon_handle* h, const void* const* x_in, void* const* x_out, const double* sumsq,
+                       const int32_t* shapes, int count, int ns_steps, const float* coeffs, void* stream) {
+  g_last_error.clear();
+  int rc;
+  if ((rc = check_common(h, shapes, count))) return rc;
+  if (!x_in || !x_out) return fail(MUON_ERR_INVALID_ARG, "x_in and x_out are required");
+  float abc[3];
+  if ((rc = check_coeffs(coeffs, ns_steps, abc))) return rc;
+  const size_t esz = h->cfg.ns_precision == MUON_NS_FP32 ? 4 : 2;
+  for (int i = 0; i < count; ++i) {
+    if ((rc = check_ptr(x_in[i], "x_in", i)) || (rc = check_ptr(x_out[i], "x_out", i))) return rc;
+    const size_t bytes = (size_t)shapes[3 * i] * (size_t)round_up_i(shapes[3 * i + 1], 8) * esz;
+    if (overlaps(x_in[i], bytes, x_out[i], bytes))
+      return fail(MUON_ERR_INVALID_ARG, "matrix " + std::to_string(i) + ": x_in and x_out overlap");
+  }
+  DeviceGuard g(h->device);
+  if (!g.ok) return fail(MUON_ERR_CUDA, "cudaSetDevice failed");
+  if ((rc = ensure_plan(h, shapes, count))) return rc;
+  DevPlan& P = *h->plan;
+  std::vector<MatBind> hb((size_t)count);
+  for (int i = 0; i < count; ++i) {
+    std::memset(&hb[i], 0, sizeof(MatBind));
+    hb[i].xin = x_in[i];
+    hb[i].xout = x_out[i];
+    hb[i].active = 1;
+  }
+  void* d_binds = nullptr;
+  if ((rc = h->binds.get(hb.data(), sizeof(MatBind) * count, &d_binds))) return rc;
+  const MatBind* db = static_cast<const MatBind*>(d_binds);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  int launches = 0;
+  if (ns_steps == 0) {
+    MUON_CUDA_TRY(launch_scale_copy(elem_launch(P, db), BUF_IN, BUF_OUT, sumsq, esz == 4, st));
+    h->last_launches = 1;
+    return MUON_OK;
+  }
+  const TmapBlob* d_in = nullptr;
+  if (esz == 2) {
+    std::vector<TmapBlob> maps((size_t)count * kInMapsPerMat);
+    for (int i = 0; i < count; ++i)
+      if ((rc = encode_x_triple(maps.data() + (size_t)i * kInMapsPerMat, x_in[i], P.mats[i]))) return rc;
+    void* dm = nullptr;
+    if ((rc = h->in_maps.get(maps.data(), sizeof(TmapBlob) * maps.size(), &dm))) return rc;
+    d_in = static_cast<const TmapBlob*>(dm);
+  }
+  int res = BUF_IN;
+  if ((rc = enqueue_ns(h, db, hb, d_in, sumsq, ns_steps, abc, BUF_IN, BUF_OUT, st, &launches, &res))) return rc;
+  h->last_launches = launches;
+  return MUON_OK;
+}
+
+int muon_apply(muon_handle* h, float* const* params, const void* const* o, const double* sumsq,
+               const int32_t* shapes, int count, float lr, float wd, void* stream) {
+  g_last_error.clear();
+  int rc;
+  if ((rc = check_common(h, shapes, count))) return rc;
+  if (!params || !o) return fail(MUON_ERR_INVALID_ARG, "params and o are required");
+  if (!std::isfinite(lr) || !std::isfinite(wd)) return fail(MUON_ERR_INVALID_ARG, "lr and wd must be finite");
+  for (int i = 0; i < count; ++i) {
+    if (!o[i]) continue;
+    if ((rc = check_ptr(params[i], "params", i)) || (rc = check_ptr(o[i], "o", i))) return rc;
+  }
+  DeviceGuard g(h->device);
+  if (!g.ok) return fail(MUON_ERR_CUDA, "cudaSetDevice failed");
+  if ((rc = ensure_plan(h, shapes, count))) return rc;
+  DevPlan& P = *h->plan;
+  std::vector<MatBind> hb((size_t)count);
+  for (int i = 0; i < count; ++i) {
+    std::memset(&hb[i], 0, sizeof(MatBind));
+    hb[i].p = params[i];
+    hb[i].xin = o[i];
+    hb[i].active = o[i] != nullptr;
+  }
+  void* d_binds = nullptr;
+  if ((rc = h->binds.get(hb.data(), sizeof(MatBind) * count, &d_binds))) return rc;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  MUON_CUDA_TRY(launch_apply(elem_launch(P, static_cast<const MatBind*>(d_binds)), BUF_IN, lr, wd,
+                             h->cfg.scale_mode, h->cfg.extra_scale, sumsq, h->cfg.ns_precision == MUON_NS_FP32, st));
+  h->last_launches = 1;
+  return MUON_OK;
+}
+
+int muon_plan_query(const int32_t* shapes, int count, int ns_precision, int64_t* ws_bytes, int64_t* region_offsets,
+                    int32_t* ntiles, int32_t* tiles, int64_t* chunk_prefix) {
+  g_last_error.clear();
+  HostPlan hp;
+  std::string why;
+  if (!build_plan(shapes, count, ns_precision, hp, why)) return fail(MUON_ERR_INVALID_ARG, why);
+  if (ws_bytes) *ws_bytes = hp.ws_bytes;
+  if (region_offsets) std::memcpy(region_offsets, hp.region_off.data(), sizeof(int64_t) * hp.region_off.size());
+  if (ntiles)
+    for (int p = 0; p < 3; ++p) ntiles[p] = (int32_t)hp.tiles[p].size();
+  if (tiles) {
+    size_t k = 0;
+    for (int p = 0; p < 3; ++p)
+      for (const TileRec& t : hp.tiles[p]) {
+        tiles[3 * k] = t.mat;
+        tiles[3 * k + 1] = t.ti;
+        tiles[3 * k + 2] = t.tj;
+        ++k;
+      }
+  }
+  if (chunk_prefix)
+    for (int i = 0; i <= count; ++i) chunk_prefix[i] = hp.prefix[i];
+  return MUON_OK;
+}
+
+int muon_workspace_size(muon_handle* h, const int32_t* shapes, int count, size_t* bytes) {
+  g_last_error.clear();
+  if (!h || !bytes) return fail(MUON_ERR_INVALID_ARG, "handle and bytes are required");
+  HostPlan hp;
+  std::string why;
+  if (!build_plan(shapes, count, h->cfg.ns_precision, hp, why)) return fail(MUON_ERR_INVALID_ARG, why);
+  *bytes = (size_t)hp.ws_bytes;
+  return MUON_OK;
+}
+
+int muon_workspace_ptr(muon_handle* h, void** base, size_t* bytes) {
+  g_last_error.clear();
+  if (!h || !base || !bytes) return fail(MUON_ERR_INVALID_ARG, "handle, base and bytes are required");
+  *base = h->plan ? h->plan->ws : nullptr;
+  *bytes = h->plan ? h->plan->ws_size : 0;
+  return MUON_OK;
+}
+
+int muon_get_status(muon_handle* h, void* stream, int32_t* error_word, uint64_t* nonfinite_count) {
+  g_last_error.clear();
+  if (!h) return fail(MUON_ERR_INVALID_ARG, "handle is NULL");
+  DeviceGuard g(h->device);
+  MUON_CUDA_TRY(cudaStreamSynchronize(static_cast<cudaStream_t>(stream)));
+  DevStatus s;
+  MUON_CUDA_TRY(cudaMemcpy(&s, h->status, sizeof(s), cudaMemcpyDeviceToHost));
+  MUON_CUDA_TRY(cudaMemset(h->status, 0, sizeof(DevStatus)));
+  if (error_word) *error_word = s.error_word;
+  if (nonfinite_count) *nonfinite_count = s.nonfinite;
+  if (s.error_word) return fail(MUON_ERR_TIMEOUT, "a device-side wait expired (code " + std::to_string(s.error_word) + ")");
+  if (s.nonfinite) return fail(MUON_ERR_NONFINITE, std::to_string(s.nonfinite) + " non-finite update entries");
+  return MUON_OK;
+}
+
+int muon_last_launch_count(muon_handle* h, int32_t* launches) {
+  if (!h || !launches) return fail(MUON_ERR_INVALID_ARG, "handle and launches are required");
+  *launches = h->last_launches;
+  return MUON_OK;
+}
+
+}  // extern "C"

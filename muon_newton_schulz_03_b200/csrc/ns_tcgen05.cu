@@ -1,0 +1,399 @@
+// Newton-Schulz phases on the 5th-generation tensor cores (sm_100a).
+//
+// One quintic step ("About Muon: Why Not Adam", sections "The lemma that
+// makes it possible" and "The whole thing, in about forty lines") is three
+// grouped launches of this persistent kernel over all matrices of a call:
+//   GRAM : A = X X^T            (wide, X is s x l)   or  X^T X  (tall)
+//   POLY : B = b A + c A A      (A symmetric)
+//   COMB : X' = a X + B X       (wide)               or  a X + X B  (tall;
+//                                                         B is symmetric)
+// Gram and polynomial outputs are symmetric: only tiles on or right of the
+// 256-block diagonal are computed; off-diagonal tiles are written twice,
+// directly and transposed. Tall matrices (m > n) are never transposed in
+// memory: the Gram reads X with M/N-major operand tiles, and the combine
+// computes X B instead of B X^T.
+// The Frobenius normalisation X0 = Y/(||u|| + eps) of the first step is
+// folded into its epilogues: A0 = alpha^2 Y Y^T and X1 = alpha (a Y + B0 Y).
+//
+// Structure of one CTA (192 threads, one CTA per SM, persistent over a
+// static round-robin tile list):
+//   warp 0     : bulk-tensor (TMA) producer, 4-stage shared-memory ring
+//   warp 1     : tensor-memory allocator and single-thread tcgen05.mma issuer
+//   warps 2..5 : epilogue; tcgen05.ld of a 128 x 256 fp32 accumulator,
+//                fused combine, bf16 round-to-nearest-even stores
+// Two accumulators in tensor memory (2 x 256 columns) let the epilogue of
+// one tile overlap the main loop of the next.
+// Every wait is bounded: on expiry the error word is set, every role stops,
+// in-flight copies and MMAs are drained and tensor memory is freed.
+#include <cstdio>
+
+#include "common.cuh"
+#include "kernels.h"
+
+namespace muon {
+
+namespace {
+
+constexpr int BM = 128, BN = 256, BK = 64;
+constexpr int kStages = 4;
+constexpr int kABytes = BM * BK * 2;            // 16 KiB
+constexpr int kBBytes = BN * BK * 2;            // 32 KiB
+constexpr int kStageBytes = kABytes + kBBytes;  // 48 KiB
+constexpr int kMnChunkBytes = 64 * BK * 2;      // one 64 (M/N) x 64 (K) box, 8 KiB
+constexpr int kThreads = 192;
+constexpr int kTmemCols = 2 * BN;               // two fp32 accumulators
+
+struct __align__(1024) SmemLayout {
+  uint8_t stage[kStages][kStageBytes];
+  uint64_t full[kStages];
+  uint64_t empty[kStages];
+  uint64_t acc_full[2];
+  uint64_t acc_empty[2];
+  uint64_t drain;
+  uint32_t tmem_base;
+};
+
+struct NsArgs {
+  NsLaunch L;
+  int phase, src_sel, dst_sel, first;
+  float a, b, c;
+};
+
+// Everything a role needs to know about one tile.
+struct TileJob {
+  int mat, ti, tj;
+  int kblocks;
+  const void* map_a;
+  const void* map_b;
+  int a_mn, b_mn;      // operand majorness: 0 = K-major, 1 = M/N-major
+  int a_coord, b_coord;  // K-major: first row; M/N-major: first M/N index
+};
+
+__device__ __forceinline__ const TmapBlob* src_maps(const NsLaunch& L, int mat, int src_sel) {
+  if (src_sel == BUF_IN) return L.in_maps + (size_t)mat * kInMapsPerMat;
+  return L.maps + (size_t)mat * kMapsPerMat + (src_sel == BUF_X0 ? MAP_X0 : MAP_X1);
+}
+
+__device__ __forceinline__ TileJob decode(const NsArgs& A, const int4 t, const MatPlan& mp) {
+  TileJob j;
+  j.mat = t.x;
+  j.ti = t.y;
+  j.tj = t.z;
+  const TmapBlob* own = A.L.maps + (size_t)j.mat * kMapsPerMat;
+  if (A.phase == PHASE_GRAM) {
+    const TmapBlob* xs = src_maps(A.L, j.mat, A.src_sel);
+    j.kblocks = (mp.l + BK - 1) / BK;
+    if (!mp.tall) {  // A[i][j] = sum_k X[i][k] X[j][k]
+      j.map_a = xs + MAP_K128; j.a_mn = 0; j.a_coord = j.ti * BM;
+      j.map_b = xs + MAP_K256; j.b_mn = 0; j.b_coord = j.tj * BN;
+    } else {         // A[i][j] = sum_k X[k][i] X[k][j]
+      j.map_a = xs + MAP_MN; j.a_mn = 1; j.a_coord = j.ti * BM;
+      j.map_b = xs + MAP_MN; j.b_mn = 1; j.b_coord = j.tj * BN;
+    }
+  } else if (A.phase == PHASE_POLY) {  // (A A)[i][j] = sum_k A[i][k] A[j][k]
+    j.kblocks = (mp.s + BK - 1) / BK;
+    j.map_a = own + MAP_A_K128; j.a_mn = 0; j.a_coord = j.ti * BM;
+    j.map_b = own + MAP_A_K256; j.b_mn = 0; j.b_coord = j.tj * BN;
+  } else {
+    const TmapBlob* xs = src_maps(A.L, j.mat, A.src_sel);
+    j.kblocks = (mp.s + BK - 1) / BK;
+    if (!mp.tall) {  // (B X)[r][c] = sum_k B[r][k] X[k][c]
+      j.map_a = own + MAP_B_K128; j.a_mn = 0; j.a_coord = j.ti * BM;
+      j.map_b = xs + MAP_MN;      j.b_mn = 1; j.b_coord = j.tj * BN;
+    } else {         // (X B)[r][c] = sum_k X[r][k] B[c][k]
+      j.map_a = xs + MAP_K128;    j.a_mn = 0; j.a_coord = j.ti * BM;
+      j.map_b = own + MAP_B_K256; j.b_mn = 0; j.b_coord = j.tj * BN;
+    }
+  }
+  return j;
+}
+
+// Wait with only a time limit (used while draining after an abort).
+__device__ __forceinline__ bool mbar_wait_drain(uint64_t* bar, uint32_t parity, uint64_t timeout_ns) {
+  const uint64_t t0 = global_timer_ns();
+  while (!mbar_try_wait(bar, parity)) {
+    if (global_timer_ns() - t0 > timeout_ns) return false;
+  }
+  return true;
+}
+
+__device__ __forceinline__ void store_bf16x32(__nv_bfloat16* dst, const float (&o)[32]) {
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    uint4 raw;
+    __nv_bfloat162* h = reinterpret_cast<__nv_bfloat162*>(&raw);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) h[i] = __floats2bfloat162_rn(o[8 * q + 2 * i], o[8 * q + 2 * i + 1]);
+    reinterpret_cast<uint4*>(dst)[q] = raw;
+  }
+}
+
+__device__ __forceinline__ void load_bf16x32(const __nv_bfloat16* src, float (&o)[32]) {
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    uint4 raw = reinterpret_cast<const uint4*>(src)[q];
+    const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&raw);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      float2 f = __bfloat1622float2(h[i]);
+      o[8 * q + 2 * i] = f.x;
+      o[8 * q + 2 * i + 1] = f.y;
+    }
+  }
+}
+
+__global__ void __launch_bounds__(kThreads, 1) ns_phase_kernel(const __grid_constant__ NsArgs args) {
+  extern __shared__ uint8_t smem_raw[];
+  SmemLayout& sm = *reinterpret_cast<SmemLayout*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const NsLaunch& L = args.L;
+  int* err = &L.status->error_word;
+  const uint64_t tmo = L.timeout_ns;
+  // Clean-up waits get at least half a second whatever the wait limit.
+  const uint64_t drain_tmo = tmo > 500000000ull ? tmo : 500000000ull;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&sm.full[s], 1);
+      mbar_init(&sm.empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&sm.acc_full[b], 1);
+      mbar_init(&sm.acc_empty[b], 4);
+    }
+    mbar_init(&sm.drain, 1);
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(&sm.tmem_base, kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = sm.tmem_base;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------------
+    // Producer
+    // ------------------------------------------------------------------
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      uint32_t armed = 0;            // bit s: stage s has been filled at least once
+      uint32_t last_parity = 0;      // bit s: parity of the last fill of stage s
+      bool ok = true;
+      for (int t = blockIdx.x; t < L.ntiles && ok; t += gridDim.x) {
+        const int4 tile = L.tiles[t];
+        if (!L.binds[tile.x].active) continue;
+        const MatPlan mp = L.plans[tile.x];
+        const TileJob j = decode(args, tile, mp);
+        for (int kb = 0; kb < j.kblocks; ++kb) {
+          if (!mbar_wait_bounded(&sm.empty[stage], phase ^ 1u, err, tmo, WAIT_TMA_EMPTY)) { ok = false; break; }
+          mbar_arrive_expect_tx(&sm.full[stage], kStageBytes);
+          uint8_t* sa = sm.stage[stage];
+          uint8_t* sb = sa + kABytes;
+          const int k0 = kb * BK;
+          if (!j.a_mn) {
+            tma_load_2d(sa, j.map_a, &sm.full[stage], k0, j.a_coord);
+          } else {
+#pragma unroll
+            for (int c = 0; c < BM / 64; ++c)
+              tma_load_2d(sa + c * kMnChunkBytes, j.map_a, &sm.full[stage], j.a_coord + 64 * c, k0);
+          }
+          if (!j.b_mn) {
+            tma_load_2d(sb, j.map_b, &sm.full[stage], k0, j.b_coord);
+          } else {
+#pragma unroll
+            for (int c = 0; c < BN / 64; ++c)
+              tma_load_2d(sb + c * kMnChunkBytes, j.map_b, &sm.full[stage], j.b_coord + 64 * c, k0);
+          }
+          armed |= 1u << stage;
+          last_parity = (last_parity & ~(1u << stage)) | (phase << stage);
+          if (++stage == kStages) { stage = 0; phase ^= 1u; }
+        }
+      }
+      if (!ok) {
+        // Let every copy this thread started land before the CTA exits.
+        for (int s = 0; s < kStages; ++s)
+          if (armed & (1u << s)) mbar_wait_drain(&sm.full[s], (last_parity >> s) & 1u, drain_tmo);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------------
+    // MMA issuer
+    // ------------------------------------------------------------------
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      int acc = 0;
+      uint32_t acc_phase = 0;
+      bool ok = true;
+      bool issued = false;
+      for (int t = blockIdx.x; t < L.ntiles && ok; t += gridDim.x) {
+        const int4 tile = L.tiles[t];
+        if (!L.binds[tile.x].active) continue;
+        const MatPlan mp = L.plans[tile.x];
+        const TileJob j = decode(args, tile, mp);
+        if (!mbar_wait_bounded(&sm.acc_empty[acc], acc_phase ^ 1u, err, tmo, WAIT_ACC_EMPTY)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BN);
+        const uint32_t idesc = umma_idesc_bf16(BM, BN, j.a_mn, j.b_mn);
+        for (int kb = 0; kb < j.kblocks; ++kb) {
+          if (!mbar_wait_bounded(&sm.full[stage], phase, err, tmo, WAIT_TMA_FULL)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t sa = smem_u32(sm.stage[stage]);
+          const uint32_t sb = sa + kABytes;
+#pragma unroll
+          for (int k16 = 0; k16 < BK / 16; ++k16) {
+            const uint64_t da = j.a_mn ? umma_desc_sw128(sa + k16 * 2048, kMnChunkBytes, 1024)
+                                       : umma_desc_sw128(sa + k16 * 32, 16, 1024);
+            const uint64_t db = j.b_mn ? umma_desc_sw128(sb + k16 * 2048, kMnChunkBytes, 1024)
+                                       : umma_desc_sw128(sb + k16 * 32, 16, 1024);
+            tc_mma_bf16(d_tmem, da, db, idesc, (kb | k16) != 0);
+          }
+          issued = true;
+          tc_commit(&sm.empty[stage]);      // frees the stage once these MMAs finish
+          if (++stage == kStages) { stage = 0; phase ^= 1u; }
+        }
+        if (!ok) break;
+        tc_commit(&sm.acc_full[acc]);       // accumulator ready for the epilogue
+        if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
+      }
+      if (!ok && issued) {
+        tc_commit(&sm.drain);
+        mbar_wait_drain(&sm.drain, 0, drain_tmo);
+      }
+    }
+  } else {
+    // ------------------------------------------------------------------
+    // Epilogue (warps 2..5): warp w reads tensor-memory lanes 32*(w%4)..+31
+    // ------------------------------------------------------------------
+    const int quarter = warp & 3;
+    const int row_in_tile = quarter * 32 + lane;
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    for (int t = blockIdx.x; t < L.ntiles; t += gridDim.x) {
+      const int4 tile = L.tiles[t];
+      const MatBind mb = L.binds[tile.x];
+      if (!mb.active) continue;
+      const MatPlan mp = L.plans[tile.x];
+      if (!mbar_wait_bounded(&sm.acc_full[acc], acc_phase, err, tmo, WAIT_ACC_FULL)) break;
+      tc_fence_after();
+
+      const int ti = tile.y, tj = tile.z;
+      const int phase = args.phase;
+      int rows, cols, ld;
+      __nv_bfloat16* out;
+      const __nv_bfloat16* aux = nullptr;
+      int aux_ld = 0;
+      float sc = 1.0f;
+      if (phase == PHASE_GRAM) {
+        rows = cols = mp.s; ld = mp.lds; out = static_cast<__nv_bfloat16*>(mp.a);
+        if (args.first) { const double al = inv_norm(L.sumsq, tile.x); sc = (float)(al * al); }
+      } else if (phase == PHASE_POLY) {
+        rows = cols = mp.s; ld = mp.lds; out = static_cast<__nv_bfloat16*>(mp.b);
+        aux = static_cast<const __nv_bfloat16*>(mp.a); aux_ld = mp.lds;
+      } else {
+        rows = mp.m; cols = mp.n; ld = mp.ldx;
+        out = static_cast<__nv_bfloat16*>(const_cast<void*>(sel_buf(mp, mb, args.dst_sel)));
+        aux = static_cast<const __nv_bfloat16*>(sel_buf(mp, mb, args.src_sel)); aux_ld = mp.ldx;
+        if (args.first) sc = (float)inv_norm(L.sumsq, tile.x);
+      }
+      const bool mirror = (phase != PHASE_COMB) && (tj > (ti >> 1));
+      const int row = ti * BM + row_in_tile;
+      const bool row_ok = row < rows;
+      const uint32_t t_base = tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(acc * BN);
+      const float ca = args.a, cb = args.b, cc = args.c;
+
+#pragma unroll 1
+      for (int ch = 0; ch < BN / 32; ++ch) {
+        const int col0 = tj * BN + ch * 32;
+        if (col0 >= cols) break;                       // warp-uniform
+        float v[32];
+        tmem_ld_32x32b_x32(t_base + (uint32_t)(ch * 32), v);
+        const bool full_chunk = col0 + 32 <= cols;
+        float o[32];
+        if (phase == PHASE_GRAM) {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) o[i] = v[i] * sc;
+        } else {
+          float x[32];
+          if (row_ok && full_chunk) {
+            load_bf16x32(aux + (size_t)row * aux_ld + col0, x);
+          } else {
+#pragma unroll
+            for (int i = 0; i < 32; ++i)
+              x[i] = (row_ok && col0 + i < cols) ? __bfloat162float(aux[(size_t)row * aux_ld + col0 + i]) : 0.0f;
+          }
+          if (phase == PHASE_POLY) {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) o[i] = fmaf(cb, x[i], cc * v[i]);
+          } else {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) o[i] = sc * fmaf(ca, x[i], v[i]);
+          }
+        }
+        if (row_ok) {
+          __nv_bfloat16* dst = out + (size_t)row * ld + col0;
+          if (full_chunk) {
+            store_bf16x32(dst, o);
+          } else {
+#pragma unroll
+            for (int i = 0; i < 32; ++i)
+              if (col0 + i < cols) dst[i] = __float2bfloat16_rn(o[i]);
+          }
+        }
+        if (mirror && row_ok) {
+          // Transposed copy: for a fixed column the 32 lanes write 32
+          // consecutive elements of one output row.
+#pragma unroll
+          for (int i = 0; i < 32; ++i)
+            if (col0 + i < cols) out[(size_t)(col0 + i) * ld + row] = __float2bfloat16_rn(o[i]);
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sm.acc_empty[acc]);
+      if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, kTmemCols);
+  }
+}
+
+}  // namespace
+
+int ns_bf16_smem_bytes() { return (int)sizeof(SmemLayout) + 1024; }
+
+cudaError_t launch_ns_phase_bf16(const NsLaunch& L, int phase, int src_sel, int dst_sel, int first, float a,
+                                 float b, float c, cudaStream_t st) {
+  if (L.ntiles <= 0) return cudaSuccess;
+  static bool attr_set = false;
+  const int smem = ns_bf16_smem_bytes();
+  if (!attr_set) {
+    cudaError_t e = cudaFuncSetAttribute(ns_phase_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    attr_set = true;
+  }
+  NsArgs args;
+  args.L = L;
+  args.phase = phase;
+  args.src_sel = src_sel;
+  args.dst_sel = dst_sel;
+  args.first = first;
+  args.a = a;
+  args.b = b;
+  args.c = c;
+  const int grid = L.grid < L.ntiles ? L.grid : L.ntiles;
+  ns_phase_kernel<<<grid, kThreads, smem, st>>>(args);
+  return cudaGetLastError();
+}
+
+}  // namespace muon

@@ -1,0 +1,109 @@
+// Plan builder. The rules (restated independently by the test oracle):
+//  * orientation: m > n is tall, s = min(m, n), l = max(m, n) ("About Muon:
+//    Why Not Adam", section "The whole thing, in about forty lines": the
+//    iteration runs on the short side, square matrices are not transposed);
+//  * storage: X buffers m x round_up(n, 8), A and B s x round_up(s, 8), so
+//    every row starts on a 16-byte boundary as the bulk-tensor copy engine
+//    requires; the workspace starts with one double per matrix (sum of
+//    squares) padded to 1024 bytes, followed by all X0, all X1, all A and
+//    all B regions, each aligned to 1024 bytes;
+//  * tiles of 128 x 256: for the symmetric Gram and polynomial outputs only
+//    tiles whose 256-column block is on or right of the 256-block diagonal
+//    (tj >= ti / 2); for the combine every tile, column block outer for wide
+//    matrices and row block outer for tall ones (each wave of CTAs then
+//    shares the large X panel in L2); each phase's list is ordered by the
+//    matrix's reduction length, longest first, ties by matrix index;
+//  * elementwise: kElemChunk elements per block, prefix over matrices.
+#include "plan.h"
+
+#include <algorithm>
+#include <numeric>
+
+namespace muon {
+
+namespace {
+
+int64_t round_up64(int64_t x, int64_t k) { return (x + k - 1) / k * k; }
+int ceil_div_i(int x, int k) { return (x + k - 1) / k; }
+
+void sym_tiles(int mat, int s, std::vector<TileRec>& out) {
+  const int rt = ceil_div_i(s, kTileM), ct = ceil_div_i(s, kTileN);
+  for (int ti = 0; ti < rt; ++ti)
+    for (int tj = ti / 2; tj < ct; ++tj) out.push_back({mat, ti, tj});
+}
+
+void comb_tiles(int mat, int m, int n, std::vector<TileRec>& out) {
+  const int rt = ceil_div_i(m, kTileM), ct = ceil_div_i(n, kTileN);
+  if (m <= n) {
+    for (int tj = 0; tj < ct; ++tj)
+      for (int ti = 0; ti < rt; ++ti) out.push_back({mat, ti, tj});
+  } else {
+    for (int ti = 0; ti < rt; ++ti)
+      for (int tj = 0; tj < ct; ++tj) out.push_back({mat, ti, tj});
+  }
+}
+
+}  // namespace
+
+bool build_plan(const int32_t* shapes, int count, int prec, HostPlan& P, std::string& why) {
+  if (shapes == nullptr) { why = "shapes is NULL"; return false; }
+  if (count < 1) { why = "count must be >= 1"; return false; }
+  if (prec != 0 && prec != 1) { why = "ns_precision must be 0 (bf16) or 1 (fp32)"; return false; }
+  P = HostPlan();
+  P.count = count;
+  P.prec = prec;
+  P.m.resize(count);
+  P.n.resize(count);
+  P.mats.resize(count);
+  for (int i = 0; i < count; ++i) {
+    const int m = shapes[3 * i], n = shapes[3 * i + 1], fl = shapes[3 * i + 2];
+    if (m < 1 || n < 1 || m > kMaxDim || n > kMaxDim) {
+      why = "matrix " + std::to_string(i) + ": m and n must be in [1, " + std::to_string(kMaxDim) + "], got " +
+            std::to_string(m) + " x " + std::to_string(n);
+      return false;
+    }
+    if (fl & ~1) { why = "matrix " + std::to_string(i) + ": unknown flag bits"; return false; }
+    P.m[i] = m;
+    P.n[i] = n;
+    MatPlan& mp = P.mats[i];
+    mp = MatPlan();
+    mp.m = m;
+    mp.n = n;
+    mp.s = std::min(m, n);
+    mp.l = std::max(m, n);
+    mp.tall = m > n ? 1 : 0;
+    mp.ldx = round_up_i(n, 8);
+    mp.lds = round_up_i(mp.s, 8);
+    mp.numel = (long long)m * (long long)n;
+  }
+  const int64_t elem = prec == 0 ? 2 : 4;
+  P.head_bytes = round_up64(8 * (int64_t)count, kRegionAlign);
+  int64_t off = P.head_bytes;
+  P.region_off.assign((size_t)count * 4, 0);
+  for (int which = 0; which < 4; ++which) {
+    for (int i = 0; i < count; ++i) {
+      const MatPlan& mp = P.mats[i];
+      const int64_t bytes = (which < 2 ? (int64_t)mp.m * mp.ldx : (int64_t)mp.s * mp.lds) * elem;
+      P.region_off[(size_t)i * 4 + which] = off;
+      off = round_up64(off + bytes, kRegionAlign);
+    }
+  }
+  P.ws_bytes = off;
+
+  std::vector<int> order(count);
+  auto sorted_by = [&](auto key) {
+    std::iota(order.begin(), order.end(), 0);
+    std::stable_sort(order.begin(), order.end(), [&](int x, int y) { return key(x) > key(y); });
+    return order;
+  };
+  for (int i : sorted_by([&](int i) { return P.mats[i].l; })) sym_tiles(i, P.mats[i].s, P.tiles[0]);
+  for (int i : sorted_by([&](int i) { return P.mats[i].s; })) sym_tiles(i, P.mats[i].s, P.tiles[1]);
+  for (int i : sorted_by([&](int i) { return P.mats[i].s; })) comb_tiles(i, P.m[i], P.n[i], P.tiles[2]);
+
+  P.prefix.assign((size_t)count + 1, 0);
+  for (int i = 0; i < count; ++i)
+    P.prefix[i + 1] = P.prefix[i] + ceil_div_ll(P.mats[i].numel, kElemChunk);
+  return true;
+}
+
+}  // namespace muon

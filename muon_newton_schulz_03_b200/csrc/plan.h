@@ -1,0 +1,39 @@
+// Host-side plan builder: geometry, workspace layout, tile lists and the
+// elementwise chunk prefix for a shape table. Pure C++ (no CUDA calls), so
+// the integer tables can be produced and checked without a GPU.
+#pragma once
+
+#include <cstdint>
+#include <string>
+#include <vector>
+
+#include "common.cuh"
+
+namespace muon {
+
+constexpr int kTileM = 128;     // output rows per tile
+constexpr int kTileN = 256;     // output columns per tile
+constexpr int kRegionAlign = 1024;
+constexpr int kMaxDim = 1 << 20;
+
+struct TileRec {
+  int mat, ti, tj;
+};
+
+struct HostPlan {
+  int count = 0;
+  int prec = 0;                       // 0 bf16, 1 fp32
+  std::vector<int> m, n;
+  std::vector<MatPlan> mats;          // workspace pointers left null
+  std::vector<int64_t> region_off;    // count * 4: X0, X1, A, B
+  int64_t head_bytes = 0;             // sum-of-squares block
+  int64_t ws_bytes = 0;
+  std::vector<TileRec> tiles[3];      // Gram, polynomial, combine
+  std::vector<long long> prefix;      // count + 1
+};
+
+// Validates the shape table (m, n in [1, kMaxDim], flags in {0, 1}) and
+// builds the plan. Returns false with a message on invalid input.
+bool build_plan(const int32_t* shapes, int count, int prec, HostPlan& out, std::string& why);
+
+}  // namespace muon

@@ -17,8 +17,7 @@ bulk-tensor copy engine requires):
   * X ping-pong buffers X0, X1: m rows, ldx = round_up(n, 8).
   * Gram A and polynomial B: s rows, lds = round_up(s, 8).
 The workspace begins with one float64 sum-of-squares accumulator per
-matrix, then an int32 error word, 4 bytes of padding and a uint64
-non-finite counter, padded to 1024 bytes; then all X0 regions, all X1
+matrix, padded to 1024 bytes; then all X0 regions, all X1
 regions, all A regions, all B regions, each region aligned to 1024 bytes.
 
 Tiles. Output tiles are BM = 128 rows by BN = 256 columns.
@@ -66,7 +65,7 @@ def matrix_geometry(m: int, n: int):
 def workspace_layout(shapes, elem_bytes: int = 2):
     """Byte offsets (X0, X1, A, B) per matrix and the total workspace size."""
     count = len(shapes)
-    head = round_up(8 * count + 16, ALIGN)
+    head = round_up(8 * count, ALIGN)
     off = head
     regions = [[0, 0, 0, 0] for _ in range(count)]
     for which in range(4):

@@ -1,0 +1,92 @@
+"""Helpers shared by the GPU parity tests (inputs, comparisons)."""
+
+import numpy as np
+import torch
+
+import muon_newton_schulz_03_b200 as muon
+import workloads as W
+
+DEV = torch.device("cuda:0")
+
+# Tolerances (relative Frobenius unless stated), from the stated gates:
+TOL_BF16_NS = 2e-2      # bf16 Newton-Schulz vs the float64 oracle
+TOL_FP32_NS = 1e-4      # fp32 debug Newton-Schulz vs the float64 oracle
+TOL_ELEM = 1e-6         # elementwise stages vs the float64 oracle
+
+
+def rel(a, b):
+    a = np.asarray(a, dtype=np.float64)
+    b = np.asarray(b, dtype=np.float64)
+    nb = np.linalg.norm(b)
+    return np.linalg.norm(a - b) / (nb if nb > 0 else 1.0)
+
+
+def to64(t):
+    return t.detach().to("cpu", torch.float64).numpy()
+
+
+def cuda_f32(a):
+    return torch.as_tensor(np.asarray(a), dtype=torch.float32).to(DEV)
+
+
+def cuda_bf16(a):
+    return torch.as_tensor(np.asarray(a), dtype=torch.float32).to(torch.bfloat16).to(DEV)
+
+
+def x_buffer(m, n, dtype=torch.bfloat16, fill=None):
+    buf = muon.x_layout(m, n, dtype, DEV)
+    if fill is not None:
+        buf.zero_()
+        buf[:, :n] = torch.as_tensor(np.asarray(fill), dtype=torch.float32).to(dtype).to(DEV)
+    return buf
+
+
+def bf16_ulp(x):
+    """Spacing of bf16 numbers at |x| (for normal values)."""
+    ax = np.abs(np.asarray(x, dtype=np.float64))
+    e = np.floor(np.log2(np.where(ax > 0, ax, 1.0)))
+    return np.where(ax > 0, 2.0 ** (e - 7), 2.0 ** -133)
+
+
+def make_set(config, shapes, grad_dtype, seed_base=0):
+    """CPU-generated inputs: list of (p, g, m) float64 arrays and torch CUDA tensors."""
+    cpu, dev = [], []
+    for i, (m, n) in enumerate(shapes):
+        seed = W.seed_for(config, i // 7, i % 7) + seed_base
+        g = W.gradient_cpu(config, m, n, seed)
+        p = W.param_cpu(m, n, seed)
+        mom = np.zeros((m, n))
+        gt = (cuda_bf16(g) if grad_dtype == torch.bfloat16 else cuda_f32(g))
+        pt, mt = cuda_f32(p), cuda_f32(mom)
+        cpu.append((to64(pt), to64(gt), to64(mt)))
+        dev.append((pt, gt, mt))
+    return cpu, dev
+
+
+def workspace_matrix(opt, shapes, index, region, dtype=torch.bfloat16):
+    """View of one workspace region (0: X0, 1: X1, 2: A, 3: B) of matrix `index`."""
+    plan = muon.plan_query(shapes, opt.ns_precision)
+    base, size = opt.workspace()
+    off = plan["region_offsets"][index][region]
+    m, n = shapes[index]
+    s = min(m, n)
+    rows, cols = (m, muon.round_up(n, 8)) if region < 2 else (s, muon.round_up(s, 8))
+    esz = 2 if dtype == torch.bfloat16 else 4
+    nbytes = rows * cols * esz
+    assert off + nbytes <= size
+    return device_view(base + off, (rows, cols), dtype).clone()
+
+
+class _CudaArray:
+    def __init__(self, ptr, shape, typestr):
+        self.__cuda_array_interface__ = {"shape": tuple(shape), "typestr": typestr, "data": (int(ptr), False),
+                                         "version": 3, "strides": None}
+
+
+def device_view(ptr, shape, dtype):
+    """A torch tensor aliasing raw device memory (bf16 or fp32)."""
+    torch.cuda.synchronize()
+    if dtype == torch.bfloat16:
+        t = torch.as_tensor(_CudaArray(ptr, shape, "<i2"), device=DEV)
+        return t.view(torch.bfloat16)
+    return torch.as_tensor(_CudaArray(ptr, shape, "<f4"), device=DEV)

@@ -1,0 +1,150 @@
+"""Host-side checks of the C ABI (no GPU needed).
+
+* the shared library builds, loads and exports every function that
+  include/muon_ns.h declares;
+* the integer plan tables match the independent restatement in
+  oracle/plan_tables.py bit for bit, for the workload shape sets and for
+  ragged shapes;
+* the tile lists cover every output entry exactly once (brute force);
+* invalid arguments are rejected with MUON_ERR_INVALID_ARG, and a missing
+  GPU is reported, not crashed on.
+"""
+
+import os
+import re
+
+import numpy as np
+import pytest
+
+import muon_newton_schulz_03_b200 as muon
+from muon_newton_schulz_03_b200 import _lib
+from oracle import plan_tables as PT
+import workloads as W
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared_functions():
+    names = set()
+    for fn in os.listdir(os.path.join(ROOT, "include")):
+        if fn.endswith(".h"):
+            text = open(os.path.join(ROOT, "include", fn)).read()
+            text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+            names |= set(re.findall(r"\b(muon_[a-z_0-9]+)\s*\(", text))
+    return names
+
+
+def test_library_exports_every_declared_function():
+    lib = muon.load()
+    declared = _declared_functions()
+    assert len(declared) >= 15
+    for name in declared:
+        assert hasattr(lib, name), f"{name} declared in include/ but not exported"
+    assert declared == set(_lib.EXPORTED)
+    assert b"sm_100a" in lib.muon_version()
+
+
+SHAPE_SETS = {
+    "single": W.single_shapes(),
+    "gpt2": W.gpt2_shapes(),
+    "llama3": W.llama3_8b_shapes(),
+    "moe": W.moe_shapes(),
+    "ragged": [(1, 1), (1, 7), (7, 1), (3, 5), (127, 129), (129, 127), (300, 300), (513, 257), (64, 1000),
+               (1000, 64), (256, 256), (255, 257)],
+}
+
+
+@pytest.mark.parametrize("name", sorted(SHAPE_SETS))
+@pytest.mark.parametrize("prec", ["bf16", "fp32"])
+def test_plan_tables_bit_exact(name, prec):
+    shapes = SHAPE_SETS[name]
+    got = muon.plan_query(shapes, prec)
+    regions, ws = PT.workspace_layout(shapes, 2 if prec == "bf16" else 4)
+    assert got["ws_bytes"] == ws
+    assert got["region_offsets"] == regions
+    gram, poly, comb = PT.tile_lists(shapes)
+    assert got["tiles"][0] == gram
+    assert got["tiles"][1] == poly
+    assert got["tiles"][2] == comb
+    assert got["chunk_prefix"] == PT.chunk_prefix(shapes)
+
+
+@pytest.mark.parametrize("shape", [(1, 1), (5, 3), (130, 300), (300, 130), (512, 512), (600, 257), (257, 600)])
+def test_tiles_cover_each_entry_once(shape):
+    m, n = shape
+    got = muon.plan_query([shape])
+    s = min(m, n)
+    # Symmetric phases: direct writes of each listed tile plus transposed
+    # writes of the tiles strictly right of the 256-block diagonal.
+    for tiles in got["tiles"][:2]:
+        cover = np.zeros((s, s), dtype=np.int64)
+        for (_, ti, tj) in tiles:
+            r0, c0 = ti * PT.BM, tj * PT.BN
+            r1, c1 = min(r0 + PT.BM, s), min(c0 + PT.BN, s)
+            cover[r0:r1, c0:c1] += 1
+            if tj > ti // 2:
+                cover[c0:c1, r0:r1] += 1
+        assert np.all(cover == 1)
+    cover = np.zeros((m, n), dtype=np.int64)
+    for (_, ti, tj) in got["tiles"][2]:
+        cover[ti * PT.BM:(ti + 1) * PT.BM, tj * PT.BN:(tj + 1) * PT.BN] += 1
+    assert np.all(cover == 1)
+
+
+def test_workspace_regions_aligned_and_disjoint():
+    shapes = SHAPE_SETS["ragged"]
+    got = muon.plan_query(shapes)
+    spans = []
+    for (m, n), offs in zip(shapes, got["region_offsets"]):
+        s = min(m, n)
+        sizes = [m * muon.round_up(n, 8) * 2] * 2 + [s * muon.round_up(s, 8) * 2] * 2
+        for o, sz in zip(offs, sizes):
+            assert o % 1024 == 0
+            spans.append((o, o + sz))
+    spans.sort()
+    assert spans[0][0] >= 8 * len(shapes)
+    for (a0, a1), (b0, b1) in zip(spans, spans[1:]):
+        assert a1 <= b0
+    assert spans[-1][1] <= got["ws_bytes"]
+
+
+@pytest.mark.parametrize("bad", [[(0, 4)], [(4, 0)], [(-1, 4)], [(4, 1 << 21)], [(4, 4, 2)]])
+def test_plan_rejects_invalid_shapes(bad):
+    with pytest.raises(muon.MuonError) as e:
+        muon.plan_query(bad)
+    assert e.value.code == 1
+
+
+def test_plan_rejects_empty_and_bad_precision():
+    lib = muon.load()
+    import ctypes
+    arr = (ctypes.c_int32 * 3)(4, 4, 0)
+    assert lib.muon_plan_query(arr, 0, 0, None, None, None, None, None) == 1
+    assert lib.muon_plan_query(arr, 1, 7, None, None, None, None, None) == 1
+    assert lib.muon_plan_query(None, 1, 0, None, None, None, None, None) == 1
+    assert b"shapes" in lib.muon_last_error()
+
+
+def test_config_defaults():
+    cfg = _lib.MuonConfig()
+    lib = muon.load()
+    import ctypes
+    assert lib.muon_config_init(ctypes.byref(cfg)) == 0
+    assert cfg.scale_mode == 0 and cfg.extra_scale == 1.0 and cfg.ns_precision == 0
+    assert cfg.wait_timeout_s == 2.0 and cfg.num_sms == 0
+    assert lib.muon_config_init(None) == 1
+
+
+def test_init_without_gpu_reports_no_device():
+    torch = pytest.importorskip("torch")
+    if torch.cuda.is_available():
+        pytest.skip("a GPU is present")
+    with pytest.raises(muon.MuonError) as e:
+        muon.Muon(device=0)
+    assert e.value.code == 6
+
+
+def test_null_handle_rejected():
+    lib = muon.load()
+    assert lib.muon_step(None, None, None, None, None, 1, 0.1, 0.9, 1, 0.0, 5, None, None) == 1
+    assert lib.muon_destroy(None) == 0

@@ -1,0 +1,270 @@
+"""GPU parity of each stage of the step against the float64 oracle.
+
+Stage 1 (momentum, Nesterov, norm, cast), stage 2 (Newton-Schulz on the
+tensor cores, and the fp32 debug path), stage 3 (apply), each called
+through the C ABI on seeded inputs of several tile counts with ragged tails.
+"""
+
+import numpy as np
+import pytest
+import torch
+
+import muon_newton_schulz_03_b200 as muon
+from oracle import muon_oracle as O
+
+from gpu_helpers import (DEV, TOL_BF16_NS, TOL_ELEM, TOL_FP32_NS, bf16_ulp, cuda_bf16, cuda_f32, rel, to64,
+                         x_buffer)
+
+pytestmark = pytest.mark.gpu
+
+RAGGED = [(1, 1), (3, 5), (5, 3), (1, 300), (300, 1), (127, 129), (129, 127), (64, 64), (256, 512), (512, 256),
+          (384, 384), (200, 1000), (1000, 200), (520, 520), (768, 2304)]
+
+
+@pytest.fixture(scope="module")
+def opt_bf16():
+    h = muon.Muon(device=0)
+    yield h
+    h.close()
+
+
+@pytest.fixture(scope="module")
+def opt_fp32():
+    h = muon.Muon(device=0, ns_precision="fp32")
+    yield h
+    h.close()
+
+
+def _assert_status_clean(opt):
+    code, ew, nf = opt.status()
+    assert (code, ew, nf) == (0, 0, 0), f"device status {code} error word {ew} non-finite {nf}"
+
+
+# ---------------------------------------------------------------------------
+# Stage 1
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("grad_dtype", [torch.float32, torch.bfloat16])
+@pytest.mark.parametrize("nesterov", [True, False])
+def test_momentum_norm_matches_oracle(opt_bf16, grad_dtype, nesterov):
+    rng = np.random.default_rng(1)
+    shapes = RAGGED
+    beta = np.float32(0.95)
+    gs, ms, ys, gd, md = [], [], [], [], []
+    for (m, n) in shapes:
+        g = rng.standard_normal((m, n)) * 1e-2
+        mom = rng.standard_normal((m, n)) * 1e-2
+        gt = cuda_bf16(g) if grad_dtype == torch.bfloat16 else cuda_f32(g)
+        mt = cuda_f32(mom)
+        gs.append(to64(gt)); ms.append(to64(mt))
+        gd.append(gt); md.append(mt); ys.append(x_buffer(m, n))
+    # one skipped matrix
+    gd[3] = None
+    sumsq = torch.full((len(shapes),), -1.0, dtype=torch.float64, device=DEV)
+    opt_bf16.momentum_norm(gd, md, ys, sumsq, beta=float(beta), nesterov=nesterov)
+    torch.cuda.synchronize()
+    ss = sumsq.cpu().numpy()
+    for i, (m, n) in enumerate(shapes):
+        if i == 3:
+            assert np.array_equal(to64(md[i]), ms[i])
+            assert ss[i] == 0.0
+            continue
+        m_ref = O.momentum_update(ms[i], gs[i], float(beta))
+        u_ref = O.nesterov_blend(gs[i], m_ref, float(beta), nesterov)
+        assert rel(to64(md[i]), m_ref) <= TOL_ELEM
+        nu_ref = np.linalg.norm(u_ref)
+        assert abs(np.sqrt(ss[i]) - nu_ref) <= TOL_ELEM * nu_ref
+        y = to64(ys[i][:, :n])
+        y_ref = O.bf16_round(u_ref)
+        assert np.all(np.abs(y - y_ref) <= bf16_ulp(y_ref)), f"matrix {i}: cast off by more than one bf16 ulp"
+
+
+def test_momentum_norm_fp32_output(opt_fp32):
+    rng = np.random.default_rng(2)
+    shapes = [(33, 70), (128, 256), (7, 8)]
+    gd = [cuda_f32(rng.standard_normal(s)) for s in shapes]
+    md = [cuda_f32(rng.standard_normal(s)) for s in shapes]
+    g64 = [to64(t) for t in gd]
+    m64 = [to64(t) for t in md]
+    ys = [x_buffer(m, n, torch.float32) for (m, n) in shapes]
+    sumsq = torch.zeros(len(shapes), dtype=torch.float64, device=DEV)
+    opt_fp32.momentum_norm(gd, md, ys, sumsq, beta=0.9, nesterov=True)
+    torch.cuda.synchronize()
+    for i, (m, n) in enumerate(shapes):
+        m_ref = O.momentum_update(m64[i], g64[i], float(np.float32(0.9)))
+        u_ref = O.nesterov_blend(g64[i], m_ref, float(np.float32(0.9)))
+        assert rel(to64(ys[i][:, :n]), u_ref) <= TOL_ELEM
+        assert rel(to64(md[i]), m_ref) <= TOL_ELEM
+
+
+# ---------------------------------------------------------------------------
+# Stage 3
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("mode", ["moonlight", "jordan", "bernstein", "none"])
+def test_apply_matches_oracle(mode):
+    opt = muon.Muon(device=0, scale_mode=mode, extra_scale=1.25)
+    rng = np.random.default_rng(3)
+    shapes = RAGGED
+    pd, od, p64, o64 = [], [], [], []
+    for (m, n) in shapes:
+        pt = cuda_f32(rng.standard_normal((m, n)) * 0.02)
+        ob = x_buffer(m, n, fill=rng.standard_normal((m, n)) * 0.05)
+        pd.append(pt); od.append(ob); p64.append(to64(pt)); o64.append(to64(ob[:, :n]))
+    od[2] = None
+    lr, wd = np.float32(2e-4), np.float32(0.1)
+    opt.apply(pd, od, lr=float(lr), wd=float(wd))
+    torch.cuda.synchronize()
+    for i, (m, n) in enumerate(shapes):
+        got = to64(pd[i])
+        if i == 2:
+            assert np.array_equal(got, p64[i])
+            continue
+        scale = O.update_scale(m, n, O.__dict__["SCALE_" + mode.upper()], float(np.float32(1.25)))
+        ref = O.apply_update(p64[i], o64[i], float(lr), float(wd), scale)
+        assert rel(got, ref) <= TOL_ELEM, f"matrix {i} {m}x{n}"
+    opt.close()
+
+
+def test_apply_with_norm_scale(opt_bf16):
+    rng = np.random.default_rng(4)
+    shapes = [(40, 72), (72, 40)]
+    pd = [cuda_f32(rng.standard_normal(s)) for s in shapes]
+    p64 = [to64(t) for t in pd]
+    ob = [x_buffer(m, n, fill=rng.standard_normal((m, n))) for (m, n) in shapes]
+    ss = np.array([4.0, 0.25])
+    sumsq = torch.tensor(ss, dtype=torch.float64, device=DEV)
+    opt_bf16.apply(pd, ob, lr=0.01, wd=0.0, sumsq=sumsq)
+    torch.cuda.synchronize()
+    for i, (m, n) in enumerate(shapes):
+        o = to64(ob[i][:, :n]) / (np.sqrt(ss[i]) + O.EPS)
+        ref = O.apply_update(p64[i], o, float(np.float32(0.01)), 0.0, O.update_scale(m, n))
+        assert rel(to64(pd[i]), ref) <= TOL_ELEM
+
+
+# ---------------------------------------------------------------------------
+# Stage 2: Newton-Schulz
+# ---------------------------------------------------------------------------
+
+def _ns_inputs(shapes, seed, scale=1.0):
+    rng = np.random.default_rng(seed)
+    xin, x64 = [], []
+    for (m, n) in shapes:
+        x = rng.standard_normal((m, n)) * scale
+        buf = x_buffer(m, n, fill=x)
+        xin.append(buf)
+        x64.append(to64(buf[:, :n]))
+    return xin, x64
+
+
+def test_ns_identity_combine_is_exact(opt_bf16):
+    # (a, b, c) = (1, 0, 0): B = 0, so X1 = 1 * X + 0 * X exactly. Exercises
+    # every tile's combine epilogue addressing (direct, ragged tails, tall).
+    shapes = RAGGED
+    xin, x64 = _ns_inputs(shapes, 5)
+    xout = [x_buffer(m, n) for (m, n) in shapes]
+    opt_bf16.newton_schulz(xin, xout, shapes, None, ns_steps=1, coeffs=(1.0, 0.0, 0.0))
+    torch.cuda.synchronize()
+    for i, (m, n) in enumerate(shapes):
+        assert np.array_equal(to64(xout[i][:, :n]), x64[i]), f"matrix {i} {m}x{n}"
+    _assert_status_clean(opt_bf16)
+
+
+@pytest.mark.parametrize("coeffs", [(0.0, 1.0, 0.0), (0.0, 0.0, 1.0), (0.5, -0.25, 0.125)])
+def test_ns_single_step_phases(opt_bf16, coeffs):
+    # One step with chosen coefficients isolates the Gram (b), the polynomial
+    # product (c) and the combine (a) against float64 products of the same
+    # bf16 input; alpha = 1 (no norm).
+    shapes = RAGGED
+    xin, x64 = _ns_inputs(shapes, 6, scale=0.05)
+    xout = [x_buffer(m, n) for (m, n) in shapes]
+    opt_bf16.newton_schulz(xin, xout, shapes, None, ns_steps=1, coeffs=coeffs)
+    torch.cuda.synchronize()
+    for i, (m, n) in enumerate(shapes):
+        ref = O.ns_only(x64[i], 1, coeffs)
+        emu = _emulated_ns_only(x64[i], 1, coeffs)
+        got = to64(xout[i][:, :n])
+        assert rel(got, ref) <= TOL_BF16_NS, f"matrix {i} {m}x{n}: {rel(got, ref):.3e}"
+        assert rel(got, emu) <= 5e-3, f"matrix {i} {m}x{n} vs bf16-emulating oracle: {rel(got, emu):.3e}"
+    _assert_status_clean(opt_bf16)
+
+
+def _emulated_ns_only(X, steps, coeffs):
+    """Oracle NS with bf16 rounding at the GPU's rounding points, alpha = 1."""
+    X = np.asarray(X, dtype=np.float64)
+    t = X.shape[0] > X.shape[1]
+    if t:
+        X = X.T
+    a, b, c = coeffs
+    for _ in range(steps):
+        A = O.bf16_round(X @ X.T)
+        B = O.bf16_round(b * A + c * (A @ A))
+        X = O.bf16_round(a * X + B @ X)
+    return X.T if t else X
+
+
+@pytest.mark.parametrize("steps", [1, 2, 5])
+def test_ns_bf16_matches_oracle(opt_bf16, steps):
+    shapes = RAGGED
+    xin, x64 = _ns_inputs(shapes, 7 + steps)
+    sumsq = torch.tensor([np.sum(x ** 2) for x in x64], dtype=torch.float64, device=DEV)
+    xout = [x_buffer(m, n) for (m, n) in shapes]
+    opt_bf16.newton_schulz(xin, xout, shapes, sumsq, ns_steps=steps)
+    torch.cuda.synchronize()
+    for i, (m, n) in enumerate(shapes):
+        ref = O.newton_schulz(x64[i], steps)
+        got = to64(xout[i][:, :n])
+        assert rel(got, ref) <= TOL_BF16_NS, f"matrix {i} {m}x{n}: {rel(got, ref):.3e}"
+    # Inputs were not modified.
+    for i, (m, n) in enumerate(shapes):
+        assert np.array_equal(to64(xin[i][:, :n]), x64[i])
+    _assert_status_clean(opt_bf16)
+
+
+def test_ns_zero_steps_scales(opt_bf16):
+    shapes = [(10, 20), (20, 10)]
+    xin, x64 = _ns_inputs(shapes, 9)
+    sumsq = torch.tensor([np.sum(x ** 2) for x in x64], dtype=torch.float64, device=DEV)
+    xout = [x_buffer(m, n) for (m, n) in shapes]
+    opt_bf16.newton_schulz(xin, xout, shapes, sumsq, ns_steps=0)
+    torch.cuda.synchronize()
+    for i, (m, n) in enumerate(shapes):
+        ref = O.newton_schulz(x64[i], 0)
+        assert rel(to64(xout[i][:, :n]), ref) <= 4e-3
+
+
+@pytest.mark.parametrize("steps", [1, 5])
+def test_ns_fp32_matches_oracle(opt_fp32, steps):
+    rng = np.random.default_rng(10)
+    shapes = RAGGED
+    xin, x64 = [], []
+    for (m, n) in shapes:
+        buf = x_buffer(m, n, torch.float32, fill=rng.standard_normal((m, n)))
+        xin.append(buf)
+        x64.append(to64(buf[:, :n]))
+    sumsq = torch.tensor([np.sum(x ** 2) for x in x64], dtype=torch.float64, device=DEV)
+    xout = [x_buffer(m, n, torch.float32) for (m, n) in shapes]
+    opt_fp32.newton_schulz(xin, xout, shapes, sumsq, ns_steps=steps)
+    torch.cuda.synchronize()
+    for i, (m, n) in enumerate(shapes):
+        ref = O.newton_schulz(x64[i], steps)
+        got = to64(xout[i][:, :n])
+        assert rel(got, ref) <= TOL_FP32_NS, f"matrix {i} {m}x{n}: {rel(got, ref):.3e}"
+
+
+def test_ns_gram_is_symmetric_in_workspace(opt_bf16):
+    # The Gram tiles right of the diagonal are mirrored: A must be exactly
+    # symmetric, and equal to the float64 Gram of the bf16 input at bf16 level.
+    from gpu_helpers import workspace_matrix
+    shapes = [(600, 900), (900, 600), (513, 513)]
+    xin, x64 = _ns_inputs(shapes, 11, scale=0.03)
+    xout = [x_buffer(m, n) for (m, n) in shapes]
+    opt_bf16.newton_schulz(xin, xout, shapes, None, ns_steps=1)
+    torch.cuda.synchronize()
+    for i, (m, n) in enumerate(shapes):
+        s = min(m, n)
+        A = to64(workspace_matrix(opt_bf16, shapes, i, 2)[:, :s])
+        assert np.array_equal(A, A.T)
+        X = x64[i] if m <= n else x64[i].T
+        ref = X @ X.T
+        assert rel(A, ref) <= 4e-3

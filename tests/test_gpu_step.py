@@ -1,0 +1,299 @@
+"""GPU parity of the whole Muon step (muon_step through the C ABI).
+
+* the single 256 x 512 workload and the GPT-2-small set in full;
+* the Llama-3-8B and MoE sets at full size in the launch configuration the
+  benchmark times, checked on sampled matrices that the oracle recomputes;
+* edge cases: skipped matrices, zero gradients, zero iterations, NaNs,
+  repeated steps (momentum carried), CUDA-graph replay, status word.
+"""
+
+import numpy as np
+import pytest
+import torch
+
+import muon_newton_schulz_03_b200 as muon
+import workloads as W
+from oracle import muon_oracle as O
+
+from gpu_helpers import (DEV, TOL_BF16_NS, TOL_ELEM, TOL_FP32_NS, cuda_bf16, cuda_f32, make_set, rel, to64,
+                         workspace_matrix)
+
+pytestmark = pytest.mark.gpu
+
+F32 = lambda v: float(np.float32(v))  # noqa: E731  (scalars as the kernels see them)
+
+
+def _check_step(cpu, dev, shapes, opt, *, lr, beta, wd, nesterov=True, ns_steps=5, scale_mode=O.SCALE_MOONLIGHT,
+                tol=TOL_BF16_NS, check_o=True, indices=None):
+    indices = range(len(shapes)) if indices is None else indices
+    worst = 0.0
+    for i in indices:
+        m, n = shapes[i]
+        p0, g, m0 = cpu[i]
+        p_ref, m_ref, o_ref, nu = O.muon_step_matrix(p0, g, m0, lr=F32(lr), beta=F32(beta), nesterov=nesterov,
+                                                     wd=F32(wd), ns_steps=ns_steps, scale_mode=scale_mode)
+        p_gpu, _, m_gpu = (to64(t) for t in dev[i])
+        assert rel(m_gpu, m_ref) <= TOL_ELEM, f"momentum of matrix {i}"
+        dp_ref = p_ref - p0
+        dp_gpu = p_gpu - p0
+        e = rel(dp_gpu, dp_ref)
+        worst = max(worst, e)
+        assert e <= tol, f"matrix {i} {m}x{n}: update off by {e:.3e}"
+        if check_o and ns_steps > 0:
+            dtype = torch.bfloat16 if opt.ns_precision == "bf16" else torch.float32
+            o_gpu = to64(workspace_matrix(opt, shapes, i, ns_steps % 2, dtype)[:, :n])
+            eo = rel(o_gpu, o_ref)
+            assert eo <= tol, f"matrix {i}: O off by {eo:.3e}"
+            # p' itself at the elementwise gate, with the oracle fed the GPU's O.
+            scale = O.update_scale(m, n, scale_mode)
+            p_from_o = O.apply_update(p0, o_gpu, F32(lr), F32(wd), scale)
+            assert rel(p_gpu, p_from_o) <= TOL_ELEM
+    return worst
+
+
+@pytest.mark.parametrize("prec,tol", [("bf16", TOL_BF16_NS), ("fp32", TOL_FP32_NS)])
+def test_single_matrix_workload(prec, tol):
+    # One 256 x 512 fp32 gradient, zero momentum, beta 0.95 Nesterov, 5 steps,
+    # lr 0.02, wd 0, Jordan scale (the lr 0.02 pairing).
+    shapes = W.single_shapes()
+    cpu, dev = make_set(W.CONFIG_SINGLE, shapes, torch.float32)
+    opt = muon.Muon(device=0, scale_mode="jordan", ns_precision=prec)
+    opt.step([d[0] for d in dev], [d[1] for d in dev], [d[2] for d in dev], lr=0.02, beta=0.95, wd=0.0)
+    torch.cuda.synchronize()
+    _check_step(cpu, dev, shapes, opt, lr=0.02, beta=0.95, wd=0.0, scale_mode=O.SCALE_JORDAN, tol=tol)
+    assert opt.status() == (0, 0, 0)
+    assert opt.last_launch_count() == (17 if prec == "bf16" else 1 + 15 + 1)
+    opt.close()
+
+
+@pytest.mark.parametrize("prec,tol", [("bf16", TOL_BF16_NS), ("fp32", TOL_FP32_NS)])
+def test_gpt2_small_set(prec, tol):
+    shapes = W.gpt2_shapes()
+    cpu, dev = make_set(W.CONFIG_GPT2, shapes, torch.float32)
+    opt = muon.Muon(device=0, ns_precision=prec)
+    opt.step([d[0] for d in dev], [d[1] for d in dev], [d[2] for d in dev], lr=2e-4, beta=0.95, wd=0.1)
+    torch.cuda.synchronize()
+    idx = range(len(shapes)) if prec == "bf16" else range(4)
+    _check_step(cpu, dev, shapes, opt, lr=2e-4, beta=0.95, wd=0.1, tol=tol, indices=idx)
+    assert opt.status() == (0, 0, 0)
+    opt.close()
+
+
+def test_warm_momentum_three_steps():
+    # Three consecutive steps with fresh gradients: the momentum carried on
+    # the GPU matches the oracle's recurrence.
+    shapes = [(256, 768), (768, 256)]
+    opt = muon.Muon(device=0)
+    rng = np.random.default_rng(20)
+    p = [cuda_f32(rng.standard_normal(s) * 0.02) for s in shapes]
+    mo = [torch.zeros(s, dtype=torch.float32, device=DEV) for s in shapes]
+    p64 = [to64(t) for t in p]
+    p_start = [x.copy() for x in p64]
+    m64 = [np.zeros(s) for s in shapes]
+    for step in range(3):
+        g = [cuda_f32(W.gradient_cpu(W.CONFIG_GPT2, m, n, 100 + 10 * step + i)) for i, (m, n) in enumerate(shapes)]
+        opt.step(p, g, mo, lr=2e-4, beta=0.95, wd=0.1)
+        for i in range(len(shapes)):
+            p64[i], m64[i], _, _ = O.muon_step_matrix(p64[i], to64(g[i]), m64[i], lr=F32(2e-4), beta=F32(0.95),
+                                                      wd=F32(0.1))
+    torch.cuda.synchronize()
+    for i in range(len(shapes)):
+        assert rel(to64(mo[i]), m64[i]) <= 1e-6
+        # total displacement over the three steps
+        assert rel(to64(p[i]) - p_start[i], p64[i] - p_start[i]) <= TOL_BF16_NS
+    opt.close()
+
+
+def test_skipped_zero_and_nan_gradients():
+    shapes = [(64, 96), (96, 64), (32, 32), (48, 80)]
+    opt = muon.Muon(device=0, check_nonfinite=True)
+    rng = np.random.default_rng(21)
+    p = [cuda_f32(rng.standard_normal(s)) for s in shapes]
+    mo = [cuda_f32(rng.standard_normal(s) * 0.1) for s in shapes]
+    p0 = [to64(t) for t in p]
+    m0 = [to64(t) for t in mo]
+    g = [None, torch.zeros(shapes[1], dtype=torch.float32, device=DEV),
+         cuda_f32(rng.standard_normal(shapes[2])), cuda_f32(rng.standard_normal(shapes[3]))]
+    opt.step(p, g, mo, lr=0.01, beta=0.9, wd=0.5, nesterov=False)
+    torch.cuda.synchronize()
+    # Skipped: untouched.
+    assert np.array_equal(to64(p[0]), p0[0]) and np.array_equal(to64(mo[0]), m0[0])
+    # Zero gradient with non-zero momentum and Nesterov off: u = 0.9 m; a
+    # plain Muon step of that direction.
+    ref, mref, _, _ = O.muon_step_matrix(p0[1], np.zeros(shapes[1]), m0[1], lr=F32(0.01), beta=F32(0.9),
+                                         wd=F32(0.5), nesterov=False)
+    assert rel(to64(p[1]) - p0[1], ref - p0[1]) <= TOL_BF16_NS
+    assert opt.status() == (0, 0, 0)
+    # A NaN is counted and reported.
+    g[2][3, 4] = float("nan")
+    g[3][0, 0] = float("inf")
+    opt.step(p, g, mo, lr=0.01, beta=0.9, wd=0.5)
+    code, ew, nf = opt.status()
+    assert code == 5 and ew == 0 and nf == 2
+    assert opt.status() == (0, 0, 0)  # cleared
+    opt.close()
+
+
+def test_truly_zero_state_gives_pure_decay():
+    shapes = [(40, 60)]
+    opt = muon.Muon(device=0)
+    p = [cuda_f32(np.random.default_rng(22).standard_normal(shapes[0]))]
+    p0 = to64(p[0])
+    opt.step(p, [torch.zeros(shapes[0], device=DEV)], [torch.zeros(shapes[0], device=DEV)], lr=0.1, wd=0.2)
+    torch.cuda.synchronize()
+    assert rel(to64(p[0]), p0 * (1 - F32(0.1) * F32(0.2))) <= TOL_ELEM
+    opt.close()
+
+
+def test_zero_iterations():
+    shapes = [(30, 50), (50, 30)]
+    cpu, dev = make_set(W.CONFIG_GPT2, shapes, torch.float32)
+    opt = muon.Muon(device=0)
+    opt.step([d[0] for d in dev], [d[1] for d in dev], [d[2] for d in dev], lr=0.01, ns_steps=0)
+    torch.cuda.synchronize()
+    _check_step(cpu, dev, shapes, opt, lr=0.01, beta=0.95, wd=0.1, ns_steps=0, tol=4e-3, check_o=False)
+    opt.close()
+
+
+def test_repeat_runs_agree_and_graph_replay():
+    shapes = W.gpt2_shapes()[:8]
+    cpu, dev = make_set(W.CONFIG_GPT2, shapes, torch.float32)
+    base_p = [d[0].clone() for d in dev]
+    outs = []
+    opt = muon.Muon(device=0)
+    for _ in range(2):
+        p = [t.clone() for t in base_p]
+        mo = [torch.zeros_like(t) for t in base_p]
+        opt.step(p, [d[1] for d in dev], mo, lr=2e-4)
+        torch.cuda.synchronize()
+        outs.append([to64(t) for t in p])
+    for a, b in zip(*outs):
+        assert np.max(np.abs(a - b)) <= 1e-9
+    # Capture the same call (same pointers: no table upload) in a CUDA graph.
+    p = [t.clone() for t in base_p]
+    mo = [torch.zeros_like(t) for t in base_p]
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        opt.step(p, [d[1] for d in dev], mo, lr=2e-4)       # warm: plan and tables exist
+    torch.cuda.current_stream().wait_stream(s)
+    torch.cuda.synchronize()
+    for t, b in zip(p, base_p):
+        t.copy_(b)
+    for t in mo:
+        t.zero_()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        opt.step(p, [d[1] for d in dev], mo, lr=2e-4)
+    for t, b in zip(p, base_p):
+        t.copy_(b)
+    for t in mo:
+        t.zero_()
+    graph.replay()
+    torch.cuda.synchronize()
+    for a, b in zip(outs[0], p):
+        assert np.max(np.abs(a - to64(b))) <= 1e-9
+    opt.close()
+
+
+def test_step_host_matches_device_step():
+    shapes = [(128, 384), (384, 128), (100, 100)]
+    cpu, dev = make_set(W.CONFIG_GPT2, shapes, torch.bfloat16)
+    hp = [d[0].cpu().pin_memory() for d in dev]
+    hg = [d[1].cpu().pin_memory() for d in dev]
+    hm = [d[2].cpu().pin_memory() for d in dev]
+    opt = muon.Muon(device=0)
+    opt.step_host(hp, hg, hm, lr=2e-4)
+    torch.cuda.synchronize()
+    opt.step([d[0] for d in dev], [d[1] for d in dev], [d[2] for d in dev], lr=2e-4)
+    torch.cuda.synchronize()
+    for i in range(len(shapes)):
+        assert torch.equal(hp[i], dev[i][0].cpu())
+        assert torch.equal(hm[i], dev[i][2].cpu())
+    opt.close()
+
+
+def test_bounded_wait_expiry_reports_timeout_and_recovers():
+    # A wait limit far below any real wait makes the first pending wait run
+    # out: the kernel records the error word, drains its copies and MMAs,
+    # frees tensor memory and returns. The context stays usable.
+    shapes = [(512, 1024), (1024, 512)]
+    cpu, dev = make_set(W.CONFIG_GPT2, shapes, torch.float32)
+    opt = muon.Muon(device=0, wait_timeout_s=1e-9)
+    opt.step([d[0].clone() for d in dev], [d[1] for d in dev], [d[2].clone() for d in dev], lr=2e-4)
+    code, ew, nf = opt.status()
+    assert code == 4 and ew in (1, 2, 3, 4)
+    opt.close()
+    ok = muon.Muon(device=0)
+    ok.step([d[0] for d in dev], [d[1] for d in dev], [d[2] for d in dev], lr=2e-4)
+    torch.cuda.synchronize()
+    _check_step(cpu, dev, shapes, ok, lr=2e-4, beta=0.95, wd=0.1)
+    assert ok.status() == (0, 0, 0)
+    ok.close()
+
+
+def test_invalid_arguments_rejected():
+    opt = muon.Muon(device=0)
+    p = torch.zeros((8, 8), device=DEV)
+    with pytest.raises(muon.MuonError) as e:
+        opt.step([p], [p], [p], lr=0.1)        # overlapping buffers
+    assert e.value.code == 1
+    with pytest.raises(muon.MuonError):
+        opt.step([p], [torch.zeros((8, 8), device=DEV)], [torch.zeros((8, 8), device=DEV)], lr=0.1, beta=1.5)
+    with pytest.raises(muon.MuonError):
+        opt.step([p], [torch.zeros((8, 8), device=DEV)], [torch.zeros((8, 8), device=DEV)], lr=0.1, ns_steps=65)
+    big = torch.zeros(64, device=DEV)
+    with pytest.raises(muon.MuonError):   # misaligned pointer
+        opt.step([big[1:].view(7, 9)], [torch.zeros((7, 9), device=DEV)], [torch.zeros((7, 9), device=DEV)], lr=0.1)
+    opt.close()
+
+
+# ---------------------------------------------------------------------------
+# Full-size sets in the benchmark's launch configuration, sampled matrices
+# ---------------------------------------------------------------------------
+
+def _full_set_sampled(config, shapes, grad_dtype, sample, lr=2e-4, wd=0.1):
+    dev = []
+    cpu = {}
+    for i, (m, n) in enumerate(shapes):
+        seed = W.seed_for(config, i // 7, i % 7)
+        if i in sample:
+            g = W.gradient_cpu(config, m, n, seed)
+            p = W.param_cpu(m, n, seed)
+            gt = cuda_bf16(g) if grad_dtype == torch.bfloat16 else cuda_f32(g)
+            pt = cuda_f32(p)
+            cpu[i] = (to64(pt), to64(gt), np.zeros((m, n)))
+        else:
+            gt = W.gradient_gpu(config, m, n, seed, DEV, grad_dtype)
+            pt = W.param_gpu(m, n, seed, DEV)
+        dev.append((pt, gt, torch.zeros((m, n), dtype=torch.float32, device=DEV)))
+    opt = muon.Muon(device=0)
+    opt.step([d[0] for d in dev], [d[1] for d in dev], [d[2] for d in dev], lr=lr, beta=0.95, wd=wd)
+    torch.cuda.synchronize()
+    assert opt.status() == (0, 0, 0)
+    errs = []
+    for i in sample:
+        m, n = shapes[i]
+        p0, g, m0 = cpu[i]
+        p_ref, m_ref, o_ref, _ = O.muon_step_matrix(p0, g, m0, lr=F32(lr), beta=F32(0.95), wd=F32(wd))
+        p_gpu, m_gpu = to64(dev[i][0]), to64(dev[i][2])
+        assert rel(m_gpu, m_ref) <= TOL_ELEM
+        e = rel(p_gpu - p0, p_ref - p0)
+        errs.append(e)
+        assert e <= TOL_BF16_NS, f"matrix {i} {m}x{n}: {e:.3e}"
+    opt.close()
+    return errs
+
+
+@pytest.mark.slow
+def test_llama3_8b_set_sampled():
+    shapes = W.llama3_8b_shapes()
+    # layer 0 q (square), k (wide, small), gate (tall), and layer 31 down (wide)
+    _full_set_sampled(W.CONFIG_LLAMA, shapes, torch.bfloat16, sample=[0, 1, 4, 223])
+
+
+@pytest.mark.slow
+def test_moe_set_sampled():
+    shapes = W.moe_shapes()
+    # three experts: gate (wide) and down (tall)
+    _full_set_sampled(W.CONFIG_MOE, shapes, torch.bfloat16, sample=[0, 5, 382])
