@@ -1,0 +1,468 @@
+"""Throughput of the Muon step on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload llama3|gpt2|moe|single]
+                    [--impl ours|reference] [--no-e2e] [--no-cpu-baseline]
+
+One "step" is one Muon optimizer step over the whole matrix set of the
+workload: momentum/Nesterov/norm/cast, five quintic Newton-Schulz iterations
+on the tensor cores, scale + weight decay + write. Default workload: the
+Llama-3-8B hidden-matrix set (224 matrices, 6.98 G elements, bf16 grads,
+fp32 params and momenta), synthetic inputs generated on the device from
+seeds (workloads/). Inputs (70 GB) are far larger than L2, so no L2 flush is
+needed between steps.
+
+Metric: Muon steps/s for the whole job (weak scaling: with N GPUs every rank
+runs its own full set, no collective on the data path), with NS TFLOP/s
+(nominal 5 (4 s^2 l + 2 s^3) per matrix) and its fraction of peak.
+Rank 0 prints one JSON line.
+
+--impl reference times the float64 CPU oracle (the reference arm of this
+method) on a bounded sample of the same workload, scaled to steps/s.
+"""
+
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import workloads as W  # noqa: E402
+
+DATASHEET_BF16_TFLOPS = 2250.0
+DATASHEET_HBM_GBS = 8000.0
+FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+WORKLOADS = {
+    "llama3": (W.CONFIG_LLAMA, W.llama3_8b_shapes, "bf16", "Llama-3-8B hidden matrices: 32 x {q 4096x4096, "
+               "k 1024x4096, v 1024x4096, o 4096x4096, gate 14336x4096, up 14336x4096, down 4096x14336}"),
+    "gpt2": (W.CONFIG_GPT2, W.gpt2_shapes, "fp32", "GPT-2-small hidden matrices: 12 x {QKV 2304x768, "
+             "O 768x768, up 3072x768, down 768x3072}"),
+    "moe": (W.CONFIG_MOE, W.moe_shapes, "bf16", "MoE layer: 128 experts x {gate 2048x7168, up 2048x7168, "
+            "down 7168x2048}"),
+    "single": (W.CONFIG_SINGLE, W.single_shapes, "fp32", "one 256x512 gradient"),
+}
+LR, BETA, WD = 2e-4, 0.95, 0.1
+NS_STEPS = 5
+METRIC = "Muon steps/sec and NS TFLOP/s (% of B200 dense BF16 peak) per matrix set"
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return {k: float(p[k]) for k in FALLBACK}, "measured"
+    except Exception:
+        return dict(FALLBACK), "fallback"
+
+
+def kernel_source_hash():
+    h = hashlib.sha256()
+    for rel in ("muon_newton_schulz_03_b200/csrc/ns_tcgen05.cu", "muon_newton_schulz_03_b200/csrc/common.cuh"):
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(workload):
+    """DRAM bytes per launch of the Newton-Schulz kernel from a committed ncu
+    summary, if it was taken on the current kernel source; else None."""
+    path = os.path.join(ROOT, "profiles", f"ns_phase_kernel_{workload}.md")
+    try:
+        text = open(path).read()
+    except OSError:
+        return None
+    vals = {}
+    for line in text.splitlines():
+        line = line.strip().strip("|").strip()
+        if line.startswith("kernel_source_hash:"):
+            vals["hash"] = line.split(":", 1)[1].strip()
+        if line.startswith("traffic_bytes_per_launch:"):
+            vals["traffic"] = float(line.split(":", 1)[1].strip())
+    if vals.get("hash") == kernel_source_hash() and "traffic" in vals:
+        return vals["traffic"]
+    return None
+
+
+class ClockSampler:
+    """nvidia-smi clock/throttle sampling during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *exc):
+        self.out = ""
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.out, _ = self.proc.communicate(timeout=5)
+            except Exception:
+                self.proc.kill()
+                self.out = ""
+
+    def summary(self):
+        rows = []
+        for line in (self.out or "").splitlines():
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                rows.append((float(parts[1]), float(parts[2]), parts[5:9], parts[4]))
+            except ValueError:
+                continue
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"], "samples": 0}
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = set()
+        for r in rows:
+            for nm, v in zip(names, r[2]):
+                if v.lower().startswith("active"):
+                    reasons.add(nm)
+        return {"sm_mhz": statistics.median(r[0] for r in rows), "sm_max_mhz": max(r[1] for r in rows),
+                "reasons": sorted(reasons), "samples": len(rows)}
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle timing (baseline and reference arm)
+# ---------------------------------------------------------------------------
+
+def oracle_sample(workload):
+    """The bounded CPU sample of a workload: matrix indices of the set."""
+    if workload == "llama3":
+        return [0, 1]          # layer 0: q 4096x4096 and k 1024x4096
+    if workload == "moe":
+        return [0, 2]          # expert 0: gate 2048x7168 and down 7168x2048
+    if workload == "gpt2":
+        return [0, 1, 2, 3]    # layer 0
+    return [0]
+
+
+def time_oracle(workload, repeats=1):
+    """Seconds for the oracle on the sample, and the sample's share of the set."""
+    import numpy as np
+    from oracle import muon_oracle as O
+    config, shapes_fn, gdt, _ = WORKLOADS[workload]
+    shapes = shapes_fn()
+    idx = oracle_sample(workload)
+    inputs = []
+    for i in idx:
+        m, n = shapes[i]
+        seed = W.seed_for(config, i // 7, i % 7)
+        g = W.gradient_cpu(config, m, n, seed).astype(np.float32).astype(np.float64)
+        inputs.append((W.param_cpu(m, n, seed), g, np.zeros((m, n))))
+    t0 = time.perf_counter()
+    for _ in range(repeats):
+        for (p, g, m) in inputs:
+            O.muon_step_matrix(p, g, m, lr=LR, beta=BETA, wd=WD, ns_steps=NS_STEPS)
+    dt = (time.perf_counter() - t0) / repeats
+    sample_flops = sum(W.ns_flops(*shapes[i]) for i in idx)
+    share = sample_flops / W.total_ns_flops(shapes)
+    return dt, share, [shapes[i] for i in idx]
+
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        info = threadpool_info()
+        return max((d.get("num_threads") or 0) for d in info) or os.cpu_count()
+    except Exception:
+        return os.cpu_count()
+
+
+def cpu_baseline(workload):
+    dt, share, sample = time_oracle(workload)
+    steps_per_s = share / dt
+    return {"value": steps_per_s, "unit": "steps/s", "cores": blas_threads(), "kind": "oracle",
+            "sample": f"float64 NumPy oracle on {len(sample)} matrices {sample} of the set "
+                      f"({share * 100:.2f}% of its nominal NS FLOPs), {dt:.2f} s, scaled to the whole set by "
+                      f"nominal NS FLOPs"}
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    _, shapes_fn, _, desc = WORKLOADS[args.workload]
+    for _ in range(args.warmup):
+        time_oracle(args.workload)
+    times = []
+    share = None
+    sample = None
+    for _ in range(args.steps):
+        dt, share, sample = time_oracle(args.workload)
+        times.append(dt / share)
+    ms = statistics.mean(times) * 1e3
+    value = 1e3 / ms
+    cores = blas_threads()
+    line = {
+        "metric": METRIC, "value": value, "unit": "steps/s", "n_gpus": args.gpus, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
+        "config": {"workload": desc, "matrices": len(shapes_fn()), "ns_steps": NS_STEPS},
+        "cpu_baseline": {"value": value, "unit": "steps/s", "cores": cores, "kind": "oracle",
+                         "sample": f"each step: the float64 oracle on {sample}, scaled by nominal NS FLOPs "
+                                   f"({share * 100:.2f}% of the set)"},
+        "e2e": {"value": value, "unit": "steps/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ---------------------------------------------------------------------------
+# GPU arm
+# ---------------------------------------------------------------------------
+
+def make_inputs(torch, workload, device, rank):
+    config, shapes_fn, gdt, _ = WORKLOADS[workload]
+    shapes = shapes_fn()
+    gdtype = torch.bfloat16 if gdt == "bf16" else torch.float32
+    params, grads, moms = [], [], []
+    for i, (m, n) in enumerate(shapes):
+        seed = W.seed_for(config, i // 7, i % 7) + 7919 * rank
+        grads.append(W.gradient_gpu(config, m, n, seed, device, gdtype))
+        params.append(W.param_gpu(m, n, seed, device))
+        moms.append(torch.zeros((m, n), dtype=torch.float32, device=device))
+    torch.cuda.synchronize()
+    return shapes, params, grads, moms, gdtype
+
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+    import muon_newton_schulz_03_b200 as muon
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        from datetime import timedelta
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=timedelta(seconds=300), device_id=torch.device("cuda", local))
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    peaks, peak_src = load_peaks()
+
+    shapes, params, grads, moms, gdtype = make_inputs(torch, args.workload, device, rank)
+    count = len(shapes)
+    nominal = W.total_ns_flops(shapes, NS_STEPS)
+    gbytes = 2 if gdtype == torch.bfloat16 else 4
+    k1_bytes = sum(W.step_bytes(m, n, gbytes)[0] for m, n in shapes)
+    k4_bytes = sum(W.step_bytes(m, n, gbytes)[1] for m, n in shapes)
+
+    opt = muon.Muon(device=local)
+    stream = torch.cuda.current_stream()
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    for _ in range(args.warmup):
+        opt.step(params, grads, moms, lr=LR, beta=BETA, wd=WD, ns_steps=NS_STEPS)
+    torch.cuda.synchronize()
+    code, ew, nf = opt.status()
+    if code != 0:
+        raise RuntimeError(f"device status {code} after warm-up (error word {ew}, non-finite {nf})")
+    launches_per_step = opt.last_launch_count()
+
+    opt.profile_enable(args.steps)
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        start.record(stream)
+        for _ in range(args.steps):
+            opt.step(params, grads, moms, lr=LR, beta=BETA, wd=WD, ns_steps=NS_STEPS)
+        end.record(stream)
+        torch.cuda.synchronize()
+    barrier()
+    elapsed_ms = start.elapsed_time(end)
+    prof = opt.profile_read()
+    opt.profile_enable(0)
+    code, ew, nf = opt.status()
+    if code != 0:
+        raise RuntimeError(f"device status {code} after timing (error word {ew}, non-finite {nf})")
+
+    ms_local = elapsed_ms / args.steps
+    if world > 1:
+        t = torch.tensor([ms_local], dtype=torch.float64, device=device)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms_step = float(t.item())
+    else:
+        ms_step = ms_local
+
+    by_kind = {}
+    for kind, ms in prof:
+        by_kind.setdefault(kind, []).append(ms)
+    ns_ms = sum(sum(by_kind.get(k, [])) for k in ("ns_gram", "ns_poly", "ns_comb")) / args.steps
+    ns_launches = sum(len(by_kind.get(k, [])) for k in ("ns_gram", "ns_poly", "ns_comb"))
+    k1_ms = statistics.mean(by_kind["momentum_norm"]) if by_kind.get("momentum_norm") else None
+    k4_ms = statistics.mean(by_kind["apply"]) if by_kind.get("apply") else None
+    ns_tflops = nominal / (ns_ms * 1e-3) / 1e12 if ns_ms > 0 else None
+    avg_ns_launch_ms = ns_ms * args.steps / ns_launches if ns_launches else None
+    per_launch_flops = nominal / (3 * NS_STEPS)
+
+    clocks = clk.summary()
+
+    # e2e: the same step through the host-buffer entry point (params, grads
+    # and momenta in pinned host memory; copies inside the timed region).
+    e2e = None
+    if not args.no_e2e:
+        e2e = run_e2e(torch, muon, opt, shapes, params, grads, moms, args, device, world, dist)
+
+    opt.close()
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(args.workload)
+
+    if rank == 0:
+        value = world * 1e3 / ms_step
+        traffic = profiled_traffic(args.workload)
+        line = {
+            "metric": METRIC,
+            "value": value,
+            "unit": "steps/s",
+            "n_gpus": world,
+            "steps": args.steps,
+            "warmup": args.warmup,
+            "ms_per_step": ms_step,
+            "higher_is_better": True,
+            "scaling": "weak",
+            "vs_baseline": None,
+            "dtype": "bf16",
+            "data": "synthetic",
+            "config": {
+                "workload": WORKLOADS[args.workload][3],
+                "matrices": count,
+                "elements": W.total_elements(shapes),
+                "grad_dtype": "bf16" if gdtype == torch.bfloat16 else "fp32",
+                "param_dtype": "fp32",
+                "ns_steps": NS_STEPS,
+                "lr": LR, "beta": BETA, "nesterov": True, "wd": WD, "scale": "moonlight 0.2*sqrt(max(m,n))",
+                "l2": "inputs larger than L2 (params, momenta, grads resident in HBM, no flush needed)",
+                "parallelism": f"replica per GPU x{world} (weak)",
+            },
+            "ns_tflops_nominal": ns_tflops,
+            "ns_frac_of_datasheet_bf16": (ns_tflops / DATASHEET_BF16_TFLOPS) if ns_tflops else None,
+            "ns_frac_of_measured_bf16": (ns_tflops / peaks["bf16_tflops_sustained"]) if ns_tflops else None,
+            "matrices_per_s": count * value,
+            "ns_ms_per_step": ns_ms,
+            "elementwise": {
+                "momentum_norm_ms": k1_ms, "momentum_norm_gbs": (k1_bytes / (k1_ms * 1e-3) / 1e9) if k1_ms else None,
+                "apply_ms": k4_ms, "apply_gbs": (k4_bytes / (k4_ms * 1e-3) / 1e9) if k4_ms else None,
+                "hbm_peak_gbs": peaks["hbm_gbs"], "peak_source": peak_src,
+            },
+            "roofline": {
+                "kernel": "ns_phase_kernel (tcgen05 Newton-Schulz phases, all matrices per launch)",
+                "bound": "tensor",
+                "achieved": ns_tflops,
+                "peak": peaks["bf16_tflops_sustained"],
+                "unit": "TFLOP/s",
+                "frac": (ns_tflops / peaks["bf16_tflops_sustained"]) if ns_tflops else None,
+                "traffic": traffic,
+                "peak_source": f"{peak_src} sustained dense bf16 (kernel timed inside a long step)",
+                "flops_per_launch_nominal": per_launch_flops,
+                "avg_launch_ms": avg_ns_launch_ms,
+                "flops_definition": "nominal 4 s^2 l + 2 s^3 per matrix per iteration (s = min(m,n), l = max)",
+            },
+            "cpu_baseline": cpu,
+            "e2e": e2e,
+            "gpu_launches": launches_per_step * args.steps,
+            "clocks": clocks,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+    return 0
+
+
+def run_e2e(torch, muon, opt, shapes, params, grads, moms, args, device, world, dist):
+    """Steps/s through muon_step_host with host buffers (copies included)."""
+    def pinned_copy(t):
+        h = torch.empty(t.shape, dtype=t.dtype, pin_memory=True)
+        h.copy_(t)
+        return h
+
+    try:
+        hp = [pinned_copy(p) for p in params]
+        hg = [pinned_copy(g) for g in grads]
+        hm = [pinned_copy(m) for m in moms]
+    except Exception as e:  # pragma: no cover - host memory limits
+        return {"value": None, "unit": "steps/s", "error": f"pinned host buffers unavailable: {e}"}
+    h2d = sum(t.numel() * t.element_size() for t in hp + hg + hm)
+    d2h = sum(t.numel() * t.element_size() for t in hp + hm)
+    # Free the device-resident copies so the staging area fits.
+    del params[:], grads[:], moms[:]
+    torch.cuda.synchronize()
+    torch.cuda.empty_cache()
+    stream = torch.cuda.current_stream()
+    steps = max(1, min(args.steps, args.e2e_steps))
+    opt.step_host(hp, hg, hm, lr=LR, beta=BETA, wd=WD, ns_steps=NS_STEPS)   # warm: staging allocation
+    torch.cuda.synchronize()
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    start.record(stream)
+    for _ in range(steps):
+        opt.step_host(hp, hg, hm, lr=LR, beta=BETA, wd=WD, ns_steps=NS_STEPS)
+    end.record(stream)
+    torch.cuda.synchronize()
+    ms = start.elapsed_time(end) / steps
+    if world > 1:
+        t = torch.tensor([ms], dtype=torch.float64, device=device)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    code, ew, _ = opt.status()
+    if code != 0:
+        return {"value": None, "unit": "steps/s", "error": f"device status {code}"}
+    return {"value": world * 1e3 / ms, "unit": "steps/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+            "ms_per_step": ms, "steps": steps,
+            "path": "muon_step_host: params, grads, momenta in pinned host memory; H2D, step, D2H of params and "
+                    "momenta on one stream"}
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.splitlines()[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--workload", choices=sorted(WORKLOADS), default="llama3")
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--e2e-steps", type=int, default=3)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    args.warmup = max(args.warmup, 3)   # at least three untimed steps
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -235,6 +235,31 @@ int muon_get_status(muon_handle* h, void* stream, int32_t* error_word,
 /* Number of kernels the last muon_step / stage call enqueued. */
 int muon_last_launch_count(muon_handle* h, int32_t* launches);
 
+/* Kernel kinds reported by muon_profile_read. */
+enum muon_kernel_kind {
+  MUON_KERNEL_MOMENTUM_NORM = 0, /* stage 1                                  */
+  MUON_KERNEL_NS_GRAM = 1,       /* tensor-core Gram phase, all matrices      */
+  MUON_KERNEL_NS_POLY = 2,       /* tensor-core polynomial phase              */
+  MUON_KERNEL_NS_COMB = 3,       /* tensor-core combine phase                 */
+  MUON_KERNEL_APPLY = 4,         /* stage 3                                   */
+  MUON_KERNEL_SCALE_COPY = 5,    /* zero-iteration Newton-Schulz stage        */
+  MUON_KERNEL_NS_FP32 = 6        /* fp32 debug phase (one matrix)             */
+};
+
+/* Per-launch timing for measurements. With max_calls > 0, each of the next
+ * max_calls step / stage calls records a CUDA event on its stream before and
+ * after every kernel it enqueues (at most 256 kernels per call); events are
+ * created here, so call this outside stream capture. max_calls = 0 stops
+ * recording and frees the events. Recording adds two event records per
+ * kernel and nothing else. */
+int muon_profile_enable(muon_handle* h, int max_calls);
+
+/* Wait for the recorded events and return, in launch order, the kind
+ * (enum muon_kernel_kind) and duration in milliseconds of up to `max`
+ * recorded kernels; *n receives the number written. Clears the record so
+ * the next calls start from an empty record (max_calls calls again). */
+int muon_profile_read(muon_handle* h, int32_t* kinds, float* ms, int max, int32_t* n);
+
 /* Thread-local text of the last error ("" if none). Never NULL. */
 const char* muon_last_error(void);
 

@@ -277,6 +277,20 @@ class Muon:
         check(self._lib.muon_workspace_ptr(self._h, ctypes.byref(base), ctypes.byref(size)))
         return base.value or 0, size.value
 
+    KERNEL_KINDS = ("momentum_norm", "ns_gram", "ns_poly", "ns_comb", "apply", "scale_copy", "ns_fp32")
+
+    def profile_enable(self, max_calls: int):
+        """Record CUDA events around every kernel of the next max_calls calls."""
+        check(self._lib.muon_profile_enable(self._h, int(max_calls)))
+
+    def profile_read(self, max_entries: int = 65536):
+        """[(kind, ms)] of the recorded kernels, in launch order; clears the record."""
+        kinds = (ctypes.c_int32 * max_entries)()
+        ms = (ctypes.c_float * max_entries)()
+        n = ctypes.c_int32()
+        check(self._lib.muon_profile_read(self._h, kinds, ms, max_entries, ctypes.byref(n)))
+        return [(self.KERNEL_KINDS[kinds[i]], ms[i]) for i in range(n.value)]
+
     def last_launch_count(self) -> int:
         n = ctypes.c_int32()
         check(self._lib.muon_last_launch_count(self._h, ctypes.byref(n)))

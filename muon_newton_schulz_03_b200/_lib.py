@@ -58,6 +58,8 @@ _SIGNATURES = {
     "muon_workspace_ptr": (c_int, [c_void_p, P(c_void_p), P(c_size_t)]),
     "muon_get_status": (c_int, [c_void_p, c_void_p, P(ctypes.c_int32), P(ctypes.c_uint64)]),
     "muon_last_launch_count": (c_int, [c_void_p, P(ctypes.c_int32)]),
+    "muon_profile_enable": (c_int, [c_void_p, c_int]),
+    "muon_profile_read": (c_int, [c_void_p, P(ctypes.c_int32), P(c_float), c_int, P(ctypes.c_int32)]),
     "muon_last_error": (c_char_p, []),
     "muon_version": (c_char_p, []),
 }

@@ -178,6 +178,13 @@ struct muon_handle {
   BlobCache binds;
   BlobCache in_maps;
   int last_launches = 0;
+  // Per-launch timing (muon_profile_enable / muon_profile_read).
+  std::vector<cudaEvent_t> prof_ev;   // 2 per slot
+  std::vector<int> prof_kind;         // per slot
+  int prof_slots = 0;                 // capacity in kernels
+  int prof_used = 0;                  // kernels recorded so far
+  int prof_calls_left = 0;            // calls that still record
+  bool prof_this_call = false;
 };
 
 namespace {
@@ -190,6 +197,35 @@ void free_plan(DevPlan* p) {
 }
 
 int64_t align_up(int64_t x, int64_t a) { return (x + a - 1) / a * a; }
+
+constexpr int kProfMaxPerCall = 256;
+
+// Marks the start of a call for the profiler.
+void prof_call_begin(muon_handle* h) {
+  h->prof_this_call = h->prof_calls_left > 0;
+  if (h->prof_this_call) --h->prof_calls_left;
+}
+
+// Records the event before a kernel; returns the slot or -1.
+int prof_before(muon_handle* h, int kind, cudaStream_t st) {
+  if (!h->prof_this_call || h->prof_used >= h->prof_slots) return -1;
+  const int slot = h->prof_used++;
+  h->prof_kind[slot] = kind;
+  cudaEventRecord(h->prof_ev[2 * slot], st);
+  return slot;
+}
+
+void prof_after(muon_handle* h, int slot, cudaStream_t st) {
+  if (slot >= 0) cudaEventRecord(h->prof_ev[2 * slot + 1], st);
+}
+
+void prof_free(muon_handle* h) {
+  for (cudaEvent_t e : h->prof_ev) cudaEventDestroy(e);
+  h->prof_ev.clear();
+  h->prof_kind.clear();
+  h->prof_slots = h->prof_used = h->prof_calls_left = 0;
+  h->prof_this_call = false;
+}
 
 // Builds (or reuses) the plan, workspace, device tables and tensor maps for
 // this shape table.
@@ -364,7 +400,9 @@ int enqueue_ns(muon_handle* h, const MatBind* d_binds, const std::vector<MatBind
       for (int ph = 0; ph < 3; ++ph) {
         L.tiles = P.d_tiles[ph];
         L.ntiles = (int)hp.tiles[ph].size();
+        const int slot = prof_before(h, MUON_KERNEL_NS_GRAM + ph, st);
         MUON_CUDA_TRY(launch_ns_phase_bf16(L, ph, src, dst, first, abc[0], abc[1], abc[2], st));
+        prof_after(h, slot, st);
         ++*launches;
       }
     } else {
@@ -373,9 +411,11 @@ int enqueue_ns(muon_handle* h, const MatBind* d_binds, const std::vector<MatBind
         const MatPlan& mp = P.mats[i];
         const float* s_ptr = static_cast<const float*>(sel_buf(mp, hbinds[i], src));
         float* d_ptr = static_cast<float*>(const_cast<void*>(sel_buf(mp, hbinds[i], dst)));
-        MUON_CUDA_TRY(launch_ns_phase_fp32(mp, i, PHASE_GRAM, s_ptr, d_ptr, sumsq, first, abc[0], abc[1], abc[2], st));
-        MUON_CUDA_TRY(launch_ns_phase_fp32(mp, i, PHASE_POLY, s_ptr, d_ptr, sumsq, first, abc[0], abc[1], abc[2], st));
-        MUON_CUDA_TRY(launch_ns_phase_fp32(mp, i, PHASE_COMB, s_ptr, d_ptr, sumsq, first, abc[0], abc[1], abc[2], st));
+        for (int ph = PHASE_GRAM; ph <= PHASE_COMB; ++ph) {
+          const int slot = prof_before(h, MUON_KERNEL_NS_FP32, st);
+          MUON_CUDA_TRY(launch_ns_phase_fp32(mp, i, ph, s_ptr, d_ptr, sumsq, first, abc[0], abc[1], abc[2], st));
+          prof_after(h, slot, st);
+        }
         *launches += 3;
       }
     }
@@ -434,13 +474,18 @@ int step_impl(muon_handle* h, float* const* params, const void* const* grads, fl
   int launches = 0;
   MUON_CUDA_TRY(cudaMemsetAsync(sumsq, 0, sizeof(double) * count, st));
   const ElemLaunch EL = elem_launch(P, db);
+  prof_call_begin(h);
+  int slot = prof_before(h, MUON_KERNEL_MOMENTUM_NORM, st);
   MUON_CUDA_TRY(launch_momentum_norm(EL, BUF_X0, beta, nesterov ? 1 : 0, sumsq, h->status, h->cfg.check_nonfinite,
                                      fp32, st));
+  prof_after(h, slot, st);
   ++launches;
   int res = BUF_X0;
   if ((rc = enqueue_ns(h, db, hb, nullptr, sumsq, ns_steps, abc, BUF_X0, -1, st, &launches, &res))) return rc;
+  slot = prof_before(h, MUON_KERNEL_APPLY, st);
   MUON_CUDA_TRY(launch_apply(EL, res, lr, wd, h->cfg.scale_mode, h->cfg.extra_scale, ns_steps == 0 ? sumsq : nullptr,
                              fp32, st));
+  prof_after(h, slot, st);
   ++launches;
   h->last_launches = launches;
   return MUON_OK;
@@ -512,6 +557,7 @@ int muon_destroy(muon_handle* h) {
     h->binds.clear();
     h->in_maps.clear();
     if (h->plan) free_plan(h->plan.get());
+    prof_free(h);
     cudaFree(h->status);
   }
   delete h;
@@ -626,9 +672,12 @@ int muon_momentum_norm(muon_handle* h, const void* const* grads, float* const* m
   if ((rc = h->binds.get(hb.data(), sizeof(MatBind) * count, &d_binds))) return rc;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   MUON_CUDA_TRY(cudaMemsetAsync(sumsq, 0, sizeof(double) * count, st));
+  prof_call_begin(h);
+  const int slot = prof_before(h, MUON_KERNEL_MOMENTUM_NORM, st);
   MUON_CUDA_TRY(launch_momentum_norm(elem_launch(P, static_cast<const MatBind*>(d_binds)), BUF_OUT, beta,
                                      nesterov ? 1 : 0, sumsq, h->status, h->cfg.check_nonfinite,
                                      h->cfg.ns_precision == MUON_NS_FP32, st));
+  prof_after(h, slot, st);
   h->last_launches = 1;
   return MUON_OK;
 }
@@ -664,8 +713,11 @@ int muon_newton_schulz(muon_handle* h, const void* const* x_in, void* const* x_o
   const MatBind* db = static_cast<const MatBind*>(d_binds);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   int launches = 0;
+  prof_call_begin(h);
   if (ns_steps == 0) {
+    const int slot = prof_before(h, MUON_KERNEL_SCALE_COPY, st);
     MUON_CUDA_TRY(launch_scale_copy(elem_launch(P, db), BUF_IN, BUF_OUT, sumsq, esz == 4, st));
+    prof_after(h, slot, st);
     h->last_launches = 1;
     return MUON_OK;
   }
@@ -709,8 +761,11 @@ int muon_apply(muon_handle* h, float* const* params, const void* const* o, const
   void* d_binds = nullptr;
   if ((rc = h->binds.get(hb.data(), sizeof(MatBind) * count, &d_binds))) return rc;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
+  prof_call_begin(h);
+  const int slot = prof_before(h, MUON_KERNEL_APPLY, st);
   MUON_CUDA_TRY(launch_apply(elem_launch(P, static_cast<const MatBind*>(d_binds)), BUF_IN, lr, wd,
                              h->cfg.scale_mode, h->cfg.extra_scale, sumsq, h->cfg.ns_precision == MUON_NS_FP32, st));
+  prof_after(h, slot, st);
   h->last_launches = 1;
   return MUON_OK;
 }
@@ -770,6 +825,49 @@ int muon_get_status(muon_handle* h, void* stream, int32_t* error_word, uint64_t*
   if (nonfinite_count) *nonfinite_count = s.nonfinite;
   if (s.error_word) return fail(MUON_ERR_TIMEOUT, "a device-side wait expired (code " + std::to_string(s.error_word) + ")");
   if (s.nonfinite) return fail(MUON_ERR_NONFINITE, std::to_string(s.nonfinite) + " non-finite update entries");
+  return MUON_OK;
+}
+
+int muon_profile_enable(muon_handle* h, int max_calls) {
+  g_last_error.clear();
+  if (!h) return fail(MUON_ERR_INVALID_ARG, "handle is NULL");
+  if (max_calls < 0 || max_calls > 4096) return fail(MUON_ERR_INVALID_ARG, "max_calls must be in [0, 4096]");
+  DeviceGuard g(h->device);
+  MUON_CUDA_TRY(cudaDeviceSynchronize());
+  prof_free(h);
+  if (max_calls == 0) return MUON_OK;
+  const int slots = max_calls * kProfMaxPerCall;
+  h->prof_ev.assign((size_t)slots * 2, nullptr);
+  h->prof_kind.assign((size_t)slots, 0);
+  for (auto& e : h->prof_ev) {
+    cudaError_t err = cudaEventCreate(&e);
+    if (err != cudaSuccess) {
+      e = nullptr;
+      prof_free(h);
+      return fail(MUON_ERR_CUDA, std::string("cudaEventCreate: ") + cudaGetErrorString(err));
+    }
+  }
+  h->prof_slots = slots;
+  h->prof_calls_left = max_calls;
+  return MUON_OK;
+}
+
+int muon_profile_read(muon_handle* h, int32_t* kinds, float* ms, int max, int32_t* n) {
+  g_last_error.clear();
+  if (!h || !n) return fail(MUON_ERR_INVALID_ARG, "handle and n are required");
+  DeviceGuard g(h->device);
+  const int used = std::min(h->prof_used, std::max(max, 0));
+  for (int k = 0; k < used; ++k) {
+    MUON_CUDA_TRY(cudaEventSynchronize(h->prof_ev[2 * k + 1]));
+    float t = 0.0f;
+    MUON_CUDA_TRY(cudaEventElapsedTime(&t, h->prof_ev[2 * k], h->prof_ev[2 * k + 1]));
+    if (kinds) kinds[k] = h->prof_kind[k];
+    if (ms) ms[k] = t;
+  }
+  *n = used;
+  const int calls = h->prof_slots / kProfMaxPerCall;
+  h->prof_used = 0;
+  h->prof_calls_left = calls;
   return MUON_OK;
 }
 

@@ -76,7 +76,11 @@ def test_momentum_norm_matches_oracle(opt_bf16, grad_dtype, nesterov):
         assert abs(np.sqrt(ss[i]) - nu_ref) <= TOL_ELEM * nu_ref
         y = to64(ys[i][:, :n])
         y_ref = O.bf16_round(u_ref)
-        assert np.all(np.abs(y - y_ref) <= bf16_ulp(y_ref)), f"matrix {i}: cast off by more than one bf16 ulp"
+        # One bf16 ulp, plus the float32 rounding of the lerp chain that
+        # produces u on the GPU (it matters where u nearly cancels).
+        fp32_err = 8 * 2.0 ** -24 * (np.abs(gs[i]) + np.abs(m_ref) + np.abs(ms[i]))
+        bad = np.abs(y - y_ref) > bf16_ulp(y_ref) + fp32_err
+        assert not bad.any(), f"matrix {i}: {bad.sum()} casts off by more than one bf16 ulp"
 
 
 def test_momentum_norm_fp32_output(opt_fp32):
