@@ -370,3 +370,19 @@ def test_emulated_bf16_close_to_exact():
     emu = O.newton_schulz(G, emulate_bf16=True)
     rel = np.linalg.norm(emu - exact) / np.linalg.norm(exact)
     assert 1e-5 < rel < 2e-2
+
+
+@pytest.mark.parametrize("shape", [(6, 10), (10, 6), (9, 9)])
+@pytest.mark.parametrize("steps", [0, 1, 5])
+def test_bf16_mode_is_exact_mode_plus_rounding(monkeypatch, shape, steps):
+    # The bf16-rounding mode differs from the exact mode only by the rounding
+    # it inserts (and by applying 1/(||G||+eps) inside the first Gram and
+    # combine, which is the same product). With rounding made the identity,
+    # both modes agree to float64 accuracy.
+    rng = np.random.default_rng(18)
+    G = rng.standard_normal(shape)
+    monkeypatch.setattr(O, "bf16_round", lambda v: np.asarray(v, dtype=np.float64))
+    a = O.newton_schulz(G, steps, emulate_bf16=True)
+    monkeypatch.undo()
+    b = O.newton_schulz(G, steps)
+    assert np.max(np.abs(a - b)) < 1e-12
