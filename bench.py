@@ -44,6 +44,8 @@ FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1
 WORKLOADS = {
     "llama3": (W.CONFIG_LLAMA, W.llama3_8b_shapes, "bf16", "Llama-3-8B hidden matrices: 32 x {q 4096x4096, "
                "k 1024x4096, v 1024x4096, o 4096x4096, gate 14336x4096, up 14336x4096, down 4096x14336}"),
+    "llama3_layer": (W.CONFIG_LLAMA, W.llama3_layer_shapes, "bf16", "one Llama-3-8B layer: {q 4096x4096, "
+                     "k 1024x4096, v 1024x4096, o 4096x4096, gate 14336x4096, up 14336x4096, down 4096x14336}"),
     "gpt2": (W.CONFIG_GPT2, W.gpt2_shapes, "fp32", "GPT-2-small hidden matrices: 12 x {QKV 2304x768, "
              "O 768x768, up 3072x768, down 768x3072}"),
     "moe": (W.CONFIG_MOE, W.moe_shapes, "bf16", "MoE layer: 128 experts x {gate 2048x7168, up 2048x7168, "
@@ -152,7 +154,7 @@ class ClockSampler:
 
 def oracle_sample(workload):
     """The bounded CPU sample of a workload: matrix indices of the set."""
-    if workload == "llama3":
+    if workload in ("llama3", "llama3_layer"):
         return [0, 1]          # layer 0: q 4096x4096 and k 1024x4096
     if workload == "moe":
         return [0, 2]          # expert 0: gate 2048x7168 and down 7168x2048

@@ -60,6 +60,11 @@ def llama3_8b_shapes():
     return out
 
 
+def llama3_layer_shapes():
+    """One layer of the Llama-3-8B set (7 matrices): the small profiling case."""
+    return llama3_8b_shapes()[:7]
+
+
 def moe_shapes(experts: int = 128):
     out = []
     for _ in range(experts):
