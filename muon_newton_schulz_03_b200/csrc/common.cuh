@@ -132,19 +132,19 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 // Wait for the phase with the given parity to complete. Gives up when the
 // shared error word is set by anyone, or after `timeout_ns` nanoseconds, in
 // which case it records `code` in the error word. Returns false on give-up.
+// (try_wait itself suspends the thread for a short, hardware-defined time
+// while the phase is incomplete, so the loop does not spin hot.)
 __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity, int* err,
                                                   uint64_t timeout_ns, int code) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = global_timer_ns();
   for (uint32_t it = 1;; ++it) {
     if (mbar_try_wait(bar, parity)) return true;
-    if ((it & 31u) == 0u) {
-      if (*reinterpret_cast<volatile int*>(err) != 0) return false;
-      if (global_timer_ns() - t0 > timeout_ns) {
-        atomicCAS(err, 0, code);
-        return false;
-      }
+    if (global_timer_ns() - t0 > timeout_ns) {
+      atomicCAS(err, 0, code);
+      return false;
     }
+    if ((it & 7u) == 0u && *reinterpret_cast<volatile int*>(err) != 0) return false;
   }
 }
 

@@ -12,7 +12,7 @@ DEV = torch.device("cuda:0")
 TOL_BF16_NS = 2e-2      # bf16 Newton-Schulz vs the float64 oracle
 TOL_FP32_NS = 1e-4      # fp32 debug Newton-Schulz vs the float64 oracle
 TOL_ELEM = 1e-6         # elementwise stages vs the float64 oracle
-TOL_BF16_EMU = 5e-3     # bf16 Newton-Schulz vs the oracle's bf16-rounding mode
+TOL_BF16_EMU = 1e-2     # bf16 Newton-Schulz vs the oracle's bf16-rounding mode
 
 
 def bf16_gate(got, exact, emulated, what=""):
@@ -20,18 +20,22 @@ def bf16_gate(got, exact, emulated, what=""):
 
     1. Against the oracle run at the pages' precision (bf16 rounding of the
        input and of every Gram / polynomial / combine output): within
-       TOL_BF16_EMU.
+       TOL_BF16_EMU. Two bf16 realizations that differ only in fp32
+       summation order (GPU) vs float64 summation (oracle) drift apart
+       through the iteration by a few 1e-3; half the gate bounds that.
     2. Against the exact float64 oracle: within TOL_BF16_NS wherever bf16
        arithmetic itself can meet that (the bf16-rounding oracle is within
-       it); otherwise no further than the bf16-rounding oracle's own
-       distance plus TOL_BF16_EMU.
+       it); otherwise no further than 1.25 times the bf16-rounding oracle's
+       own distance (inputs whose spectrum reaches below the bf16 floor,
+       tiny matrices whose few singular values land near the repelling
+       fixed points).
     Returns (err_vs_exact, err_vs_emulated, err_of_emulation).
     """
     e_emu = rel(got, emulated)
     e_exact = rel(got, exact)
     e_inherent = rel(emulated, exact)
     assert e_emu <= TOL_BF16_EMU, f"{what}: {e_emu:.3e} from the bf16-rounding oracle"
-    bound = TOL_BF16_NS if e_inherent <= TOL_BF16_NS else e_inherent + TOL_BF16_EMU
+    bound = TOL_BF16_NS if e_inherent <= TOL_BF16_NS else 1.25 * e_inherent
     assert e_exact <= bound, (f"{what}: {e_exact:.3e} from the exact oracle "
                               f"(bf16 arithmetic alone: {e_inherent:.3e})")
     return e_exact, e_emu, e_inherent
