@@ -266,6 +266,47 @@ const char* muon_last_error(void);
 /* Library version string. */
 const char* muon_version(void);
 
+/* ---- Allocation-free Newton-Schulz stage ----
+ *
+ * The pages have no counterpart to this entry point; it exists for callers
+ * that cannot allocate device memory when they run the stage: a stream being
+ * captured in global capture mode (allocation calls are refused then), a
+ * process whose device memory belongs to its own fixed-budget pool, or a
+ * latency-critical path that cannot take the implicit synchronisation an
+ * allocation may bring.
+ *
+ * Same computation and the same tensor-core kernels as muon_newton_schulz,
+ * in bf16, on the CURRENT device, with no handle. All scratch (X ping-pong
+ * buffers, Gram and polynomial matrices, tile lists, tensor maps, status
+ * word) lives in one static device array of MUON_NOALLOC_SCRATCH_BYTES that
+ * every GPU which loads this library holds until the process exits. The call
+ * allocates nothing: no cudaMalloc, no cudaFree, no allocating library call.
+ *
+ *   x_in, x_out : host arrays of `count` device pointers in X layout (bf16),
+ *                 owned by the caller; x_in is read only; they must not
+ *                 overlap.
+ *   sumsq       : device array of count doubles or NULL (as in
+ *                 muon_newton_schulz).
+ *   shapes, count, ns_steps (0..64), coeffs (NULL = default): as in
+ *                 muon_newton_schulz.
+ *   error_word  : device int32 or NULL; receives 0, or the code of a
+ *                 device-side wait that ran out (results then invalid).
+ *   stream      : cudaStream_t.
+ * A shape table whose scratch (tables plus the workspace muon_plan_query
+ * reports) exceeds MUON_NOALLOC_SCRATCH_BYTES is rejected with
+ * MUON_ERR_INVALID_ARG and a message giving both sizes.
+ * The first call on a device looks up the array's device address there
+ * (cudaGetSymbolAddress) and the device's properties; make that first call
+ * before any stream capture. Every call reuses the same array and leaves the
+ * previous call's contents in it (the status word is cleared at the start
+ * of each call, the tables are rewritten): calls whose work overlaps on the
+ * GPU (different streams, different host threads) race on it; calls on one
+ * stream are ordered. */
+#define MUON_NOALLOC_SCRATCH_BYTES (64u * 1024u * 1024u)
+int muon_newton_schulz_noalloc(const void* const* x_in, void* const* x_out, const double* sumsq,
+                               const int32_t* shapes, int count, int ns_steps, const float* coeffs,
+                               int32_t* error_word, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -60,6 +60,8 @@ _SIGNATURES = {
     "muon_last_launch_count": (c_int, [c_void_p, P(ctypes.c_int32)]),
     "muon_profile_enable": (c_int, [c_void_p, c_int]),
     "muon_profile_read": (c_int, [c_void_p, P(ctypes.c_int32), P(c_float), c_int, P(ctypes.c_int32)]),
+    "muon_newton_schulz_noalloc": (c_int, [P(c_void_p), P(c_void_p), c_void_p, P(ctypes.c_int32), c_int, c_int,
+                                           P(c_float), c_void_p, c_void_p]),
     "muon_last_error": (c_char_p, []),
     "muon_version": (c_char_p, []),
 }

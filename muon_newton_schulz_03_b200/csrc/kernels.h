@@ -2,6 +2,7 @@
 #pragma once
 
 #include <cstdint>
+#include <string>
 #include <cuda_runtime.h>
 
 #include "common.cuh"
@@ -66,5 +67,8 @@ cudaError_t launch_ns_phase_fp32(const MatPlan& mp_host, int mat, int phase, con
                                  const double* sumsq, int first, float a, float b, float c, cudaStream_t st);
 
 int ns_bf16_smem_bytes();
+
+// Sets the calling thread's muon_last_error text.
+void record_last_error(const std::string& msg);
 
 }  // namespace muon

@@ -149,6 +149,10 @@ int encode_x_triple(TmapBlob* out3, const void* base, const MatPlan& mp) {
 
 }  // namespace
 
+namespace muon {
+void record_last_error(const std::string& msg) { g_last_error = msg; }
+}  // namespace muon
+
 // ---------------------------------------------------------------------------
 // Handle
 // ---------------------------------------------------------------------------
