@@ -238,6 +238,15 @@ def run_reference(args):
 # GPU arm
 # ---------------------------------------------------------------------------
 
+def max_over_ranks(torch, dist, value, device):
+    """Largest value over all ranks (timing is reported as the slowest rank)."""
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(value)
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
 def make_inputs(torch, workload, device, rank):
     config, shapes_fn, gdt, _ = WORKLOADS[workload]
     shapes = shapes_fn()
@@ -309,13 +318,7 @@ def run_ours(args):
     if code != 0:
         raise RuntimeError(f"device status {code} after timing (error word {ew}, non-finite {nf})")
 
-    ms_local = elapsed_ms / args.steps
-    if world > 1:
-        t = torch.tensor([ms_local], dtype=torch.float64, device=device)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms_step = float(t.item())
-    else:
-        ms_step = ms_local
+    ms_step = max_over_ranks(torch, dist, elapsed_ms / args.steps, device)
 
     by_kind = {}
     for kind, ms in prof:
@@ -435,11 +438,7 @@ def run_e2e(torch, muon, opt, shapes, params, grads, moms, args, device, world, 
         opt.step_host(hp, hg, hm, lr=LR, beta=BETA, wd=WD, ns_steps=NS_STEPS)
     end.record(stream)
     torch.cuda.synchronize()
-    ms = start.elapsed_time(end) / steps
-    if world > 1:
-        t = torch.tensor([ms], dtype=torch.float64, device=device)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(torch, dist, start.elapsed_time(end) / steps, device)
     code, ew, _ = opt.status()
     if code != 0:
         return {"value": None, "unit": "steps/s", "error": f"device status {code}"}
@@ -449,18 +448,77 @@ def run_e2e(torch, muon, opt, shapes, params, grads, moms, args, device, world, 
                     "momenta on one stream"}
 
 
+def run_sweep(args):
+    """NS-only sweep: bf16 X with log-uniform singular values in [1e-4, 1],
+    five steps, every (m, n, batch) point of the sweep; one JSON line whose
+    `sweep` list holds nominal NS TFLOP/s per point."""
+    import torch
+    import muon_newton_schulz_03_b200 as muon
+    device = torch.device("cuda", int(os.environ.get("LOCAL_RANK", "0")))
+    torch.cuda.set_device(device)
+    peaks, peak_src = load_peaks()
+    batches = set(int(b) for b in args.sweep_batches.split(","))
+    opt = muon.Muon(device=device.index)
+    points = []
+    for (m, n, batch) in W.sweep_points():
+        if batch not in batches:
+            continue
+        base = W.gradient_gpu(W.CONFIG_SWEEP, m, n, W.seed_for(W.CONFIG_SWEEP, m, n), device, torch.bfloat16)
+        ld = muon.round_up(n, 8)
+        xin = []
+        for b in range(batch):
+            buf = torch.zeros((m, ld), dtype=torch.bfloat16, device=device)
+            buf[:, :n] = base if b % 2 == 0 else -base
+            xin.append(buf)
+        del base
+        xout = [torch.empty((m, ld), dtype=torch.bfloat16, device=device) for _ in range(batch)]
+        shapes = [(m, n)] * batch
+        opt.newton_schulz(xin, xout, shapes, None, ns_steps=NS_STEPS)        # plan, workspace, maps
+        torch.cuda.synchronize()
+        reps = 3
+        start = torch.cuda.Event(enable_timing=True)
+        end = torch.cuda.Event(enable_timing=True)
+        start.record()
+        for _ in range(reps):
+            opt.newton_schulz(xin, xout, shapes, None, ns_steps=NS_STEPS)
+        end.record()
+        torch.cuda.synchronize()
+        ms = start.elapsed_time(end) / reps
+        flops = batch * W.ns_flops(m, n, NS_STEPS)
+        tf = flops / (ms * 1e-3) / 1e12
+        points.append({"m": m, "n": n, "batch": batch, "ms": ms, "tflops_nominal": tf,
+                       "frac_datasheet": tf / DATASHEET_BF16_TFLOPS, "frac_measured": tf / peaks["bf16_tflops"]})
+        del xin, xout
+        torch.cuda.empty_cache()
+    code, ew, _ = opt.status()
+    opt.close()
+    if code != 0:
+        raise RuntimeError(f"device status {code} (error word {ew})")
+    vals = sorted(p["tflops_nominal"] for p in points)
+    line = {"metric": "NS-only TFLOP/s (nominal 5 (4 s^2 l + 2 s^3)) per sweep point", "value": vals[len(vals) // 2],
+            "unit": "TFLOP/s (median over points)", "n_gpus": 1, "higher_is_better": True, "dtype": "bf16",
+            "data": "synthetic", "config": {"workload": W.describe(W.CONFIG_SWEEP), "ns_steps": NS_STEPS,
+                                            "batches": sorted(batches), "peak_source": peak_src},
+            "sweep": points}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__.splitlines()[0])
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=10)
     ap.add_argument("--warmup", type=int, default=3)
-    ap.add_argument("--workload", choices=sorted(WORKLOADS), default="llama3")
+    ap.add_argument("--workload", choices=sorted(WORKLOADS) + ["sweep"], default="llama3")
+    ap.add_argument("--sweep-batches", default="1,4,16,64,256")
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args(argv)
     args.warmup = max(args.warmup, 3)   # at least three untimed steps
+    if args.workload == "sweep":
+        return run_sweep(args)
     if args.impl == "reference":
         return run_reference(args)
     return run_ours(args)

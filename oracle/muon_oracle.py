@@ -166,18 +166,21 @@ def newton_schulz(G, steps=5, coeffs=DEFAULT_COEFFS, eps=EPS,
     return X.T if transposed else X
 
 
-def ns_only(X, steps=5, coeffs=DEFAULT_COEFFS):
+def ns_only(X, steps=5, coeffs=DEFAULT_COEFFS, emulate_bf16=False):
     """The Newton-Schulz phases alone on an already-scaled X (no norm).
 
     Used for the NS-only sweep workload, whose inputs are generated with
     singular values already in [1e-4, 1]. Same orientation rule as
-    ``newton_schulz``.
+    ``newton_schulz``; with ``emulate_bf16`` the input and every Gram,
+    polynomial and combine output are rounded to bf16.
     """
     X = np.asarray(X, dtype=np.float64)
+    if emulate_bf16:
+        X = bf16_round(X)
     transposed = X.shape[0] > X.shape[1]
     if transposed:
         X = X.T
-    X = _ns_iterations(X, steps, coeffs, False)
+    X = _ns_iterations(X, steps, coeffs, emulate_bf16)
     return X.T if transposed else X
 
 

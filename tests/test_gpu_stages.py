@@ -186,24 +186,10 @@ def test_ns_single_step_phases(opt_bf16, coeffs):
     torch.cuda.synchronize()
     for i, (m, n) in enumerate(shapes):
         ref = O.ns_only(x64[i], 1, coeffs)
-        emu = _emulated_ns_only(x64[i], 1, coeffs)
+        emu = O.ns_only(x64[i], 1, coeffs, emulate_bf16=True)
         got = to64(xout[i][:, :n])
         bf16_gate(got, ref, emu, f"matrix {i} {m}x{n}")
     _assert_status_clean(opt_bf16)
-
-
-def _emulated_ns_only(X, steps, coeffs):
-    """Oracle NS with bf16 rounding at the GPU's rounding points, alpha = 1."""
-    X = np.asarray(X, dtype=np.float64)
-    t = X.shape[0] > X.shape[1]
-    if t:
-        X = X.T
-    a, b, c = coeffs
-    for _ in range(steps):
-        A = O.bf16_round(X @ X.T)
-        B = O.bf16_round(b * A + c * (A @ A))
-        X = O.bf16_round(a * X + B @ X)
-    return X.T if t else X
 
 
 @pytest.mark.parametrize("steps", [1, 2, 5])
@@ -272,3 +258,30 @@ def test_ns_gram_is_symmetric_in_workspace(opt_bf16):
         X = x64[i] if m <= n else x64[i].T
         ref = X @ X.T
         assert rel(A, ref) <= 4e-3
+
+
+SWEEP_POINTS = [(128, 128, 4), (128, 512, 2), (512, 128, 2), (256, 256, 3), (256, 2048, 1), (2048, 256, 1),
+                (1024, 1024, 1), (512, 4096, 1)]
+
+
+@pytest.mark.parametrize("point", SWEEP_POINTS, ids=lambda p: f"{p[0]}x{p[1]}x{p[2]}")
+def test_ns_only_sweep_inputs(opt_bf16, point):
+    # NS-only workload: bf16 X with log-uniform singular values in [1e-4, 1],
+    # no normalisation; five steps.
+    import workloads as W
+    m, n, batch = point
+    shapes = [(m, n)] * batch
+    xin, x64 = [], []
+    for b in range(batch):
+        x = W.gradient_cpu(W.CONFIG_SWEEP, m, n, W.seed_for(W.CONFIG_SWEEP, m // 128, n // 128, b))
+        buf = x_buffer(m, n, fill=x)
+        xin.append(buf)
+        x64.append(to64(buf[:, :n]))
+    xout = [x_buffer(m, n) for _ in shapes]
+    opt_bf16.newton_schulz(xin, xout, shapes, None, ns_steps=5)
+    torch.cuda.synchronize()
+    for b in range(batch):
+        ref = O.ns_only(x64[b], 5)
+        emu = O.ns_only(x64[b], 5, emulate_bf16=True)
+        bf16_gate(to64(xout[b][:, :n]), ref, emu, f"{m}x{n} #{b}")
+    _assert_status_clean(opt_bf16)

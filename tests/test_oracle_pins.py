@@ -386,3 +386,12 @@ def test_bf16_mode_is_exact_mode_plus_rounding(monkeypatch, shape, steps):
     monkeypatch.undo()
     b = O.newton_schulz(G, steps)
     assert np.max(np.abs(a - b)) < 1e-12
+
+
+def test_ns_only_bf16_mode_structure(monkeypatch):
+    rng = np.random.default_rng(19)
+    X = rng.standard_normal((7, 12)) * 0.1
+    monkeypatch.setattr(O, "bf16_round", lambda v: np.asarray(v, dtype=np.float64))
+    a = O.ns_only(X, 5, emulate_bf16=True)
+    monkeypatch.undo()
+    assert np.max(np.abs(a - O.ns_only(X, 5))) < 1e-13
