@@ -107,6 +107,10 @@ typedef struct muon_config {
   double wait_timeout_s;      /* limit of every device-side wait; a wait
                                  that runs out sets the error word and the
                                  kernel returns. Default 2.0 seconds       */
+  int small_path;             /* 1: matrices with min(m,n) <= 128 and
+                                 max(m,n) <= 512 run all iterations in one
+                                 on-chip kernel (one CTA each); 0: every
+                                 matrix uses the tiled phases. Default 1   */
 } muon_config;
 
 typedef struct muon_handle muon_handle;
@@ -202,18 +206,19 @@ int muon_apply(muon_handle* h, float* const* params, const void* const* o,
 /* ---- Plan, workspace and status ---- */
 
 /* Integer plan tables for a shape table, computed on the host (needs no
- * GPU). Any output pointer may be NULL.
+ * GPU). small_path as in muon_config. Any output pointer may be NULL.
  *   ws_bytes      : total workspace bytes for `ns_precision`.
  *   region_offsets: int64[count][4], byte offsets of X0, X1, A, B.
- *   ntiles        : int32[3], tile counts of the Gram, polynomial and
- *                   combine phases.
- *   tiles         : int32[ntiles[0]+ntiles[1]+ntiles[2]][3] =
+ *   ntiles        : int32[4], tile counts of the Gram, polynomial and
+ *                   combine phases, and the number of small-path matrices.
+ *   tiles         : int32[ntiles[0]+...+ntiles[3]][3] =
  *                   {matrix, row tile, column tile} for the three phases,
- *                   one after the other.
+ *                   one after the other, then {matrix, 0, 0} for each
+ *                   small-path matrix.
  *   chunk_prefix  : int64[count+1], elementwise chunks before matrix i.
  * Call once with tiles = NULL to learn ntiles. */
 int muon_plan_query(const int32_t* shapes, int count, int ns_precision,
-                    int64_t* ws_bytes, int64_t* region_offsets,
+                    int small_path, int64_t* ws_bytes, int64_t* region_offsets,
                     int32_t* ntiles, int32_t* tiles, int64_t* chunk_prefix);
 
 /* Workspace bytes the handle would allocate for this shape table
@@ -243,7 +248,8 @@ enum muon_kernel_kind {
   MUON_KERNEL_NS_COMB = 3,       /* tensor-core combine phase                 */
   MUON_KERNEL_APPLY = 4,         /* stage 3                                   */
   MUON_KERNEL_SCALE_COPY = 5,    /* zero-iteration Newton-Schulz stage        */
-  MUON_KERNEL_NS_FP32 = 6        /* fp32 debug phase (one matrix)             */
+  MUON_KERNEL_NS_FP32 = 6,       /* fp32 debug phase (one matrix)             */
+  MUON_KERNEL_NS_SMALL = 7       /* on-chip small-matrix path, all iterations */
 };
 
 /* Per-launch timing for measurements. With max_calls > 0, each of the next

@@ -86,30 +86,34 @@ def x_layout(m: int, n: int, dtype, device):
     return torch.empty((m, round_up(n, 8)), dtype=dtype, device=device)
 
 
-def plan_query(shapes, ns_precision: str = "bf16"):
+def plan_query(shapes, ns_precision: str = "bf16", small_path: bool = True):
     """Integer plan tables of a shape table (list of (m, n) or (m, n, flags)).
 
     Returns dict(ws_bytes, region_offsets [count][4], tiles (gram, poly,
-    comb lists of (mat, ti, tj)), chunk_prefix). Needs no GPU.
+    comb lists of (mat, ti, tj)), small (list of small-path matrices),
+    chunk_prefix). Needs no GPU.
     """
     lib = load()
     sh = [(int(s[0]), int(s[1]), int(s[2]) if len(s) > 2 else 0) for s in shapes]
     count = len(sh)
     arr = _shapes_array(sh)
     prec = PRECISIONS[ns_precision]
-    nt = (ctypes.c_int32 * 3)()
+    sp = int(bool(small_path))
+    nt = (ctypes.c_int32 * 4)()
     ws = ctypes.c_int64()
-    check(lib.muon_plan_query(arr, count, prec, ctypes.byref(ws), None, nt, None, None))
-    total = nt[0] + nt[1] + nt[2]
+    check(lib.muon_plan_query(arr, count, prec, sp, ctypes.byref(ws), None, nt, None, None))
+    total = nt[0] + nt[1] + nt[2] + nt[3]
     offs = (ctypes.c_int64 * (4 * count))()
     tiles = (ctypes.c_int32 * (3 * max(total, 1)))()
     pref = (ctypes.c_int64 * (count + 1))()
-    check(lib.muon_plan_query(arr, count, prec, ctypes.byref(ws), offs, nt, tiles, pref))
+    check(lib.muon_plan_query(arr, count, prec, sp, ctypes.byref(ws), offs, nt, tiles, pref))
     tl = [(tiles[3 * k], tiles[3 * k + 1], tiles[3 * k + 2]) for k in range(total)]
+    a, b, c = nt[0], nt[0] + nt[1], nt[0] + nt[1] + nt[2]
     return {
         "ws_bytes": ws.value,
         "region_offsets": [list(offs[4 * i:4 * i + 4]) for i in range(count)],
-        "tiles": (tl[:nt[0]], tl[nt[0]:nt[0] + nt[1]], tl[nt[0] + nt[1]:]),
+        "tiles": (tl[:a], tl[a:b], tl[b:c]),
+        "small": [t[0] for t in tl[c:]],
         "chunk_prefix": list(pref),
     }
 
@@ -119,7 +123,7 @@ class Muon:
 
     def __init__(self, device: int = 0, scale_mode: str = "moonlight", extra_scale: float = 1.0,
                  ns_precision: str = "bf16", check_nonfinite: bool = False, num_sms: int = 0,
-                 workspace_cap_bytes: int = 0, wait_timeout_s: float = 2.0):
+                 workspace_cap_bytes: int = 0, wait_timeout_s: float = 2.0, small_path: bool = True):
         self._lib = load()
         cfg = MuonConfig()
         check(self._lib.muon_config_init(ctypes.byref(cfg)))
@@ -130,12 +134,13 @@ class Muon:
         cfg.num_sms = int(num_sms)
         cfg.workspace_cap_bytes = int(workspace_cap_bytes)
         cfg.wait_timeout_s = float(wait_timeout_s)
+        cfg.small_path = int(bool(small_path))
         h = ctypes.c_void_p()
         check(self._lib.muon_init(int(device), ctypes.byref(cfg), ctypes.byref(h)))
         self._h = h
         self.device = device
         self.ns_precision = ns_precision
-        self.x_dtype = None
+        self.small_path = bool(small_path)
 
     # -- lifetime -----------------------------------------------------------
     def close(self):
@@ -277,7 +282,7 @@ class Muon:
         check(self._lib.muon_workspace_ptr(self._h, ctypes.byref(base), ctypes.byref(size)))
         return base.value or 0, size.value
 
-    KERNEL_KINDS = ("momentum_norm", "ns_gram", "ns_poly", "ns_comb", "apply", "scale_copy", "ns_fp32")
+    KERNEL_KINDS = ("momentum_norm", "ns_gram", "ns_poly", "ns_comb", "apply", "scale_copy", "ns_fp32", "ns_small")
 
     def profile_enable(self, max_calls: int):
         """Record CUDA events around every kernel of the next max_calls calls."""

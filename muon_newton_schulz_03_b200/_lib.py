@@ -34,6 +34,7 @@ class MuonConfig(ctypes.Structure):
         ("num_sms", c_int),
         ("workspace_cap_bytes", c_size_t),
         ("wait_timeout_s", c_double),
+        ("small_path", c_int),
     ]
 
 
@@ -52,7 +53,7 @@ _SIGNATURES = {
                                    c_int, P(c_float), c_void_p]),
     "muon_apply": (c_int, [c_void_p, P(c_void_p), P(c_void_p), c_void_p, P(ctypes.c_int32), c_int,
                            c_float, c_float, c_void_p]),
-    "muon_plan_query": (c_int, [P(ctypes.c_int32), c_int, c_int, P(ctypes.c_int64), P(ctypes.c_int64),
+    "muon_plan_query": (c_int, [P(ctypes.c_int32), c_int, c_int, c_int, P(ctypes.c_int64), P(ctypes.c_int64),
                                 P(ctypes.c_int32), P(ctypes.c_int32), P(ctypes.c_int64)]),
     "muon_workspace_size": (c_int, [c_void_p, P(ctypes.c_int32), c_int, P(c_size_t)]),
     "muon_workspace_ptr": (c_int, [c_void_p, P(c_void_p), P(c_size_t)]),

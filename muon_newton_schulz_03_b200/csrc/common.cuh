@@ -148,6 +148,16 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity
   }
 }
 
+// Wait with only a time limit (used while draining after an abort: the
+// outstanding copy or MMA must land before the CTA frees its resources).
+__device__ __forceinline__ bool mbar_wait_drain(uint64_t* bar, uint32_t parity, uint64_t timeout_ns) {
+  const uint64_t t0 = global_timer_ns();
+  while (!mbar_try_wait(bar, parity)) {
+    if (global_timer_ns() - t0 > timeout_ns) return false;
+  }
+  return true;
+}
+
 // ---------------------------------------------------------------------------
 // Bulk-tensor (TMA) loads: 2D tile, global -> shared::cta, completion on an
 // mbarrier. The tensor map lives in global memory (written by the host before

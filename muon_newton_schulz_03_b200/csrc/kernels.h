@@ -59,6 +59,23 @@ struct NsLaunch {
   unsigned long long timeout_ns;
 };
 
+// Small-matrix path: one CTA per listed matrix runs every iteration on chip.
+struct NsSmallLaunch {
+  const MatPlan* plans;      // device
+  const MatBind* binds;      // device
+  const TmapBlob* maps;      // device, kMapsPerMat per matrix
+  const TmapBlob* in_maps;   // device, kInMapsPerMat per matrix or NULL
+  const int* mats;           // device list of matrix indices
+  int nmats;
+  const double* sumsq;       // device or NULL
+  DevStatus* status;         // device
+  unsigned long long timeout_ns;
+};
+
+cudaError_t launch_ns_small(const NsSmallLaunch& L, int ns_steps, int src_sel, int final_sel, float a, float b,
+                            float c, cudaStream_t st);
+int ns_small_smem_bytes();
+
 cudaError_t launch_ns_phase_bf16(const NsLaunch& L, int phase, int src_sel, int dst_sel, int first, float a,
                                  float b, float c, cudaStream_t st);
 

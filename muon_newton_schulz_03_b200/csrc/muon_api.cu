@@ -166,6 +166,7 @@ struct DevPlan {
   MatPlan* d_mats = nullptr;
   long long* d_prefix = nullptr;
   int4* d_tiles[3] = {nullptr, nullptr, nullptr};
+  int* d_small = nullptr;
   TmapBlob* d_maps = nullptr;
   std::vector<MatPlan> mats;         // host copy with workspace pointers
   void* staging = nullptr;           // muon_step_host buffers
@@ -243,7 +244,8 @@ int ensure_plan(muon_handle* h, const int32_t* shapes, int count) {
 
   auto np = std::make_unique<DevPlan>();
   std::string why;
-  if (!build_plan(shapes, count, h->cfg.ns_precision, np->hp, why)) return fail(MUON_ERR_INVALID_ARG, why);
+  if (!build_plan(shapes, count, h->cfg.ns_precision, h->cfg.small_path != 0, np->hp, why))
+    return fail(MUON_ERR_INVALID_ARG, why);
   np->key = key;
   const HostPlan& hp = np->hp;
   if (h->cfg.workspace_cap_bytes && (size_t)hp.ws_bytes > h->cfg.workspace_cap_bytes)
@@ -286,6 +288,8 @@ int ensure_plan(muon_handle* h, const int32_t* shapes, int count) {
     o_tiles[p] = off;
     off = align_up(off + (int64_t)sizeof(int4) * std::max<size_t>(hp.tiles[p].size(), 1), 256);
   }
+  const int64_t o_small = off;
+  off = align_up(off + (int64_t)sizeof(int) * std::max<size_t>(hp.small.size(), 1), 256);
   const int64_t o_maps = off;
   if (bf16) off = align_up(off + (int64_t)sizeof(TmapBlob) * kMapsPerMat * count, 256);
   std::vector<unsigned char> host((size_t)off, 0);
@@ -296,6 +300,7 @@ int ensure_plan(muon_handle* h, const int32_t* shapes, int count) {
     for (size_t k = 0; k < hp.tiles[p].size(); ++k)
       t[k] = make_int4(hp.tiles[p][k].mat, hp.tiles[p][k].ti, hp.tiles[p][k].tj, 0);
   }
+  if (!hp.small.empty()) std::memcpy(host.data() + o_small, hp.small.data(), sizeof(int) * hp.small.size());
   if (bf16) {
     TmapBlob* maps = reinterpret_cast<TmapBlob*>(host.data() + o_maps);
     for (int i = 0; i < count; ++i) {
@@ -325,6 +330,7 @@ int ensure_plan(muon_handle* h, const int32_t* shapes, int count) {
   np->d_mats = reinterpret_cast<MatPlan*>(tb + o_mats);
   np->d_prefix = reinterpret_cast<long long*>(tb + o_pref);
   for (int p = 0; p < 3; ++p) np->d_tiles[p] = reinterpret_cast<int4*>(tb + o_tiles[p]);
+  np->d_small = reinterpret_cast<int*>(tb + o_small);
   np->d_maps = bf16 ? reinterpret_cast<TmapBlob*>(tb + o_maps) : nullptr;
   h->plan = std::move(np);
   return MUON_OK;
@@ -387,6 +393,25 @@ int enqueue_ns(muon_handle* h, const MatBind* d_binds, const std::vector<MatBind
   DevPlan& P = *h->plan;
   const HostPlan& hp = P.hp;
   const bool bf16 = h->cfg.ns_precision == MUON_NS_BF16;
+  if (bf16 && ns_steps > 0 && !hp.small.empty()) {
+    // Matrices on the small path run every iteration in one launch and land
+    // in the same buffer as the others' last step.
+    NsSmallLaunch S;
+    S.plans = P.d_mats;
+    S.binds = d_binds;
+    S.maps = P.d_maps;
+    S.in_maps = d_in_maps;
+    S.mats = P.d_small;
+    S.nmats = (int)hp.small.size();
+    S.sumsq = sumsq;
+    S.status = h->status;
+    S.timeout_ns = (unsigned long long)(h->cfg.wait_timeout_s * 1e9);
+    const int final_sel = last_dst >= 0 ? last_dst : (ns_steps % 2 == 1 ? BUF_X1 : BUF_X0);
+    const int slot = prof_before(h, MUON_KERNEL_NS_SMALL, st);
+    MUON_CUDA_TRY(launch_ns_small(S, ns_steps, first_src, final_sel, abc[0], abc[1], abc[2], st));
+    prof_after(h, slot, st);
+    ++*launches;
+  }
   int src = first_src;
   for (int t = 1; t <= ns_steps; ++t) {
     const int dst = (t == ns_steps && last_dst >= 0) ? last_dst : (t % 2 == 1 ? BUF_X1 : BUF_X0);
@@ -404,6 +429,7 @@ int enqueue_ns(muon_handle* h, const MatBind* d_binds, const std::vector<MatBind
       for (int ph = 0; ph < 3; ++ph) {
         L.tiles = P.d_tiles[ph];
         L.ntiles = (int)hp.tiles[ph].size();
+        if (L.ntiles == 0) continue;
         const int slot = prof_before(h, MUON_KERNEL_NS_GRAM + ph, st);
         MUON_CUDA_TRY(launch_ns_phase_bf16(L, ph, src, dst, first, abc[0], abc[1], abc[2], st));
         prof_after(h, slot, st);
@@ -516,6 +542,7 @@ int muon_config_init(muon_config* cfg) {
   cfg->num_sms = 0;
   cfg->workspace_cap_bytes = 0;
   cfg->wait_timeout_s = 2.0;
+  cfg->small_path = 1;
   return MUON_OK;
 }
 
@@ -774,16 +801,18 @@ int muon_apply(muon_handle* h, float* const* params, const void* const* o, const
   return MUON_OK;
 }
 
-int muon_plan_query(const int32_t* shapes, int count, int ns_precision, int64_t* ws_bytes, int64_t* region_offsets,
-                    int32_t* ntiles, int32_t* tiles, int64_t* chunk_prefix) {
+int muon_plan_query(const int32_t* shapes, int count, int ns_precision, int small_path, int64_t* ws_bytes,
+                    int64_t* region_offsets, int32_t* ntiles, int32_t* tiles, int64_t* chunk_prefix) {
   g_last_error.clear();
   HostPlan hp;
   std::string why;
-  if (!build_plan(shapes, count, ns_precision, hp, why)) return fail(MUON_ERR_INVALID_ARG, why);
+  if (!build_plan(shapes, count, ns_precision, small_path != 0, hp, why)) return fail(MUON_ERR_INVALID_ARG, why);
   if (ws_bytes) *ws_bytes = hp.ws_bytes;
   if (region_offsets) std::memcpy(region_offsets, hp.region_off.data(), sizeof(int64_t) * hp.region_off.size());
-  if (ntiles)
+  if (ntiles) {
     for (int p = 0; p < 3; ++p) ntiles[p] = (int32_t)hp.tiles[p].size();
+    ntiles[3] = (int32_t)hp.small.size();
+  }
   if (tiles) {
     size_t k = 0;
     for (int p = 0; p < 3; ++p)
@@ -793,6 +822,12 @@ int muon_plan_query(const int32_t* shapes, int count, int ns_precision, int64_t*
         tiles[3 * k + 2] = t.tj;
         ++k;
       }
+    for (int i : hp.small) {
+      tiles[3 * k] = i;
+      tiles[3 * k + 1] = 0;
+      tiles[3 * k + 2] = 0;
+      ++k;
+    }
   }
   if (chunk_prefix)
     for (int i = 0; i <= count; ++i) chunk_prefix[i] = hp.prefix[i];
@@ -804,7 +839,8 @@ int muon_workspace_size(muon_handle* h, const int32_t* shapes, int count, size_t
   if (!h || !bytes) return fail(MUON_ERR_INVALID_ARG, "handle and bytes are required");
   HostPlan hp;
   std::string why;
-  if (!build_plan(shapes, count, h->cfg.ns_precision, hp, why)) return fail(MUON_ERR_INVALID_ARG, why);
+  if (!build_plan(shapes, count, h->cfg.ns_precision, h->cfg.small_path != 0, hp, why))
+    return fail(MUON_ERR_INVALID_ARG, why);
   *bytes = (size_t)hp.ws_bytes;
   return MUON_OK;
 }

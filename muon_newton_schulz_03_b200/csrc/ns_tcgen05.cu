@@ -108,15 +108,6 @@ __device__ __forceinline__ TileJob decode(const NsArgs& A, const int4 t, const M
   return j;
 }
 
-// Wait with only a time limit (used while draining after an abort).
-__device__ __forceinline__ bool mbar_wait_drain(uint64_t* bar, uint32_t parity, uint64_t timeout_ns) {
-  const uint64_t t0 = global_timer_ns();
-  while (!mbar_try_wait(bar, parity)) {
-    if (global_timer_ns() - t0 > timeout_ns) return false;
-  }
-  return true;
-}
-
 __device__ __forceinline__ void store_bf16x32(__nv_bfloat16* dst, const float (&o)[32]) {
 #pragma unroll
   for (int q = 0; q < 4; ++q) {

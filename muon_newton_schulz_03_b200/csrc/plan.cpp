@@ -13,6 +13,9 @@
 //    matrices and row block outer for tall ones (each wave of CTAs then
 //    shares the large X panel in L2); each phase's list is ordered by the
 //    matrix's reduction length, longest first, ties by matrix index;
+//  * small path (when enabled): matrices with s <= 128 and l <= 512 are left
+//    out of the tile lists and listed, in index order, for the on-chip
+//    kernel that runs the whole iteration in one CTA;
 //  * elementwise: kElemChunk elements per block, prefix over matrices.
 #include "plan.h"
 
@@ -45,7 +48,7 @@ void comb_tiles(int mat, int m, int n, std::vector<TileRec>& out) {
 
 }  // namespace
 
-bool build_plan(const int32_t* shapes, int count, int prec, HostPlan& P, std::string& why) {
+bool build_plan(const int32_t* shapes, int count, int prec, bool small_path, HostPlan& P, std::string& why) {
   if (shapes == nullptr) { why = "shapes is NULL"; return false; }
   if (count < 1) { why = "count must be >= 1"; return false; }
   if (prec != 0 && prec != 1) { why = "ns_precision must be 0 (bf16) or 1 (fp32)"; return false; }
@@ -90,15 +93,25 @@ bool build_plan(const int32_t* shapes, int count, int prec, HostPlan& P, std::st
   }
   P.ws_bytes = off;
 
+  std::vector<char> is_small((size_t)count, 0);
+  if (small_path)
+    for (int i = 0; i < count; ++i)
+      if (P.mats[i].s <= kSmallMaxS && P.mats[i].l <= kSmallMaxL) {
+        is_small[i] = 1;
+        P.small.push_back(i);
+      }
   std::vector<int> order(count);
   auto sorted_by = [&](auto key) {
     std::iota(order.begin(), order.end(), 0);
     std::stable_sort(order.begin(), order.end(), [&](int x, int y) { return key(x) > key(y); });
     return order;
   };
-  for (int i : sorted_by([&](int i) { return P.mats[i].l; })) sym_tiles(i, P.mats[i].s, P.tiles[0]);
-  for (int i : sorted_by([&](int i) { return P.mats[i].s; })) sym_tiles(i, P.mats[i].s, P.tiles[1]);
-  for (int i : sorted_by([&](int i) { return P.mats[i].s; })) comb_tiles(i, P.m[i], P.n[i], P.tiles[2]);
+  for (int i : sorted_by([&](int i) { return P.mats[i].l; }))
+    if (!is_small[i]) sym_tiles(i, P.mats[i].s, P.tiles[0]);
+  for (int i : sorted_by([&](int i) { return P.mats[i].s; }))
+    if (!is_small[i]) sym_tiles(i, P.mats[i].s, P.tiles[1]);
+  for (int i : sorted_by([&](int i) { return P.mats[i].s; }))
+    if (!is_small[i]) comb_tiles(i, P.m[i], P.n[i], P.tiles[2]);
 
   P.prefix.assign((size_t)count + 1, 0);
   for (int i = 0; i < count; ++i)

@@ -15,6 +15,8 @@ constexpr int kTileM = 128;     // output rows per tile
 constexpr int kTileN = 256;     // output columns per tile
 constexpr int kRegionAlign = 1024;
 constexpr int kMaxDim = 1 << 20;
+constexpr int kSmallMaxS = 128;     // small path: min(m, n) <= 128 ...
+constexpr int kSmallMaxL = 512;     // ... and max(m, n) <= 512
 
 struct TileRec {
   int mat, ti, tj;
@@ -29,11 +31,14 @@ struct HostPlan {
   int64_t head_bytes = 0;             // sum-of-squares block
   int64_t ws_bytes = 0;
   std::vector<TileRec> tiles[3];      // Gram, polynomial, combine
+  std::vector<int> small;             // matrices on the on-chip small path
   std::vector<long long> prefix;      // count + 1
 };
 
 // Validates the shape table (m, n in [1, kMaxDim], flags in {0, 1}) and
-// builds the plan. Returns false with a message on invalid input.
-bool build_plan(const int32_t* shapes, int count, int prec, HostPlan& out, std::string& why);
+// builds the plan. With small_path, matrices with s <= kSmallMaxS and
+// l <= kSmallMaxL go to the on-chip small path instead of the tile lists.
+// Returns false with a message on invalid input.
+bool build_plan(const int32_t* shapes, int count, int prec, bool small_path, HostPlan& out, std::string& why);
 
 }  // namespace muon

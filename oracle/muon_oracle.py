@@ -108,7 +108,15 @@ def ns_poly_iterate(s, steps=5, coeffs=DEFAULT_COEFFS):
 # Matrix Newton-Schulz
 # ---------------------------------------------------------------------------
 
-def _ns_iterations(X, steps, coeffs, emulate_bf16):
+def _matmul(P, Q, accum_fp32):
+    """P @ Q; with accum_fp32 the operands (bf16 values, exact in float32)
+    are multiplied with float32 accumulation, as tensor cores accumulate."""
+    if not accum_fp32:
+        return P @ Q
+    return (P.astype(np.float32) @ Q.astype(np.float32)).astype(np.float64)
+
+
+def _ns_iterations(X, steps, coeffs, emulate_bf16, accum_fp32=False):
     """Run the quintic iteration on a short-side-first matrix X (s x l).
 
     Each step forms the Gram A = X X^T, the polynomial B = bA + cA^2 and the
@@ -119,14 +127,14 @@ def _ns_iterations(X, steps, coeffs, emulate_bf16):
     a, b, c = coeffs
     rnd = bf16_round if emulate_bf16 else (lambda v: v)
     for _ in range(steps):
-        A = rnd(X @ X.T)
-        B = rnd(b * A + c * (A @ A))
-        X = rnd(a * X + B @ X)
+        A = rnd(_matmul(X, X.T, accum_fp32))
+        B = rnd(b * A + c * _matmul(A, A, accum_fp32))
+        X = rnd(a * X + _matmul(B, X, accum_fp32))
     return X
 
 
 def newton_schulz(G, steps=5, coeffs=DEFAULT_COEFFS, eps=EPS,
-                  emulate_bf16=False):
+                  emulate_bf16=False, accum_fp32=False):
     """Approximate orthogonal polar factor of G (float64).
 
     "About Muon: Why Not Adam", section "The whole thing, in about forty
@@ -137,6 +145,8 @@ def newton_schulz(G, steps=5, coeffs=DEFAULT_COEFFS, eps=EPS,
     With ``emulate_bf16`` the input is rounded to bf16 before normalising and
     the normalisation factor is applied exactly where the GPU applies it
     (inside the first Gram and first combine); otherwise no rounding happens.
+    ``accum_fp32`` (with ``emulate_bf16``) accumulates the products in
+    float32 instead of float64: a second, equally valid bf16 realization.
     """
     G = np.asarray(G, dtype=np.float64)
     if G.ndim != 2:
@@ -159,14 +169,14 @@ def newton_schulz(G, steps=5, coeffs=DEFAULT_COEFFS, eps=EPS,
     if steps == 0:
         X = alpha * Y
     else:
-        A = bf16_round(alpha * alpha * (Y @ Y.T))
-        B = bf16_round(b * A + c * (A @ A))
-        X = bf16_round(alpha * (a * Y + B @ Y))
-        X = _ns_iterations(X, steps - 1, coeffs, True)
+        A = bf16_round(alpha * alpha * _matmul(Y, Y.T, accum_fp32))
+        B = bf16_round(b * A + c * _matmul(A, A, accum_fp32))
+        X = bf16_round(alpha * (a * Y + _matmul(B, Y, accum_fp32)))
+        X = _ns_iterations(X, steps - 1, coeffs, True, accum_fp32)
     return X.T if transposed else X
 
 
-def ns_only(X, steps=5, coeffs=DEFAULT_COEFFS, emulate_bf16=False):
+def ns_only(X, steps=5, coeffs=DEFAULT_COEFFS, emulate_bf16=False, accum_fp32=False):
     """The Newton-Schulz phases alone on an already-scaled X (no norm).
 
     Used for the NS-only sweep workload, whose inputs are generated with
@@ -180,7 +190,7 @@ def ns_only(X, steps=5, coeffs=DEFAULT_COEFFS, emulate_bf16=False):
     transposed = X.shape[0] > X.shape[1]
     if transposed:
         X = X.T
-    X = _ns_iterations(X, steps, coeffs, emulate_bf16)
+    X = _ns_iterations(X, steps, coeffs, emulate_bf16, accum_fp32 and emulate_bf16)
     return X.T if transposed else X
 
 
@@ -258,7 +268,7 @@ def apply_update(p, O, lr, wd, scale):
 def muon_step_matrix(p, g, m, *, lr, beta=0.95, nesterov=True, wd=0.1,
                      ns_steps=5, coeffs=DEFAULT_COEFFS,
                      scale_mode=SCALE_MOONLIGHT, extra_scale=1.0,
-                     emulate_bf16=False):
+                     emulate_bf16=False, accum_fp32=False):
     """One Muon step on one matrix. Returns (p', m', O, ||u||_F).
 
     Order: momentum, Nesterov blend, Newton-Schulz (normalise, orient,
@@ -270,7 +280,7 @@ def muon_step_matrix(p, g, m, *, lr, beta=0.95, nesterov=True, wd=0.1,
     m_new = momentum_update(m, g, beta)
     u = nesterov_blend(g, m_new, beta, nesterov)
     nu = float(np.linalg.norm(u))
-    O = newton_schulz(u, ns_steps, coeffs, EPS, emulate_bf16)
+    O = newton_schulz(u, ns_steps, coeffs, EPS, emulate_bf16, accum_fp32)
     scale = update_scale(p.shape[0], p.shape[1], scale_mode, extra_scale)
     p_new = apply_update(p, O, lr, wd, scale)
     return p_new, m_new, O, nu

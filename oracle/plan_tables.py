@@ -33,6 +33,11 @@ Tiles. Output tiles are BM = 128 rows by BN = 256 columns.
   index, then by the per-matrix order above. A tile entry is
   (matrix, ti, tj).
 
+Small path. With the small path on (the default), a matrix with
+s <= 128 and l <= 512 runs its whole iteration in one on-chip kernel: it is
+left out of the three tile lists and listed, in matrix-index order, in a
+fourth list.
+
 Elementwise chunks. The fused momentum and apply kernels give each thread
 block CHUNK = 8192 consecutive elements of one matrix; chunk_prefix[i] is
 the number of chunks of matrices 0..i-1.
@@ -92,22 +97,31 @@ def _comb_tiles(m: int, n: int):
     return [(ti, tj) for ti in range(rows) for tj in range(cols)]
 
 
-def tile_lists(shapes):
-    """(gram, poly, comb) lists of (matrix, ti, tj)."""
+SMALL_MAX_S = 128
+SMALL_MAX_L = 512
+
+
+def tile_lists(shapes, small_path=True):
+    """(gram, poly, comb) lists of (matrix, ti, tj) and the small-path list."""
     gram, poly, comb = [], [], []
     geo = [matrix_geometry(m, n) for (m, n) in shapes]
+    small = [i for i, g in enumerate(geo) if small_path and g[1] <= SMALL_MAX_S and g[2] <= SMALL_MAX_L]
+    tiled = set(range(len(shapes))) - set(small)
 
     def order(klen):
         return sorted(range(len(shapes)), key=lambda i: (-klen(i), i))
 
     for i in order(lambda i: geo[i][2]):
-        gram += [(i, ti, tj) for ti, tj in _sym_tiles(geo[i][1])]
+        if i in tiled:
+            gram += [(i, ti, tj) for ti, tj in _sym_tiles(geo[i][1])]
     for i in order(lambda i: geo[i][1]):
-        poly += [(i, ti, tj) for ti, tj in _sym_tiles(geo[i][1])]
+        if i in tiled:
+            poly += [(i, ti, tj) for ti, tj in _sym_tiles(geo[i][1])]
     for i in order(lambda i: geo[i][1]):
-        m, n = shapes[i]
-        comb += [(i, ti, tj) for ti, tj in _comb_tiles(m, n)]
-    return gram, poly, comb
+        if i in tiled:
+            m, n = shapes[i]
+            comb += [(i, ti, tj) for ti, tj in _comb_tiles(m, n)]
+    return gram, poly, comb, small
 
 
 def chunk_prefix(shapes):

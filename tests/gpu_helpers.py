@@ -15,30 +15,34 @@ TOL_ELEM = 1e-6         # elementwise stages vs the float64 oracle
 TOL_BF16_EMU = 1e-2     # bf16 Newton-Schulz vs the oracle's bf16-rounding mode
 
 
-def bf16_gate(got, exact, emulated, what=""):
+def bf16_gate(got, exact, emulated, emulated32, what=""):
     """Two-tier parity of a bf16 Newton-Schulz result.
 
-    1. Against the oracle run at the pages' precision (bf16 rounding of the
-       input and of every Gram / polynomial / combine output): within
-       TOL_BF16_EMU. Two bf16 realizations that differ only in fp32
-       summation order (GPU) vs float64 summation (oracle) drift apart
-       through the iteration by a few 1e-3; half the gate bounds that.
-    2. Against the exact float64 oracle: within TOL_BF16_NS wherever bf16
-       arithmetic itself can meet that (the bf16-rounding oracle is within
-       it); otherwise no further than 1.25 times the bf16-rounding oracle's
-       own distance (inputs whose spectrum reaches below the bf16 floor,
-       tiny matrices whose few singular values land near the repelling
-       fixed points).
-    Returns (err_vs_exact, err_vs_emulated, err_of_emulation).
+    `emulated` and `emulated32` are the oracle at the pages' precision (bf16
+    rounding of the input and of every Gram / polynomial / combine output),
+    accumulating in float64 and in float32: two equally valid bf16
+    realizations. Their distance, `spread`, measures how strongly rounding
+    differences grow through the iteration at this input (tiny for
+    well-conditioned inputs, ~1e-2 and more when singular values reach down to
+    1e-4 without normalisation).
+    1. The GPU is a bf16 realization: its distance to the nearer of the two
+       is within max(TOL_BF16_EMU, 3 * spread).
+    2. The GPU is as accurate as bf16 arithmetic allows: its distance to the
+       exact float64 oracle is within TOL_BF16_NS, or, where bf16 arithmetic
+       itself cannot meet that (the emulations' own distance `inherent`
+       exceeds it), within inherent + 3 * spread.
+    Returns (err_vs_exact, err_vs_emulated, inherent, spread).
     """
-    e_emu = rel(got, emulated)
+    e_emu = min(rel(got, emulated), rel(got, emulated32))
     e_exact = rel(got, exact)
-    e_inherent = rel(emulated, exact)
-    assert e_emu <= TOL_BF16_EMU, f"{what}: {e_emu:.3e} from the bf16-rounding oracle"
-    bound = TOL_BF16_NS if e_inherent <= TOL_BF16_NS else 1.25 * e_inherent
-    assert e_exact <= bound, (f"{what}: {e_exact:.3e} from the exact oracle "
-                              f"(bf16 arithmetic alone: {e_inherent:.3e})")
-    return e_exact, e_emu, e_inherent
+    inherent = max(rel(emulated, exact), rel(emulated32, exact))
+    spread = rel(emulated32, emulated)
+    bound1 = max(TOL_BF16_EMU, 3.0 * spread)
+    assert e_emu <= bound1, f"{what}: {e_emu:.3e} from the bf16-rounding oracle (spread {spread:.3e})"
+    bound2 = TOL_BF16_NS if inherent <= TOL_BF16_NS else inherent + 3.0 * spread
+    assert e_exact <= bound2, (f"{what}: {e_exact:.3e} from the exact oracle "
+                               f"(bf16 arithmetic alone: {inherent:.3e}, spread {spread:.3e})")
+    return e_exact, e_emu, inherent, spread
 
 
 def rel(a, b):

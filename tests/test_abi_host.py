@@ -56,23 +56,25 @@ SHAPE_SETS = {
 
 @pytest.mark.parametrize("name", sorted(SHAPE_SETS))
 @pytest.mark.parametrize("prec", ["bf16", "fp32"])
-def test_plan_tables_bit_exact(name, prec):
+@pytest.mark.parametrize("small_path", [True, False])
+def test_plan_tables_bit_exact(name, prec, small_path):
     shapes = SHAPE_SETS[name]
-    got = muon.plan_query(shapes, prec)
+    got = muon.plan_query(shapes, prec, small_path)
     regions, ws = PT.workspace_layout(shapes, 2 if prec == "bf16" else 4)
     assert got["ws_bytes"] == ws
     assert got["region_offsets"] == regions
-    gram, poly, comb = PT.tile_lists(shapes)
+    gram, poly, comb, small = PT.tile_lists(shapes, small_path)
     assert got["tiles"][0] == gram
     assert got["tiles"][1] == poly
     assert got["tiles"][2] == comb
+    assert got["small"] == small
     assert got["chunk_prefix"] == PT.chunk_prefix(shapes)
 
 
 @pytest.mark.parametrize("shape", [(1, 1), (5, 3), (130, 300), (300, 130), (512, 512), (600, 257), (257, 600)])
 def test_tiles_cover_each_entry_once(shape):
     m, n = shape
-    got = muon.plan_query([shape])
+    got = muon.plan_query([shape], small_path=False)
     s = min(m, n)
     # Symmetric phases: direct writes of each listed tile plus transposed
     # writes of the tiles strictly right of the 256-block diagonal.
@@ -119,9 +121,9 @@ def test_plan_rejects_empty_and_bad_precision():
     lib = muon.load()
     import ctypes
     arr = (ctypes.c_int32 * 3)(4, 4, 0)
-    assert lib.muon_plan_query(arr, 0, 0, None, None, None, None, None) == 1
-    assert lib.muon_plan_query(arr, 1, 7, None, None, None, None, None) == 1
-    assert lib.muon_plan_query(None, 1, 0, None, None, None, None, None) == 1
+    assert lib.muon_plan_query(arr, 0, 0, 1, None, None, None, None, None) == 1
+    assert lib.muon_plan_query(arr, 1, 7, 1, None, None, None, None, None) == 1
+    assert lib.muon_plan_query(None, 1, 0, 1, None, None, None, None, None) == 1
     assert b"shapes" in lib.muon_last_error()
 
 
@@ -131,7 +133,7 @@ def test_config_defaults():
     import ctypes
     assert lib.muon_config_init(ctypes.byref(cfg)) == 0
     assert cfg.scale_mode == 0 and cfg.extra_scale == 1.0 and cfg.ns_precision == 0
-    assert cfg.wait_timeout_s == 2.0 and cfg.num_sms == 0
+    assert cfg.wait_timeout_s == 2.0 and cfg.num_sms == 0 and cfg.small_path == 1
     assert lib.muon_config_init(None) == 1
 
 

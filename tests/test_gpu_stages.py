@@ -187,8 +187,9 @@ def test_ns_single_step_phases(opt_bf16, coeffs):
     for i, (m, n) in enumerate(shapes):
         ref = O.ns_only(x64[i], 1, coeffs)
         emu = O.ns_only(x64[i], 1, coeffs, emulate_bf16=True)
+        emu32 = O.ns_only(x64[i], 1, coeffs, emulate_bf16=True, accum_fp32=True)
         got = to64(xout[i][:, :n])
-        bf16_gate(got, ref, emu, f"matrix {i} {m}x{n}")
+        bf16_gate(got, ref, emu, emu32, f"matrix {i} {m}x{n}")
     _assert_status_clean(opt_bf16)
 
 
@@ -203,8 +204,9 @@ def test_ns_bf16_matches_oracle(opt_bf16, steps):
     for i, (m, n) in enumerate(shapes):
         ref = O.newton_schulz(x64[i], steps)
         emu = O.newton_schulz(x64[i], steps, emulate_bf16=True)
+        emu32 = O.newton_schulz(x64[i], steps, emulate_bf16=True, accum_fp32=True)
         got = to64(xout[i][:, :n])
-        bf16_gate(got, ref, emu, f"matrix {i} {m}x{n}")
+        bf16_gate(got, ref, emu, emu32, f"matrix {i} {m}x{n}")
     # Inputs were not modified.
     for i, (m, n) in enumerate(shapes):
         assert np.array_equal(to64(xin[i][:, :n]), x64[i])
@@ -283,5 +285,47 @@ def test_ns_only_sweep_inputs(opt_bf16, point):
     for b in range(batch):
         ref = O.ns_only(x64[b], 5)
         emu = O.ns_only(x64[b], 5, emulate_bf16=True)
-        bf16_gate(to64(xout[b][:, :n]), ref, emu, f"{m}x{n} #{b}")
+        emu32 = O.ns_only(x64[b], 5, emulate_bf16=True, accum_fp32=True)
+        bf16_gate(to64(xout[b][:, :n]), ref, emu, emu32, f"{m}x{n} #{b}")
     _assert_status_clean(opt_bf16)
+
+
+SMALL_SHAPES = [(1, 1), (3, 5), (5, 3), (64, 64), (100, 300), (300, 100), (128, 128), (128, 512), (512, 128),
+                (127, 129), (1, 300), (300, 1), (16, 512), (512, 16), (96, 200), (65, 65)]
+
+
+@pytest.mark.parametrize("steps", [1, 5])
+def test_small_path_matches_oracle_and_tiled_path(opt_bf16, steps):
+    # The on-chip small-matrix kernel (all iterations in one CTA) against the
+    # oracle, and against the tiled phases on the same inputs.
+    shapes = SMALL_SHAPES
+    assert muon.plan_query(shapes)["small"] == list(range(len(shapes)))
+    xin, x64 = _ns_inputs(shapes, 30 + steps)
+    sumsq = torch.tensor([np.sum(x ** 2) for x in x64], dtype=torch.float64, device=DEV)
+    out_small = [x_buffer(m, n) for (m, n) in shapes]
+    out_tiled = [x_buffer(m, n) for (m, n) in shapes]
+    opt_bf16.newton_schulz(xin, out_small, shapes, sumsq, ns_steps=steps)
+    tiled = muon.Muon(device=0, small_path=False)
+    tiled.newton_schulz(xin, out_tiled, shapes, sumsq, ns_steps=steps)
+    torch.cuda.synchronize()
+    assert opt_bf16.last_launch_count() == 1       # one launch for every small matrix
+    for i, (m, n) in enumerate(shapes):
+        got = to64(out_small[i][:, :n])
+        ref = O.newton_schulz(x64[i], steps)
+        emu = O.newton_schulz(x64[i], steps, emulate_bf16=True)
+        emu32 = O.newton_schulz(x64[i], steps, emulate_bf16=True, accum_fp32=True)
+        bf16_gate(got, ref, emu, emu32, f"small path {m}x{n}")
+        assert rel(got, to64(out_tiled[i][:, :n])) <= TOL_BF16_EMU, f"small vs tiled {m}x{n}"
+    _assert_status_clean(opt_bf16)
+    assert tiled.status() == (0, 0, 0)
+    tiled.close()
+
+
+def test_small_path_identity_is_exact(opt_bf16):
+    shapes = SMALL_SHAPES
+    xin, x64 = _ns_inputs(shapes, 40)
+    xout = [x_buffer(m, n) for (m, n) in shapes]
+    opt_bf16.newton_schulz(xin, xout, shapes, None, ns_steps=3, coeffs=(1.0, 0.0, 0.0))
+    torch.cuda.synchronize()
+    for i, (m, n) in enumerate(shapes):
+        assert np.array_equal(to64(xout[i][:, :n]), x64[i]), f"{m}x{n}"

@@ -38,10 +38,11 @@ def _check_step(cpu, dev, shapes, opt, *, lr, beta, wd, nesterov=True, ns_steps=
         dp_gpu = p_gpu - p0
         bf16 = opt.ns_precision == "bf16"
         if bf16:
-            p_emu, _, o_emu, _ = O.muon_step_matrix(p0, g, m0, lr=F32(lr), beta=F32(beta), nesterov=nesterov,
-                                                    wd=F32(wd), ns_steps=ns_steps, scale_mode=scale_mode,
-                                                    emulate_bf16=True)
-            e, _, _ = bf16_gate(dp_gpu, dp_ref, p_emu - p0, f"update of matrix {i} {m}x{n}")
+            kw = dict(lr=F32(lr), beta=F32(beta), nesterov=nesterov, wd=F32(wd), ns_steps=ns_steps,
+                      scale_mode=scale_mode, emulate_bf16=True)
+            p_emu, _, o_emu, _ = O.muon_step_matrix(p0, g, m0, **kw)
+            p_e32, _, o_e32, _ = O.muon_step_matrix(p0, g, m0, accum_fp32=True, **kw)
+            e = bf16_gate(dp_gpu, dp_ref, p_emu - p0, p_e32 - p0, f"update of matrix {i} {m}x{n}")[0]
         else:
             e = rel(dp_gpu, dp_ref)
             assert e <= tol, f"matrix {i} {m}x{n}: update off by {e:.3e}"
@@ -50,7 +51,7 @@ def _check_step(cpu, dev, shapes, opt, *, lr, beta, wd, nesterov=True, ns_steps=
             dtype = torch.bfloat16 if bf16 else torch.float32
             o_gpu = to64(workspace_matrix(opt, shapes, i, ns_steps % 2, dtype)[:, :n])
             if bf16:
-                bf16_gate(o_gpu, o_ref, o_emu, f"O of matrix {i}")
+                bf16_gate(o_gpu, o_ref, o_emu, o_e32, f"O of matrix {i}")
             else:
                 eo = rel(o_gpu, o_ref)
                 assert eo <= tol, f"matrix {i}: O off by {eo:.3e}"
@@ -134,7 +135,8 @@ def test_skipped_zero_and_nan_gradients():
     kw = dict(lr=F32(0.01), beta=F32(0.9), wd=F32(0.5), nesterov=False)
     ref, mref, _, _ = O.muon_step_matrix(p0[1], np.zeros(shapes[1]), m0[1], **kw)
     emu, _, _, _ = O.muon_step_matrix(p0[1], np.zeros(shapes[1]), m0[1], emulate_bf16=True, **kw)
-    bf16_gate(to64(p[1]) - p0[1], ref - p0[1], emu - p0[1], "zero-gradient matrix")
+    e32, _, _, _ = O.muon_step_matrix(p0[1], np.zeros(shapes[1]), m0[1], emulate_bf16=True, accum_fp32=True, **kw)
+    bf16_gate(to64(p[1]) - p0[1], ref - p0[1], emu - p0[1], e32 - p0[1], "zero-gradient matrix")
     assert opt.status() == (0, 0, 0)
     # A NaN is counted and reported.
     g[2][3, 4] = float("nan")
@@ -290,9 +292,10 @@ def _full_set_sampled(config, shapes, grad_dtype, sample, lr=2e-4, wd=0.1):
         kw = dict(lr=F32(lr), beta=F32(0.95), wd=F32(wd))
         p_ref, m_ref, o_ref, _ = O.muon_step_matrix(p0, g, m0, **kw)
         p_emu, _, _, _ = O.muon_step_matrix(p0, g, m0, emulate_bf16=True, **kw)
+        p_e32, _, _, _ = O.muon_step_matrix(p0, g, m0, emulate_bf16=True, accum_fp32=True, **kw)
         p_gpu, m_gpu = to64(dev[i][0]), to64(dev[i][2])
         assert rel(m_gpu, m_ref) <= TOL_ELEM
-        errs.append(bf16_gate(p_gpu - p0, p_ref - p0, p_emu - p0, f"matrix {i} {m}x{n}"))
+        errs.append(bf16_gate(p_gpu - p0, p_ref - p0, p_emu - p0, p_e32 - p0, f"matrix {i} {m}x{n}"))
     opt.close()
     return errs
 
@@ -309,3 +312,19 @@ def test_moe_set_sampled():
     shapes = W.moe_shapes()
     # three experts: gate (wide) and down (tall)
     _full_set_sampled(W.CONFIG_MOE, shapes, torch.bfloat16, sample=[0, 5, 382])
+
+
+def test_mixed_small_and_tiled_matrices_in_one_step():
+    # Matrices on the on-chip path and on the tiled phases in the same call:
+    # both land in the same workspace buffer before the apply kernel.
+    shapes = [(128, 512), (512, 128), (64, 64), (768, 768), (300, 100), (1024, 256), (2, 2)]
+    plan = muon.plan_query(shapes)
+    assert plan["small"] == [0, 1, 2, 4, 6]
+    cpu, dev = make_set(W.CONFIG_GPT2, shapes, torch.float32)
+    opt = muon.Muon(device=0)
+    opt.step([d[0] for d in dev], [d[1] for d in dev], [d[2] for d in dev], lr=2e-4, beta=0.95, wd=0.1)
+    torch.cuda.synchronize()
+    _check_step(cpu, dev, shapes, opt, lr=2e-4, beta=0.95, wd=0.1)
+    assert opt.last_launch_count() == 1 + 1 + 15 + 1
+    assert opt.status() == (0, 0, 0)
+    opt.close()

@@ -395,3 +395,20 @@ def test_ns_only_bf16_mode_structure(monkeypatch):
     a = O.ns_only(X, 5, emulate_bf16=True)
     monkeypatch.undo()
     assert np.max(np.abs(a - O.ns_only(X, 5))) < 1e-13
+
+
+def test_bf16_mode_fp32_accumulation_is_a_nearby_realization():
+    # On a well-conditioned input the two bf16 realizations (float64 and
+    # float32 accumulation) agree far below the bf16 gate, and with rounding
+    # made the identity the float32-accumulated mode stays within float32
+    # accuracy of the exact mode.
+    rng = np.random.default_rng(20)
+    G = (_haar(rng, 40, 40) * np.linspace(1, 0.1, 40)) @ _haar(rng, 90, 40).T
+    a = O.newton_schulz(G, emulate_bf16=True)
+    b = O.newton_schulz(G, emulate_bf16=True, accum_fp32=True)
+    assert np.linalg.norm(a - b) / np.linalg.norm(a) < 5e-3
+    monkey = pytest.MonkeyPatch()
+    monkey.setattr(O, "bf16_round", lambda v: np.asarray(v, dtype=np.float64))
+    c = O.newton_schulz(G, emulate_bf16=True, accum_fp32=True)
+    monkey.undo()
+    assert np.max(np.abs(c - O.newton_schulz(G))) < 1e-5

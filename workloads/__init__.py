@@ -189,7 +189,7 @@ def gradient_gpu(config: int, m: int, n: int, seed: int, device, dtype):
     k = len(sigma)
     U = _torch_haar(torch, gen, m, k, device)
     V = _torch_haar(torch, gen, n, k, device)
-    sig = torch.tensor(sigma, dtype=torch.float32, device=device)
+    sig = torch.tensor(np.ascontiguousarray(sigma), dtype=torch.float32, device=device)
     G = (U * sig) @ V.T
     if noise:
         G += noise * torch.randn(m, n, generator=gen, device=device, dtype=torch.float32)
