@@ -26,20 +26,23 @@ def bf16_gate(got, exact, emulated, emulated32, what=""):
     well-conditioned inputs, ~1e-2 and more when singular values reach down to
     1e-4 without normalisation).
     1. The GPU is a bf16 realization: its distance to the nearer of the two
-       is within max(TOL_BF16_EMU, 3 * spread).
+       is within max(TOL_BF16_EMU, 3 * spread, inherent / 2). The last term
+       only matters where bf16 arithmetic is far from exact (inherent above
+       the gate): there the tensor cores' accumulation makes a third
+       realization whose drift the float32 emulation does not bound.
     2. The GPU is as accurate as bf16 arithmetic allows: its distance to the
        exact float64 oracle is within TOL_BF16_NS, or, where bf16 arithmetic
        itself cannot meet that (the emulations' own distance `inherent`
-       exceeds it), within inherent + 3 * spread.
+       exceeds it), within 1.05 * inherent + 3 * spread.
     Returns (err_vs_exact, err_vs_emulated, inherent, spread).
     """
     e_emu = min(rel(got, emulated), rel(got, emulated32))
     e_exact = rel(got, exact)
     inherent = max(rel(emulated, exact), rel(emulated32, exact))
     spread = rel(emulated32, emulated)
-    bound1 = max(TOL_BF16_EMU, 3.0 * spread)
+    bound1 = max(TOL_BF16_EMU, 3.0 * spread, 0.5 * inherent if inherent > TOL_BF16_NS else 0.0)
     assert e_emu <= bound1, f"{what}: {e_emu:.3e} from the bf16-rounding oracle (spread {spread:.3e})"
-    bound2 = TOL_BF16_NS if inherent <= TOL_BF16_NS else inherent + 3.0 * spread
+    bound2 = TOL_BF16_NS if inherent <= TOL_BF16_NS else 1.05 * inherent + 3.0 * spread
     assert e_exact <= bound2, (f"{what}: {e_exact:.3e} from the exact oracle "
                                f"(bf16 arithmetic alone: {inherent:.3e}, spread {spread:.3e})")
     return e_exact, e_emu, inherent, spread
