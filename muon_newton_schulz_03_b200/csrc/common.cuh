@@ -132,19 +132,26 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 // Wait for the phase with the given parity to complete. Gives up when the
 // shared error word is set by anyone, or after `timeout_ns` nanoseconds, in
 // which case it records `code` in the error word. Returns false on give-up.
-// (try_wait itself suspends the thread for a short, hardware-defined time
-// while the phase is incomplete, so the loop does not spin hot.)
+// try_wait itself suspends the thread for a short, hardware-defined time
+// while the phase is incomplete, so the loop does not spin hot; the timer is
+// a register read every try, the shared error word (one global address for
+// every waiting warp on the GPU) is read at most every 20 microseconds.
 __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity, int* err,
                                                   uint64_t timeout_ns, int code) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = global_timer_ns();
-  for (uint32_t it = 1;; ++it) {
+  uint64_t next_check = t0 + 20000;
+  for (;;) {
     if (mbar_try_wait(bar, parity)) return true;
-    if (global_timer_ns() - t0 > timeout_ns) {
+    const uint64_t t = global_timer_ns();
+    if (t - t0 > timeout_ns) {
       atomicCAS(err, 0, code);
       return false;
     }
-    if ((it & 7u) == 0u && *reinterpret_cast<volatile int*>(err) != 0) return false;
+    if (t >= next_check) {
+      if (*reinterpret_cast<volatile int*>(err) != 0) return false;
+      next_check = t + 20000;
+    }
   }
 }
 

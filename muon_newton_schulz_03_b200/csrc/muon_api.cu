@@ -61,18 +61,34 @@ struct DevBlob {
   void* dptr = nullptr;
 };
 
+// Builds the bytes of a table on a cache miss.
+typedef int (*BlobBuilder)(const void* ctx, std::vector<unsigned char>& out);
+
 class BlobCache {
  public:
   ~BlobCache() { clear(); }
   // Returns the device copy of `bytes`, uploading it (synchronously) on a miss.
-  int get(const void* bytes, size_t n, void** out) {
-    const unsigned char* b = static_cast<const unsigned char*>(bytes);
+  int get(const void* bytes, size_t n, void** out) { return get_keyed(bytes, n, nullptr, nullptr, out); }
+
+  // Device table identified by `key`; on a miss its bytes come from
+  // build(ctx) (or are the key itself when build is NULL).
+  int get_keyed(const void* key, size_t nkey, BlobBuilder build, const void* ctx, void** out) {
+    const unsigned char* k = static_cast<const unsigned char*>(key);
     for (auto it = entries_.begin(); it != entries_.end(); ++it) {
-      if (it->key.size() == n && std::memcmp(it->key.data(), b, n) == 0) {
+      if (it->key.size() == nkey && std::memcmp(it->key.data(), k, nkey) == 0) {
         entries_.splice(entries_.begin(), entries_, it);
         *out = entries_.front().dptr;
         return MUON_OK;
       }
+    }
+    std::vector<unsigned char> content;
+    const unsigned char* src = k;
+    size_t n = nkey;
+    if (build) {
+      int rc = build(ctx, content);
+      if (rc) return rc;
+      src = content.data();
+      n = content.size();
     }
     if (entries_.size() >= kMax) {
       // The evicted table may still be read by queued work: wait for it.
@@ -81,9 +97,9 @@ class BlobCache {
       entries_.pop_back();
     }
     DevBlob e;
-    e.key.assign(b, b + n);
+    e.key.assign(k, k + nkey);
     MUON_CUDA_TRY(cudaMalloc(&e.dptr, std::max<size_t>(n, 16)));
-    cudaError_t err = cudaMemcpy(e.dptr, b, n, cudaMemcpyHostToDevice);
+    cudaError_t err = cudaMemcpy(e.dptr, src, n, cudaMemcpyHostToDevice);
     if (err != cudaSuccess) {
       cudaFree(e.dptr);
       return fail(MUON_ERR_CUDA, std::string("table upload: ") + cudaGetErrorString(err));
@@ -754,11 +770,25 @@ int muon_newton_schulz(muon_handle* h, const void* const* x_in, void* const* x_o
   }
   const TmapBlob* d_in = nullptr;
   if (esz == 2) {
-    std::vector<TmapBlob> maps((size_t)count * kInMapsPerMat);
-    for (int i = 0; i < count; ++i)
-      if ((rc = encode_x_triple(maps.data() + (size_t)i * kInMapsPerMat, x_in[i], P.mats[i]))) return rc;
+    // Tensor maps of the caller's inputs, cached by the pointer list (the
+    // plan, hence every shape, is fixed while the cache lives).
+    struct InCtx {
+      const void* const* x_in;
+      const DevPlan* plan;
+    } ctx{x_in, &P};
+    auto build = [](const void* c, std::vector<unsigned char>& out) -> int {
+      const InCtx& ic = *static_cast<const InCtx*>(c);
+      const int n = ic.plan->hp.count;
+      out.assign(sizeof(TmapBlob) * kInMapsPerMat * (size_t)n, 0);
+      TmapBlob* maps = reinterpret_cast<TmapBlob*>(out.data());
+      for (int i = 0; i < n; ++i) {
+        const int rc = encode_x_triple(maps + (size_t)i * kInMapsPerMat, ic.x_in[i], ic.plan->mats[i]);
+        if (rc) return rc;
+      }
+      return MUON_OK;
+    };
     void* dm = nullptr;
-    if ((rc = h->in_maps.get(maps.data(), sizeof(TmapBlob) * maps.size(), &dm))) return rc;
+    if ((rc = h->in_maps.get_keyed(x_in, sizeof(void*) * (size_t)count, build, &ctx, &dm))) return rc;
     d_in = static_cast<const TmapBlob*>(dm);
   }
   int res = BUF_IN;
