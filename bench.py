@@ -284,7 +284,7 @@ def run_ours(args):
     k1_bytes = sum(W.step_bytes(m, n, gbytes)[0] for m, n in shapes)
     k4_bytes = sum(W.step_bytes(m, n, gbytes)[1] for m, n in shapes)
 
-    opt = muon.Muon(device=local)
+    opt = muon.Muon(device=local, cta_pair=args.cta_pair)
     stream = torch.cuda.current_stream()
 
     def barrier():
@@ -370,6 +370,7 @@ def run_ours(args):
                 "lr": LR, "beta": BETA, "nesterov": True, "wd": WD, "scale": "moonlight 0.2*sqrt(max(m,n))",
                 "l2": "inputs larger than L2 (params, momenta, grads resident in HBM, no flush needed)",
                 "parallelism": f"replica per GPU x{world} (weak)",
+                "ns_tiles": "256x256 CTA pair (cta_group::2)" if args.cta_pair else "128x256 single CTA",
             },
             "ns_tflops_nominal": ns_tflops,
             "ns_frac_of_datasheet_bf16": (ns_tflops / DATASHEET_BF16_TFLOPS) if ns_tflops else None,
@@ -458,7 +459,7 @@ def run_sweep(args):
     torch.cuda.set_device(device)
     peaks, peak_src = load_peaks()
     batches = set(int(b) for b in args.sweep_batches.split(","))
-    opt = muon.Muon(device=device.index)
+    opt = muon.Muon(device=device.index, cta_pair=args.cta_pair)
     points = []
     for (m, n, batch) in W.sweep_points():
         if batch not in batches:
@@ -515,6 +516,8 @@ def main(argv=None):
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cta-pair", action="store_true",
+                    help="tiled phases on CTA pairs (256 x 256 tiles, cta_group::2) instead of single CTAs")
     args = ap.parse_args(argv)
     args.warmup = max(args.warmup, 3)   # at least three untimed steps
     if args.workload == "sweep":

@@ -111,7 +111,15 @@ typedef struct muon_config {
                                  max(m,n) <= 512 run all iterations in one
                                  on-chip kernel (one CTA each); 0: every
                                  matrix uses the tiled phases. Default 1   */
+  int cta_pair;               /* 1: tiled phases use 256 x 256 tiles on CTA
+                                 pairs (tcgen05 cta_group::2); 0: 128 x 256
+                                 tiles on single CTAs. Default 0 (both
+                                 measure alike on B200 under its power cap) */
 } muon_config;
+
+/* plan_flags of muon_plan_query */
+#define MUON_PLAN_SMALL_PATH 1
+#define MUON_PLAN_CTA_PAIR 2
 
 typedef struct muon_handle muon_handle;
 
@@ -206,7 +214,9 @@ int muon_apply(muon_handle* h, float* const* params, const void* const* o,
 /* ---- Plan, workspace and status ---- */
 
 /* Integer plan tables for a shape table, computed on the host (needs no
- * GPU). small_path as in muon_config. Any output pointer may be NULL.
+ * GPU). plan_flags: MUON_PLAN_SMALL_PATH and MUON_PLAN_CTA_PAIR, as the
+ * small_path and cta_pair fields of muon_config. Any output pointer may be
+ * NULL.
  *   ws_bytes      : total workspace bytes for `ns_precision`.
  *   region_offsets: int64[count][4], byte offsets of X0, X1, A, B.
  *   ntiles        : int32[4], tile counts of the Gram, polynomial and
@@ -218,7 +228,7 @@ int muon_apply(muon_handle* h, float* const* params, const void* const* o,
  *   chunk_prefix  : int64[count+1], elementwise chunks before matrix i.
  * Call once with tiles = NULL to learn ntiles. */
 int muon_plan_query(const int32_t* shapes, int count, int ns_precision,
-                    int small_path, int64_t* ws_bytes, int64_t* region_offsets,
+                    int plan_flags, int64_t* ws_bytes, int64_t* region_offsets,
                     int32_t* ntiles, int32_t* tiles, int64_t* chunk_prefix);
 
 /* Workspace bytes the handle would allocate for this shape table

@@ -86,7 +86,7 @@ def x_layout(m: int, n: int, dtype, device):
     return torch.empty((m, round_up(n, 8)), dtype=dtype, device=device)
 
 
-def plan_query(shapes, ns_precision: str = "bf16", small_path: bool = True):
+def plan_query(shapes, ns_precision: str = "bf16", small_path: bool = True, cta_pair: bool = False):
     """Integer plan tables of a shape table (list of (m, n) or (m, n, flags)).
 
     Returns dict(ws_bytes, region_offsets [count][4], tiles (gram, poly,
@@ -98,7 +98,7 @@ def plan_query(shapes, ns_precision: str = "bf16", small_path: bool = True):
     count = len(sh)
     arr = _shapes_array(sh)
     prec = PRECISIONS[ns_precision]
-    sp = int(bool(small_path))
+    sp = (1 if small_path else 0) | (2 if cta_pair else 0)
     nt = (ctypes.c_int32 * 4)()
     ws = ctypes.c_int64()
     check(lib.muon_plan_query(arr, count, prec, sp, ctypes.byref(ws), None, nt, None, None))
@@ -123,7 +123,8 @@ class Muon:
 
     def __init__(self, device: int = 0, scale_mode: str = "moonlight", extra_scale: float = 1.0,
                  ns_precision: str = "bf16", check_nonfinite: bool = False, num_sms: int = 0,
-                 workspace_cap_bytes: int = 0, wait_timeout_s: float = 2.0, small_path: bool = True):
+                 workspace_cap_bytes: int = 0, wait_timeout_s: float = 2.0, small_path: bool = True,
+                 cta_pair: bool = False):
         self._lib = load()
         cfg = MuonConfig()
         check(self._lib.muon_config_init(ctypes.byref(cfg)))
@@ -135,12 +136,14 @@ class Muon:
         cfg.workspace_cap_bytes = int(workspace_cap_bytes)
         cfg.wait_timeout_s = float(wait_timeout_s)
         cfg.small_path = int(bool(small_path))
+        cfg.cta_pair = int(bool(cta_pair))
         h = ctypes.c_void_p()
         check(self._lib.muon_init(int(device), ctypes.byref(cfg), ctypes.byref(h)))
         self._h = h
         self.device = device
         self.ns_precision = ns_precision
         self.small_path = bool(small_path)
+        self.cta_pair = bool(cta_pair)
 
     # -- lifetime -----------------------------------------------------------
     def close(self):

@@ -76,6 +76,11 @@ cudaError_t launch_ns_small(const NsSmallLaunch& L, int ns_steps, int src_sel, i
                             float c, cudaStream_t st);
 int ns_small_smem_bytes();
 
+cudaError_t launch_ns_phase_pair(const NsLaunch& L, int phase, int src_sel, int dst_sel, int first, float a,
+                                 float b, float c, cudaStream_t st);
+int ns_pair_smem_bytes();
+int ns_pair_clusters_resident();
+
 cudaError_t launch_ns_phase_bf16(const NsLaunch& L, int phase, int src_sel, int dst_sel, int first, float a,
                                  float b, float c, cudaStream_t st);
 

@@ -260,7 +260,7 @@ int ensure_plan(muon_handle* h, const int32_t* shapes, int count) {
 
   auto np = std::make_unique<DevPlan>();
   std::string why;
-  if (!build_plan(shapes, count, h->cfg.ns_precision, h->cfg.small_path != 0, np->hp, why))
+  if (!build_plan(shapes, count, h->cfg.ns_precision, h->cfg.small_path != 0, h->cfg.cta_pair != 0, np->hp, why))
     return fail(MUON_ERR_INVALID_ARG, why);
   np->key = key;
   const HostPlan& hp = np->hp;
@@ -447,7 +447,10 @@ int enqueue_ns(muon_handle* h, const MatBind* d_binds, const std::vector<MatBind
         L.ntiles = (int)hp.tiles[ph].size();
         if (L.ntiles == 0) continue;
         const int slot = prof_before(h, MUON_KERNEL_NS_GRAM + ph, st);
-        MUON_CUDA_TRY(launch_ns_phase_bf16(L, ph, src, dst, first, abc[0], abc[1], abc[2], st));
+        if (hp.tile_m == kTileMPair)
+          MUON_CUDA_TRY(launch_ns_phase_pair(L, ph, src, dst, first, abc[0], abc[1], abc[2], st));
+        else
+          MUON_CUDA_TRY(launch_ns_phase_bf16(L, ph, src, dst, first, abc[0], abc[1], abc[2], st));
         prof_after(h, slot, st);
         ++*launches;
       }
@@ -559,6 +562,7 @@ int muon_config_init(muon_config* cfg) {
   cfg->workspace_cap_bytes = 0;
   cfg->wait_timeout_s = 2.0;
   cfg->small_path = 1;
+  cfg->cta_pair = 0;
   return MUON_OK;
 }
 
@@ -831,12 +835,15 @@ int muon_apply(muon_handle* h, float* const* params, const void* const* o, const
   return MUON_OK;
 }
 
-int muon_plan_query(const int32_t* shapes, int count, int ns_precision, int small_path, int64_t* ws_bytes,
+int muon_plan_query(const int32_t* shapes, int count, int ns_precision, int plan_flags, int64_t* ws_bytes,
                     int64_t* region_offsets, int32_t* ntiles, int32_t* tiles, int64_t* chunk_prefix) {
   g_last_error.clear();
+  if (plan_flags & ~(MUON_PLAN_SMALL_PATH | MUON_PLAN_CTA_PAIR)) return fail(MUON_ERR_INVALID_ARG, "unknown plan flags");
   HostPlan hp;
   std::string why;
-  if (!build_plan(shapes, count, ns_precision, small_path != 0, hp, why)) return fail(MUON_ERR_INVALID_ARG, why);
+  if (!build_plan(shapes, count, ns_precision, (plan_flags & MUON_PLAN_SMALL_PATH) != 0,
+                  (plan_flags & MUON_PLAN_CTA_PAIR) != 0, hp, why))
+    return fail(MUON_ERR_INVALID_ARG, why);
   if (ws_bytes) *ws_bytes = hp.ws_bytes;
   if (region_offsets) std::memcpy(region_offsets, hp.region_off.data(), sizeof(int64_t) * hp.region_off.size());
   if (ntiles) {
@@ -869,7 +876,7 @@ int muon_workspace_size(muon_handle* h, const int32_t* shapes, int count, size_t
   if (!h || !bytes) return fail(MUON_ERR_INVALID_ARG, "handle and bytes are required");
   HostPlan hp;
   std::string why;
-  if (!build_plan(shapes, count, h->cfg.ns_precision, h->cfg.small_path != 0, hp, why))
+  if (!build_plan(shapes, count, h->cfg.ns_precision, h->cfg.small_path != 0, h->cfg.cta_pair != 0, hp, why))
     return fail(MUON_ERR_INVALID_ARG, why);
   *bytes = (size_t)hp.ws_bytes;
   return MUON_OK;

@@ -142,7 +142,7 @@ extern "C" int muon_newton_schulz_noalloc(const void* const* x_in, void* const* 
   const float* abc = coeffs ? coeffs : def;
   HostPlan hp;
   std::string why;
-  if (!build_plan(shapes, count, 0, /*small_path=*/false, hp, why)) return noalloc_fail(MUON_ERR_INVALID_ARG, why);
+  if (!build_plan(shapes, count, 0, /*small_path=*/false, /*pair_tiles=*/false, hp, why)) return noalloc_fail(MUON_ERR_INVALID_ARG, why);
   for (int i = 0; i < count; ++i) {
     const void* a = x_in[i];
     const void* b = x_out[i];

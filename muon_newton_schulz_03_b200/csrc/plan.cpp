@@ -7,9 +7,10 @@
 //    requires; the workspace starts with one double per matrix (sum of
 //    squares) padded to 1024 bytes, followed by all X0, all X1, all A and
 //    all B regions, each aligned to 1024 bytes;
-//  * tiles of 128 x 256: for the symmetric Gram and polynomial outputs only
-//    tiles whose 256-column block is on or right of the 256-block diagonal
-//    (tj >= ti / 2); for the combine every tile, column block outer for wide
+//  * tiles of BM x 256 (BM = 128 for single-CTA tiles, 256 for CTA pairs):
+//    for the symmetric Gram and polynomial outputs only tiles whose
+//    256-column block is on or right of the 256-block diagonal
+//    (tj >= ti * BM / 256); for the combine every tile, column block outer for wide
 //    matrices and row block outer for tall ones (each wave of CTAs then
 //    shares the large X panel in L2); each phase's list is ordered by the
 //    matrix's reduction length, longest first, ties by matrix index;
@@ -29,14 +30,14 @@ namespace {
 int64_t round_up64(int64_t x, int64_t k) { return (x + k - 1) / k * k; }
 int ceil_div_i(int x, int k) { return (x + k - 1) / k; }
 
-void sym_tiles(int mat, int s, std::vector<TileRec>& out) {
-  const int rt = ceil_div_i(s, kTileM), ct = ceil_div_i(s, kTileN);
+void sym_tiles(int mat, int s, int bm, std::vector<TileRec>& out) {
+  const int rt = ceil_div_i(s, bm), ct = ceil_div_i(s, kTileN);
   for (int ti = 0; ti < rt; ++ti)
-    for (int tj = ti / 2; tj < ct; ++tj) out.push_back({mat, ti, tj});
+    for (int tj = ti * bm / kTileN; tj < ct; ++tj) out.push_back({mat, ti, tj});
 }
 
-void comb_tiles(int mat, int m, int n, std::vector<TileRec>& out) {
-  const int rt = ceil_div_i(m, kTileM), ct = ceil_div_i(n, kTileN);
+void comb_tiles(int mat, int m, int n, int bm, std::vector<TileRec>& out) {
+  const int rt = ceil_div_i(m, bm), ct = ceil_div_i(n, kTileN);
   if (m <= n) {
     for (int tj = 0; tj < ct; ++tj)
       for (int ti = 0; ti < rt; ++ti) out.push_back({mat, ti, tj});
@@ -48,13 +49,16 @@ void comb_tiles(int mat, int m, int n, std::vector<TileRec>& out) {
 
 }  // namespace
 
-bool build_plan(const int32_t* shapes, int count, int prec, bool small_path, HostPlan& P, std::string& why) {
+bool build_plan(const int32_t* shapes, int count, int prec, bool small_path, bool pair_tiles, HostPlan& P,
+                std::string& why) {
   if (shapes == nullptr) { why = "shapes is NULL"; return false; }
   if (count < 1) { why = "count must be >= 1"; return false; }
   if (prec != 0 && prec != 1) { why = "ns_precision must be 0 (bf16) or 1 (fp32)"; return false; }
   P = HostPlan();
   P.count = count;
   P.prec = prec;
+  P.tile_m = pair_tiles ? kTileMPair : kTileM;
+  const int bm = P.tile_m;
   P.m.resize(count);
   P.n.resize(count);
   P.mats.resize(count);
@@ -107,11 +111,11 @@ bool build_plan(const int32_t* shapes, int count, int prec, bool small_path, Hos
     return order;
   };
   for (int i : sorted_by([&](int i) { return P.mats[i].l; }))
-    if (!is_small[i]) sym_tiles(i, P.mats[i].s, P.tiles[0]);
+    if (!is_small[i]) sym_tiles(i, P.mats[i].s, bm, P.tiles[0]);
   for (int i : sorted_by([&](int i) { return P.mats[i].s; }))
-    if (!is_small[i]) sym_tiles(i, P.mats[i].s, P.tiles[1]);
+    if (!is_small[i]) sym_tiles(i, P.mats[i].s, bm, P.tiles[1]);
   for (int i : sorted_by([&](int i) { return P.mats[i].s; }))
-    if (!is_small[i]) comb_tiles(i, P.m[i], P.n[i], P.tiles[2]);
+    if (!is_small[i]) comb_tiles(i, P.m[i], P.n[i], bm, P.tiles[2]);
 
   P.prefix.assign((size_t)count + 1, 0);
   for (int i = 0; i < count; ++i)

@@ -11,7 +11,8 @@
 
 namespace muon {
 
-constexpr int kTileM = 128;     // output rows per tile
+constexpr int kTileM = 128;     // output rows per tile (single-CTA tiles)
+constexpr int kTileMPair = 256; // output rows per tile (CTA-pair tiles)
 constexpr int kTileN = 256;     // output columns per tile
 constexpr int kRegionAlign = 1024;
 constexpr int kMaxDim = 1 << 20;
@@ -32,13 +33,16 @@ struct HostPlan {
   int64_t ws_bytes = 0;
   std::vector<TileRec> tiles[3];      // Gram, polynomial, combine
   std::vector<int> small;             // matrices on the on-chip small path
+  int tile_m = kTileM;                // 128 (single CTA) or 256 (CTA pair)
   std::vector<long long> prefix;      // count + 1
 };
 
 // Validates the shape table (m, n in [1, kMaxDim], flags in {0, 1}) and
 // builds the plan. With small_path, matrices with s <= kSmallMaxS and
 // l <= kSmallMaxL go to the on-chip small path instead of the tile lists.
-// Returns false with a message on invalid input.
-bool build_plan(const int32_t* shapes, int count, int prec, bool small_path, HostPlan& out, std::string& why);
+// With pair_tiles the tiles are 256 x 256 (one per CTA pair), else
+// 128 x 256. Returns false with a message on invalid input.
+bool build_plan(const int32_t* shapes, int count, int prec, bool small_path, bool pair_tiles, HostPlan& out,
+                std::string& why);
 
 }  // namespace muon

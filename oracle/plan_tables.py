@@ -20,13 +20,15 @@ The workspace begins with one float64 sum-of-squares accumulator per
 matrix, padded to 1024 bytes; then all X0 regions, all X1
 regions, all A regions, all B regions, each region aligned to 1024 bytes.
 
-Tiles. Output tiles are BM = 128 rows by BN = 256 columns.
+Tiles. Output tiles are BM rows by BN = 256 columns: BM = 128 on single
+CTAs, BM = 256 on CTA pairs.
   * Gram and polynomial (both symmetric s x s): tile (ti, tj) is listed iff
-    tj >= ti // 2, i.e. its 256-wide column block is on or right of the
-    256-block diagonal. Off-diagonal tiles are also written transposed, so
-    each entry is produced once.
+    tj >= ti * BM // 256, i.e. its 256-wide column block is on or right of
+    the 256-block diagonal. Tiles whose column block starts at or after the
+    end of their row block are also written transposed, so each entry is
+    produced once.
   * Combine (output in the original m x n layout): every tile of the
-    ceil(m/128) x ceil(n/256) grid. For wide matrices (m <= n) the column
+    ceil(m/BM) x ceil(n/256) grid. For wide matrices (m <= n) the column
     block is the outer loop, for tall ones the row block.
   Each phase's list is ordered by the matrix's reduction length K
   (descending; Gram: K = l, polynomial and combine: K = s), ties by matrix
@@ -82,16 +84,24 @@ def workspace_layout(shapes, elem_bytes: int = 2):
     return regions, off
 
 
-def _sym_tiles(s: int):
+BM_PAIR = 256
+
+
+def _sym_tiles(s: int, bm: int):
     out = []
-    for ti in range(ceil_div(s, BM)):
-        for tj in range(ti // 2, ceil_div(s, BN)):
+    for ti in range(ceil_div(s, bm)):
+        for tj in range(ti * bm // BN, ceil_div(s, BN)):
             out.append((ti, tj))
     return out
 
 
-def _comb_tiles(m: int, n: int):
-    rows, cols = ceil_div(m, BM), ceil_div(n, BN)
+def mirrored(ti: int, tj: int, bm: int) -> bool:
+    """Whether a symmetric tile is also written transposed."""
+    return tj * BN >= (ti + 1) * bm
+
+
+def _comb_tiles(m: int, n: int, bm: int):
+    rows, cols = ceil_div(m, bm), ceil_div(n, BN)
     if m <= n:   # wide: column block outer
         return [(ti, tj) for tj in range(cols) for ti in range(rows)]
     return [(ti, tj) for ti in range(rows) for tj in range(cols)]
@@ -101,8 +111,9 @@ SMALL_MAX_S = 128
 SMALL_MAX_L = 512
 
 
-def tile_lists(shapes, small_path=True):
+def tile_lists(shapes, small_path=True, pair=False):
     """(gram, poly, comb) lists of (matrix, ti, tj) and the small-path list."""
+    bm = BM_PAIR if pair else BM
     gram, poly, comb = [], [], []
     geo = [matrix_geometry(m, n) for (m, n) in shapes]
     small = [i for i, g in enumerate(geo) if small_path and g[1] <= SMALL_MAX_S and g[2] <= SMALL_MAX_L]
@@ -113,14 +124,14 @@ def tile_lists(shapes, small_path=True):
 
     for i in order(lambda i: geo[i][2]):
         if i in tiled:
-            gram += [(i, ti, tj) for ti, tj in _sym_tiles(geo[i][1])]
+            gram += [(i, ti, tj) for ti, tj in _sym_tiles(geo[i][1], bm)]
     for i in order(lambda i: geo[i][1]):
         if i in tiled:
-            poly += [(i, ti, tj) for ti, tj in _sym_tiles(geo[i][1])]
+            poly += [(i, ti, tj) for ti, tj in _sym_tiles(geo[i][1], bm)]
     for i in order(lambda i: geo[i][1]):
         if i in tiled:
             m, n = shapes[i]
-            comb += [(i, ti, tj) for ti, tj in _comb_tiles(m, n)]
+            comb += [(i, ti, tj) for ti, tj in _comb_tiles(m, n, bm)]
     return gram, poly, comb, small
 
 

@@ -57,13 +57,14 @@ SHAPE_SETS = {
 @pytest.mark.parametrize("name", sorted(SHAPE_SETS))
 @pytest.mark.parametrize("prec", ["bf16", "fp32"])
 @pytest.mark.parametrize("small_path", [True, False])
-def test_plan_tables_bit_exact(name, prec, small_path):
+@pytest.mark.parametrize("pair", [True, False])
+def test_plan_tables_bit_exact(name, prec, small_path, pair):
     shapes = SHAPE_SETS[name]
-    got = muon.plan_query(shapes, prec, small_path)
+    got = muon.plan_query(shapes, prec, small_path, pair)
     regions, ws = PT.workspace_layout(shapes, 2 if prec == "bf16" else 4)
     assert got["ws_bytes"] == ws
     assert got["region_offsets"] == regions
-    gram, poly, comb, small = PT.tile_lists(shapes, small_path)
+    gram, poly, comb, small = PT.tile_lists(shapes, small_path, pair)
     assert got["tiles"][0] == gram
     assert got["tiles"][1] == poly
     assert got["tiles"][2] == comb
@@ -71,25 +72,28 @@ def test_plan_tables_bit_exact(name, prec, small_path):
     assert got["chunk_prefix"] == PT.chunk_prefix(shapes)
 
 
-@pytest.mark.parametrize("shape", [(1, 1), (5, 3), (130, 300), (300, 130), (512, 512), (600, 257), (257, 600)])
-def test_tiles_cover_each_entry_once(shape):
+@pytest.mark.parametrize("shape", [(1, 1), (5, 3), (130, 300), (300, 130), (512, 512), (600, 257), (257, 600),
+                                   (1000, 700)])
+@pytest.mark.parametrize("pair", [False, True])
+def test_tiles_cover_each_entry_once(shape, pair):
     m, n = shape
-    got = muon.plan_query([shape], small_path=False)
+    bm = PT.BM_PAIR if pair else PT.BM
+    got = muon.plan_query([shape], small_path=False, cta_pair=pair)
     s = min(m, n)
     # Symmetric phases: direct writes of each listed tile plus transposed
-    # writes of the tiles strictly right of the 256-block diagonal.
+    # writes of the tiles whose column block starts after their row block.
     for tiles in got["tiles"][:2]:
         cover = np.zeros((s, s), dtype=np.int64)
         for (_, ti, tj) in tiles:
-            r0, c0 = ti * PT.BM, tj * PT.BN
-            r1, c1 = min(r0 + PT.BM, s), min(c0 + PT.BN, s)
+            r0, c0 = ti * bm, tj * PT.BN
+            r1, c1 = min(r0 + bm, s), min(c0 + PT.BN, s)
             cover[r0:r1, c0:c1] += 1
-            if tj > ti // 2:
+            if PT.mirrored(ti, tj, bm):
                 cover[c0:c1, r0:r1] += 1
         assert np.all(cover == 1)
     cover = np.zeros((m, n), dtype=np.int64)
     for (_, ti, tj) in got["tiles"][2]:
-        cover[ti * PT.BM:(ti + 1) * PT.BM, tj * PT.BN:(tj + 1) * PT.BN] += 1
+        cover[ti * bm:(ti + 1) * bm, tj * PT.BN:(tj + 1) * PT.BN] += 1
     assert np.all(cover == 1)
 
 
@@ -125,6 +129,8 @@ def test_plan_rejects_empty_and_bad_precision():
     assert lib.muon_plan_query(arr, 1, 7, 1, None, None, None, None, None) == 1
     assert lib.muon_plan_query(None, 1, 0, 1, None, None, None, None, None) == 1
     assert b"shapes" in lib.muon_last_error()
+    assert lib.muon_plan_query(arr, 1, 0, 8, None, None, None, None, None) == 1
+    assert b"flags" in lib.muon_last_error()
 
 
 def test_config_defaults():
@@ -133,7 +139,7 @@ def test_config_defaults():
     import ctypes
     assert lib.muon_config_init(ctypes.byref(cfg)) == 0
     assert cfg.scale_mode == 0 and cfg.extra_scale == 1.0 and cfg.ns_precision == 0
-    assert cfg.wait_timeout_s == 2.0 and cfg.num_sms == 0 and cfg.small_path == 1
+    assert cfg.wait_timeout_s == 2.0 and cfg.num_sms == 0 and cfg.small_path == 1 and cfg.cta_pair == 0
     assert lib.muon_config_init(None) == 1
 
 

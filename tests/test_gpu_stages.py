@@ -29,6 +29,15 @@ def opt_bf16():
 
 
 @pytest.fixture(scope="module")
+def opts():
+    """Handles for both tiled-phase kernels: single CTAs (default) and CTA pairs."""
+    hs = {"pair": muon.Muon(device=0, cta_pair=True), "single": muon.Muon(device=0)}
+    yield hs
+    for h in hs.values():
+        h.close()
+
+
+@pytest.fixture(scope="module")
 def opt_fp32():
     h = muon.Muon(device=0, ns_precision="fp32")
     yield h
@@ -161,9 +170,11 @@ def _ns_inputs(shapes, seed, scale=1.0):
     return xin, x64
 
 
-def test_ns_identity_combine_is_exact(opt_bf16):
+@pytest.mark.parametrize("kind", ["pair", "single"])
+def test_ns_identity_combine_is_exact(opts, kind):
     # (a, b, c) = (1, 0, 0): B = 0, so X1 = 1 * X + 0 * X exactly. Exercises
     # every tile's combine epilogue addressing (direct, ragged tails, tall).
+    opt_bf16 = opts[kind]
     shapes = RAGGED
     xin, x64 = _ns_inputs(shapes, 5)
     xout = [x_buffer(m, n) for (m, n) in shapes]
@@ -174,8 +185,10 @@ def test_ns_identity_combine_is_exact(opt_bf16):
     _assert_status_clean(opt_bf16)
 
 
+@pytest.mark.parametrize("kind", ["pair", "single"])
 @pytest.mark.parametrize("coeffs", [(0.0, 1.0, 0.0), (0.0, 0.0, 1.0), (0.5, -0.25, 0.125)])
-def test_ns_single_step_phases(opt_bf16, coeffs):
+def test_ns_single_step_phases(opts, kind, coeffs):
+    opt_bf16 = opts[kind]
     # One step with chosen coefficients isolates the Gram (b), the polynomial
     # product (c) and the combine (a) against float64 products of the same
     # bf16 input; alpha = 1 (no norm).
@@ -193,8 +206,10 @@ def test_ns_single_step_phases(opt_bf16, coeffs):
     _assert_status_clean(opt_bf16)
 
 
+@pytest.mark.parametrize("kind", ["pair", "single"])
 @pytest.mark.parametrize("steps", [1, 2, 5])
-def test_ns_bf16_matches_oracle(opt_bf16, steps):
+def test_ns_bf16_matches_oracle(opts, kind, steps):
+    opt_bf16 = opts[kind]
     shapes = RAGGED
     xin, x64 = _ns_inputs(shapes, 7 + steps)
     sumsq = torch.tensor([np.sum(x ** 2) for x in x64], dtype=torch.float64, device=DEV)
@@ -244,11 +259,13 @@ def test_ns_fp32_matches_oracle(opt_fp32, steps):
         assert rel(got, ref) <= TOL_FP32_NS, f"matrix {i} {m}x{n}: {rel(got, ref):.3e}"
 
 
-def test_ns_gram_is_symmetric_in_workspace(opt_bf16):
+@pytest.mark.parametrize("kind", ["pair", "single"])
+def test_ns_gram_is_symmetric_in_workspace(opts, kind):
     # The Gram tiles right of the diagonal are mirrored: A must be exactly
     # symmetric, and equal to the float64 Gram of the bf16 input at bf16 level.
     from gpu_helpers import workspace_matrix
-    shapes = [(600, 900), (900, 600), (513, 513)]
+    opt_bf16 = opts[kind]
+    shapes = [(600, 900), (900, 600), (513, 513), (1100, 300)]
     xin, x64 = _ns_inputs(shapes, 11, scale=0.03)
     xout = [x_buffer(m, n) for (m, n) in shapes]
     opt_bf16.newton_schulz(xin, xout, shapes, None, ns_steps=1)

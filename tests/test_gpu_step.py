@@ -77,11 +77,12 @@ def test_single_matrix_workload(prec, tol):
     opt.close()
 
 
-@pytest.mark.parametrize("prec,tol", [("bf16", TOL_BF16_NS), ("fp32", TOL_FP32_NS)])
-def test_gpt2_small_set(prec, tol):
+@pytest.mark.parametrize("prec,tol,pair", [("bf16", TOL_BF16_NS, True), ("bf16", TOL_BF16_NS, False),
+                                           ("fp32", TOL_FP32_NS, True)])
+def test_gpt2_small_set(prec, tol, pair):
     shapes = W.gpt2_shapes()
     cpu, dev = make_set(W.CONFIG_GPT2, shapes, torch.float32)
-    opt = muon.Muon(device=0, ns_precision=prec)
+    opt = muon.Muon(device=0, ns_precision=prec, cta_pair=pair)
     opt.step([d[0] for d in dev], [d[1] for d in dev], [d[2] for d in dev], lr=2e-4, beta=0.95, wd=0.1)
     torch.cuda.synchronize()
     idx = range(len(shapes)) if prec == "bf16" else range(4)
