@@ -445,8 +445,8 @@ def run_e2e(torch, muon, opt, shapes, params, grads, moms, args, device, world, 
         return {"value": None, "unit": "steps/s", "error": f"device status {code}"}
     return {"value": world * 1e3 / ms, "unit": "steps/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
             "ms_per_step": ms, "steps": steps,
-            "path": "muon_step_host: params, grads, momenta in pinned host memory; H2D, step, D2H of params and "
-                    "momenta on one stream"}
+            "path": "muon_step_host: params, grads, momenta in pinned host memory; 8 chunks pipelined over "
+                    "copy-in, compute and copy-out streams; the caller's stream waits for the last copy-out"}
 
 
 def run_sweep(args):

@@ -165,12 +165,16 @@ int muon_step(muon_handle* h, float* const* params, const void* const* grads,
               float lr, float beta, int nesterov, float wd, int ns_steps,
               const float* coeffs, void* stream);
 
-/* Same step with every tensor in HOST memory (pinned memory gives
- * asynchronous copies): the library copies params, grads and momenta to
- * its own device staging area, runs muon_step there and copies params and
- * momenta back, all on `stream`. The host buffers must stay valid and
- * untouched until the stream completes. Staging is allocated on first use
- * per shape table and counts against the workspace cap. */
+/* Same step with every tensor in HOST memory. The matrices are split into
+ * up to 8 chunks of consecutive matrices with about equal element counts;
+ * while chunk c is computed, chunk c+1 is copied in and chunk c-1 copied
+ * out, on three library streams (copy-in, compute, copy-out) that start
+ * after the work already queued on `stream`; `stream` waits for the last
+ * copy-out. Pinned host memory is needed for the copies to overlap. Only
+ * matrices with a gradient are copied. The host buffers must stay valid and
+ * untouched until `stream` reaches that point, and calls on one handle must
+ * be ordered by the caller (one stream). Staging (three chunk slots) is
+ * allocated on first use per shape table and counts against the cap. */
 int muon_step_host(muon_handle* h, float* const* params,
                    const void* const* grads, float* const* momenta,
                    const int32_t* shapes, int count, float lr, float beta,

@@ -108,11 +108,11 @@ __device__ __forceinline__ float momentum_u(float g, float& m, float beta, float
 template <bool kFp32Out>
 __global__ void __launch_bounds__(kThreads) k1_momentum_norm(
     const MatPlan* __restrict__ plans, const MatBind* __restrict__ binds, const long long* __restrict__ prefix,
-    int count, int ysel, float beta, int nesterov, double* __restrict__ sumsq, DevStatus* status,
-    int check_nonfinite) {
+    int count, long long block_base, int ysel, float beta, int nesterov, double* __restrict__ sumsq,
+    DevStatus* status, int check_nonfinite) {
   __shared__ double red[kThreads / 32];
   __shared__ unsigned redc[kThreads / 32];
-  const long long blk = blockIdx.x;
+  const long long blk = (long long)blockIdx.x + block_base;
   const int mat = find_matrix(prefix, count, blk);
   const MatBind mb = binds[mat];
   if (!mb.active || mb.g == nullptr) return;
@@ -183,10 +183,11 @@ __device__ __forceinline__ float update_scale_dev(int m, int n, int mode, float 
 template <bool kFp32In>
 __global__ void __launch_bounds__(kThreads) k4_apply(const MatPlan* __restrict__ plans,
                                                      const MatBind* __restrict__ binds,
-                                                     const long long* __restrict__ prefix, int count, int osel,
-                                                     float lr, float wd, int scale_mode, float extra_scale,
+                                                     const long long* __restrict__ prefix, int count,
+                                                     long long block_base, int osel, float lr, float wd,
+                                                     int scale_mode, float extra_scale,
                                                      const double* __restrict__ sumsq) {
-  const long long blk = blockIdx.x;
+  const long long blk = (long long)blockIdx.x + block_base;
   const int mat = find_matrix(prefix, count, blk);
   const MatBind mb = binds[mat];
   if (!mb.active) return;
@@ -225,8 +226,9 @@ template <bool kFp32>
 __global__ void __launch_bounds__(kThreads) k0_scale_copy(const MatPlan* __restrict__ plans,
                                                           const MatBind* __restrict__ binds,
                                                           const long long* __restrict__ prefix, int count,
-                                                          int isel, int osel, const double* __restrict__ sumsq) {
-  const long long blk = blockIdx.x;
+                                                          long long block_base, int isel, int osel,
+                                                          const double* __restrict__ sumsq) {
+  const long long blk = (long long)blockIdx.x + block_base;
   const int mat = find_matrix(prefix, count, blk);
   const MatBind mb = binds[mat];
   if (!mb.active) return;
@@ -252,11 +254,11 @@ cudaError_t launch_momentum_norm(const ElemLaunch& L, int ysel, float beta, int 
                                  DevStatus* status, int check_nonfinite, bool fp32_out, cudaStream_t st) {
   if (L.nblocks <= 0) return cudaSuccess;
   if (fp32_out)
-    k1_momentum_norm<true><<<(unsigned)L.nblocks, kThreads, 0, st>>>(L.plans, L.binds, L.prefix, L.count, ysel,
+    k1_momentum_norm<true><<<(unsigned)L.nblocks, kThreads, 0, st>>>(L.plans, L.binds, L.prefix, L.count, L.block_base, ysel,
                                                                       beta, nesterov, sumsq, status,
                                                                       check_nonfinite);
   else
-    k1_momentum_norm<false><<<(unsigned)L.nblocks, kThreads, 0, st>>>(L.plans, L.binds, L.prefix, L.count, ysel,
+    k1_momentum_norm<false><<<(unsigned)L.nblocks, kThreads, 0, st>>>(L.plans, L.binds, L.prefix, L.count, L.block_base, ysel,
                                                                        beta, nesterov, sumsq, status,
                                                                        check_nonfinite);
   return cudaGetLastError();
@@ -266,10 +268,10 @@ cudaError_t launch_apply(const ElemLaunch& L, int osel, float lr, float wd, int 
                          const double* sumsq, bool fp32_in, cudaStream_t st) {
   if (L.nblocks <= 0) return cudaSuccess;
   if (fp32_in)
-    k4_apply<true><<<(unsigned)L.nblocks, kThreads, 0, st>>>(L.plans, L.binds, L.prefix, L.count, osel, lr, wd,
+    k4_apply<true><<<(unsigned)L.nblocks, kThreads, 0, st>>>(L.plans, L.binds, L.prefix, L.count, L.block_base, osel, lr, wd,
                                                              scale_mode, extra_scale, sumsq);
   else
-    k4_apply<false><<<(unsigned)L.nblocks, kThreads, 0, st>>>(L.plans, L.binds, L.prefix, L.count, osel, lr, wd,
+    k4_apply<false><<<(unsigned)L.nblocks, kThreads, 0, st>>>(L.plans, L.binds, L.prefix, L.count, L.block_base, osel, lr, wd,
                                                               scale_mode, extra_scale, sumsq);
   return cudaGetLastError();
 }
@@ -278,10 +280,10 @@ cudaError_t launch_scale_copy(const ElemLaunch& L, int isel, int osel, const dou
                               cudaStream_t st) {
   if (L.nblocks <= 0) return cudaSuccess;
   if (fp32)
-    k0_scale_copy<true><<<(unsigned)L.nblocks, kThreads, 0, st>>>(L.plans, L.binds, L.prefix, L.count, isel, osel,
+    k0_scale_copy<true><<<(unsigned)L.nblocks, kThreads, 0, st>>>(L.plans, L.binds, L.prefix, L.count, L.block_base, isel, osel,
                                                                   sumsq);
   else
-    k0_scale_copy<false><<<(unsigned)L.nblocks, kThreads, 0, st>>>(L.plans, L.binds, L.prefix, L.count, isel,
+    k0_scale_copy<false><<<(unsigned)L.nblocks, kThreads, 0, st>>>(L.plans, L.binds, L.prefix, L.count, L.block_base, isel,
                                                                    osel, sumsq);
   return cudaGetLastError();
 }

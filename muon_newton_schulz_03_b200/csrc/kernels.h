@@ -15,7 +15,8 @@ struct ElemLaunch {
   const MatBind* binds;     // device
   const long long* prefix;  // device, count + 1 entries
   int count;
-  long long nblocks;        // prefix[count]
+  long long block_base;     // first chunk of the launch (0 for a whole set)
+  long long nblocks;        // chunks in the launch (prefix[count] for a whole set)
 };
 
 cudaError_t launch_momentum_norm(const ElemLaunch& L, int ysel, float beta, int nesterov, double* sumsq,

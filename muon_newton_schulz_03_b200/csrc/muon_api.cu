@@ -185,10 +185,32 @@ struct DevPlan {
   int* d_small = nullptr;
   TmapBlob* d_maps = nullptr;
   std::vector<MatPlan> mats;         // host copy with workspace pointers
-  void* staging = nullptr;           // muon_step_host buffers
+  // Chunks for the pipelined host-buffer step: consecutive matrices with
+  // about equal element counts, each with its own slice of every tile list.
+  std::vector<int> chunk_bounds;                 // nchunks + 1
+  int4* d_chunk_tiles[3] = {nullptr, nullptr, nullptr};
+  std::vector<int> chunk_tile_off[3];            // nchunks + 1 each
+  int* d_chunk_small = nullptr;
+  std::vector<int> chunk_small_off;              // nchunks + 1
+  void* staging = nullptr;                       // muon_step_host: kStagingSlots slots
   size_t staging_size = 0;
-  std::vector<int64_t> staging_off;  // count * 3: param, grad, momentum
+  size_t slot_bytes = 0;
+  std::vector<int64_t> staging_off;              // count * 3: param, grad, momentum (within the slot)
 };
+
+// Work of one enqueue: matrices [m0, m1), elementwise chunks [blk0, blk1),
+// and the matching tile lists.
+struct WorkRange {
+  int m0 = 0, m1 = 0;
+  long long blk0 = 0, blk1 = 0;
+  const int4* tiles[3] = {nullptr, nullptr, nullptr};
+  int ntiles[3] = {0, 0, 0};
+  const int* small = nullptr;
+  int nsmall = 0;
+};
+
+constexpr int kHostChunks = 8;      // chunks of the pipelined host-buffer step
+constexpr int kStagingSlots = 3;    // staging slots in flight (H2D, compute, D2H)
 
 struct muon_handle {
   int device = 0;
@@ -206,6 +228,9 @@ struct muon_handle {
   int prof_used = 0;                  // kernels recorded so far
   int prof_calls_left = 0;            // calls that still record
   bool prof_this_call = false;
+  // Pipelined host-buffer step: copy-in, compute and copy-out streams.
+  cudaStream_t hs[3] = {nullptr, nullptr, nullptr};
+  std::vector<cudaEvent_t> hev;       // 3 per chunk + 1
 };
 
 namespace {
@@ -306,6 +331,49 @@ int ensure_plan(muon_handle* h, const int32_t* shapes, int count) {
   }
   const int64_t o_small = off;
   off = align_up(off + (int64_t)sizeof(int) * std::max<size_t>(hp.small.size(), 1), 256);
+  // Chunk partition and per-chunk slices of the tile lists.
+  {
+    const int nch = std::min(count, kHostChunks);
+    long long total = 0;
+    for (int i = 0; i < count; ++i) total += np->mats[i].numel;
+    np->chunk_bounds.assign(1, 0);
+    long long cum = 0;
+    for (int i = 0; i < count; ++i) {
+      cum += np->mats[i].numel;
+      const int made = (int)np->chunk_bounds.size() - 1;
+      const int left_m = count - (i + 1), left_c = nch - (made + 1);
+      if (made + 1 < nch && (cum * nch >= total * (long long)(made + 1) || left_m == left_c))
+        np->chunk_bounds.push_back(i + 1);
+    }
+    np->chunk_bounds.push_back(count);
+  }
+  const int nch = (int)np->chunk_bounds.size() - 1;
+  std::vector<int> chunk_of((size_t)count);
+  for (int c = 0; c < nch; ++c)
+    for (int i = np->chunk_bounds[c]; i < np->chunk_bounds[c + 1]; ++i) chunk_of[i] = c;
+  std::vector<TileRec> chunk_tiles[3];
+  for (int p = 0; p < 3; ++p) {
+    np->chunk_tile_off[p].assign(1, 0);
+    for (int c = 0; c < nch; ++c) {
+      for (const TileRec& t : hp.tiles[p])
+        if (chunk_of[t.mat] == c) chunk_tiles[p].push_back(t);
+      np->chunk_tile_off[p].push_back((int)chunk_tiles[p].size());
+    }
+  }
+  std::vector<int> chunk_small;
+  np->chunk_small_off.assign(1, 0);
+  for (int c = 0; c < nch; ++c) {
+    for (int i : hp.small)
+      if (chunk_of[i] == c) chunk_small.push_back(i);
+    np->chunk_small_off.push_back((int)chunk_small.size());
+  }
+  int64_t o_ctiles[3];
+  for (int p = 0; p < 3; ++p) {
+    o_ctiles[p] = off;
+    off = align_up(off + (int64_t)sizeof(int4) * std::max<size_t>(chunk_tiles[p].size(), 1), 256);
+  }
+  const int64_t o_csmall = off;
+  off = align_up(off + (int64_t)sizeof(int) * std::max<size_t>(chunk_small.size(), 1), 256);
   const int64_t o_maps = off;
   if (bf16) off = align_up(off + (int64_t)sizeof(TmapBlob) * kMapsPerMat * count, 256);
   std::vector<unsigned char> host((size_t)off, 0);
@@ -317,6 +385,13 @@ int ensure_plan(muon_handle* h, const int32_t* shapes, int count) {
       t[k] = make_int4(hp.tiles[p][k].mat, hp.tiles[p][k].ti, hp.tiles[p][k].tj, 0);
   }
   if (!hp.small.empty()) std::memcpy(host.data() + o_small, hp.small.data(), sizeof(int) * hp.small.size());
+  for (int p = 0; p < 3; ++p) {
+    int4* t = reinterpret_cast<int4*>(host.data() + o_ctiles[p]);
+    for (size_t k = 0; k < chunk_tiles[p].size(); ++k)
+      t[k] = make_int4(chunk_tiles[p][k].mat, chunk_tiles[p][k].ti, chunk_tiles[p][k].tj, 0);
+  }
+  if (!chunk_small.empty())
+    std::memcpy(host.data() + o_csmall, chunk_small.data(), sizeof(int) * chunk_small.size());
   if (bf16) {
     TmapBlob* maps = reinterpret_cast<TmapBlob*>(host.data() + o_maps);
     for (int i = 0; i < count; ++i) {
@@ -347,6 +422,8 @@ int ensure_plan(muon_handle* h, const int32_t* shapes, int count) {
   np->d_prefix = reinterpret_cast<long long*>(tb + o_pref);
   for (int p = 0; p < 3; ++p) np->d_tiles[p] = reinterpret_cast<int4*>(tb + o_tiles[p]);
   np->d_small = reinterpret_cast<int*>(tb + o_small);
+  for (int p = 0; p < 3; ++p) np->d_chunk_tiles[p] = reinterpret_cast<int4*>(tb + o_ctiles[p]);
+  np->d_chunk_small = reinterpret_cast<int*>(tb + o_csmall);
   np->d_maps = bf16 ? reinterpret_cast<TmapBlob*>(tb + o_maps) : nullptr;
   h->plan = std::move(np);
   return MUON_OK;
@@ -395,21 +472,59 @@ ElemLaunch elem_launch(const DevPlan& P, const MatBind* d_binds) {
   L.binds = d_binds;
   L.prefix = P.d_prefix;
   L.count = P.hp.count;
+  L.block_base = 0;
   L.nblocks = P.hp.prefix[P.hp.count];
   return L;
+}
+
+ElemLaunch elem_launch(const DevPlan& P, const MatBind* d_binds, const WorkRange& R) {
+  ElemLaunch L = elem_launch(P, d_binds);
+  L.block_base = R.blk0;
+  L.nblocks = R.blk1 - R.blk0;
+  return L;
+}
+
+WorkRange full_range(const DevPlan& P) {
+  WorkRange R;
+  R.m0 = 0;
+  R.m1 = P.hp.count;
+  R.blk0 = 0;
+  R.blk1 = P.hp.prefix[P.hp.count];
+  for (int p = 0; p < 3; ++p) {
+    R.tiles[p] = P.d_tiles[p];
+    R.ntiles[p] = (int)P.hp.tiles[p].size();
+  }
+  R.small = P.d_small;
+  R.nsmall = (int)P.hp.small.size();
+  return R;
+}
+
+WorkRange chunk_range(const DevPlan& P, int c) {
+  WorkRange R;
+  R.m0 = P.chunk_bounds[c];
+  R.m1 = P.chunk_bounds[c + 1];
+  R.blk0 = P.hp.prefix[R.m0];
+  R.blk1 = P.hp.prefix[R.m1];
+  for (int p = 0; p < 3; ++p) {
+    R.tiles[p] = P.d_chunk_tiles[p] + P.chunk_tile_off[p][c];
+    R.ntiles[p] = P.chunk_tile_off[p][c + 1] - P.chunk_tile_off[p][c];
+  }
+  R.small = P.d_chunk_small + P.chunk_small_off[c];
+  R.nsmall = P.chunk_small_off[c + 1] - P.chunk_small_off[c];
+  return R;
 }
 
 // Enqueue `ns_steps` Newton-Schulz iterations. The input of step 1 is
 // `first_src`; intermediate results alternate X1, X0, X1, ...; the result of
 // the last step goes to `last_dst` (or stays in the ping-pong buffers when
 // last_dst < 0). *result receives the selector of the result buffer.
-int enqueue_ns(muon_handle* h, const MatBind* d_binds, const std::vector<MatBind>& hbinds,
+int enqueue_ns(muon_handle* h, const MatBind* d_binds, const std::vector<MatBind>& hbinds, const WorkRange& R,
                const TmapBlob* d_in_maps, const double* sumsq, int ns_steps, const float* abc, int first_src,
                int last_dst, cudaStream_t st, int* launches, int* result) {
   DevPlan& P = *h->plan;
   const HostPlan& hp = P.hp;
   const bool bf16 = h->cfg.ns_precision == MUON_NS_BF16;
-  if (bf16 && ns_steps > 0 && !hp.small.empty()) {
+  if (bf16 && ns_steps > 0 && R.nsmall > 0) {
     // Matrices on the small path run every iteration in one launch and land
     // in the same buffer as the others' last step.
     NsSmallLaunch S;
@@ -417,8 +532,8 @@ int enqueue_ns(muon_handle* h, const MatBind* d_binds, const std::vector<MatBind
     S.binds = d_binds;
     S.maps = P.d_maps;
     S.in_maps = d_in_maps;
-    S.mats = P.d_small;
-    S.nmats = (int)hp.small.size();
+    S.mats = R.small;
+    S.nmats = R.nsmall;
     S.sumsq = sumsq;
     S.status = h->status;
     S.timeout_ns = (unsigned long long)(h->cfg.wait_timeout_s * 1e9);
@@ -443,8 +558,8 @@ int enqueue_ns(muon_handle* h, const MatBind* d_binds, const std::vector<MatBind
       L.grid = h->num_sms;
       L.timeout_ns = (unsigned long long)(h->cfg.wait_timeout_s * 1e9);
       for (int ph = 0; ph < 3; ++ph) {
-        L.tiles = P.d_tiles[ph];
-        L.ntiles = (int)hp.tiles[ph].size();
+        L.tiles = R.tiles[ph];
+        L.ntiles = R.ntiles[ph];
         if (L.ntiles == 0) continue;
         const int slot = prof_before(h, MUON_KERNEL_NS_GRAM + ph, st);
         if (hp.tile_m == kTileMPair)
@@ -455,7 +570,7 @@ int enqueue_ns(muon_handle* h, const MatBind* d_binds, const std::vector<MatBind
         ++*launches;
       }
     } else {
-      for (int i = 0; i < hp.count; ++i) {
+      for (int i = R.m0; i < R.m1; ++i) {
         if (!hbinds[i].active) continue;
         const MatPlan& mp = P.mats[i];
         const float* s_ptr = static_cast<const float*>(sel_buf(mp, hbinds[i], src));
@@ -499,13 +614,10 @@ int check_scalars(float lr, float beta, float wd) {
   return MUON_OK;
 }
 
-int step_impl(muon_handle* h, float* const* params, const void* const* grads, float* const* momenta,
-              const int32_t* shapes, int count, float lr, float beta, int nesterov, float wd, int ns_steps,
-              const float* abc, cudaStream_t st) {
-  int rc;
-  if ((rc = ensure_plan(h, shapes, count))) return rc;
-  DevPlan& P = *h->plan;
-  std::vector<MatBind> hb((size_t)count);
+// Device pointer table of a step (cached by content).
+int step_binds(muon_handle* h, float* const* params, const void* const* grads, float* const* momenta,
+               const int32_t* shapes, int count, std::vector<MatBind>& hb, const MatBind** db) {
+  hb.assign((size_t)count, MatBind());
   for (int i = 0; i < count; ++i) {
     MatBind& b = hb[i];
     std::memset(&b, 0, sizeof(b));
@@ -516,26 +628,50 @@ int step_impl(muon_handle* h, float* const* params, const void* const* grads, fl
     b.active = grads[i] != nullptr;
   }
   void* d_binds = nullptr;
+  int rc;
   if ((rc = h->binds.get(hb.data(), sizeof(MatBind) * count, &d_binds))) return rc;
-  const MatBind* db = static_cast<const MatBind*>(d_binds);
+  *db = static_cast<const MatBind*>(d_binds);
+  return MUON_OK;
+}
+
+// Momentum/norm/cast, Newton-Schulz and apply for the matrices of R.
+int enqueue_step_range(muon_handle* h, const MatBind* db, const std::vector<MatBind>& hb, const WorkRange& R,
+                       float lr, float beta, int nesterov, float wd, int ns_steps, const float* abc, cudaStream_t st,
+                       int* launches) {
+  DevPlan& P = *h->plan;
   double* sumsq = static_cast<double*>(P.ws);
   const bool fp32 = h->cfg.ns_precision == MUON_NS_FP32;
-  int launches = 0;
-  MUON_CUDA_TRY(cudaMemsetAsync(sumsq, 0, sizeof(double) * count, st));
-  const ElemLaunch EL = elem_launch(P, db);
-  prof_call_begin(h);
+  int rc;
+  MUON_CUDA_TRY(cudaMemsetAsync(sumsq + R.m0, 0, sizeof(double) * (size_t)(R.m1 - R.m0), st));
+  const ElemLaunch EL = elem_launch(P, db, R);
   int slot = prof_before(h, MUON_KERNEL_MOMENTUM_NORM, st);
   MUON_CUDA_TRY(launch_momentum_norm(EL, BUF_X0, beta, nesterov ? 1 : 0, sumsq, h->status, h->cfg.check_nonfinite,
                                      fp32, st));
   prof_after(h, slot, st);
-  ++launches;
+  ++*launches;
   int res = BUF_X0;
-  if ((rc = enqueue_ns(h, db, hb, nullptr, sumsq, ns_steps, abc, BUF_X0, -1, st, &launches, &res))) return rc;
+  if ((rc = enqueue_ns(h, db, hb, R, nullptr, sumsq, ns_steps, abc, BUF_X0, -1, st, launches, &res))) return rc;
   slot = prof_before(h, MUON_KERNEL_APPLY, st);
   MUON_CUDA_TRY(launch_apply(EL, res, lr, wd, h->cfg.scale_mode, h->cfg.extra_scale, ns_steps == 0 ? sumsq : nullptr,
                              fp32, st));
   prof_after(h, slot, st);
-  ++launches;
+  ++*launches;
+  return MUON_OK;
+}
+
+int step_impl(muon_handle* h, float* const* params, const void* const* grads, float* const* momenta,
+              const int32_t* shapes, int count, float lr, float beta, int nesterov, float wd, int ns_steps,
+              const float* abc, cudaStream_t st) {
+  int rc;
+  if ((rc = ensure_plan(h, shapes, count))) return rc;
+  std::vector<MatBind> hb;
+  const MatBind* db = nullptr;
+  if ((rc = step_binds(h, params, grads, momenta, shapes, count, hb, &db))) return rc;
+  int launches = 0;
+  prof_call_begin(h);
+  if ((rc = enqueue_step_range(h, db, hb, full_range(*h->plan), lr, beta, nesterov, wd, ns_steps, abc, st,
+                               &launches)))
+    return rc;
   h->last_launches = launches;
   return MUON_OK;
 }
@@ -609,6 +745,9 @@ int muon_destroy(muon_handle* h) {
     h->in_maps.clear();
     if (h->plan) free_plan(h->plan.get());
     prof_free(h);
+    for (cudaEvent_t e : h->hev) cudaEventDestroy(e);
+    for (int k = 0; k < 3; ++k)
+      if (h->hs[k]) cudaStreamDestroy(h->hs[k]);
     cudaFree(h->status);
   }
   delete h;
@@ -647,48 +786,100 @@ int muon_step_host(muon_handle* h, float* const* params, const void* const* grad
   if (!g.ok) return fail(MUON_ERR_CUDA, "cudaSetDevice failed");
   if ((rc = ensure_plan(h, shapes, count))) return rc;
   DevPlan& P = *h->plan;
+  const int nch = (int)P.chunk_bounds.size() - 1;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
+
+  // Staging: kStagingSlots slots, each holding one chunk's params, grads and
+  // momenta (4 bytes per element each); chunk c uses slot c % kStagingSlots.
   if (!P.staging) {
     P.staging_off.assign((size_t)count * 3, 0);
-    int64_t off = 0;
-    for (int i = 0; i < count; ++i) {
-      const int64_t numel = P.mats[i].numel;
-      for (int k = 0; k < 3; ++k) {
-        P.staging_off[(size_t)i * 3 + k] = off;
-        off = align_up(off + numel * 4, 256);
-      }
+    size_t slot = 0;
+    for (int c = 0; c < nch; ++c) {
+      int64_t off = 0;
+      for (int i = P.chunk_bounds[c]; i < P.chunk_bounds[c + 1]; ++i)
+        for (int k = 0; k < 3; ++k) {
+          P.staging_off[(size_t)i * 3 + k] = off;
+          off = align_up(off + P.mats[i].numel * 4, 256);
+        }
+      slot = std::max(slot, (size_t)off);
     }
-    if (h->cfg.workspace_cap_bytes && (size_t)(off + P.hp.ws_bytes) > h->cfg.workspace_cap_bytes)
+    const int slots = std::min(nch, kStagingSlots);
+    const size_t total = slot * (size_t)slots;
+    if (h->cfg.workspace_cap_bytes && total + (size_t)P.hp.ws_bytes > h->cfg.workspace_cap_bytes)
       return fail(MUON_ERR_OOM, "staging plus workspace exceed the cap");
-    cudaError_t e = cudaMalloc(&P.staging, (size_t)off);
+    cudaError_t e = cudaMalloc(&P.staging, total);
     if (e != cudaSuccess) {
       cudaGetLastError();
       P.staging = nullptr;
-      return fail(MUON_ERR_OOM, "staging allocation of " + std::to_string(off) + " bytes failed");
+      return fail(MUON_ERR_OOM, "staging allocation of " + std::to_string(total) + " bytes failed");
     }
-    P.staging_size = (size_t)off;
+    P.staging_size = total;
+    P.slot_bytes = slot;
   }
+  for (int k = 0; k < 3; ++k)
+    if (!h->hs[k]) MUON_CUDA_TRY(cudaStreamCreateWithFlags(&h->hs[k], cudaStreamNonBlocking));
+  while ((int)h->hev.size() < 3 * nch + 1) {
+    cudaEvent_t ev;
+    MUON_CUDA_TRY(cudaEventCreateWithFlags(&ev, cudaEventDisableTiming));
+    h->hev.push_back(ev);
+  }
+  cudaEvent_t ev_begin = h->hev[3 * nch];
+  auto ev_in = [&](int c) { return h->hev[3 * c]; };
+  auto ev_comp = [&](int c) { return h->hev[3 * c + 1]; };
+  auto ev_out = [&](int c) { return h->hev[3 * c + 2]; };
+
+  // Device pointers of every matrix inside its chunk's slot.
   std::vector<float*> dp(count), dm(count);
   std::vector<const void*> dg(count);
   char* sb = static_cast<char*>(P.staging);
-  for (int i = 0; i < count; ++i) {
-    const size_t numel = (size_t)P.mats[i].numel;
-    const size_t gbytes = numel * ((shapes[3 * i + 2] & 1) ? 2 : 4);
-    dp[i] = reinterpret_cast<float*>(sb + P.staging_off[(size_t)i * 3 + 0]);
-    dg[i] = grads[i] ? sb + P.staging_off[(size_t)i * 3 + 1] : nullptr;
-    dm[i] = reinterpret_cast<float*>(sb + P.staging_off[(size_t)i * 3 + 2]);
-    MUON_CUDA_TRY(cudaMemcpyAsync(dp[i], params[i], numel * 4, cudaMemcpyHostToDevice, st));
-    MUON_CUDA_TRY(cudaMemcpyAsync(dm[i], momenta[i], numel * 4, cudaMemcpyHostToDevice, st));
-    if (grads[i]) MUON_CUDA_TRY(cudaMemcpyAsync(const_cast<void*>(dg[i]), grads[i], gbytes, cudaMemcpyHostToDevice, st));
+  for (int c = 0; c < nch; ++c) {
+    char* slot = sb + (size_t)(c % kStagingSlots) * P.slot_bytes;
+    for (int i = P.chunk_bounds[c]; i < P.chunk_bounds[c + 1]; ++i) {
+      dp[i] = reinterpret_cast<float*>(slot + P.staging_off[(size_t)i * 3 + 0]);
+      dg[i] = grads[i] ? slot + P.staging_off[(size_t)i * 3 + 1] : nullptr;
+      dm[i] = reinterpret_cast<float*>(slot + P.staging_off[(size_t)i * 3 + 2]);
+    }
   }
-  if ((rc = step_impl(h, dp.data(), dg.data(), dm.data(), shapes, count, lr, beta, nesterov, wd, ns_steps, abc, st)))
-    return rc;
-  for (int i = 0; i < count; ++i) {
-    if (!grads[i]) continue;
-    const size_t numel = (size_t)P.mats[i].numel;
-    MUON_CUDA_TRY(cudaMemcpyAsync(params[i], dp[i], numel * 4, cudaMemcpyDeviceToHost, st));
-    MUON_CUDA_TRY(cudaMemcpyAsync(momenta[i], dm[i], numel * 4, cudaMemcpyDeviceToHost, st));
+  std::vector<MatBind> hb;
+  const MatBind* db = nullptr;
+  if ((rc = step_binds(h, dp.data(), dg.data(), dm.data(), shapes, count, hb, &db))) return rc;
+
+  cudaStream_t s_in = h->hs[0], s_comp = h->hs[1], s_out = h->hs[2];
+  MUON_CUDA_TRY(cudaEventRecord(ev_begin, st));
+  for (int k = 0; k < 3; ++k) MUON_CUDA_TRY(cudaStreamWaitEvent(h->hs[k], ev_begin, 0));
+  int launches = 0;
+  prof_call_begin(h);
+  for (int c = 0; c < nch; ++c) {
+    // Copy-in (after the slot's previous chunk has been copied out).
+    if (c >= kStagingSlots) MUON_CUDA_TRY(cudaStreamWaitEvent(s_in, ev_out(c - kStagingSlots), 0));
+    for (int i = P.chunk_bounds[c]; i < P.chunk_bounds[c + 1]; ++i) {
+      if (!grads[i]) continue;
+      const size_t numel = (size_t)P.mats[i].numel;
+      const size_t gbytes = numel * ((shapes[3 * i + 2] & 1) ? 2 : 4);
+      MUON_CUDA_TRY(cudaMemcpyAsync(dp[i], params[i], numel * 4, cudaMemcpyHostToDevice, s_in));
+      MUON_CUDA_TRY(cudaMemcpyAsync(dm[i], momenta[i], numel * 4, cudaMemcpyHostToDevice, s_in));
+      MUON_CUDA_TRY(cudaMemcpyAsync(const_cast<void*>(dg[i]), grads[i], gbytes, cudaMemcpyHostToDevice, s_in));
+    }
+    MUON_CUDA_TRY(cudaEventRecord(ev_in(c), s_in));
+    // Compute.
+    MUON_CUDA_TRY(cudaStreamWaitEvent(s_comp, ev_in(c), 0));
+    if ((rc = enqueue_step_range(h, db, hb, chunk_range(P, c), lr, beta, nesterov, wd, ns_steps, abc, s_comp,
+                                 &launches)))
+      return rc;
+    MUON_CUDA_TRY(cudaEventRecord(ev_comp(c), s_comp));
+    // Copy-out.
+    MUON_CUDA_TRY(cudaStreamWaitEvent(s_out, ev_comp(c), 0));
+    for (int i = P.chunk_bounds[c]; i < P.chunk_bounds[c + 1]; ++i) {
+      if (!grads[i]) continue;
+      const size_t numel = (size_t)P.mats[i].numel;
+      MUON_CUDA_TRY(cudaMemcpyAsync(params[i], dp[i], numel * 4, cudaMemcpyDeviceToHost, s_out));
+      MUON_CUDA_TRY(cudaMemcpyAsync(momenta[i], dm[i], numel * 4, cudaMemcpyDeviceToHost, s_out));
+    }
+    MUON_CUDA_TRY(cudaEventRecord(ev_out(c), s_out));
   }
+  // The caller's stream resumes once every chunk is back in host memory.
+  MUON_CUDA_TRY(cudaStreamWaitEvent(st, ev_out(nch - 1), 0));
+  h->last_launches = launches;
   return MUON_OK;
 }
 
@@ -796,7 +987,8 @@ int muon_newton_schulz(muon_handle* h, const void* const* x_in, void* const* x_o
     d_in = static_cast<const TmapBlob*>(dm);
   }
   int res = BUF_IN;
-  if ((rc = enqueue_ns(h, db, hb, d_in, sumsq, ns_steps, abc, BUF_IN, BUF_OUT, st, &launches, &res))) return rc;
+  if ((rc = enqueue_ns(h, db, hb, full_range(P), d_in, sumsq, ns_steps, abc, BUF_IN, BUF_OUT, st, &launches, &res)))
+    return rc;
   h->last_launches = launches;
   return MUON_OK;
 }
