@@ -165,6 +165,32 @@ int muon_step(muon_handle* h, float* const* params, const void* const* grads,
               float lr, float beta, int nesterov, float wd, int ns_steps,
               const float* coeffs, void* stream);
 
+/* muon_step with a coefficient schedule: coeff_table is a host array of
+ * table_rows x 3 floats (a, b, c); table_rows = 1 applies one triple to every
+ * iteration, table_rows = ns_steps gives iteration t its own row. A sequence
+ * of odd polynomials still acts on the singular values only ("About Muon:
+ * Why Not Adam", "The lemma that makes it possible"); the pages name
+ * Chebyshev-type compositions ("Gram Newton-Schulz" section) but print no
+ * coefficients, so none are built in. Otherwise identical to muon_step. */
+int muon_step_schedule(muon_handle* h, float* const* params,
+                       const void* const* grads, float* const* momenta,
+                       const int32_t* shapes, int count, float lr, float beta,
+                       int nesterov, float wd, int ns_steps,
+                       const float* coeff_table, int table_rows, void* stream);
+
+/* QK-Clip after a Muon step ("The Optimizer Wars", MuonClip): for every
+ * weight i (fp32 W_q or W_k, device pointer, rows x cols, updated in place)
+ * with shapes[i] = {rows, cols, head_rows} (rows a multiple of head_rows),
+ * the rows of head h are multiplied by sqrt(tau / s_max[i][h]) when
+ * s_max[i][h] > tau (gamma_h = min(1, tau / S_max^h) applied as
+ * sqrt(gamma_h) to each of W_q^h and W_k^h), else left unchanged (NaN
+ * included). s_max is a host array of device float arrays, one per weight,
+ * rows / head_rows entries each: the largest attention logit per head seen
+ * in the step, tracked by the caller's forward pass. tau > 0 (the pages use
+ * 100). One kernel per weight. */
+int muon_qk_clip(muon_handle* h, float* const* weights, const int32_t* shapes,
+                 const float* const* s_max, int count, float tau, void* stream);
+
 /* Same step with every tensor in HOST memory. The matrices are split into
  * up to 8 chunks of consecutive matrices with about equal element counts;
  * while chunk c is computed, chunk c+1 is copied in and chunk c-1 copied

@@ -22,8 +22,8 @@ import ctypes
 
 from ._lib import EXPORTED, MuonConfig, MuonError, check, lib_path, load
 
-__all__ = ["Muon", "MuonError", "plan_query", "x_layout", "round_up", "SCALE_MODES", "DEFAULT_COEFFS",
-           "EXPORTED", "lib_path", "load"]
+__all__ = ["Muon", "MuonError", "plan_query", "x_layout", "round_up", "split_rows", "SCALE_MODES",
+           "DEFAULT_COEFFS", "EXPORTED", "lib_path", "load"]
 
 DEFAULT_COEFFS = (3.4445, -4.7750, 2.0315)
 SCALE_MODES = {"moonlight": 0, "jordan": 1, "bernstein": 2, "none": 3}
@@ -84,6 +84,34 @@ def x_layout(m: int, n: int, dtype, device):
     """An empty X-layout buffer: row-major m x round_up(n, 8)."""
     import torch
     return torch.empty((m, round_up(n, 8)), dtype=dtype, device=device)
+
+
+def _blocks(rows, spec):
+    if spec is None:
+        return [rows]
+    if isinstance(spec, int):
+        if spec < 1 or rows % spec:
+            raise ValueError(f"row split {spec} does not divide {rows} rows")
+        return [spec] * (rows // spec)
+    spec = [int(h) for h in spec]
+    if sum(spec) != rows or min(spec) < 1:
+        raise ValueError(f"row blocks {spec} do not sum to {rows} rows")
+    return spec
+
+
+def split_rows(params, grads, momenta, row_splits):
+    """Row-block views for split Muon (see Muon.step)."""
+    if len(row_splits) != len(params):
+        raise ValueError("row_splits needs one entry per matrix")
+    P, G, M = [], [], []
+    for p, g, m, spec in zip(params, grads, momenta, row_splits):
+        r0 = 0
+        for h in _blocks(p.shape[0], spec):
+            P.append(p[r0:r0 + h])
+            G.append(None if g is None else g[r0:r0 + h])
+            M.append(m[r0:r0 + h])
+            r0 += h
+    return P, G, M
 
 
 def plan_query(shapes, ns_precision: str = "bf16", small_path: bool = True, cta_pair: bool = False):
@@ -169,12 +197,18 @@ class Muon:
 
     # -- full step ----------------------------------------------------------
     def step(self, params, grads, momenta, lr, beta=0.95, nesterov=True, wd=0.1, ns_steps=5, coeffs=None,
-             stream=None):
+             stream=None, row_splits=None):
         """One Muon step, in place on params and momenta (lists of CUDA tensors).
 
-        A ``None`` gradient skips its matrix.
+        A ``None`` gradient skips its matrix. ``row_splits`` (optional, one
+        entry per matrix) requests split Muon: ``None`` keeps the matrix whole,
+        an int h cuts it into row blocks of h rows, a list gives the block
+        heights; every block is then a Muon matrix of its own (its rows are
+        contiguous, so the blocks are passed as views, no copy).
         """
         import torch
+        if row_splits is not None:
+            params, grads, momenta = split_rows(params, grads, momenta, row_splits)
         shapes, pp, gp, mp = [], [], [], []
         for i, (p, g, m) in enumerate(zip(params, grads, momenta, strict=True)):
             _check_2d(p, f"params[{i}]", (torch.float32,))
@@ -192,6 +226,48 @@ class Muon:
         check(self._lib.muon_step(self._h, _ptr_array(pp), _ptr_array(gp), _ptr_array(mp), _shapes_array(shapes),
                                   len(shapes), float(lr), float(beta), int(bool(nesterov)), float(wd),
                                   int(ns_steps), _coeffs(coeffs), _stream_handle(stream)))
+
+    def step_schedule(self, params, grads, momenta, coeff_table, lr, beta=0.95, nesterov=True, wd=0.1,
+                      stream=None):
+        """One Muon step whose Newton-Schulz iteration t uses coeff_table[t] = (a, b, c)."""
+        import torch
+        rows = [tuple(float(v) for v in r) for r in coeff_table]
+        if not rows or any(len(r) != 3 for r in rows):
+            raise ValueError("coeff_table must be a non-empty list of (a, b, c)")
+        table = (ctypes.c_float * (3 * len(rows)))(*[v for r in rows for v in r])
+        shapes, pp, gp, mp = [], [], [], []
+        for i, (p, g, m) in enumerate(zip(params, grads, momenta, strict=True)):
+            _check_2d(p, f"params[{i}]", (torch.float32,))
+            _check_2d(m, f"momenta[{i}]", (torch.float32,), p.device)
+            flag = 0
+            if g is not None:
+                _check_2d(g, f"grads[{i}]", (torch.float32, torch.bfloat16), p.device)
+                flag = FLAG_GRAD_BF16 if g.dtype == torch.bfloat16 else 0
+            shapes.append((p.shape[0], p.shape[1], flag))
+            pp.append(p.data_ptr()); gp.append(_ptr(g)); mp.append(m.data_ptr())
+        check(self._lib.muon_step_schedule(self._h, _ptr_array(pp), _ptr_array(gp), _ptr_array(mp),
+                                           _shapes_array(shapes), len(shapes), float(lr), float(beta),
+                                           int(bool(nesterov)), float(wd), len(rows), table, len(rows),
+                                           _stream_handle(stream)))
+
+    def qk_clip(self, weights, s_max, head_rows, tau=100.0, stream=None):
+        """QK-Clip in place on W_q / W_k weights (fp32 CUDA tensors).
+
+        s_max: one float32 CUDA tensor per weight with the largest attention
+        logit of each head; head_rows: rows per head (int or one per weight).
+        """
+        import torch
+        if isinstance(head_rows, int):
+            head_rows = [head_rows] * len(weights)
+        shapes = []
+        for i, (w, s, hr) in enumerate(zip(weights, s_max, head_rows, strict=True)):
+            _check_2d(w, f"weights[{i}]", (torch.float32,))
+            if s.dtype != torch.float32 or not s.is_contiguous() or s.numel() * hr != w.shape[0]:
+                raise ValueError(f"s_max[{i}] must be a contiguous float32 tensor with one entry per head")
+            shapes.append((w.shape[0], w.shape[1], int(hr)))
+        check(self._lib.muon_qk_clip(self._h, _ptr_array([w.data_ptr() for w in weights]), _shapes_array(shapes),
+                                     _ptr_array([s.data_ptr() for s in s_max]), len(weights), float(tau),
+                                     _stream_handle(stream)))
 
     def step_host(self, params, grads, momenta, lr, beta=0.95, nesterov=True, wd=0.1, ns_steps=5,
                   coeffs=None, stream=None):

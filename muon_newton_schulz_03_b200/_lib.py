@@ -46,6 +46,9 @@ _SIGNATURES = {
     "muon_destroy": (c_int, [c_void_p]),
     "muon_step": (c_int, [c_void_p, P(c_void_p), P(c_void_p), P(c_void_p), P(ctypes.c_int32), c_int,
                           c_float, c_float, c_int, c_float, c_int, P(c_float), c_void_p]),
+    "muon_step_schedule": (c_int, [c_void_p, P(c_void_p), P(c_void_p), P(c_void_p), P(ctypes.c_int32), c_int,
+                                   c_float, c_float, c_int, c_float, c_int, P(c_float), c_int, c_void_p]),
+    "muon_qk_clip": (c_int, [c_void_p, P(c_void_p), P(ctypes.c_int32), P(c_void_p), c_int, c_float, c_void_p]),
     "muon_step_host": (c_int, [c_void_p, P(c_void_p), P(c_void_p), P(c_void_p), P(ctypes.c_int32), c_int,
                                c_float, c_float, c_int, c_float, c_int, P(c_float), c_void_p]),
     "muon_momentum_norm": (c_int, [c_void_p, P(c_void_p), P(c_void_p), P(c_void_p), c_void_p,

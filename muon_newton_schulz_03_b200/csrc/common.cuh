@@ -66,6 +66,7 @@ enum WaitCode : int {
 };
 
 constexpr int kElemChunk = 8192;  // elements per block in the elementwise kernels
+constexpr int kMaxNsSteps = 64;   // Newton-Schulz iterations per call
 constexpr double kNormEps = 1e-7; // added to ||u||_F before dividing
 
 __host__ __device__ inline long long ceil_div_ll(long long a, long long b) { return (a + b - 1) / b; }

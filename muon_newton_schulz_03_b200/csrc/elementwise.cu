@@ -248,7 +248,30 @@ __global__ void __launch_bounds__(kThreads) k0_scale_copy(const MatPlan* __restr
   }
 }
 
+// QK-Clip ("The Optimizer Wars", MuonClip): after the update, the rows of
+// head h of W_q or W_k are multiplied by sqrt(gamma_h), gamma_h =
+// min(1, tau / S_max^h), so the head's q.k logits shrink by gamma_h.
+__global__ void __launch_bounds__(kThreads) k5_qk_clip(float* __restrict__ w, long long rows, long long cols,
+                                                       int head_rows, const float* __restrict__ s_max, float tau) {
+  const long long n = rows * cols;
+  for (long long e = (long long)blockIdx.x * kThreads + threadIdx.x; e < n; e += (long long)gridDim.x * kThreads) {
+    const long long r = e / cols;
+    const float s = s_max[r / head_rows];
+    if (s > tau) w[e] *= sqrtf(tau / s);     // false for NaN: no clip
+  }
+}
+
 }  // namespace
+
+cudaError_t launch_qk_clip(float* w, long long rows, long long cols, int head_rows, const float* s_max, float tau,
+                           cudaStream_t st) {
+  const long long n = rows * cols;
+  if (n <= 0) return cudaSuccess;
+  long long blocks = (n + kThreads - 1) / kThreads;
+  if (blocks > 148 * 16) blocks = 148 * 16;
+  k5_qk_clip<<<(unsigned)blocks, kThreads, 0, st>>>(w, rows, cols, head_rows, s_max, tau);
+  return cudaGetLastError();
+}
 
 cudaError_t launch_momentum_norm(const ElemLaunch& L, int ysel, float beta, int nesterov, double* sumsq,
                                  DevStatus* status, int check_nonfinite, bool fp32_out, cudaStream_t st) {

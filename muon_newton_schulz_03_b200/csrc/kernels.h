@@ -23,6 +23,10 @@ cudaError_t launch_momentum_norm(const ElemLaunch& L, int ysel, float beta, int 
                                  DevStatus* status, int check_nonfinite, bool fp32_out, cudaStream_t st);
 cudaError_t launch_apply(const ElemLaunch& L, int osel, float lr, float wd, int scale_mode, float extra_scale,
                          const double* sumsq, bool fp32_in, cudaStream_t st);
+// QK-Clip: rows of head h scaled by sqrt(tau / s_max[h]) when s_max[h] > tau.
+cudaError_t launch_qk_clip(float* w, long long rows, long long cols, int head_rows, const float* s_max, float tau,
+                           cudaStream_t st);
+
 cudaError_t launch_scale_copy(const ElemLaunch& L, int isel, int osel, const double* sumsq, bool fp32,
                               cudaStream_t st);
 
@@ -73,8 +77,9 @@ struct NsSmallLaunch {
   unsigned long long timeout_ns;
 };
 
-cudaError_t launch_ns_small(const NsSmallLaunch& L, int ns_steps, int src_sel, int final_sel, float a, float b,
-                            float c, cudaStream_t st);
+// abc: ns_steps rows of (a, b, c).
+cudaError_t launch_ns_small(const NsSmallLaunch& L, int ns_steps, int src_sel, int final_sel, const float* abc,
+                            cudaStream_t st);
 int ns_small_smem_bytes();
 
 cudaError_t launch_ns_phase_pair(const NsLaunch& L, int phase, int src_sel, int dst_sel, int first, float a,

@@ -455,13 +455,19 @@ int check_common(muon_handle* h, const int32_t* shapes, int count) {
   return MUON_OK;
 }
 
-int check_coeffs(const float* coeffs, int ns_steps, float* abc) {
-  if (ns_steps < 0 || ns_steps > 64) return fail(MUON_ERR_INVALID_ARG, "ns_steps must be in [0, 64]");
+// Fills abc with ns_steps rows of (a, b, c): `rows` = 1 repeats one triple,
+// `rows` = ns_steps gives one per step; NULL = the default triple.
+int check_coeffs(const float* coeffs, int ns_steps, float* abc, int rows = 1) {
+  if (ns_steps < 0 || ns_steps > kMaxNsSteps) return fail(MUON_ERR_INVALID_ARG, "ns_steps must be in [0, 64]");
+  if (rows != 1 && rows != ns_steps)
+    return fail(MUON_ERR_INVALID_ARG, "a coefficient table needs 1 or ns_steps rows");
   const float def[3] = {3.4445f, -4.7750f, 2.0315f};
-  const float* c = coeffs ? coeffs : def;
-  for (int k = 0; k < 3; ++k) {
-    if (!std::isfinite(c[k])) return fail(MUON_ERR_INVALID_ARG, "coefficients must be finite");
-    abc[k] = c[k];
+  for (int t = 0; t < std::max(ns_steps, 1); ++t) {
+    const float* c = coeffs ? coeffs + 3 * (rows == 1 ? 0 : t) : def;
+    for (int k = 0; k < 3; ++k) {
+      if (!std::isfinite(c[k])) return fail(MUON_ERR_INVALID_ARG, "coefficients must be finite");
+      abc[3 * t + k] = c[k];
+    }
   }
   return MUON_OK;
 }
@@ -539,7 +545,7 @@ int enqueue_ns(muon_handle* h, const MatBind* d_binds, const std::vector<MatBind
     S.timeout_ns = (unsigned long long)(h->cfg.wait_timeout_s * 1e9);
     const int final_sel = last_dst >= 0 ? last_dst : (ns_steps % 2 == 1 ? BUF_X1 : BUF_X0);
     const int slot = prof_before(h, MUON_KERNEL_NS_SMALL, st);
-    MUON_CUDA_TRY(launch_ns_small(S, ns_steps, first_src, final_sel, abc[0], abc[1], abc[2], st));
+    MUON_CUDA_TRY(launch_ns_small(S, ns_steps, first_src, final_sel, abc, st));
     prof_after(h, slot, st);
     ++*launches;
   }
@@ -547,6 +553,7 @@ int enqueue_ns(muon_handle* h, const MatBind* d_binds, const std::vector<MatBind
   for (int t = 1; t <= ns_steps; ++t) {
     const int dst = (t == ns_steps && last_dst >= 0) ? last_dst : (t % 2 == 1 ? BUF_X1 : BUF_X0);
     const int first = t == 1 ? 1 : 0;
+    const float* c3 = abc + 3 * (t - 1);
     if (bf16) {
       NsLaunch L;
       L.plans = P.d_mats;
@@ -563,9 +570,9 @@ int enqueue_ns(muon_handle* h, const MatBind* d_binds, const std::vector<MatBind
         if (L.ntiles == 0) continue;
         const int slot = prof_before(h, MUON_KERNEL_NS_GRAM + ph, st);
         if (hp.tile_m == kTileMPair)
-          MUON_CUDA_TRY(launch_ns_phase_pair(L, ph, src, dst, first, abc[0], abc[1], abc[2], st));
+          MUON_CUDA_TRY(launch_ns_phase_pair(L, ph, src, dst, first, c3[0], c3[1], c3[2], st));
         else
-          MUON_CUDA_TRY(launch_ns_phase_bf16(L, ph, src, dst, first, abc[0], abc[1], abc[2], st));
+          MUON_CUDA_TRY(launch_ns_phase_bf16(L, ph, src, dst, first, c3[0], c3[1], c3[2], st));
         prof_after(h, slot, st);
         ++*launches;
       }
@@ -577,7 +584,7 @@ int enqueue_ns(muon_handle* h, const MatBind* d_binds, const std::vector<MatBind
         float* d_ptr = static_cast<float*>(const_cast<void*>(sel_buf(mp, hbinds[i], dst)));
         for (int ph = PHASE_GRAM; ph <= PHASE_COMB; ++ph) {
           const int slot = prof_before(h, MUON_KERNEL_NS_FP32, st);
-          MUON_CUDA_TRY(launch_ns_phase_fp32(mp, i, ph, s_ptr, d_ptr, sumsq, first, abc[0], abc[1], abc[2], st));
+          MUON_CUDA_TRY(launch_ns_phase_fp32(mp, i, ph, s_ptr, d_ptr, sumsq, first, c3[0], c3[1], c3[2], st));
           prof_after(h, slot, st);
         }
         *launches += 3;
@@ -762,12 +769,53 @@ int muon_step(muon_handle* h, float* const* params, const void* const* grads, fl
   if ((rc = check_common(h, shapes, count))) return rc;
   if ((rc = check_step_ptrs(params, grads, momenta, shapes, count))) return rc;
   if ((rc = check_scalars(lr, beta, wd))) return rc;
-  float abc[3];
+  float abc[3 * kMaxNsSteps];
   if ((rc = check_coeffs(coeffs, ns_steps, abc))) return rc;
   DeviceGuard g(h->device);
   if (!g.ok) return fail(MUON_ERR_CUDA, "cudaSetDevice failed");
   return step_impl(h, params, grads, momenta, shapes, count, lr, beta, nesterov, wd, ns_steps, abc,
                    static_cast<cudaStream_t>(stream));
+}
+
+int muon_step_schedule(muon_handle* h, float* const* params, const void* const* grads, float* const* momenta,
+                       const int32_t* shapes, int count, float lr, float beta, int nesterov, float wd, int ns_steps,
+                       const float* coeff_table, int table_rows, void* stream) {
+  g_last_error.clear();
+  int rc;
+  if ((rc = check_common(h, shapes, count))) return rc;
+  if ((rc = check_step_ptrs(params, grads, momenta, shapes, count))) return rc;
+  if ((rc = check_scalars(lr, beta, wd))) return rc;
+  if (!coeff_table) return fail(MUON_ERR_INVALID_ARG, "coeff_table is required");
+  float abc[3 * kMaxNsSteps];
+  if ((rc = check_coeffs(coeff_table, ns_steps, abc, table_rows))) return rc;
+  DeviceGuard g(h->device);
+  if (!g.ok) return fail(MUON_ERR_CUDA, "cudaSetDevice failed");
+  return step_impl(h, params, grads, momenta, shapes, count, lr, beta, nesterov, wd, ns_steps, abc,
+                   static_cast<cudaStream_t>(stream));
+}
+
+int muon_qk_clip(muon_handle* h, float* const* weights, const int32_t* shapes, const float* const* s_max, int count,
+                 float tau, void* stream) {
+  g_last_error.clear();
+  if (!h) return fail(MUON_ERR_INVALID_ARG, "handle is NULL");
+  if (!weights || !shapes || !s_max || count < 1) return fail(MUON_ERR_INVALID_ARG, "weights, shapes, s_max, count");
+  if (!(tau > 0.0f) || !std::isfinite(tau)) return fail(MUON_ERR_INVALID_ARG, "tau must be positive and finite");
+  int rc;
+  for (int i = 0; i < count; ++i) {
+    const int rows = shapes[3 * i], cols = shapes[3 * i + 1], hr = shapes[3 * i + 2];
+    if (rows < 1 || cols < 1 || hr < 1 || rows % hr)
+      return fail(MUON_ERR_INVALID_ARG, "matrix " + std::to_string(i) + ": rows must be a positive multiple of head_rows");
+    if ((rc = check_ptr(weights[i], "weights", i))) return rc;
+    if (!s_max[i] || reinterpret_cast<uintptr_t>(s_max[i]) % 4)
+      return fail(MUON_ERR_INVALID_ARG, "s_max[" + std::to_string(i) + "] is NULL or misaligned");
+  }
+  DeviceGuard g(h->device);
+  if (!g.ok) return fail(MUON_ERR_CUDA, "cudaSetDevice failed");
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  for (int i = 0; i < count; ++i)
+    MUON_CUDA_TRY(launch_qk_clip(weights[i], shapes[3 * i], shapes[3 * i + 1], shapes[3 * i + 2], s_max[i], tau, st));
+  h->last_launches = count;
+  return MUON_OK;
 }
 
 int muon_step_host(muon_handle* h, float* const* params, const void* const* grads, float* const* momenta,
@@ -780,7 +828,7 @@ int muon_step_host(muon_handle* h, float* const* params, const void* const* grad
   for (int i = 0; i < count; ++i)
     if (!params[i] || !momenta[i]) return fail(MUON_ERR_INVALID_ARG, "host params and momenta must be non-NULL");
   if ((rc = check_scalars(lr, beta, wd))) return rc;
-  float abc[3];
+  float abc[3 * kMaxNsSteps];
   if ((rc = check_coeffs(coeffs, ns_steps, abc))) return rc;
   DeviceGuard g(h->device);
   if (!g.ok) return fail(MUON_ERR_CUDA, "cudaSetDevice failed");
@@ -930,7 +978,7 @@ int muon_newton_schulz(muon_handle* h, const void* const* x_in, void* const* x_o
   int rc;
   if ((rc = check_common(h, shapes, count))) return rc;
   if (!x_in || !x_out) return fail(MUON_ERR_INVALID_ARG, "x_in and x_out are required");
-  float abc[3];
+  float abc[3 * kMaxNsSteps];
   if ((rc = check_coeffs(coeffs, ns_steps, abc))) return rc;
   const size_t esz = h->cfg.ns_precision == MUON_NS_FP32 ? 4 : 2;
   for (int i = 0; i < count; ++i) {

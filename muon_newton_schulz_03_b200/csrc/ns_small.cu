@@ -50,7 +50,7 @@ struct __align__(1024) SmallSmem {
 struct SmallArgs {
   NsSmallLaunch L;
   int ns_steps, src_sel, final_sel;
-  float a, b, c;
+  float coef[kMaxNsSteps][3];   // (a, b, c) of every step
 };
 
 __device__ __forceinline__ uint32_t swz(int r, int c, int chunk_stride) {
@@ -153,6 +153,7 @@ __global__ void __launch_bounds__(kThreads, 1) ns_small_kernel(const __grid_cons
   for (int t = 1; t <= args.ns_steps && ok; ++t) {
     const bool first = t == 1;
     const bool last = t == args.ns_steps;
+    const float ca = args.coef[t - 1][0], cb = args.coef[t - 1][1], cc = args.coef[t - 1][2];
 
     // ---------------- Gram: TMEM columns [0, 128) ----------------
     if (tid == 0) {
@@ -223,7 +224,7 @@ __global__ void __launch_bounds__(kThreads, 1) ns_small_kernel(const __grid_cons
       tmem_ld_32x32b_x32(lane_base + (uint32_t)c0, av);          // A (fp32, before rounding)
       tmem_ld_32x32b_x32(lane_base + 128u + (uint32_t)c0, pv);   // A A
 #pragma unroll
-      for (int i = 0; i < 32; ++i) pv[i] = fmaf(args.b, bf16r(av[i] * sc_gram), args.c * pv[i]);
+      for (int i = 0; i < 32; ++i) pv[i] = fmaf(cb, bf16r(av[i] * sc_gram), cc * pv[i]);
       sts_row32(sm.b, row, c0, kChunk, pv);
     }
     fence_proxy_async_smem();
@@ -278,7 +279,7 @@ __global__ void __launch_bounds__(kThreads, 1) ns_small_kernel(const __grid_cons
         tmem_ld_32x32b_x32(lane_base + (uint32_t)(blk * 128 + c0), v);
         lds_row32(sm.x, r, c0, x_cs, x);
 #pragma unroll
-        for (int i = 0; i < 32; ++i) v[i] = sc * fmaf(args.a, x[i], v[i]);
+        for (int i = 0; i < 32; ++i) v[i] = sc * fmaf(ca, x[i], v[i]);
         if (!last) {
           sts_row32(sm.x, r, c0, x_cs, v);
         } else if (r < mp.m && c0 < mp.n) {
@@ -315,9 +316,10 @@ __global__ void __launch_bounds__(kThreads, 1) ns_small_kernel(const __grid_cons
 
 int ns_small_smem_bytes() { return (int)sizeof(SmallSmem) + 1024; }
 
-cudaError_t launch_ns_small(const NsSmallLaunch& L, int ns_steps, int src_sel, int final_sel, float a, float b,
-                            float c, cudaStream_t st) {
+cudaError_t launch_ns_small(const NsSmallLaunch& L, int ns_steps, int src_sel, int final_sel, const float* abc,
+                            cudaStream_t st) {
   if (L.nmats <= 0 || ns_steps <= 0) return cudaSuccess;
+  if (ns_steps > kMaxNsSteps) return cudaErrorInvalidValue;
   static bool attr_set = false;
   const int smem = ns_small_smem_bytes();
   if (!attr_set) {
@@ -330,9 +332,8 @@ cudaError_t launch_ns_small(const NsSmallLaunch& L, int ns_steps, int src_sel, i
   args.ns_steps = ns_steps;
   args.src_sel = src_sel;
   args.final_sel = final_sel;
-  args.a = a;
-  args.b = b;
-  args.c = c;
+  for (int t = 0; t < ns_steps; ++t)
+    for (int k = 0; k < 3; ++k) args.coef[t][k] = abc[3 * t + k];
   ns_small_kernel<<<L.nmats, kThreads, smem, st>>>(args);
   return cudaGetLastError();
 }

@@ -30,13 +30,16 @@ from .muon_oracle import (  # noqa: F401
     SCALE_NONE,
     apply_update,
     bf16_round,
+    coeff_rows,
     momentum_update,
     muon_step,
     muon_step_matrix,
+    muon_step_matrix_split,
     nesterov_blend,
     newton_schulz,
     ns_only,
     ns_poly,
     ns_poly_iterate,
+    qk_clip,
     update_scale,
 )

@@ -116,17 +116,33 @@ def _matmul(P, Q, accum_fp32):
     return (P.astype(np.float32) @ Q.astype(np.float32)).astype(np.float64)
 
 
-def _ns_iterations(X, steps, coeffs, emulate_bf16, accum_fp32=False):
+def coeff_rows(coeffs, steps):
+    """Per-step (a, b, c): one triple for every step, or a table of `steps`
+    triples (a schedule of different odd polynomials, "About Muon: Why Not
+    Adam", section "Gram Newton-Schulz": Chebyshev-type schemes compose
+    different odd polynomials)."""
+    arr = np.asarray(coeffs, dtype=np.float64)
+    if arr.ndim == 1:
+        if arr.shape != (3,):
+            raise ValueError("coefficients must be (a, b, c) or a table of them")
+        return [tuple(arr)] * steps
+    if arr.shape != (steps, 3):
+        raise ValueError(f"a coefficient table needs {steps} rows of (a, b, c)")
+    return [tuple(r) for r in arr]
+
+
+def _ns_iterations(X, steps, coeffs, emulate_bf16, accum_fp32=False, start=0):
     """Run the quintic iteration on a short-side-first matrix X (s x l).
 
     Each step forms the Gram A = X X^T, the polynomial B = bA + cA^2 and the
     combine X <- aX + BX. This equals aX + bX(X^T X) + cX(X^T X)^2 because
     (X X^T)^k X = X (X^T X)^k ("About Muon: Why Not Adam", section "The lemma
-    that makes it possible").
+    that makes it possible"). ``coeffs`` holds one triple per step (see
+    coeff_rows); steps ``start..steps-1`` are run.
     """
-    a, b, c = coeffs
     rnd = bf16_round if emulate_bf16 else (lambda v: v)
-    for _ in range(steps):
+    for k in range(start, steps):
+        a, b, c = coeffs[k]
         A = rnd(_matmul(X, X.T, accum_fp32))
         B = rnd(b * A + c * _matmul(A, A, accum_fp32))
         X = rnd(a * X + _matmul(B, X, accum_fp32))
@@ -151,12 +167,13 @@ def newton_schulz(G, steps=5, coeffs=DEFAULT_COEFFS, eps=EPS,
     G = np.asarray(G, dtype=np.float64)
     if G.ndim != 2:
         raise ValueError("Newton-Schulz is defined for 2D matrices only")
+    rows = coeff_rows(coeffs, steps)
     transposed = G.shape[0] > G.shape[1]
     if not emulate_bf16:
         X = G / (np.linalg.norm(G) + eps)
         if transposed:
             X = X.T
-        X = _ns_iterations(X, steps, coeffs, False)
+        X = _ns_iterations(X, steps, rows, False)
         return X.T if transposed else X
 
     # bf16-emulating diagnostic: Y = bf16(G); alpha = 1/(||G|| + eps) is
@@ -165,14 +182,14 @@ def newton_schulz(G, steps=5, coeffs=DEFAULT_COEFFS, eps=EPS,
     Y = bf16_round(G)
     if transposed:
         Y = Y.T
-    a, b, c = coeffs
     if steps == 0:
         X = alpha * Y
     else:
+        a, b, c = rows[0]
         A = bf16_round(alpha * alpha * _matmul(Y, Y.T, accum_fp32))
         B = bf16_round(b * A + c * _matmul(A, A, accum_fp32))
         X = bf16_round(alpha * (a * Y + _matmul(B, Y, accum_fp32)))
-        X = _ns_iterations(X, steps - 1, coeffs, True, accum_fp32)
+        X = _ns_iterations(X, steps, rows, True, accum_fp32, start=1)
     return X.T if transposed else X
 
 
@@ -190,7 +207,7 @@ def ns_only(X, steps=5, coeffs=DEFAULT_COEFFS, emulate_bf16=False, accum_fp32=Fa
     transposed = X.shape[0] > X.shape[1]
     if transposed:
         X = X.T
-    X = _ns_iterations(X, steps, coeffs, emulate_bf16, accum_fp32 and emulate_bf16)
+    X = _ns_iterations(X, steps, coeff_rows(coeffs, steps), emulate_bf16, accum_fp32 and emulate_bf16)
     return X.T if transposed else X
 
 
@@ -284,6 +301,50 @@ def muon_step_matrix(p, g, m, *, lr, beta=0.95, nesterov=True, wd=0.1,
     scale = update_scale(p.shape[0], p.shape[1], scale_mode, extra_scale)
     p_new = apply_update(p, O, lr, wd, scale)
     return p_new, m_new, O, nu
+
+
+def qk_clip(w, s_max, tau, head_rows):
+    """QK-Clip on one projection weight (rows = heads x head_rows).
+
+    "The Optimizer Wars", section on MuonClip: after the Muon update, a head
+    whose largest attention logit S_max^h exceeded tau gets
+    gamma_h = min(1, tau / S_max^h), applied as sqrt(gamma_h) to that head's
+    rows of W_q and of W_k, so their product shrinks by gamma_h. Heads at or
+    below tau (and non-finite S_max) are left unchanged.
+    """
+    w = np.asarray(w, dtype=np.float64).copy()
+    s_max = np.asarray(s_max, dtype=np.float64)
+    if w.shape[0] != head_rows * len(s_max):
+        raise ValueError("rows must be heads x head_rows")
+    for h, s in enumerate(s_max):
+        if np.isfinite(s) and s > tau:
+            w[h * head_rows:(h + 1) * head_rows] *= np.sqrt(tau / s)
+    return w
+
+
+def muon_step_matrix_split(p, g, m, row_blocks, **kw):
+    """Split Muon on one matrix: each row block is a Muon matrix of its own.
+
+    "Why Muon Works", section 7.3 (QKV / MLA split): orthogonalise Q, K, V,
+    or each head's rows, separately and put the blocks back together; "The
+    Optimizer Wars", "Muon Split" and "Per-Head Muon": the projection matrix
+    is cut into per-head blocks before orthogonalisation. Reading: momentum,
+    normalisation, Newton-Schulz, scale (from the block's own shape, which
+    keeps Moonlight's entry RMS of 0.2) and the write all act per block.
+    ``row_blocks`` lists the block heights (summing to the row count).
+    Returns (p', m', O, norms) with O concatenated and one norm per block.
+    """
+    p = np.asarray(p, dtype=np.float64)
+    if sum(row_blocks) != p.shape[0] or min(row_blocks) < 1:
+        raise ValueError("row blocks must be positive and sum to the row count")
+    outs = []
+    r0 = 0
+    for h in row_blocks:
+        sl = slice(r0, r0 + h)
+        outs.append(muon_step_matrix(p[sl], np.asarray(g)[sl], np.asarray(m)[sl], **kw))
+        r0 += h
+    return (np.concatenate([o[0] for o in outs]), np.concatenate([o[1] for o in outs]),
+            np.concatenate([o[2] for o in outs]), [o[3] for o in outs])
 
 
 def muon_step(params, grads, momenta, *, lr, beta=0.95, nesterov=True,

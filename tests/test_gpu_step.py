@@ -346,3 +346,81 @@ def test_mixed_small_and_tiled_matrices_in_one_step():
     assert opt.last_launch_count() == 1 + 1 + 15 + 1
     assert opt.status() == (0, 0, 0)
     opt.close()
+
+
+def test_split_muon_qkv_and_per_head():
+    # QKV fused weight cut into Q, K, V; an attention output projection cut
+    # per head (12 heads of 64 rows); one matrix kept whole.
+    shapes = [(2304, 768), (768, 768), (768, 3072)]
+    splits = [768, 64, None]
+    cpu, dev = make_set(W.CONFIG_GPT2, shapes, torch.float32)
+    opt = muon.Muon(device=0)
+    opt.step([d[0] for d in dev], [d[1] for d in dev], [d[2] for d in dev], lr=2e-4, wd=0.1, row_splits=splits)
+    torch.cuda.synchronize()
+    assert opt.status() == (0, 0, 0)
+    assert opt.last_launch_count() >= 17
+    for i, (m, n) in enumerate(shapes):
+        p0, g, m0 = cpu[i]
+        blocks = [m] if splits[i] is None else [splits[i]] * (m // splits[i])
+        kw = dict(lr=F32(2e-4), beta=F32(0.95), wd=F32(0.1))
+        p_ref, m_ref, _, _ = O.muon_step_matrix_split(p0, g, m0, blocks, **kw)
+        p_emu, _, _, _ = O.muon_step_matrix_split(p0, g, m0, blocks, emulate_bf16=True, **kw)
+        p_e32, _, _, _ = O.muon_step_matrix_split(p0, g, m0, blocks, emulate_bf16=True, accum_fp32=True, **kw)
+        assert rel(to64(dev[i][2]), m_ref) <= TOL_ELEM
+        bf16_gate(to64(dev[i][0]) - p0, p_ref - p0, p_emu - p0, p_e32 - p0, f"split matrix {i}")
+    opt.close()
+
+
+def test_coefficient_schedule():
+    shapes = [(256, 768), (768, 256), (100, 300), (512, 512)]
+    cpu, dev = make_set(W.CONFIG_GPT2, shapes, torch.float32)
+    base = [(d[0].clone(), d[2].clone()) for d in dev]
+    opt = muon.Muon(device=0)
+    # A constant table is the plain step, bit for bit.
+    opt.step_schedule([d[0] for d in dev], [d[1] for d in dev], [d[2] for d in dev], [O.DEFAULT_COEFFS] * 5, lr=2e-4)
+    torch.cuda.synchronize()
+    p_sched = [to64(d[0]) for d in dev]
+    for d, (p0, m0) in zip(dev, base):
+        d[0].copy_(p0)
+        d[2].copy_(m0)
+    opt.step([d[0] for d in dev], [d[1] for d in dev], [d[2] for d in dev], lr=2e-4)
+    torch.cuda.synchronize()
+    for a, d in zip(p_sched, dev):
+        assert np.max(np.abs(a - to64(d[0]))) <= 1e-6 * np.max(np.abs(a))
+    # A varying table against the oracle.
+    table = [(3.4445, -4.7750, 2.0315), (3.0, -3.2, 1.2), (2.5, -2.0, 0.6), (1.875, -1.25, 0.375)]
+    for d, (p0, m0) in zip(dev, base):
+        d[0].copy_(p0)
+        d[2].copy_(m0)
+    opt.step_schedule([d[0] for d in dev], [d[1] for d in dev], [d[2] for d in dev], table, lr=2e-4)
+    torch.cuda.synchronize()
+    for i, (m, n) in enumerate(shapes):
+        p0, g, m0 = cpu[i]
+        kw = dict(lr=F32(2e-4), beta=F32(0.95), wd=F32(0.1), ns_steps=4,
+                  coeffs=[tuple(float(np.float32(v)) for v in r) for r in table])
+        p_ref = O.muon_step_matrix(p0, g, m0, **kw)[0]
+        p_emu = O.muon_step_matrix(p0, g, m0, emulate_bf16=True, **kw)[0]
+        p_e32 = O.muon_step_matrix(p0, g, m0, emulate_bf16=True, accum_fp32=True, **kw)[0]
+        bf16_gate(to64(dev[i][0]) - p0, p_ref - p0, p_emu - p0, p_e32 - p0, f"schedule matrix {i}")
+    with pytest.raises(ValueError):
+        opt.step_schedule([d[0] for d in dev], [d[1] for d in dev], [d[2] for d in dev], [], lr=2e-4)
+    assert opt.status() == (0, 0, 0)
+    opt.close()
+
+
+def test_qk_clip_matches_oracle():
+    rng = np.random.default_rng(31)
+    heads, d, dm = 8, 64, 512
+    wq = cuda_f32(rng.standard_normal((heads * d, dm)) * 0.02)
+    wk = cuda_f32(rng.standard_normal((heads // 2 * d, dm)) * 0.02)       # grouped K heads
+    sq = torch.tensor([250.0, 30.0, 101.0, 100.0, float("nan"), 5000.0, -3.0, 99.9], dtype=torch.float32,
+                      device=DEV)
+    sk = torch.tensor([250.0, 101.0, 5000.0, 99.9], dtype=torch.float32, device=DEV)
+    q0, k0 = to64(wq), to64(wk)
+    opt = muon.Muon(device=0)
+    opt.qk_clip([wq, wk], [sq, sk], [d, d], tau=100.0)
+    torch.cuda.synchronize()
+    assert rel(to64(wq), O.qk_clip(q0, sq.cpu().numpy(), 100.0, d)) <= TOL_ELEM
+    assert rel(to64(wk), O.qk_clip(k0, sk.cpu().numpy(), 100.0, d)) <= TOL_ELEM
+    assert np.array_equal(to64(wq)[64:128], q0[64:128])          # 30 < tau: untouched
+    opt.close()

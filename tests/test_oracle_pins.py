@@ -412,3 +412,100 @@ def test_bf16_mode_fp32_accumulation_is_a_nearby_realization():
     c = O.newton_schulz(G, emulate_bf16=True, accum_fp32=True)
     monkey.undo()
     assert np.max(np.abs(c - O.newton_schulz(G))) < 1e-5
+
+
+# ---------------------------------------------------------------------------
+# Split Muon ("Why Muon Works", section 7.3; "The Optimizer Wars", Muon
+# Split / Per-Head Muon): each row block is orthogonalised on its own.
+# ---------------------------------------------------------------------------
+
+def test_split_with_one_block_is_plain_step():
+    rng = np.random.default_rng(21)
+    p, g = rng.standard_normal((12, 20)), rng.standard_normal((12, 20))
+    a = O.muon_step_matrix(p, g, np.zeros_like(p), lr=0.1)
+    b = O.muon_step_matrix_split(p, g, np.zeros_like(p), [12], lr=0.1)
+    assert np.array_equal(a[0], b[0]) and np.array_equal(a[2], b[2])
+
+
+def test_split_blocks_follow_their_own_svd():
+    # Every block of O equals U_h f^5(sigma_h / (||u_h|| + eps)) V_h^T of its
+    # own block's SVD, and block norms are the blocks' own.
+    rng = np.random.default_rng(22)
+    g = rng.standard_normal((24, 16))
+    blocks = [8, 8, 8]
+    _, _, o, norms = O.muon_step_matrix_split(np.zeros_like(g), g, np.zeros_like(g), blocks, lr=0.1, beta=0.0,
+                                              nesterov=False, wd=0.0)
+    r0 = 0
+    for h, nu in zip(blocks, norms):
+        gb = g[r0:r0 + h]
+        U, sig, Vt = np.linalg.svd(gb, full_matrices=False)
+        x = sig / (np.linalg.norm(gb) + O.EPS)
+        a, b, c = O.DEFAULT_COEFFS
+        for _ in range(5):
+            x = a * x + b * x ** 3 + c * x ** 5
+        assert np.max(np.abs(o[r0:r0 + h] - (U * x) @ Vt)) < 1e-12
+        assert abs(nu - np.linalg.norm(gb)) < 1e-12
+        r0 += h
+    # Not the same as orthogonalising the whole matrix.
+    whole = O.newton_schulz(g)
+    assert np.max(np.abs(whole - o)) > 1e-3
+
+
+def test_split_rejects_bad_blocks():
+    with pytest.raises(ValueError):
+        O.muon_step_matrix_split(np.zeros((6, 4)), np.zeros((6, 4)), np.zeros((6, 4)), [4, 4], lr=0.1)
+
+
+# ---------------------------------------------------------------------------
+# Coefficient schedules: a sequence of odd polynomials still acts on the
+# singular values only (lemma), and convergent members reach the polar factor.
+# ---------------------------------------------------------------------------
+
+def test_schedule_of_constant_rows_equals_triple():
+    rng = np.random.default_rng(23)
+    G = rng.standard_normal((10, 14))
+    assert np.array_equal(O.newton_schulz(G, 4, [O.DEFAULT_COEFFS] * 4), O.newton_schulz(G, 4))
+
+
+def test_schedule_follows_composed_scalar_polynomials():
+    rng = np.random.default_rng(24)
+    G = rng.standard_normal((9, 13))
+    table = [(3.4445, -4.7750, 2.0315), (1.875, -1.25, 0.375), (1.5, -0.5, 0.0), (2.0, -1.5, 0.5)]
+    U, sig, Vt = np.linalg.svd(G, full_matrices=False)
+    x = sig / (np.linalg.norm(G) + O.EPS)
+    for a, b, c in table:
+        x = a * x + b * x ** 3 + c * x ** 5
+    assert np.max(np.abs(O.newton_schulz(G, 4, table) - (U * x) @ Vt)) < 1e-12
+    for mode in (False, True):
+        with pytest.raises(ValueError):
+            O.newton_schulz(G, 3, table, emulate_bf16=mode)
+
+
+def test_alternating_convergent_schedule_gives_polar_factor():
+    rng = np.random.default_rng(25)
+    U, V = _haar(rng, 12, 12), _haar(rng, 20, 12)
+    G = (U * np.linspace(1.0, 0.3, 12)) @ V.T
+    table = [(1.5, -0.5, 0.0), (15 / 8, -10 / 8, 3 / 8)] * 20
+    assert np.max(np.abs(O.newton_schulz(G, 40, table) - U @ V.T)) < 1e-10
+
+
+# ---------------------------------------------------------------------------
+# QK-Clip ("The Optimizer Wars", MuonClip): the q.k logit of a clipped head
+# scales by gamma_h = tau / S_max^h; other heads are untouched.
+# ---------------------------------------------------------------------------
+
+def test_qk_clip_scales_head_logits_by_gamma():
+    rng = np.random.default_rng(26)
+    heads, d, dm = 4, 8, 16
+    wq, wk = rng.standard_normal((heads * d, dm)), rng.standard_normal((heads * d, dm))
+    s_max = np.array([250.0, 50.0, 100.0, np.nan])
+    tau = 100.0
+    wq2, wk2 = O.qk_clip(wq, s_max, tau, d), O.qk_clip(wk, s_max, tau, d)
+    x, y = rng.standard_normal(dm), rng.standard_normal(dm)
+    for h in range(heads):
+        sl = slice(h * d, (h + 1) * d)
+        before = (wq[sl] @ x) @ (wk[sl] @ y)
+        after = (wq2[sl] @ x) @ (wk2[sl] @ y)
+        gamma = min(1.0, tau / s_max[h]) if np.isfinite(s_max[h]) else 1.0
+        assert after == pytest.approx(gamma * before, rel=1e-12)
+    assert np.array_equal(wq2[8:24], wq[8:24])
