@@ -286,13 +286,22 @@ def run_ours(args):
 
     opt = muon.Muon(device=local, cta_pair=args.cta_pair)
     stream = torch.cuda.current_stream()
+    stepper = opt
+    if args.layerwise:
+        # One matrix set for the whole job: each rank updates the matrices it
+        # owns and broadcasts them (layer-wise distributed Muon).
+        from muon_newton_schulz_03_b200.distributed import LayerwiseMuon
+        if world == 1:
+            dist.init_process_group("nccl", init_method="tcp://127.0.0.1:29511", rank=0, world_size=1,
+                                    device_id=device)
+        stepper = LayerwiseMuon(opt)
 
     def barrier():
         if world > 1:
             dist.barrier()
 
     for _ in range(args.warmup):
-        opt.step(params, grads, moms, lr=LR, beta=BETA, wd=WD, ns_steps=NS_STEPS)
+        stepper.step(params, grads, moms, lr=LR, beta=BETA, wd=WD, ns_steps=NS_STEPS)
     torch.cuda.synchronize()
     code, ew, nf = opt.status()
     if code != 0:
@@ -307,7 +316,7 @@ def run_ours(args):
     with ClockSampler(local) as clk:
         start.record(stream)
         for _ in range(args.steps):
-            opt.step(params, grads, moms, lr=LR, beta=BETA, wd=WD, ns_steps=NS_STEPS)
+            stepper.step(params, grads, moms, lr=LR, beta=BETA, wd=WD, ns_steps=NS_STEPS)
         end.record(stream)
         torch.cuda.synchronize()
     barrier()
@@ -345,7 +354,7 @@ def run_ours(args):
         cpu = cpu_baseline(args.workload)
 
     if rank == 0:
-        value = world * 1e3 / ms_step
+        value = (1 if args.layerwise else world) * 1e3 / ms_step
         traffic = profiled_traffic(args.workload)
         line = {
             "metric": METRIC,
@@ -356,7 +365,7 @@ def run_ours(args):
             "warmup": args.warmup,
             "ms_per_step": ms_step,
             "higher_is_better": True,
-            "scaling": "weak",
+            "scaling": "strong" if args.layerwise else "weak",
             "vs_baseline": None,
             "dtype": "bf16",
             "data": "synthetic",
@@ -369,7 +378,8 @@ def run_ours(args):
                 "ns_steps": NS_STEPS,
                 "lr": LR, "beta": BETA, "nesterov": True, "wd": WD, "scale": "moonlight 0.2*sqrt(max(m,n))",
                 "l2": "inputs larger than L2 (params, momenta, grads resident in HBM, no flush needed)",
-                "parallelism": f"replica per GPU x{world} (weak)",
+                "parallelism": (f"layer-wise ownership over {world} GPUs + broadcast (strong)" if args.layerwise
+                                else f"replica per GPU x{world} (weak)"),
                 "ns_tiles": "256x256 CTA pair (cta_group::2)" if args.cta_pair else "128x256 single CTA",
             },
             "ns_tflops_nominal": ns_tflops,
@@ -401,7 +411,7 @@ def run_ours(args):
             "clocks": clocks,
         }
         print(json.dumps(line), flush=True)
-    if world > 1:
+    if dist.is_initialized():
         dist.destroy_process_group()
     return 0
 
@@ -516,6 +526,8 @@ def main(argv=None):
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--layerwise", action="store_true",
+                    help="one matrix set per job, whole matrices owned by ranks, broadcast after the update")
     ap.add_argument("--cta-pair", action="store_true",
                     help="tiled phases on CTA pairs (256 x 256 tiles, cta_group::2) instead of single CTAs")
     args = ap.parse_args(argv)

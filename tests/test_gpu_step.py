@@ -424,3 +424,29 @@ def test_qk_clip_matches_oracle():
     assert rel(to64(wk), O.qk_clip(k0, sk.cpu().numpy(), 100.0, d)) <= TOL_ELEM
     assert np.array_equal(to64(wq)[64:128], q0[64:128])          # 30 < tau: untouched
     opt.close()
+
+
+def test_layerwise_single_rank_equals_plain_step():
+    # The layer-wise distributed wrapper over an NCCL group of one rank:
+    # every matrix is owned locally, the broadcasts are to self.
+    import socket
+    import torch.distributed as dist
+    from muon_newton_schulz_03_b200.distributed import LayerwiseMuon
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        port = s.getsockname()[1]
+    dist.init_process_group("nccl", init_method=f"tcp://127.0.0.1:{port}", rank=0, world_size=1)
+    try:
+        shapes = [(256, 768), (768, 256), (64, 64)]
+        cpu, dev = make_set(W.CONFIG_GPT2, shapes, torch.float32)
+        twin = [(d[0].clone(), d[1], d[2].clone()) for d in dev]
+        opt = muon.Muon(device=0)
+        LayerwiseMuon(opt).step([d[0] for d in dev], [d[1] for d in dev], [d[2] for d in dev], lr=2e-4)
+        opt.step([t[0] for t in twin], [t[1] for t in twin], [t[2] for t in twin], lr=2e-4)
+        torch.cuda.synchronize()
+        for d, t in zip(dev, twin):
+            assert torch.max(torch.abs(d[0] - t[0])) <= 1e-6 * torch.max(torch.abs(t[0]))
+            assert torch.equal(d[2], t[2])
+        opt.close()
+    finally:
+        dist.destroy_process_group()
