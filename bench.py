@@ -279,12 +279,13 @@ def run_ours(args):
 
     shapes, params, grads, moms, gdtype = make_inputs(torch, args.workload, device, rank)
     count = len(shapes)
-    nominal = W.total_ns_flops(shapes, NS_STEPS)
+    gram = args.ns_algorithm == "gram"
+    nominal = W.total_ns_flops(shapes, NS_STEPS, gram)
     gbytes = 2 if gdtype == torch.bfloat16 else 4
     k1_bytes = sum(W.step_bytes(m, n, gbytes)[0] for m, n in shapes)
     k4_bytes = sum(W.step_bytes(m, n, gbytes)[1] for m, n in shapes)
 
-    opt = muon.Muon(device=local, cta_pair=args.cta_pair)
+    opt = muon.Muon(device=local, cta_pair=args.cta_pair, ns_algorithm=args.ns_algorithm)
     stream = torch.cuda.current_stream()
     stepper = opt
     if args.layerwise:
@@ -338,7 +339,7 @@ def run_ours(args):
     k4_ms = statistics.mean(by_kind["apply"]) if by_kind.get("apply") else None
     ns_tflops = nominal / (ns_ms * 1e-3) / 1e12 if ns_ms > 0 else None
     avg_ns_launch_ms = ns_ms * args.steps / ns_launches if ns_launches else None
-    per_launch_flops = nominal / (3 * NS_STEPS)
+    per_launch_flops = nominal * args.steps / ns_launches if ns_launches else None
 
     clocks = clk.summary()
 
@@ -355,7 +356,7 @@ def run_ours(args):
 
     if rank == 0:
         value = (1 if args.layerwise else world) * 1e3 / ms_step
-        traffic = profiled_traffic(args.workload)
+        traffic = None if gram else profiled_traffic(args.workload)
         line = {
             "metric": METRIC,
             "value": value,
@@ -381,6 +382,7 @@ def run_ours(args):
                 "parallelism": (f"layer-wise ownership over {world} GPUs + broadcast (strong)" if args.layerwise
                                 else f"replica per GPU x{world} (weak)"),
                 "ns_tiles": "256x256 CTA pair (cta_group::2)" if args.cta_pair else "128x256 single CTA",
+                "ns_algorithm": ("Gram form, segments of 2 steps" if gram else "standard"),
             },
             "ns_tflops_nominal": ns_tflops,
             "ns_frac_of_datasheet_bf16": (ns_tflops / DATASHEET_BF16_TFLOPS) if ns_tflops else None,
@@ -403,7 +405,9 @@ def run_ours(args):
                 "peak_source": f"{peak_src} sustained dense bf16 (kernel timed inside a long step)",
                 "flops_per_launch_nominal": per_launch_flops,
                 "avg_launch_ms": avg_ns_launch_ms,
-                "flops_definition": "nominal 4 s^2 l + 2 s^3 per matrix per iteration (s = min(m,n), l = max)",
+                "flops_definition": ("Gram form: nominal 4 s^2 l + 10 s^3 per two-step segment, 4 s^2 l + 2 s^3 per "
+                                     "one-step segment (s = min(m,n), l = max)" if gram else
+                                     "nominal 4 s^2 l + 2 s^3 per matrix per iteration (s = min(m,n), l = max)"),
             },
             "cpu_baseline": cpu,
             "e2e": e2e,
@@ -530,6 +534,8 @@ def main(argv=None):
                     help="one matrix set per job, whole matrices owned by ranks, broadcast after the update")
     ap.add_argument("--cta-pair", action="store_true",
                     help="tiled phases on CTA pairs (256 x 256 tiles, cta_group::2) instead of single CTAs")
+    ap.add_argument("--ns-algorithm", choices=["standard", "gram"], default="standard",
+                    help="form of the Newton-Schulz iteration (the Gram form iterates on the s x s Gram)")
     args = ap.parse_args(argv)
     args.warmup = max(args.warmup, 3)   # at least three untimed steps
     if args.workload == "sweep":

@@ -93,6 +93,19 @@ enum muon_ns_precision {
   MUON_NS_FP32 = 1  /* debug: fp32 operands and FFMA accumulation          */
 };
 
+/* Form of the Newton-Schulz iteration. */
+enum muon_ns_algorithm {
+  MUON_NS_STANDARD = 0, /* X <- aX + (bA + cA^2)X, A = X X^T, each step
+                           ("About Muon: Why Not Adam", "The whole thing,
+                           in about forty lines")                          */
+  MUON_NS_GRAM = 1      /* the same polynomial iterated on the s x s Gram
+                           ("About Muon: Why Not Adam", "Gram
+                           Newton-Schulz"), in segments of two steps: a
+                           fresh Gram every second step; equal in exact
+                           arithmetic, fewer FLOPs when max(m,n) >> min(m,n).
+                           bf16 and single-CTA tiles only                  */
+};
+
 #define MUON_FLAG_GRAD_BF16 1
 
 typedef struct muon_config {
@@ -111,6 +124,7 @@ typedef struct muon_config {
                                  max(m,n) <= 512 run all iterations in one
                                  on-chip kernel (one CTA each); 0: every
                                  matrix uses the tiled phases. Default 1   */
+  int ns_algorithm;           /* enum muon_ns_algorithm; default STANDARD  */
   int cta_pair;               /* 1: tiled phases use 256 x 256 tiles on CTA
                                  pairs (tcgen05 cta_group::2); 0: 128 x 256
                                  tiles on single CTAs. Default 0 (both

@@ -28,6 +28,7 @@ __all__ = ["Muon", "MuonError", "plan_query", "x_layout", "round_up", "split_row
 DEFAULT_COEFFS = (3.4445, -4.7750, 2.0315)
 SCALE_MODES = {"moonlight": 0, "jordan": 1, "bernstein": 2, "none": 3}
 PRECISIONS = {"bf16": 0, "fp32": 1}
+ALGORITHMS = {"standard": 0, "gram": 1}
 FLAG_GRAD_BF16 = 1
 
 
@@ -152,7 +153,7 @@ class Muon:
     def __init__(self, device: int = 0, scale_mode: str = "moonlight", extra_scale: float = 1.0,
                  ns_precision: str = "bf16", check_nonfinite: bool = False, num_sms: int = 0,
                  workspace_cap_bytes: int = 0, wait_timeout_s: float = 2.0, small_path: bool = True,
-                 cta_pair: bool = False):
+                 cta_pair: bool = False, ns_algorithm: str = "standard"):
         self._lib = load()
         cfg = MuonConfig()
         check(self._lib.muon_config_init(ctypes.byref(cfg)))
@@ -165,6 +166,7 @@ class Muon:
         cfg.wait_timeout_s = float(wait_timeout_s)
         cfg.small_path = int(bool(small_path))
         cfg.cta_pair = int(bool(cta_pair))
+        cfg.ns_algorithm = ALGORITHMS[ns_algorithm]
         h = ctypes.c_void_p()
         check(self._lib.muon_init(int(device), ctypes.byref(cfg), ctypes.byref(h)))
         self._h = h
@@ -172,6 +174,7 @@ class Muon:
         self.ns_precision = ns_precision
         self.small_path = bool(small_path)
         self.cta_pair = bool(cta_pair)
+        self.ns_algorithm = ns_algorithm
 
     # -- lifetime -----------------------------------------------------------
     def close(self):

@@ -35,6 +35,7 @@ class MuonConfig(ctypes.Structure):
         ("workspace_cap_bytes", c_size_t),
         ("wait_timeout_s", c_double),
         ("small_path", c_int),
+        ("ns_algorithm", c_int),
         ("cta_pair", c_int),
     ]
 

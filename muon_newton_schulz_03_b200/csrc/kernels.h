@@ -30,8 +30,29 @@ cudaError_t launch_qk_clip(float* w, long long rows, long long cols, int head_ro
 cudaError_t launch_scale_copy(const ElemLaunch& L, int isel, int osel, const double* sumsq, bool fp32,
                               cudaStream_t st);
 
-// Newton-Schulz phases.
-enum NsPhase : int { PHASE_GRAM = 0, PHASE_POLY = 1, PHASE_COMB = 2 };
+// Newton-Schulz phases. PHASE_SYM is the product of two symmetric s x s
+// buffers used by the Gram form of the iteration.
+enum NsPhase : int { PHASE_GRAM = 0, PHASE_POLY = 1, PHASE_COMB = 2, PHASE_SYM = 3 };
+
+// The s x s buffers of a matrix: the Gram A and polynomial B of the plan,
+// and T and B1, used only by the Gram form.
+enum SymBuf : int { SB_A = 0, SB_B = 1, SB_T = 2, SB_B1 = 3, SB_NONE = -1 };
+
+struct GramBufs {
+  void* t;
+  void* b1;
+};
+constexpr int kGramMapsPerMat = 4;   // T (K-major 128- and 256-row boxes), B1 (same)
+
+// Operands and epilogue of one launch beyond the phase itself.
+struct PhaseSpec {
+  int poly_out = SB_B;                 // POLY: where B = bA + cA^2 goes
+  int sym_l = SB_A, sym_r = SB_A;      // SYM: D = L R (both symmetric)
+  int sym_out = SB_T;
+  int aux1 = SB_NONE, aux2 = SB_NONE;  // SYM: out = D + e1 aux1 + e2 aux2
+  float e1 = 0.0f, e2 = 0.0f;
+  int comb_b = SB_B;                   // COMB: left operand (SB_B or SB_T)
+};
 
 // Tensor maps of one matrix (bf16 path). Each CUtensorMap is 128 bytes and
 // must be 64-byte aligned in global memory.
@@ -62,6 +83,8 @@ struct NsLaunch {
   DevStatus* status;         // device
   int grid;                  // persistent CTAs
   unsigned long long timeout_ns;
+  const TmapBlob* gmaps = nullptr;   // device, kGramMapsPerMat per matrix (Gram form only)
+  const GramBufs* gbufs = nullptr;   // device, one per matrix (Gram form only)
 };
 
 // Small-matrix path: one CTA per listed matrix runs every iteration on chip.
@@ -88,7 +111,7 @@ int ns_pair_smem_bytes();
 int ns_pair_clusters_resident();
 
 cudaError_t launch_ns_phase_bf16(const NsLaunch& L, int phase, int src_sel, int dst_sel, int first, float a,
-                                 float b, float c, cudaStream_t st);
+                                 float b, float c, cudaStream_t st, const PhaseSpec& spec = PhaseSpec());
 
 // fp32 debug Newton-Schulz: one launch per matrix and phase.
 cudaError_t launch_ns_phase_fp32(const MatPlan& mp_host, int mat, int phase, const float* src, float* dst,

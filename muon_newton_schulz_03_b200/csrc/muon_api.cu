@@ -192,6 +192,9 @@ struct DevPlan {
   std::vector<int> chunk_tile_off[3];            // nchunks + 1 each
   int* d_chunk_small = nullptr;
   std::vector<int> chunk_small_off;              // nchunks + 1
+  void* gram_ws = nullptr;                       // Gram form: T and B1 per matrix
+  GramBufs* d_gbufs = nullptr;                   // device table of T / B1 pointers
+  TmapBlob* d_gmaps = nullptr;                   // device, kGramMapsPerMat per matrix
   void* staging = nullptr;                       // muon_step_host: kStagingSlots slots
   size_t staging_size = 0;
   size_t slot_bytes = 0;
@@ -240,9 +243,63 @@ void free_plan(DevPlan* p) {
   cudaFree(p->ws);
   cudaFree(p->tables);
   cudaFree(p->staging);
+  cudaFree(p->gram_ws);
+  cudaFree(p->d_gbufs);
 }
 
+
 int64_t align_up(int64_t x, int64_t a) { return (x + a - 1) / a * a; }
+
+// Extra s x s buffers (T, B1), their pointer table and tensor maps for the
+// Gram form of the iteration, for the matrices of the tile lists (the small
+// path keeps its matrices on chip).
+int ensure_gram_buffers(DevPlan& P) {
+  if (P.gram_ws || P.d_gbufs) return MUON_OK;
+  const int count = P.hp.count;
+  std::vector<char> tiled((size_t)count, 1);
+  for (int i : P.hp.small) tiled[(size_t)i] = 0;
+  std::vector<int64_t> off((size_t)count * 2, -1);
+  int64_t total = 0;
+  for (int i = 0; i < count; ++i)
+    if (tiled[(size_t)i])
+      for (int k = 0; k < 2; ++k) {
+        off[(size_t)i * 2 + k] = total;
+        total = align_up(total + (int64_t)P.mats[i].s * P.mats[i].lds * 2, kRegionAlign);
+      }
+  if (total > 0) {
+    cudaError_t e = cudaMalloc(&P.gram_ws, (size_t)total);
+    if (e != cudaSuccess) {
+      cudaGetLastError();
+      P.gram_ws = nullptr;
+      return fail(MUON_ERR_OOM, "Gram-form buffers of " + std::to_string(total) + " bytes failed to allocate");
+    }
+  }
+  const size_t tab_bytes = align_up(sizeof(GramBufs) * (size_t)count, 256);
+  const size_t map_bytes = sizeof(TmapBlob) * kGramMapsPerMat * (size_t)count;
+  std::vector<unsigned char> host(tab_bytes + map_bytes, 0);
+  GramBufs* gb = reinterpret_cast<GramBufs*>(host.data());
+  TmapBlob* gm = reinterpret_cast<TmapBlob*>(host.data() + tab_bytes);
+  char* base = static_cast<char*>(P.gram_ws);
+  for (int i = 0; i < count; ++i) {
+    if (!tiled[(size_t)i]) continue;
+    const MatPlan& mp = P.mats[i];
+    gb[i].t = base + off[(size_t)i * 2];
+    gb[i].b1 = base + off[(size_t)i * 2 + 1];
+    TmapBlob* m = gm + (size_t)i * kGramMapsPerMat;
+    int rc;
+    if ((rc = encode_map(m + 0, gb[i].t, mp.s, mp.s, mp.lds, 64, 128)) ||
+        (rc = encode_map(m + 1, gb[i].t, mp.s, mp.s, mp.lds, 64, 256)) ||
+        (rc = encode_map(m + 2, gb[i].b1, mp.s, mp.s, mp.lds, 64, 128)) ||
+        (rc = encode_map(m + 3, gb[i].b1, mp.s, mp.s, mp.lds, 64, 256)))
+      return rc;
+  }
+  void* d = nullptr;
+  MUON_CUDA_TRY(cudaMalloc(&d, host.size()));
+  P.d_gbufs = static_cast<GramBufs*>(d);
+  MUON_CUDA_TRY(cudaMemcpy(d, host.data(), host.size(), cudaMemcpyHostToDevice));
+  P.d_gmaps = reinterpret_cast<TmapBlob*>(static_cast<char*>(d) + tab_bytes);
+  return MUON_OK;
+}
 
 constexpr int kProfMaxPerCall = 256;
 
@@ -425,6 +482,12 @@ int ensure_plan(muon_handle* h, const int32_t* shapes, int count) {
   for (int p = 0; p < 3; ++p) np->d_chunk_tiles[p] = reinterpret_cast<int4*>(tb + o_ctiles[p]);
   np->d_chunk_small = reinterpret_cast<int*>(tb + o_csmall);
   np->d_maps = bf16 ? reinterpret_cast<TmapBlob*>(tb + o_maps) : nullptr;
+  // Gram-form buffers are made with the plan so that a captured step never
+  // allocates.
+  if (bf16 && h->cfg.ns_algorithm == MUON_NS_GRAM) {
+    const int rc = ensure_gram_buffers(*np);
+    if (rc) { free_plan(np.get()); return rc; }
+  }
   h->plan = std::move(np);
   return MUON_OK;
 }
@@ -543,11 +606,86 @@ int enqueue_ns(muon_handle* h, const MatBind* d_binds, const std::vector<MatBind
     S.sumsq = sumsq;
     S.status = h->status;
     S.timeout_ns = (unsigned long long)(h->cfg.wait_timeout_s * 1e9);
-    const int final_sel = last_dst >= 0 ? last_dst : (ns_steps % 2 == 1 ? BUF_X1 : BUF_X0);
+    const int flips = h->cfg.ns_algorithm == MUON_NS_GRAM ? (ns_steps + 1) / 2 : ns_steps;
+    const int final_sel = last_dst >= 0 ? last_dst : (flips % 2 == 1 ? BUF_X1 : BUF_X0);
     const int slot = prof_before(h, MUON_KERNEL_NS_SMALL, st);
     MUON_CUDA_TRY(launch_ns_small(S, ns_steps, first_src, final_sel, abc, st));
     prof_after(h, slot, st);
     ++*launches;
+  }
+  if (bf16 && h->cfg.ns_algorithm == MUON_NS_GRAM && ns_steps > 0) {
+    // Gram form, segments of two steps (one of one at an odd end):
+    //   A = X X^T; B0 = b0 A + c0 A^2;                       (GRAM, POLY)
+    //   T = a0 A + B0 A; A = a0 T + T B0;                    (SYM, SYM)
+    //   B1 = b1 A + c1 A^2;                                  (POLY)
+    //   T = a1 B0 + a0 B1 + B1 B0;  X' = a0 a1 X + T X        (SYM, COMB)
+    // a one-step segment is the plain step X' = a0 X + B0 X.
+    int rc;
+    if ((rc = ensure_gram_buffers(P))) return rc;
+    NsLaunch L;
+    L.plans = P.d_mats;
+    L.binds = d_binds;
+    L.maps = P.d_maps;
+    L.in_maps = d_in_maps;
+    L.sumsq = sumsq;
+    L.status = h->status;
+    L.grid = h->num_sms;
+    L.timeout_ns = (unsigned long long)(h->cfg.wait_timeout_s * 1e9);
+    L.gmaps = P.d_gmaps;
+    L.gbufs = P.d_gbufs;
+    auto run = [&](int phase, int src_sel, int dst_sel, int first, float a, float b, float c,
+                   const PhaseSpec& spec) -> int {
+      const int list = phase == PHASE_SYM ? PHASE_POLY : phase;
+      L.tiles = R.tiles[list];
+      L.ntiles = R.ntiles[list];
+      if (L.ntiles == 0) return MUON_OK;
+      const int kind = phase == PHASE_SYM ? MUON_KERNEL_NS_POLY : MUON_KERNEL_NS_GRAM + phase;
+      const int slot = prof_before(h, kind, st);
+      MUON_CUDA_TRY(launch_ns_phase_bf16(L, phase, src_sel, dst_sel, first, a, b, c, st, spec));
+      prof_after(h, slot, st);
+      ++*launches;
+      return MUON_OK;
+    };
+    int src = first_src;
+    bool first = true;
+    for (int k = 0; k < ns_steps;) {
+      const int len = std::min(2, ns_steps - k);
+      const bool last = k + len == ns_steps;
+      const int dst = (last && last_dst >= 0) ? last_dst : (src == BUF_X1 ? BUF_X0 : BUF_X1);
+      const float* c0 = abc + 3 * k;
+      PhaseSpec sp;
+      if ((rc = run(PHASE_GRAM, src, dst, first, 0.f, 0.f, 0.f, sp))) return rc;
+      sp.poly_out = SB_B;
+      if ((rc = run(PHASE_POLY, src, dst, 0, 0.f, c0[1], c0[2], sp))) return rc;
+      if (len == 2) {
+        const float* c1 = abc + 3 * (k + 1);
+        PhaseSpec s1;
+        s1.sym_l = SB_B; s1.sym_r = SB_A; s1.sym_out = SB_T; s1.aux1 = SB_A; s1.e1 = c0[0];
+        if ((rc = run(PHASE_SYM, src, dst, 0, 0.f, 0.f, 0.f, s1))) return rc;
+        PhaseSpec s2;
+        s2.sym_l = SB_T; s2.sym_r = SB_B; s2.sym_out = SB_A; s2.aux1 = SB_T; s2.e1 = c0[0];
+        if ((rc = run(PHASE_SYM, src, dst, 0, 0.f, 0.f, 0.f, s2))) return rc;
+        PhaseSpec s3;
+        s3.poly_out = SB_B1;
+        if ((rc = run(PHASE_POLY, src, dst, 0, 0.f, c1[1], c1[2], s3))) return rc;
+        PhaseSpec s4;
+        s4.sym_l = SB_B1; s4.sym_r = SB_B; s4.sym_out = SB_T;
+        s4.aux1 = SB_B; s4.e1 = c1[0]; s4.aux2 = SB_B1; s4.e2 = c0[0];
+        if ((rc = run(PHASE_SYM, src, dst, 0, 0.f, 0.f, 0.f, s4))) return rc;
+        PhaseSpec s5;
+        s5.comb_b = SB_T;
+        if ((rc = run(PHASE_COMB, src, dst, first, c0[0] * c1[0], 0.f, 0.f, s5))) return rc;
+      } else {
+        PhaseSpec s5;
+        s5.comb_b = SB_B;
+        if ((rc = run(PHASE_COMB, src, dst, first, c0[0], 0.f, 0.f, s5))) return rc;
+      }
+      src = dst;
+      first = false;
+      k += len;
+    }
+    *result = src;
+    return MUON_OK;
   }
   int src = first_src;
   for (int t = 1; t <= ns_steps; ++t) {
@@ -706,6 +844,7 @@ int muon_config_init(muon_config* cfg) {
   cfg->wait_timeout_s = 2.0;
   cfg->small_path = 1;
   cfg->cta_pair = 0;
+  cfg->ns_algorithm = MUON_NS_STANDARD;
   return MUON_OK;
 }
 
@@ -720,6 +859,10 @@ int muon_init(int device, const muon_config* cfg, muon_handle** out) {
   if (!(c.wait_timeout_s > 0.0 && c.wait_timeout_s <= 600.0))
     return fail(MUON_ERR_INVALID_ARG, "wait_timeout_s must be in (0, 600]");
   if (c.num_sms < 0) return fail(MUON_ERR_INVALID_ARG, "num_sms must be >= 0");
+  if (c.ns_algorithm != MUON_NS_STANDARD && c.ns_algorithm != MUON_NS_GRAM)
+    return fail(MUON_ERR_INVALID_ARG, "unknown ns_algorithm");
+  if (c.ns_algorithm == MUON_NS_GRAM && (c.ns_precision != MUON_NS_BF16 || c.cta_pair))
+    return fail(MUON_ERR_INVALID_ARG, "the Gram form runs in bf16 on single-CTA tiles (ns_precision 0, cta_pair 0)");
   int ndev = 0;
   if (cudaGetDeviceCount(&ndev) != cudaSuccess || ndev == 0) {
     cudaGetLastError();

@@ -57,6 +57,7 @@ struct NsArgs {
   NsLaunch L;
   int phase, src_sel, dst_sel, first;
   float a, b, c;
+  PhaseSpec spec;
 };
 
 // Everything a role needs to know about one tile.
@@ -72,6 +73,21 @@ struct TileJob {
 __device__ __forceinline__ const TmapBlob* src_maps(const NsLaunch& L, int mat, int src_sel) {
   if (src_sel == BUF_IN) return L.in_maps + (size_t)mat * kInMapsPerMat;
   return L.maps + (size_t)mat * kMapsPerMat + (src_sel == BUF_X0 ? MAP_X0 : MAP_X1);
+}
+
+// Tensor map of an s x s buffer: K-major box of 128 rows (or 256).
+__device__ __forceinline__ const TmapBlob* sym_map(const NsLaunch& L, int mat, int id, bool rows256) {
+  if (id == SB_A) return L.maps + (size_t)mat * kMapsPerMat + (rows256 ? MAP_A_K256 : MAP_A_K128);
+  if (id == SB_B) return L.maps + (size_t)mat * kMapsPerMat + (rows256 ? MAP_B_K256 : MAP_B_K128);
+  return L.gmaps + (size_t)mat * kGramMapsPerMat + (id == SB_T ? 0 : 2) + (rows256 ? 1 : 0);
+}
+
+__device__ __forceinline__ __nv_bfloat16* sym_ptr(const NsLaunch& L, const MatPlan& mp, int mat, int id) {
+  if (id == SB_A) return static_cast<__nv_bfloat16*>(mp.a);
+  if (id == SB_B) return static_cast<__nv_bfloat16*>(mp.b);
+  if (id == SB_T) return static_cast<__nv_bfloat16*>(L.gbufs[mat].t);
+  if (id == SB_B1) return static_cast<__nv_bfloat16*>(L.gbufs[mat].b1);
+  return nullptr;
 }
 
 __device__ __forceinline__ TileJob decode(const NsArgs& A, const int4 t, const MatPlan& mp) {
@@ -94,15 +110,19 @@ __device__ __forceinline__ TileJob decode(const NsArgs& A, const int4 t, const M
     j.kblocks = (mp.s + BK - 1) / BK;
     j.map_a = own + MAP_A_K128; j.a_mn = 0; j.a_coord = j.ti * BM;
     j.map_b = own + MAP_A_K256; j.b_mn = 0; j.b_coord = j.tj * BN;
+  } else if (A.phase == PHASE_SYM) {   // (L R)[i][j] = sum_k L[i][k] R[j][k], R symmetric
+    j.kblocks = (mp.s + BK - 1) / BK;
+    j.map_a = sym_map(A.L, j.mat, A.spec.sym_l, false); j.a_mn = 0; j.a_coord = j.ti * BM;
+    j.map_b = sym_map(A.L, j.mat, A.spec.sym_r, true);  j.b_mn = 0; j.b_coord = j.tj * BN;
   } else {
     const TmapBlob* xs = src_maps(A.L, j.mat, A.src_sel);
     j.kblocks = (mp.s + BK - 1) / BK;
     if (!mp.tall) {  // (B X)[r][c] = sum_k B[r][k] X[k][c]
-      j.map_a = own + MAP_B_K128; j.a_mn = 0; j.a_coord = j.ti * BM;
+      j.map_a = sym_map(A.L, j.mat, A.spec.comb_b, false); j.a_mn = 0; j.a_coord = j.ti * BM;
       j.map_b = xs + MAP_MN;      j.b_mn = 1; j.b_coord = j.tj * BN;
     } else {         // (X B)[r][c] = sum_k X[r][k] B[c][k]
       j.map_a = xs + MAP_K128;    j.a_mn = 0; j.a_coord = j.ti * BM;
-      j.map_b = own + MAP_B_K256; j.b_mn = 0; j.b_coord = j.tj * BN;
+      j.map_b = sym_map(A.L, j.mat, A.spec.comb_b, true); j.b_mn = 0; j.b_coord = j.tj * BN;
     }
   }
   return j;
@@ -278,14 +298,19 @@ __global__ void __launch_bounds__(kThreads, 1) ns_phase_kernel(const __grid_cons
       int rows, cols, ld;
       __nv_bfloat16* out;
       const __nv_bfloat16* aux = nullptr;
+      const __nv_bfloat16* aux2 = nullptr;
       int aux_ld = 0;
       float sc = 1.0f;
       if (phase == PHASE_GRAM) {
         rows = cols = mp.s; ld = mp.lds; out = static_cast<__nv_bfloat16*>(mp.a);
         if (args.first) { const double al = inv_norm(L.sumsq, tile.x); sc = (float)(al * al); }
       } else if (phase == PHASE_POLY) {
-        rows = cols = mp.s; ld = mp.lds; out = static_cast<__nv_bfloat16*>(mp.b);
+        rows = cols = mp.s; ld = mp.lds; out = sym_ptr(L, mp, tile.x, args.spec.poly_out);
         aux = static_cast<const __nv_bfloat16*>(mp.a); aux_ld = mp.lds;
+      } else if (phase == PHASE_SYM) {
+        rows = cols = mp.s; ld = mp.lds; out = sym_ptr(L, mp, tile.x, args.spec.sym_out);
+        aux = sym_ptr(L, mp, tile.x, args.spec.aux1); aux2 = sym_ptr(L, mp, tile.x, args.spec.aux2);
+        aux_ld = mp.lds;
       } else {
         rows = mp.m; cols = mp.n; ld = mp.ldx;
         out = static_cast<__nv_bfloat16*>(const_cast<void*>(sel_buf(mp, mb, args.dst_sel)));
@@ -293,6 +318,7 @@ __global__ void __launch_bounds__(kThreads, 1) ns_phase_kernel(const __grid_cons
         if (args.first) sc = (float)inv_norm(L.sumsq, tile.x);
       }
       const bool mirror = (phase != PHASE_COMB) && (tj > (ti >> 1));
+      const float e1 = args.spec.e1, e2 = args.spec.e2;
       const int row = ti * BM + row_in_tile;
       const bool row_ok = row < rows;
       const uint32_t t_base = tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(acc * BN);
@@ -306,7 +332,7 @@ __global__ void __launch_bounds__(kThreads, 1) ns_phase_kernel(const __grid_cons
         tmem_ld_32x32b_x32(t_base + (uint32_t)(ch * 32), v);
         const bool full_chunk = col0 + 32 <= cols;
         float o[32];
-        if (phase == PHASE_GRAM) {
+        if (phase == PHASE_GRAM || (phase == PHASE_SYM && aux == nullptr)) {
 #pragma unroll
           for (int i = 0; i < 32; ++i) o[i] = v[i] * sc;
         } else {
@@ -318,7 +344,24 @@ __global__ void __launch_bounds__(kThreads, 1) ns_phase_kernel(const __grid_cons
             for (int i = 0; i < 32; ++i)
               x[i] = (row_ok && col0 + i < cols) ? __bfloat162float(aux[(size_t)row * aux_ld + col0 + i]) : 0.0f;
           }
-          if (phase == PHASE_POLY) {
+          if (phase == PHASE_SYM) {
+            if (aux2 != nullptr) {
+              float y[32];
+              if (row_ok && full_chunk) {
+                load_bf16x32(aux2 + (size_t)row * aux_ld + col0, y);
+              } else {
+#pragma unroll
+                for (int i = 0; i < 32; ++i)
+                  y[i] = (row_ok && col0 + i < cols) ? __bfloat162float(aux2[(size_t)row * aux_ld + col0 + i])
+                                                     : 0.0f;
+              }
+#pragma unroll
+              for (int i = 0; i < 32; ++i) o[i] = fmaf(e1, x[i], fmaf(e2, y[i], v[i]));
+            } else {
+#pragma unroll
+              for (int i = 0; i < 32; ++i) o[i] = fmaf(e1, x[i], v[i]);
+            }
+          } else if (phase == PHASE_POLY) {
 #pragma unroll
             for (int i = 0; i < 32; ++i) o[i] = fmaf(cb, x[i], cc * v[i]);
           } else {
@@ -364,7 +407,7 @@ __global__ void __launch_bounds__(kThreads, 1) ns_phase_kernel(const __grid_cons
 int ns_bf16_smem_bytes() { return (int)sizeof(SmemLayout) + 1024; }
 
 cudaError_t launch_ns_phase_bf16(const NsLaunch& L, int phase, int src_sel, int dst_sel, int first, float a,
-                                 float b, float c, cudaStream_t st) {
+                                 float b, float c, cudaStream_t st, const PhaseSpec& spec) {
   if (L.ntiles <= 0) return cudaSuccess;
   static bool attr_set = false;
   const int smem = ns_bf16_smem_bytes();
@@ -382,6 +425,7 @@ cudaError_t launch_ns_phase_bf16(const NsLaunch& L, int phase, int src_sel, int 
   args.a = a;
   args.b = b;
   args.c = c;
+  args.spec = spec;
   const int grid = L.grid < L.ntiles ? L.grid : L.ntiles;
   ns_phase_kernel<<<grid, kThreads, smem, st>>>(args);
   return cudaGetLastError();

@@ -31,6 +31,7 @@ from .muon_oracle import (  # noqa: F401
     apply_update,
     bf16_round,
     coeff_rows,
+    gram_newton_schulz,
     momentum_update,
     muon_step,
     muon_step_matrix,

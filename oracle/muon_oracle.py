@@ -193,6 +193,75 @@ def newton_schulz(G, steps=5, coeffs=DEFAULT_COEFFS, eps=EPS,
     return X.T if transposed else X
 
 
+def gram_newton_schulz(G, steps=5, coeffs=DEFAULT_COEFFS, eps=EPS, emulate_bf16=False, accum_fp32=False,
+                       segment=2):
+    """Gram Newton-Schulz ("About Muon: Why Not Adam", section "Gram
+    Newton-Schulz"): the same odd polynomial, iterated on the small Gram.
+
+    With X the normalised short-side-first matrix, a segment of L steps
+    forms A = X X^T once and then, for each step, B = bA + cA^2 (so the
+    plain step is X <- (aI + B) X); the segment's product
+    Q = (a_L I + B_L) ... (a_1 I + B_1) is applied to X at the end, and the
+    Gram is carried between the steps of a segment as A <- P A P (the Gram
+    of P X, P = aI + B commutes with A). In exact arithmetic every segment
+    length gives ``newton_schulz``. Reading: segments of 2 steps (a fresh
+    Gram every second step) keep bf16 rounding from accumulating in the
+    carried Gram; ``segment=None`` runs all steps in one segment (exact mode
+    only). The aI parts are never stored: with B0, B1 the two steps' B,
+      R = a0 A + B0 A,   A1 = a0 R + R B0,
+      Q - a0 a1 I = a1 B0 + a0 B1 + B1 B0,
+      X' = a0 a1 X + (Q - a0 a1 I) X.
+    With ``emulate_bf16`` each of A, B0, R, A1, B1, Q - a0 a1 I and X' is
+    rounded to bf16 (the normalisation folded into the first segment's Gram
+    as alpha^2 and its final product as alpha).
+    """
+    G = np.asarray(G, dtype=np.float64)
+    if G.ndim != 2:
+        raise ValueError("Newton-Schulz is defined for 2D matrices only")
+    rows = coeff_rows(coeffs, steps)
+    seg = steps if segment is None else int(segment)
+    if emulate_bf16 and not 1 <= seg <= 2:
+        raise ValueError("the bf16 mode restates segments of 1 or 2 steps")
+    rnd = bf16_round if emulate_bf16 else (lambda v: v)
+    acc = accum_fp32 and emulate_bf16
+    transposed = G.shape[0] > G.shape[1]
+    alpha = 1.0 / (np.linalg.norm(G) + eps)
+    X = bf16_round(G) if emulate_bf16 else G
+    if transposed:
+        X = X.T
+    if steps == 0:
+        X = alpha * X
+        return X.T if transposed else X
+    k, sc = 0, alpha
+    while k < steps:
+        L = min(max(seg, 1), steps - k)
+        A = rnd(sc * sc * _matmul(X, X.T, acc))
+        if emulate_bf16 or L <= 2:
+            a0, b0, c0 = rows[k]
+            B0 = rnd(b0 * A + c0 * _matmul(A, A, acc))
+            if L == 1:
+                X = rnd(sc * (a0 * X + _matmul(B0, X, acc)))
+            else:
+                a1, b1, c1 = rows[k + 1]
+                R = rnd(a0 * A + _matmul(B0, A, acc))
+                A1 = rnd(a0 * R + _matmul(R, B0, acc))
+                B1 = rnd(b1 * A1 + c1 * _matmul(A1, A1, acc))
+                Qd = rnd(a1 * B0 + a0 * B1 + _matmul(B1, B0, acc))
+                X = rnd(sc * (a0 * a1 * X + _matmul(Qd, X, acc)))
+        else:
+            eye = np.eye(A.shape[0])
+            Q = None
+            for j in range(L):
+                a, b, c = rows[k + j]
+                P = a * eye + b * A + c * (A @ A)
+                Q = P if Q is None else P @ Q
+                A = P @ A @ P
+            X = sc * (Q @ X)
+        k += L
+        sc = 1.0
+    return X.T if transposed else X
+
+
 def ns_only(X, steps=5, coeffs=DEFAULT_COEFFS, emulate_bf16=False, accum_fp32=False):
     """The Newton-Schulz phases alone on an already-scaled X (no norm).
 
@@ -285,8 +354,11 @@ def apply_update(p, O, lr, wd, scale):
 def muon_step_matrix(p, g, m, *, lr, beta=0.95, nesterov=True, wd=0.1,
                      ns_steps=5, coeffs=DEFAULT_COEFFS,
                      scale_mode=SCALE_MOONLIGHT, extra_scale=1.0,
-                     emulate_bf16=False, accum_fp32=False):
+                     emulate_bf16=False, accum_fp32=False, gram=False):
     """One Muon step on one matrix. Returns (p', m', O, ||u||_F).
+
+    ``gram`` selects the Gram form of Newton-Schulz (same result in exact
+    arithmetic).
 
     Order: momentum, Nesterov blend, Newton-Schulz (normalise, orient,
     iterate, orient back), scale, decoupled weight decay, write.
@@ -297,7 +369,10 @@ def muon_step_matrix(p, g, m, *, lr, beta=0.95, nesterov=True, wd=0.1,
     m_new = momentum_update(m, g, beta)
     u = nesterov_blend(g, m_new, beta, nesterov)
     nu = float(np.linalg.norm(u))
-    O = newton_schulz(u, ns_steps, coeffs, EPS, emulate_bf16, accum_fp32)
+    if gram:
+        O = gram_newton_schulz(u, ns_steps, coeffs, EPS, emulate_bf16, accum_fp32)
+    else:
+        O = newton_schulz(u, ns_steps, coeffs, EPS, emulate_bf16, accum_fp32)
     scale = update_scale(p.shape[0], p.shape[1], scale_mode, extra_scale)
     p_new = apply_update(p, O, lr, wd, scale)
     return p_new, m_new, O, nu

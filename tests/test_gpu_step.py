@@ -24,12 +24,13 @@ F32 = lambda v: float(np.float32(v))  # noqa: E731  (scalars as the kernels see 
 
 
 def _check_step(cpu, dev, shapes, opt, *, lr, beta, wd, nesterov=True, ns_steps=5, scale_mode=O.SCALE_MOONLIGHT,
-                tol=TOL_BF16_NS, check_o=True, indices=None):
+                tol=TOL_BF16_NS, check_o=True, indices=None, gram_mats=()):
     indices = range(len(shapes)) if indices is None else indices
     worst = 0.0
     for i in indices:
         m, n = shapes[i]
         p0, g, m0 = cpu[i]
+        gram = i in gram_mats
         p_ref, m_ref, o_ref, nu = O.muon_step_matrix(p0, g, m0, lr=F32(lr), beta=F32(beta), nesterov=nesterov,
                                                      wd=F32(wd), ns_steps=ns_steps, scale_mode=scale_mode)
         p_gpu, _, m_gpu = (to64(t) for t in dev[i])
@@ -39,7 +40,7 @@ def _check_step(cpu, dev, shapes, opt, *, lr, beta, wd, nesterov=True, ns_steps=
         bf16 = opt.ns_precision == "bf16"
         if bf16:
             kw = dict(lr=F32(lr), beta=F32(beta), nesterov=nesterov, wd=F32(wd), ns_steps=ns_steps,
-                      scale_mode=scale_mode, emulate_bf16=True)
+                      scale_mode=scale_mode, emulate_bf16=True, gram=gram)
             p_emu, _, o_emu, _ = O.muon_step_matrix(p0, g, m0, **kw)
             p_e32, _, o_e32, _ = O.muon_step_matrix(p0, g, m0, accum_fp32=True, **kw)
             e = bf16_gate(dp_gpu, dp_ref, p_emu - p0, p_e32 - p0, f"update of matrix {i} {m}x{n}")[0]
@@ -49,7 +50,8 @@ def _check_step(cpu, dev, shapes, opt, *, lr, beta, wd, nesterov=True, ns_steps=
         worst = max(worst, e)
         if check_o and ns_steps > 0:
             dtype = torch.bfloat16 if bf16 else torch.float32
-            o_gpu = to64(workspace_matrix(opt, shapes, i, ns_steps % 2, dtype)[:, :n])
+            flips = (ns_steps + 1) // 2 if gram_mats else ns_steps
+            o_gpu = to64(workspace_matrix(opt, shapes, i, flips % 2, dtype)[:, :n])
             if bf16:
                 bf16_gate(o_gpu, o_ref, o_emu, o_e32, f"O of matrix {i}")
             else:
@@ -346,6 +348,32 @@ def test_mixed_small_and_tiled_matrices_in_one_step():
     assert opt.last_launch_count() == 1 + 1 + 15 + 1
     assert opt.status() == (0, 0, 0)
     opt.close()
+
+
+@pytest.mark.parametrize("ns_steps", [5, 4, 1])
+def test_gram_form_step(ns_steps):
+    # The Gram form on the tiled phases: wide, tall, square and ragged
+    # matrices, one-step and two-step segments. The small path (kept in the
+    # standard form) handles the small matrices of the same call.
+    shapes = [(256, 1024), (1024, 256), (384, 384), (300, 1000), (1000, 300), (600, 257), (128, 512), (64, 96)]
+    plan = muon.plan_query(shapes)
+    cpu, dev = make_set(W.CONFIG_GPT2, shapes, torch.float32)
+    opt = muon.Muon(device=0, ns_algorithm="gram")
+    opt.step([d[0] for d in dev], [d[1] for d in dev], [d[2] for d in dev], lr=2e-4, beta=0.95, wd=0.1,
+             ns_steps=ns_steps)
+    torch.cuda.synchronize()
+    tiled = [i for i in range(len(shapes)) if i not in plan["small"]]
+    _check_step(cpu, dev, shapes, opt, lr=2e-4, beta=0.95, wd=0.1, ns_steps=ns_steps, gram_mats=tiled)
+    segs2, segs1 = ns_steps // 2, ns_steps % 2
+    assert opt.last_launch_count() == 1 + 1 + 7 * segs2 + 3 * segs1 + 1
+    assert opt.status() == (0, 0, 0)
+    opt.close()
+
+
+def test_gram_form_rejected_with_fp32_or_pairs():
+    for kw in (dict(ns_precision="fp32"), dict(cta_pair=True)):
+        with pytest.raises(muon.MuonError):
+            muon.Muon(device=0, ns_algorithm="gram", **kw)
 
 
 def test_split_muon_qkv_and_per_head():

@@ -509,3 +509,47 @@ def test_qk_clip_scales_head_logits_by_gamma():
         gamma = min(1.0, tau / s_max[h]) if np.isfinite(s_max[h]) else 1.0
         assert after == pytest.approx(gamma * before, rel=1e-12)
     assert np.array_equal(wq2[8:24], wq[8:24])
+
+
+# ---------------------------------------------------------------------------
+# Gram Newton-Schulz ("About Muon: Why Not Adam", section "Gram
+# Newton-Schulz"): in exact arithmetic it returns the same matrix.
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("shape", [(3, 5), (8, 8), (16, 4), (33, 17), (20, 70), (1, 9)])
+@pytest.mark.parametrize("steps", [0, 1, 2, 5])
+@pytest.mark.parametrize("segment", [1, 2, None])
+def test_gram_ns_equals_standard_ns(shape, steps, segment):
+    rng = np.random.default_rng(hash(shape) % 2 ** 32 + 7 * steps)
+    G = rng.standard_normal(shape)
+    U, sig, Vt = np.linalg.svd(G, full_matrices=False)
+    x = sig / (np.linalg.norm(G) + O.EPS)
+    a, b, c = O.DEFAULT_COEFFS
+    for _ in range(steps):
+        x = a * x + b * x ** 3 + c * x ** 5
+    got = O.gram_newton_schulz(G, steps, segment=segment)
+    assert np.max(np.abs(got - (U * x) @ Vt)) < 1e-11
+    assert np.max(np.abs(got - O.newton_schulz(G, steps))) < 1e-11
+
+
+def test_gram_ns_segment_one_is_the_standard_bf16_iteration():
+    rng = np.random.default_rng(29)
+    G = rng.standard_normal((24, 56))
+    assert np.array_equal(O.gram_newton_schulz(G, 5, emulate_bf16=True, segment=1),
+                          O.newton_schulz(G, 5, emulate_bf16=True))
+
+
+def test_gram_ns_with_schedule_and_bf16_structure(monkeypatch):
+    rng = np.random.default_rng(27)
+    G = rng.standard_normal((12, 30))
+    table = [(3.4445, -4.7750, 2.0315), (1.875, -1.25, 0.375), (1.5, -0.5, 0.0)]
+    assert np.max(np.abs(O.gram_newton_schulz(G, 3, table) - O.newton_schulz(G, 3, table))) < 1e-11
+    monkeypatch.setattr(O, "bf16_round", lambda v: np.asarray(v, dtype=np.float64))
+    a = O.gram_newton_schulz(G, 5, emulate_bf16=True)
+    monkeypatch.undo()
+    assert np.max(np.abs(a - O.newton_schulz(G, 5))) < 1e-11
+    rng = np.random.default_rng(28)
+    p, g = rng.standard_normal((10, 40)), rng.standard_normal((10, 40))
+    r1 = O.muon_step_matrix(p, g, np.zeros_like(p), lr=0.1, gram=True)
+    r2 = O.muon_step_matrix(p, g, np.zeros_like(p), lr=0.1)
+    assert np.max(np.abs(r1[0] - r2[0])) < 1e-12

@@ -209,6 +209,15 @@ def ns_flops(m: int, n: int, steps: int = 5) -> float:
     return steps * (4.0 * s * s * l + 2.0 * s ** 3)
 
 
+def gram_ns_flops(m: int, n: int, steps: int = 5) -> float:
+    """Nominal FLOPs of the Gram form in segments of two steps: per
+    two-step segment one Gram and one final product (2 s^2 l each) and five
+    s x s products (2 s^3 each); a one-step segment is the plain step."""
+    s, l = min(m, n), max(m, n)
+    two, one = steps // 2, steps % 2
+    return two * (4.0 * s * s * l + 10.0 * s ** 3) + one * (4.0 * s * s * l + 2.0 * s ** 3)
+
+
 def step_bytes(m: int, n: int, grad_bytes: int) -> tuple:
     """Algorithmic HBM bytes of the two elementwise kernels per matrix.
 
@@ -233,8 +242,9 @@ def total_elements(shapes) -> int:
     return int(sum(m * n for m, n in shapes))
 
 
-def total_ns_flops(shapes, steps: int = 5) -> float:
-    return float(sum(ns_flops(m, n, steps) for m, n in shapes))
+def total_ns_flops(shapes, steps: int = 5, gram: bool = False) -> float:
+    f = gram_ns_flops if gram else ns_flops
+    return float(sum(f(m, n, steps) for m, n in shapes))
 
 
 __all__ = [name for name in dir() if not name.startswith("_") and name not in ("annotations", "math", "np")]
