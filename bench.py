@@ -330,11 +330,40 @@ def run_ours(args):
 
     ms_step = max_over_ranks(torch, dist, elapsed_ms / args.steps, device)
 
+    # The same step captured once in a CUDA graph and replayed (no host work
+    # per step: launch overhead and host-side checks drop out).
+    graph_ms = None
+    if not args.layerwise and not args.no_graph:
+        side = torch.cuda.Stream(device)
+        side.wait_stream(stream)
+        with torch.cuda.stream(side):
+            opt.step(params, grads, moms, lr=LR, beta=BETA, wd=WD, ns_steps=NS_STEPS)
+        stream.wait_stream(side)
+        torch.cuda.synchronize()
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            opt.step(params, grads, moms, lr=LR, beta=BETA, wd=WD, ns_steps=NS_STEPS)
+        for _ in range(2):
+            graph.replay()
+        barrier()
+        torch.cuda.synchronize()
+        start.record(stream)
+        for _ in range(args.steps):
+            graph.replay()
+        end.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        graph_ms = max_over_ranks(torch, dist, start.elapsed_time(end) / args.steps, device)
+        del graph
+        code, ew, nf = opt.status()
+        if code != 0:
+            raise RuntimeError(f"device status {code} after graph replay (error word {ew}, non-finite {nf})")
+
     by_kind = {}
     for kind, ms in prof:
         by_kind.setdefault(kind, []).append(ms)
-    ns_ms = sum(sum(by_kind.get(k, [])) for k in ("ns_gram", "ns_poly", "ns_comb")) / args.steps
-    ns_launches = sum(len(by_kind.get(k, [])) for k in ("ns_gram", "ns_poly", "ns_comb"))
+    ns_ms = sum(sum(by_kind.get(k, [])) for k in ("ns_gram", "ns_poly", "ns_comb", "ns_sym")) / args.steps
+    ns_launches = sum(len(by_kind.get(k, [])) for k in ("ns_gram", "ns_poly", "ns_comb", "ns_sym"))
     k1_ms = statistics.mean(by_kind["momentum_norm"]) if by_kind.get("momentum_norm") else None
     k4_ms = statistics.mean(by_kind["apply"]) if by_kind.get("apply") else None
     ns_tflops = nominal / (ns_ms * 1e-3) / 1e12 if ns_ms > 0 else None
@@ -409,6 +438,9 @@ def run_ours(args):
                                      "one-step segment (s = min(m,n), l = max)" if gram else
                                      "nominal 4 s^2 l + 2 s^3 per matrix per iteration (s = min(m,n), l = max)"),
             },
+            "graph": ({"ms_per_step": graph_ms, "value": (1 if args.layerwise else world) * 1e3 / graph_ms,
+                       "unit": "steps/s", "note": "one step captured in a CUDA graph, replayed"}
+                      if graph_ms else None),
             "cpu_baseline": cpu,
             "e2e": e2e,
             "gpu_launches": launches_per_step * args.steps,
@@ -530,6 +562,7 @@ def main(argv=None):
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-graph", action="store_true", help="skip the CUDA-graph replay timing")
     ap.add_argument("--layerwise", action="store_true",
                     help="one matrix set per job, whole matrices owned by ranks, broadcast after the update")
     ap.add_argument("--cta-pair", action="store_true",

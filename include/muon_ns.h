@@ -125,6 +125,11 @@ typedef struct muon_config {
                                  on-chip kernel (one CTA each); 0: every
                                  matrix uses the tiled phases. Default 1   */
   int ns_algorithm;           /* enum muon_ns_algorithm; default STANDARD  */
+  int deterministic;          /* 1: the per-matrix sum of squares is added
+                                 in a fixed order (per-block partials, then
+                                 one more launch), so repeated steps on the
+                                 same inputs are bitwise identical; 0
+                                 (default): one double atomic per block    */
   int cta_pair;               /* 1: tiled phases use 256 x 256 tiles on CTA
                                  pairs (tcgen05 cta_group::2); 0: 128 x 256
                                  tiles on single CTAs. Default 0 (both
@@ -303,7 +308,9 @@ enum muon_kernel_kind {
   MUON_KERNEL_APPLY = 4,         /* stage 3                                   */
   MUON_KERNEL_SCALE_COPY = 5,    /* zero-iteration Newton-Schulz stage        */
   MUON_KERNEL_NS_FP32 = 6,       /* fp32 debug phase (one matrix)             */
-  MUON_KERNEL_NS_SMALL = 7       /* on-chip small-matrix path, all iterations */
+  MUON_KERNEL_NS_SMALL = 7,      /* on-chip small-matrix path, all iterations */
+  MUON_KERNEL_NORM_REDUCE = 8,   /* fixed-order norm sum (deterministic mode) */
+  MUON_KERNEL_NS_SYM = 9         /* symmetric-product phase of the Gram form  */
 };
 
 /* Per-launch timing for measurements. With max_calls > 0, each of the next

@@ -153,7 +153,7 @@ class Muon:
     def __init__(self, device: int = 0, scale_mode: str = "moonlight", extra_scale: float = 1.0,
                  ns_precision: str = "bf16", check_nonfinite: bool = False, num_sms: int = 0,
                  workspace_cap_bytes: int = 0, wait_timeout_s: float = 2.0, small_path: bool = True,
-                 cta_pair: bool = False, ns_algorithm: str = "standard"):
+                 cta_pair: bool = False, ns_algorithm: str = "standard", deterministic: bool = False):
         self._lib = load()
         cfg = MuonConfig()
         check(self._lib.muon_config_init(ctypes.byref(cfg)))
@@ -167,6 +167,7 @@ class Muon:
         cfg.small_path = int(bool(small_path))
         cfg.cta_pair = int(bool(cta_pair))
         cfg.ns_algorithm = ALGORITHMS[ns_algorithm]
+        cfg.deterministic = int(bool(deterministic))
         h = ctypes.c_void_p()
         check(self._lib.muon_init(int(device), ctypes.byref(cfg), ctypes.byref(h)))
         self._h = h
@@ -364,7 +365,8 @@ class Muon:
         check(self._lib.muon_workspace_ptr(self._h, ctypes.byref(base), ctypes.byref(size)))
         return base.value or 0, size.value
 
-    KERNEL_KINDS = ("momentum_norm", "ns_gram", "ns_poly", "ns_comb", "apply", "scale_copy", "ns_fp32", "ns_small")
+    KERNEL_KINDS = ("momentum_norm", "ns_gram", "ns_poly", "ns_comb", "apply", "scale_copy", "ns_fp32", "ns_small",
+                    "norm_reduce", "ns_sym")
 
     def profile_enable(self, max_calls: int):
         """Record CUDA events around every kernel of the next max_calls calls."""

@@ -36,6 +36,7 @@ class MuonConfig(ctypes.Structure):
         ("wait_timeout_s", c_double),
         ("small_path", c_int),
         ("ns_algorithm", c_int),
+        ("deterministic", c_int),
         ("cta_pair", c_int),
     ]
 

@@ -109,7 +109,7 @@ template <bool kFp32Out>
 __global__ void __launch_bounds__(kThreads) k1_momentum_norm(
     const MatPlan* __restrict__ plans, const MatBind* __restrict__ binds, const long long* __restrict__ prefix,
     int count, long long block_base, int ysel, float beta, int nesterov, double* __restrict__ sumsq,
-    DevStatus* status, int check_nonfinite) {
+    double* __restrict__ partials, DevStatus* status, int check_nonfinite) {
   __shared__ double red[kThreads / 32];
   __shared__ unsigned redc[kThreads / 32];
   const long long blk = (long long)blockIdx.x + block_base;
@@ -160,12 +160,34 @@ __global__ void __launch_bounds__(kThreads) k1_momentum_norm(
     }
   }
   const double tot = block_sum(acc, red);
-  if (threadIdx.x == 0) atomicAdd(sumsq + mat, tot);
+  if (threadIdx.x == 0) {
+    if (partials != nullptr) partials[blk] = tot;   // fixed-order sum later
+    else atomicAdd(sumsq + mat, tot);
+  }
   if (check_nonfinite) {
     __syncthreads();
     const unsigned nb = block_count(bad, redc);
     if (threadIdx.x == 0 && nb) atomicAdd(&status->nonfinite, (unsigned long long)nb);
   }
+}
+
+// Deterministic norm: one warp per matrix adds that matrix's per-block
+// partial sums in a fixed order (lane-strided, then a fixed shuffle tree).
+__global__ void __launch_bounds__(kThreads) k1b_reduce_partials(const MatBind* __restrict__ binds,
+                                                                const long long* __restrict__ prefix, int m0,
+                                                                int m1, const double* __restrict__ partials,
+                                                                double* __restrict__ sumsq) {
+  const int mat = m0 + (int)((blockIdx.x * (unsigned)kThreads + threadIdx.x) >> 5);
+  const int lane = threadIdx.x & 31;
+  if (mat >= m1) return;
+  const MatBind mb = binds[mat];
+  if (!mb.active || mb.g == nullptr) return;
+  const long long b0 = prefix[mat], b1 = prefix[mat + 1];
+  double v = 0.0;
+  for (long long b = b0 + lane; b < b1; b += 32) v += partials[b];
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  if (lane == 0) sumsq[mat] = v;
 }
 
 __device__ __forceinline__ float update_scale_dev(int m, int n, int mode, float extra) {
@@ -274,16 +296,26 @@ cudaError_t launch_qk_clip(float* w, long long rows, long long cols, int head_ro
 }
 
 cudaError_t launch_momentum_norm(const ElemLaunch& L, int ysel, float beta, int nesterov, double* sumsq,
-                                 DevStatus* status, int check_nonfinite, bool fp32_out, cudaStream_t st) {
+                                 double* partials, DevStatus* status, int check_nonfinite, bool fp32_out,
+                                 cudaStream_t st) {
   if (L.nblocks <= 0) return cudaSuccess;
   if (fp32_out)
-    k1_momentum_norm<true><<<(unsigned)L.nblocks, kThreads, 0, st>>>(L.plans, L.binds, L.prefix, L.count, L.block_base, ysel,
-                                                                      beta, nesterov, sumsq, status,
-                                                                      check_nonfinite);
+    k1_momentum_norm<true><<<(unsigned)L.nblocks, kThreads, 0, st>>>(L.plans, L.binds, L.prefix, L.count,
+                                                                      L.block_base, ysel, beta, nesterov, sumsq,
+                                                                      partials, status, check_nonfinite);
   else
-    k1_momentum_norm<false><<<(unsigned)L.nblocks, kThreads, 0, st>>>(L.plans, L.binds, L.prefix, L.count, L.block_base, ysel,
-                                                                       beta, nesterov, sumsq, status,
-                                                                       check_nonfinite);
+    k1_momentum_norm<false><<<(unsigned)L.nblocks, kThreads, 0, st>>>(L.plans, L.binds, L.prefix, L.count,
+                                                                       L.block_base, ysel, beta, nesterov, sumsq,
+                                                                       partials, status, check_nonfinite);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_reduce_partials(const ElemLaunch& L, int m0, int m1, const double* partials, double* sumsq,
+                                   cudaStream_t st) {
+  if (m1 <= m0) return cudaSuccess;
+  const int warps_per_block = kThreads / 32;
+  const unsigned grid = (unsigned)((m1 - m0 + warps_per_block - 1) / warps_per_block);
+  k1b_reduce_partials<<<grid, kThreads, 0, st>>>(L.binds, L.prefix, m0, m1, partials, sumsq);
   return cudaGetLastError();
 }
 

@@ -19,8 +19,14 @@ struct ElemLaunch {
   long long nblocks;        // chunks in the launch (prefix[count] for a whole set)
 };
 
+// partials == nullptr: one double atomic per block into sumsq; else each
+// block stores its partial at partials[block] and launch_reduce_partials
+// adds them per matrix in a fixed order (bitwise reproducible norms).
 cudaError_t launch_momentum_norm(const ElemLaunch& L, int ysel, float beta, int nesterov, double* sumsq,
-                                 DevStatus* status, int check_nonfinite, bool fp32_out, cudaStream_t st);
+                                 double* partials, DevStatus* status, int check_nonfinite, bool fp32_out,
+                                 cudaStream_t st);
+cudaError_t launch_reduce_partials(const ElemLaunch& L, int m0, int m1, const double* partials, double* sumsq,
+                                   cudaStream_t st);
 cudaError_t launch_apply(const ElemLaunch& L, int osel, float lr, float wd, int scale_mode, float extra_scale,
                          const double* sumsq, bool fp32_in, cudaStream_t st);
 // QK-Clip: rows of head h scaled by sqrt(tau / s_max[h]) when s_max[h] > tau.
@@ -42,7 +48,9 @@ struct GramBufs {
   void* t;
   void* b1;
 };
-constexpr int kGramMapsPerMat = 4;   // T (K-major 128- and 256-row boxes), B1 (same)
+// T (K-major 128- and 256-row boxes), B1 (same), then the 32 x 32 store
+// boxes of T and B1.
+constexpr int kGramMapsPerMat = 6;
 
 // Operands and epilogue of one launch beyond the phase itself.
 struct PhaseSpec {
@@ -68,7 +76,9 @@ enum MapIdx : int {
   MAP_K128 = 0, MAP_K256 = 1, MAP_MN = 2,   // offsets inside a triple
   MAP_A_K128 = 6, MAP_A_K256 = 7,
   MAP_B_K128 = 8, MAP_B_K256 = 9,
-  kMapsPerMat = 10,
+  // 32 x 32 boxes with 64-byte swizzle for the epilogue's bulk stores
+  MAP_X0_ST = 10, MAP_X1_ST = 11, MAP_A_ST = 12, MAP_B_ST = 13,
+  kMapsPerMat = 14,
   kInMapsPerMat = 3
 };
 
@@ -84,6 +94,8 @@ struct NsLaunch {
   int grid;                  // persistent CTAs
   unsigned long long timeout_ns;
   const TmapBlob* gmaps = nullptr;   // device, kGramMapsPerMat per matrix (Gram form only)
+  int tma_store = 0;                 // 1: the *_ST store maps are present, stage outputs
+                                     //    in shared memory and write them with bulk stores
   const GramBufs* gbufs = nullptr;   // device, one per matrix (Gram form only)
 };
 

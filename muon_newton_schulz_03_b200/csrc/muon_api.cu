@@ -138,7 +138,8 @@ EncodeTiledFn get_encode_fn() {
 
 // 2D bf16 row-major tensor (rows x cols, leading dimension ld elements),
 // 128-byte swizzle, box of box_cols (inner) x box_rows.
-int encode_map(TmapBlob* out, const void* base, int rows, int cols, int ld, int box_cols, int box_rows) {
+int encode_map(TmapBlob* out, const void* base, int rows, int cols, int ld, int box_cols, int box_rows,
+               CUtensorMapSwizzle swizzle = CU_TENSOR_MAP_SWIZZLE_128B) {
   static_assert(sizeof(CUtensorMap) == sizeof(TmapBlob), "tensor map size");
   EncodeTiledFn enc = get_encode_fn();
   if (!enc) return fail(MUON_ERR_CUDA, "cuTensorMapEncodeTiled is not available");
@@ -147,7 +148,7 @@ int encode_map(TmapBlob* out, const void* base, int rows, int cols, int ld, int 
   cuuint32_t box[2] = {(cuuint32_t)box_cols, (cuuint32_t)box_rows};
   cuuint32_t estr[2] = {1, 1};
   CUresult r = enc(reinterpret_cast<CUtensorMap*>(out), CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base),
-                   dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle,
                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return fail(MUON_ERR_CUDA, "cuTensorMapEncodeTiled failed: " + std::to_string((int)r));
   return MUON_OK;
@@ -161,6 +162,11 @@ int encode_x_triple(TmapBlob* out3, const void* base, const MatPlan& mp) {
   if ((rc = encode_map(out3 + MAP_K256, base, mp.m, mp.n, mp.ldx, 64, 256))) return rc;
   if ((rc = encode_map(out3 + MAP_MN, base, mp.m, mp.n, mp.ldx, 64, 64))) return rc;
   return MUON_OK;
+}
+
+// 32 x 32 store box with 64-byte swizzle (the epilogue's staging layout).
+int encode_store_map(TmapBlob* out, const void* base, int rows, int cols, int ld) {
+  return encode_map(out, base, rows, cols, ld, 32, 32, CU_TENSOR_MAP_SWIZZLE_64B);
 }
 
 }  // namespace
@@ -192,6 +198,7 @@ struct DevPlan {
   std::vector<int> chunk_tile_off[3];            // nchunks + 1 each
   int* d_chunk_small = nullptr;
   std::vector<int> chunk_small_off;              // nchunks + 1
+  double* partials = nullptr;                    // deterministic norm: one per K1 block
   void* gram_ws = nullptr;                       // Gram form: T and B1 per matrix
   GramBufs* d_gbufs = nullptr;                   // device table of T / B1 pointers
   TmapBlob* d_gmaps = nullptr;                   // device, kGramMapsPerMat per matrix
@@ -245,6 +252,7 @@ void free_plan(DevPlan* p) {
   cudaFree(p->staging);
   cudaFree(p->gram_ws);
   cudaFree(p->d_gbufs);
+  cudaFree(p->partials);
 }
 
 
@@ -290,7 +298,9 @@ int ensure_gram_buffers(DevPlan& P) {
     if ((rc = encode_map(m + 0, gb[i].t, mp.s, mp.s, mp.lds, 64, 128)) ||
         (rc = encode_map(m + 1, gb[i].t, mp.s, mp.s, mp.lds, 64, 256)) ||
         (rc = encode_map(m + 2, gb[i].b1, mp.s, mp.s, mp.lds, 64, 128)) ||
-        (rc = encode_map(m + 3, gb[i].b1, mp.s, mp.s, mp.lds, 64, 256)))
+        (rc = encode_map(m + 3, gb[i].b1, mp.s, mp.s, mp.lds, 64, 256)) ||
+        (rc = encode_store_map(m + 4, gb[i].t, mp.s, mp.s, mp.lds)) ||
+        (rc = encode_store_map(m + 5, gb[i].b1, mp.s, mp.s, mp.lds)))
       return rc;
   }
   void* d = nullptr;
@@ -461,6 +471,13 @@ int ensure_plan(muon_handle* h, const int32_t* shapes, int count) {
       if ((rc = encode_map(mm + MAP_A_K256, mp.a, mp.s, mp.s, mp.lds, 64, 256))) { free_plan(np.get()); return rc; }
       if ((rc = encode_map(mm + MAP_B_K128, mp.b, mp.s, mp.s, mp.lds, 64, 128))) { free_plan(np.get()); return rc; }
       if ((rc = encode_map(mm + MAP_B_K256, mp.b, mp.s, mp.s, mp.lds, 64, 256))) { free_plan(np.get()); return rc; }
+      if ((rc = encode_store_map(mm + MAP_X0_ST, mp.x0, mp.m, mp.n, mp.ldx)) ||
+          (rc = encode_store_map(mm + MAP_X1_ST, mp.x1, mp.m, mp.n, mp.ldx)) ||
+          (rc = encode_store_map(mm + MAP_A_ST, mp.a, mp.s, mp.s, mp.lds)) ||
+          (rc = encode_store_map(mm + MAP_B_ST, mp.b, mp.s, mp.s, mp.lds))) {
+        free_plan(np.get());
+        return rc;
+      }
     }
   }
   e = cudaMalloc(&np->tables, (size_t)off);
@@ -482,6 +499,15 @@ int ensure_plan(muon_handle* h, const int32_t* shapes, int count) {
   for (int p = 0; p < 3; ++p) np->d_chunk_tiles[p] = reinterpret_cast<int4*>(tb + o_ctiles[p]);
   np->d_chunk_small = reinterpret_cast<int*>(tb + o_csmall);
   np->d_maps = bf16 ? reinterpret_cast<TmapBlob*>(tb + o_maps) : nullptr;
+  if (h->cfg.deterministic) {
+    const size_t nb = sizeof(double) * (size_t)std::max<long long>(hp.prefix[count], 1);
+    if (cudaMalloc(reinterpret_cast<void**>(&np->partials), nb) != cudaSuccess) {
+      cudaGetLastError();
+      np->partials = nullptr;
+      free_plan(np.get());
+      return fail(MUON_ERR_OOM, "norm partials of " + std::to_string(nb) + " bytes failed to allocate");
+    }
+  }
   // Gram-form buffers are made with the plan so that a captured step never
   // allocates.
   if (bf16 && h->cfg.ns_algorithm == MUON_NS_GRAM) {
@@ -633,13 +659,14 @@ int enqueue_ns(muon_handle* h, const MatBind* d_binds, const std::vector<MatBind
     L.timeout_ns = (unsigned long long)(h->cfg.wait_timeout_s * 1e9);
     L.gmaps = P.d_gmaps;
     L.gbufs = P.d_gbufs;
+    L.tma_store = 1;
     auto run = [&](int phase, int src_sel, int dst_sel, int first, float a, float b, float c,
                    const PhaseSpec& spec) -> int {
       const int list = phase == PHASE_SYM ? PHASE_POLY : phase;
       L.tiles = R.tiles[list];
       L.ntiles = R.ntiles[list];
       if (L.ntiles == 0) return MUON_OK;
-      const int kind = phase == PHASE_SYM ? MUON_KERNEL_NS_POLY : MUON_KERNEL_NS_GRAM + phase;
+      const int kind = phase == PHASE_SYM ? MUON_KERNEL_NS_SYM : MUON_KERNEL_NS_GRAM + phase;
       const int slot = prof_before(h, kind, st);
       MUON_CUDA_TRY(launch_ns_phase_bf16(L, phase, src_sel, dst_sel, first, a, b, c, st, spec));
       prof_after(h, slot, st);
@@ -702,6 +729,7 @@ int enqueue_ns(muon_handle* h, const MatBind* d_binds, const std::vector<MatBind
       L.status = h->status;
       L.grid = h->num_sms;
       L.timeout_ns = (unsigned long long)(h->cfg.wait_timeout_s * 1e9);
+      L.tma_store = 1;
       for (int ph = 0; ph < 3; ++ph) {
         L.tiles = R.tiles[ph];
         L.ntiles = R.ntiles[ph];
@@ -790,10 +818,16 @@ int enqueue_step_range(muon_handle* h, const MatBind* db, const std::vector<MatB
   MUON_CUDA_TRY(cudaMemsetAsync(sumsq + R.m0, 0, sizeof(double) * (size_t)(R.m1 - R.m0), st));
   const ElemLaunch EL = elem_launch(P, db, R);
   int slot = prof_before(h, MUON_KERNEL_MOMENTUM_NORM, st);
-  MUON_CUDA_TRY(launch_momentum_norm(EL, BUF_X0, beta, nesterov ? 1 : 0, sumsq, h->status, h->cfg.check_nonfinite,
-                                     fp32, st));
+  MUON_CUDA_TRY(launch_momentum_norm(EL, BUF_X0, beta, nesterov ? 1 : 0, sumsq, P.partials, h->status,
+                                     h->cfg.check_nonfinite, fp32, st));
   prof_after(h, slot, st);
   ++*launches;
+  if (P.partials) {
+    slot = prof_before(h, MUON_KERNEL_NORM_REDUCE, st);
+    MUON_CUDA_TRY(launch_reduce_partials(EL, R.m0, R.m1, P.partials, sumsq, st));
+    prof_after(h, slot, st);
+    ++*launches;
+  }
   int res = BUF_X0;
   if ((rc = enqueue_ns(h, db, hb, R, nullptr, sumsq, ns_steps, abc, BUF_X0, -1, st, launches, &res))) return rc;
   slot = prof_before(h, MUON_KERNEL_APPLY, st);
@@ -845,6 +879,7 @@ int muon_config_init(muon_config* cfg) {
   cfg->small_path = 1;
   cfg->cta_pair = 0;
   cfg->ns_algorithm = MUON_NS_STANDARD;
+  cfg->deterministic = 0;
   return MUON_OK;
 }
 
@@ -859,6 +894,7 @@ int muon_init(int device, const muon_config* cfg, muon_handle** out) {
   if (!(c.wait_timeout_s > 0.0 && c.wait_timeout_s <= 600.0))
     return fail(MUON_ERR_INVALID_ARG, "wait_timeout_s must be in (0, 600]");
   if (c.num_sms < 0) return fail(MUON_ERR_INVALID_ARG, "num_sms must be >= 0");
+  if (c.deterministic != 0 && c.deterministic != 1) return fail(MUON_ERR_INVALID_ARG, "deterministic must be 0 or 1");
   if (c.ns_algorithm != MUON_NS_STANDARD && c.ns_algorithm != MUON_NS_GRAM)
     return fail(MUON_ERR_INVALID_ARG, "unknown ns_algorithm");
   if (c.ns_algorithm == MUON_NS_GRAM && (c.ns_precision != MUON_NS_BF16 || c.cta_pair))
@@ -1106,12 +1142,18 @@ int muon_momentum_norm(muon_handle* h, const void* const* grads, float* const* m
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   MUON_CUDA_TRY(cudaMemsetAsync(sumsq, 0, sizeof(double) * count, st));
   prof_call_begin(h);
-  const int slot = prof_before(h, MUON_KERNEL_MOMENTUM_NORM, st);
-  MUON_CUDA_TRY(launch_momentum_norm(elem_launch(P, static_cast<const MatBind*>(d_binds)), BUF_OUT, beta,
-                                     nesterov ? 1 : 0, sumsq, h->status, h->cfg.check_nonfinite,
-                                     h->cfg.ns_precision == MUON_NS_FP32, st));
+  const ElemLaunch EL = elem_launch(P, static_cast<const MatBind*>(d_binds));
+  int slot = prof_before(h, MUON_KERNEL_MOMENTUM_NORM, st);
+  MUON_CUDA_TRY(launch_momentum_norm(EL, BUF_OUT, beta, nesterov ? 1 : 0, sumsq, P.partials, h->status,
+                                     h->cfg.check_nonfinite, h->cfg.ns_precision == MUON_NS_FP32, st));
   prof_after(h, slot, st);
   h->last_launches = 1;
+  if (P.partials) {
+    slot = prof_before(h, MUON_KERNEL_NORM_REDUCE, st);
+    MUON_CUDA_TRY(launch_reduce_partials(EL, 0, count, P.partials, sumsq, st));
+    prof_after(h, slot, st);
+    h->last_launches = 2;
+  }
   return MUON_OK;
 }
 

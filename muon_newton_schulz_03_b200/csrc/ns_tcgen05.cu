@@ -42,9 +42,14 @@ constexpr int kStageBytes = kABytes + kBBytes;  // 48 KiB
 constexpr int kMnChunkBytes = 64 * BK * 2;      // one 64 (M/N) x 64 (K) box, 8 KiB
 constexpr int kThreads = 192;
 constexpr int kTmemCols = 2 * BN;               // two fp32 accumulators
+constexpr int kOutBox = 32;                     // bulk-store box: 32 rows x 32 columns
+constexpr int kOutStageBytes = kOutBox * kOutBox * 2;
 
 struct __align__(1024) SmemLayout {
   uint8_t stage[kStages][kStageBytes];
+  // Epilogue staging for bulk stores: per epilogue warp two direct and two
+  // transposed 32 x 32 bf16 blocks (64-byte rows, 64-byte swizzle).
+  uint8_t ostage[4][4][kOutStageBytes];
   uint64_t full[kStages];
   uint64_t empty[kStages];
   uint64_t acc_full[2];
@@ -88,6 +93,20 @@ __device__ __forceinline__ __nv_bfloat16* sym_ptr(const NsLaunch& L, const MatPl
   if (id == SB_T) return static_cast<__nv_bfloat16*>(L.gbufs[mat].t);
   if (id == SB_B1) return static_cast<__nv_bfloat16*>(L.gbufs[mat].b1);
   return nullptr;
+}
+
+// Store map (32 x 32 box) of an s x s buffer.
+__device__ __forceinline__ const TmapBlob* sym_store_map(const NsLaunch& L, int mat, int id) {
+  if (id == SB_A) return L.maps + (size_t)mat * kMapsPerMat + MAP_A_ST;
+  if (id == SB_B) return L.maps + (size_t)mat * kMapsPerMat + MAP_B_ST;
+  return L.gmaps + (size_t)mat * kGramMapsPerMat + (id == SB_T ? 4 : 5);
+}
+
+// Byte offset of the 16-byte group `q` of row `r` in a 32 x 32 bf16 block
+// with 64-byte rows and the 64-byte swizzle of the bulk-tensor unit (the
+// group index is XORed with bits 1..2 of the row).
+__device__ __forceinline__ uint32_t sw64_offset(int r, int q) {
+  return (uint32_t)(r * 64 + ((q ^ ((r >> 1) & 3)) << 4));
 }
 
 __device__ __forceinline__ TileJob decode(const NsArgs& A, const int4 t, const MatPlan& mp) {
@@ -285,6 +304,8 @@ __global__ void __launch_bounds__(kThreads, 1) ns_phase_kernel(const __grid_cons
     const int row_in_tile = quarter * 32 + lane;
     int acc = 0;
     uint32_t acc_phase = 0;
+    int obuf = 0;   // staging block pair used by this warp's next chunk
+    const bool tma_out = L.tma_store != 0 && !(args.phase == PHASE_COMB && args.dst_sel == BUF_OUT);
     for (int t = blockIdx.x; t < L.ntiles; t += gridDim.x) {
       const int4 tile = L.tiles[t];
       const MatBind mb = L.binds[tile.x];
@@ -318,6 +339,14 @@ __global__ void __launch_bounds__(kThreads, 1) ns_phase_kernel(const __grid_cons
         if (args.first) sc = (float)inv_norm(L.sumsq, tile.x);
       }
       const bool mirror = (phase != PHASE_COMB) && (tj > (ti >> 1));
+      const TmapBlob* st_map = nullptr;
+      if (tma_out) {
+        if (phase == PHASE_GRAM) st_map = sym_store_map(L, tile.x, SB_A);
+        else if (phase == PHASE_POLY) st_map = sym_store_map(L, tile.x, args.spec.poly_out);
+        else if (phase == PHASE_SYM) st_map = sym_store_map(L, tile.x, args.spec.sym_out);
+        else st_map = L.maps + (size_t)tile.x * kMapsPerMat + (args.dst_sel == BUF_X0 ? MAP_X0_ST : MAP_X1_ST);
+      }
+      const int warp_row0 = ti * BM + quarter * 32;
       const float e1 = args.spec.e1, e2 = args.spec.e2;
       const int row = ti * BM + row_in_tile;
       const bool row_ok = row < rows;
@@ -369,6 +398,43 @@ __global__ void __launch_bounds__(kThreads, 1) ns_phase_kernel(const __grid_cons
             for (int i = 0; i < 32; ++i) o[i] = sc * fmaf(ca, x[i], v[i]);
           }
         }
+        if (tma_out) {
+          // Stage the 32 x 32 block (and its transpose) in shared memory and
+          // write it with bulk stores; the tensor map clips rows and columns
+          // beyond the matrix.
+          uint8_t* dbuf = sm.ostage[quarter][obuf];
+          uint8_t* mbuf = sm.ostage[quarter][2 + obuf];
+          if (lane == 0) bulk_wait_group_read<1>();   // the pair used two chunks ago is free
+          __syncwarp();
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            uint4 raw;
+            __nv_bfloat162* h = reinterpret_cast<__nv_bfloat162*>(&raw);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) h[i] = __floats2bfloat162_rn(o[8 * q + 2 * i], o[8 * q + 2 * i + 1]);
+            *reinterpret_cast<uint4*>(dbuf + sw64_offset(lane, q)) = raw;
+          }
+          if (mirror) {
+            // Element (j, lane) of the transposed block: for a fixed j the
+            // warp writes one 64-byte row.
+            const uint32_t in_group = (uint32_t)(lane & 7) * 2;
+#pragma unroll
+            for (int j = 0; j < 32; ++j)
+              *reinterpret_cast<__nv_bfloat16*>(mbuf + sw64_offset(j, lane >> 3) + in_group) =
+                  __float2bfloat16_rn(o[j]);
+          }
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            if (warp_row0 < rows) {
+              tma_store_2d(st_map, dbuf, col0, warp_row0);
+              if (mirror) tma_store_2d(st_map, mbuf, warp_row0, col0);
+            }
+            bulk_commit_group();
+          }
+          obuf ^= 1;
+          continue;
+        }
         if (row_ok) {
           __nv_bfloat16* dst = out + (size_t)row * ld + col0;
           if (full_chunk) {
@@ -392,6 +458,8 @@ __global__ void __launch_bounds__(kThreads, 1) ns_phase_kernel(const __grid_cons
       if (lane == 0) mbar_arrive(&sm.acc_empty[acc]);
       if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
     }
+    // Bulk stores read this CTA's shared memory: let them finish.
+    if (tma_out && lane == 0) bulk_wait_group_all();
   }
 
   tc_fence_before();

@@ -140,7 +140,7 @@ def test_config_defaults():
     assert lib.muon_config_init(ctypes.byref(cfg)) == 0
     assert cfg.scale_mode == 0 and cfg.extra_scale == 1.0 and cfg.ns_precision == 0
     assert cfg.wait_timeout_s == 2.0 and cfg.num_sms == 0 and cfg.small_path == 1 and cfg.cta_pair == 0
-    assert cfg.ns_algorithm == 0
+    assert cfg.ns_algorithm == 0 and cfg.deterministic == 0
     assert lib.muon_config_init(None) == 1
 
 

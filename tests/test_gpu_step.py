@@ -16,7 +16,7 @@ import workloads as W
 from oracle import muon_oracle as O
 
 from gpu_helpers import (DEV, TOL_BF16_NS, TOL_ELEM, TOL_FP32_NS, bf16_gate, cuda_bf16, cuda_f32, make_set, rel,
-                         to64, workspace_matrix)
+                         to64, workspace_matrix, x_buffer)
 
 pytestmark = pytest.mark.gpu
 
@@ -368,6 +368,37 @@ def test_gram_form_step(ns_steps):
     assert opt.last_launch_count() == 1 + 1 + 7 * segs2 + 3 * segs1 + 1
     assert opt.status() == (0, 0, 0)
     opt.close()
+
+
+def test_deterministic_norm_is_bitwise_repeatable():
+    # Fixed-order norm sums: two steps on identical copies of the inputs give
+    # identical bits, and the step still meets the oracle's gates.
+    shapes = [(2304, 768), (768, 3072), (300, 1000), (64, 96), (4096, 1024)]
+    cpu, dev = make_set(W.CONFIG_GPT2, shapes, torch.float32)
+    twin = [(p.clone(), g.clone(), m.clone()) for (p, g, m) in dev]
+    opt = muon.Muon(device=0, deterministic=True)
+    for d in (dev, twin):
+        opt.step([x[0] for x in d], [x[1] for x in d], [x[2] for x in d], lr=2e-4, beta=0.95, wd=0.1)
+    torch.cuda.synchronize()
+    for (p, _, m), (p2, _, m2) in zip(dev, twin):
+        assert torch.equal(p, p2) and torch.equal(m, m2)
+    _check_step(cpu, dev, shapes, opt, lr=2e-4, beta=0.95, wd=0.1)
+    assert opt.last_launch_count() == 1 + 1 + 1 + 15 + 1   # K1, fixed-order sum, small path, phases, apply
+    # The stage entry point: the same sums as the atomic mode to fp64 rounding.
+    ref = muon.Muon(device=0)
+    sums = []
+    for o in (opt, ref):
+        moms = [torch.zeros(s, dtype=torch.float32, device=DEV) for s in shapes]
+        ys = [x_buffer(m, n) for (m, n) in shapes]
+        ss = torch.zeros(len(shapes), dtype=torch.float64, device=DEV)
+        o.momentum_norm([x[1] for x in twin], moms, ys, ss, beta=0.95)
+        sums.append(ss.cpu().numpy())
+    torch.cuda.synchronize()
+    assert opt.last_launch_count() == 2
+    assert np.allclose(sums[0], sums[1], rtol=1e-13, atol=0)
+    assert opt.status() == (0, 0, 0)
+    opt.close()
+    ref.close()
 
 
 def test_gram_form_rejected_with_fp32_or_pairs():
