@@ -43,9 +43,13 @@ constexpr int kStageBytes = 2 * kHalfBytes;  // A half + B half
 constexpr int kMnChunkBytes = 64 * BK * 2;   // one 64 x 64 M/N-major box
 constexpr int kThreads = 192;
 constexpr int kTmemCols = 2 * BN;            // two 256-column fp32 accumulators
+constexpr int kOutStageBytes = 32 * 32 * 2;  // one 32 x 32 bf16 bulk-store block
 
 struct __align__(1024) PairSmem {
   uint8_t stage[kStages][kStageBytes];
+  // Epilogue staging for bulk stores: per epilogue warp two direct and two
+  // transposed 32 x 32 blocks (64-byte rows, 64-byte swizzle).
+  uint8_t ostage[4][4][kOutStageBytes];
   uint64_t full[kStages];      // leader only: both CTAs' copies of the stage landed
   uint64_t empty[kStages];     // MMAs reading the stage are done (both CTAs)
   uint64_t acc_full[2];        // accumulator ready (both CTAs)
@@ -107,6 +111,12 @@ __device__ __forceinline__ PairJob decode_pair(const PairArgs& A, const int4 t, 
   j.a_coord = ra;
   j.b_coord = rb;
   return j;
+}
+
+// Byte offset of 16-byte group q of row r in a 32 x 32 bf16 block with
+// 64-byte rows under the bulk-tensor unit's 64-byte swizzle.
+__device__ __forceinline__ uint32_t sw64_off(int r, int q) {
+  return (uint32_t)(r * 64 + ((q ^ ((r >> 1) & 3)) << 4));
 }
 
 __device__ __forceinline__ void store_row32(__nv_bfloat16* dst, const float (&o)[32]) {
@@ -279,6 +289,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     const uint32_t leader_acc_empty0 = map_shared_rank(&sm.acc_empty[0], 0);
     int acc = 0;
     uint32_t acc_phase = 0;
+    int obuf = 0;
+    const bool tma_out = L.tma_store != 0 && !(args.phase == PHASE_COMB && args.dst_sel == BUF_OUT);
     for (int t = cid; t < L.ntiles; t += ncl) {
       const int4 tile = L.tiles[t];
       const MatBind mb = L.binds[tile.x];
@@ -307,6 +319,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         if (args.first) sc = (float)inv_norm(L.sumsq, tile.x);
       }
       const bool mirror = (phase != PHASE_COMB) && (tj > ti);
+      const TmapBlob* own_maps = L.maps + (size_t)tile.x * kMapsPerMat;
+      const TmapBlob* st_map = phase == PHASE_GRAM ? own_maps + MAP_A_ST
+                               : phase == PHASE_POLY ? own_maps + MAP_B_ST
+                               : own_maps + (args.dst_sel == BUF_X0 ? MAP_X0_ST : MAP_X1_ST);
+      const int warp_row0 = ti * BM + rank * kHalf + quarter * 32;
       const int row = ti * BM + rank * kHalf + row_in_half;
       const bool row_ok = row < rows;
       const uint32_t t_base = tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(acc * BN);
@@ -340,6 +357,37 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             for (int i = 0; i < 32; ++i) o[i] = sc * fmaf(ca, x[i], v[i]);
           }
         }
+        if (tma_out) {
+          uint8_t* dbuf = sm.ostage[quarter][obuf];
+          uint8_t* mbuf = sm.ostage[quarter][2 + obuf];
+          if (lane == 0) bulk_wait_group_read<1>();   // the pair used two chunks ago is free
+          __syncwarp();
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            uint4 raw;
+            __nv_bfloat162* h = reinterpret_cast<__nv_bfloat162*>(&raw);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) h[i] = __floats2bfloat162_rn(o[8 * q + 2 * i], o[8 * q + 2 * i + 1]);
+            *reinterpret_cast<uint4*>(dbuf + sw64_off(lane, q)) = raw;
+          }
+          if (mirror) {
+            const uint32_t in_group = (uint32_t)(lane & 7) * 2;
+#pragma unroll
+            for (int j = 0; j < 32; ++j)
+              *reinterpret_cast<__nv_bfloat16*>(mbuf + sw64_off(j, lane >> 3) + in_group) = __float2bfloat16_rn(o[j]);
+          }
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            if (warp_row0 < rows) {
+              tma_store_2d(st_map, dbuf, col0, warp_row0);
+              if (mirror) tma_store_2d(st_map, mbuf, warp_row0, col0);
+            }
+            bulk_commit_group();
+          }
+          obuf ^= 1;
+          continue;
+        }
         if (row_ok) {
           __nv_bfloat16* dst = out + (size_t)row * ld + col0;
           if (full_chunk) {
@@ -361,6 +409,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       if (lane == 0) mbar_arrive_cluster(leader_acc_empty0 + (uint32_t)(acc * sizeof(uint64_t)));
       if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
     }
+    if (tma_out && lane == 0) bulk_wait_group_all();
   }
 
   tc_fence_before();
