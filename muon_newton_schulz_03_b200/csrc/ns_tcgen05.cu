@@ -172,6 +172,43 @@ __device__ __forceinline__ void load_bf16x32(const __nv_bfloat16* src, float (&o
   }
 }
 
+// 32 consecutive bf16 of one row, as raw 16-byte groups; entries past the
+// last column (or of a row past the last row) read as zero.
+__device__ __forceinline__ void load_aux_chunk(const __nv_bfloat16* row_ptr, int col0, int cols, bool row_ok,
+                                               uint4 (&r)[4]) {
+  if (row_ok && col0 + 32 <= cols) {
+    const uint4* p = reinterpret_cast<const uint4*>(row_ptr + col0);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) r[q] = p[q];
+  } else {
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      uint32_t w[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int c0 = col0 + 8 * q + 2 * i;
+        const uint32_t lo = (row_ok && c0 < cols) ? (uint32_t)__bfloat16_as_ushort(row_ptr[c0]) : 0u;
+        const uint32_t hi = (row_ok && c0 + 1 < cols) ? (uint32_t)__bfloat16_as_ushort(row_ptr[c0 + 1]) : 0u;
+        w[i] = lo | (hi << 16);
+      }
+      r[q] = make_uint4(w[0], w[1], w[2], w[3]);
+    }
+  }
+}
+
+__device__ __forceinline__ void unpack_bf16x32(const uint4 (&r)[4], float (&o)[32]) {
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&r[q]);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float2 f = __bfloat1622float2(h[i]);
+      o[8 * q + 2 * i] = f.x;
+      o[8 * q + 2 * i + 1] = f.y;
+    }
+  }
+}
+
 __global__ void __launch_bounds__(kThreads, 1) ns_phase_kernel(const __grid_constant__ NsArgs args) {
   extern __shared__ uint8_t smem_raw[];
   SmemLayout& sm = *reinterpret_cast<SmemLayout*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -311,9 +348,10 @@ __global__ void __launch_bounds__(kThreads, 1) ns_phase_kernel(const __grid_cons
       const MatBind mb = L.binds[tile.x];
       if (!mb.active) continue;
       const MatPlan mp = L.plans[tile.x];
-      if (!mbar_wait_bounded(&sm.acc_full[acc], acc_phase, err, tmo, WAIT_ACC_FULL)) break;
-      tc_fence_after();
 
+      // Everything that does not need the accumulator is set up before
+      // waiting for it, and the first chunk of the auxiliary operand is
+      // already on its way.
       const int ti = tile.y, tj = tile.z;
       const int phase = args.phase;
       int rows, cols, ld;
@@ -352,27 +390,29 @@ __global__ void __launch_bounds__(kThreads, 1) ns_phase_kernel(const __grid_cons
       const bool row_ok = row < rows;
       const uint32_t t_base = tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(acc * BN);
       const float ca = args.a, cb = args.b, cc = args.c;
+      const __nv_bfloat16* aux_row = aux != nullptr ? aux + (size_t)row * aux_ld : nullptr;
+      uint4 xa[4], xb[4];   // packed bf16 auxiliary values of the current and the next chunk
+      if (aux_row != nullptr) load_aux_chunk(aux_row, tj * BN, cols, row_ok, xa);
 
-#pragma unroll 1
-      for (int ch = 0; ch < BN / 32; ++ch) {
+      if (!mbar_wait_bounded(&sm.acc_full[acc], acc_phase, err, tmo, WAIT_ACC_FULL)) break;
+      tc_fence_after();
+
+      // One 32-column chunk: returns false past the last column.
+      auto chunk = [&](int ch, const uint4 (&cur)[4], uint4 (&nxt)[4]) -> bool {
         const int col0 = tj * BN + ch * 32;
-        if (col0 >= cols) break;                       // warp-uniform
+        if (col0 >= cols) return false;                // warp-uniform
+        if (aux_row != nullptr && ch + 1 < BN / 32 && col0 + 32 < cols)
+          load_aux_chunk(aux_row, col0 + 32, cols, row_ok, nxt);
         float v[32];
         tmem_ld_32x32b_x32(t_base + (uint32_t)(ch * 32), v);
         const bool full_chunk = col0 + 32 <= cols;
         float o[32];
-        if (phase == PHASE_GRAM || (phase == PHASE_SYM && aux == nullptr)) {
+        if (aux_row == nullptr) {
 #pragma unroll
           for (int i = 0; i < 32; ++i) o[i] = v[i] * sc;
         } else {
           float x[32];
-          if (row_ok && full_chunk) {
-            load_bf16x32(aux + (size_t)row * aux_ld + col0, x);
-          } else {
-#pragma unroll
-            for (int i = 0; i < 32; ++i)
-              x[i] = (row_ok && col0 + i < cols) ? __bfloat162float(aux[(size_t)row * aux_ld + col0 + i]) : 0.0f;
-          }
+          unpack_bf16x32(cur, x);
           if (phase == PHASE_SYM) {
             if (aux2 != nullptr) {
               float y[32];
@@ -433,7 +473,7 @@ __global__ void __launch_bounds__(kThreads, 1) ns_phase_kernel(const __grid_cons
             bulk_commit_group();
           }
           obuf ^= 1;
-          continue;
+          return true;
         }
         if (row_ok) {
           __nv_bfloat16* dst = out + (size_t)row * ld + col0;
@@ -452,6 +492,13 @@ __global__ void __launch_bounds__(kThreads, 1) ns_phase_kernel(const __grid_cons
           for (int i = 0; i < 32; ++i)
             if (col0 + i < cols) out[(size_t)(col0 + i) * ld + row] = __float2bfloat16_rn(o[i]);
         }
+        return true;
+      };
+      // Chunks in pairs so that the two auxiliary buffers stay in registers.
+#pragma unroll 1
+      for (int ch = 0; ch < BN / 32; ch += 2) {
+        if (!chunk(ch, xa, xb)) break;
+        if (!chunk(ch + 1, xb, xa)) break;
       }
       tc_fence_before();
       __syncwarp();
