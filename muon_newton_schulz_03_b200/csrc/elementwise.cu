@@ -125,7 +125,35 @@ __global__ void __launch_bounds__(kThreads) k1_momentum_norm(
 
   double acc = 0.0;
   unsigned bad = 0;
-  if ((mp.n % kVec) == 0) {
+  if ((mp.n % kVec) == 0 && e1 - e0 == kElemChunk) {
+    // Whole chunk, dense X layout: the loads of vector step it + 1 are issued
+    // before the stores of step it, so each thread keeps two steps in flight.
+    const long long eb = e0 + (long long)threadIdx.x * kVec;
+    float g[2][8], m[2][8];
+    auto load = [&](int it, int b) {
+      const long long e = eb + (long long)it * kThreads * kVec;
+      if (g_bf16) load8_bf16(static_cast<const __nv_bfloat16*>(mb.g) + e, g[b]);
+      else load8_f32(static_cast<const float*>(mb.g) + e, g[b]);
+      load8_f32(mb.mom + e, m[b]);
+    };
+    load(0, 0);
+#pragma unroll
+    for (int it = 0; it < kIters; ++it) {
+      const int b = it & 1;
+      if (it + 1 < kIters) load(it + 1, b ^ 1);
+      const long long e = eb + (long long)it * kThreads * kVec;
+      float u[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        u[i] = momentum_u(g[b][i], m[b][i], beta, omb, nesterov);
+        acc += (double)u[i] * (double)u[i];
+        if (check_nonfinite) bad += !isfinite(u[i]);
+      }
+      store8_f32(mb.mom + e, m[b]);
+      if (kFp32Out) store8_f32(static_cast<float*>(ybase) + e, u);
+      else store8_bf16(static_cast<__nv_bfloat16*>(ybase) + e, u);
+    }
+  } else if ((mp.n % kVec) == 0) {
     // ldx == n: the X layout is dense, element e maps to offset e.
     for (int it = 0; it < kIters; ++it) {
       const long long e = e0 + ((long long)it * kThreads + threadIdx.x) * kVec;
@@ -221,7 +249,27 @@ __global__ void __launch_bounds__(kThreads) k4_apply(const MatPlan* __restrict__
   const float decay = 1.0f - lr * wd;
   const float step = (float)((double)lr * (double)update_scale_dev(mp.m, mp.n, scale_mode, extra_scale) *
                              inv_norm(sumsq, mat));
-  if ((mp.n % kVec) == 0) {
+  if ((mp.n % kVec) == 0 && e1 - e0 == kElemChunk) {
+    // Whole chunk: two vector steps in flight per thread, as in K1.
+    const long long eb = e0 + (long long)threadIdx.x * kVec;
+    float p[2][8], o[2][8];
+    auto load = [&](int it, int b) {
+      const long long e = eb + (long long)it * kThreads * kVec;
+      load8_f32(mb.p + e, p[b]);
+      if (kFp32In) load8_f32(static_cast<const float*>(obase) + e, o[b]);
+      else load8_bf16(static_cast<const __nv_bfloat16*>(obase) + e, o[b]);
+    };
+    load(0, 0);
+#pragma unroll
+    for (int it = 0; it < kIters; ++it) {
+      const int b = it & 1;
+      if (it + 1 < kIters) load(it + 1, b ^ 1);
+      const long long e = eb + (long long)it * kThreads * kVec;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) p[b][i] = fmaf(p[b][i], decay, -step * o[b][i]);
+      store8_f32(mb.p + e, p[b]);
+    }
+  } else if ((mp.n % kVec) == 0) {
     for (int it = 0; it < kIters; ++it) {
       const long long e = e0 + ((long long)it * kThreads + threadIdx.x) * kVec;
       if (e >= e1) break;
