@@ -563,10 +563,31 @@ def run_sweep(args):
             opt.newton_schulz(xin, xout, shapes, None, ns_steps=NS_STEPS)
         end.record()
         torch.cuda.synchronize()
+        ms_eager = start.elapsed_time(end) / reps
+        # The same call captured in a CUDA graph: the device time without the
+        # per-call host work (argument checks and marshalling of `batch`
+        # tensors), which dominates the eager time of small batched points.
+        side = torch.cuda.Stream(device)
+        side.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(side):
+            opt.newton_schulz(xin, xout, shapes, None, ns_steps=NS_STEPS)
+        torch.cuda.current_stream().wait_stream(side)
+        torch.cuda.synchronize()
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            opt.newton_schulz(xin, xout, shapes, None, ns_steps=NS_STEPS)
+        graph.replay()
+        torch.cuda.synchronize()
+        start.record()
+        for _ in range(reps):
+            graph.replay()
+        end.record()
+        torch.cuda.synchronize()
         ms = start.elapsed_time(end) / reps
+        del graph
         flops = batch * W.ns_flops(m, n, NS_STEPS)
         tf = flops / (ms * 1e-3) / 1e12
-        points.append({"m": m, "n": n, "batch": batch, "ms": ms, "tflops_nominal": tf,
+        points.append({"m": m, "n": n, "batch": batch, "ms": ms, "ms_eager": ms_eager, "tflops_nominal": tf,
                        "frac_datasheet": tf / DATASHEET_BF16_TFLOPS, "frac_measured": tf / peaks["bf16_tflops"]})
         del xin, xout
         torch.cuda.empty_cache()
@@ -578,6 +599,7 @@ def run_sweep(args):
     line = {"metric": "NS-only TFLOP/s (nominal 5 (4 s^2 l + 2 s^3)) per sweep point", "value": vals[len(vals) // 2],
             "unit": "TFLOP/s (median over points)", "n_gpus": 1, "higher_is_better": True, "dtype": "bf16",
             "data": "synthetic", "config": {"workload": W.describe(W.CONFIG_SWEEP), "ns_steps": NS_STEPS,
+                                            "timing": "CUDA-graph replay of the call (ms); eager call (ms_eager)",
                                             "batches": sorted(batches), "peak_source": peak_src},
             "sweep": points}
     print(json.dumps(line), flush=True)

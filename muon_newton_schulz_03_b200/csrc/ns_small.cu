@@ -57,10 +57,6 @@ __device__ __forceinline__ uint32_t swz(int r, int c, int chunk_stride) {
   return (uint32_t)((c >> 6) * chunk_stride + r * 128 + ((((c & 63) >> 3) ^ (r & 7)) << 4) + ((c & 7) << 1));
 }
 
-__device__ __forceinline__ void fence_proxy_async_smem() {
-  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-}
-
 // 32 bf16 from an image row (r, c0..c0+31), c0 a multiple of 32.
 __device__ __forceinline__ void lds_row32(const uint8_t* img, int r, int c0, int cs, float (&o)[32]) {
 #pragma unroll
