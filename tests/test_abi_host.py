@@ -157,3 +157,29 @@ def test_null_handle_rejected():
     lib = muon.load()
     assert lib.muon_step(None, None, None, None, None, 1, 0.1, 0.9, 1, 0.0, 5, None, None) == 1
     assert lib.muon_destroy(None) == 0
+
+
+@pytest.mark.parametrize("field,value", [("ns_algorithm", 2), ("deterministic", 2)])
+def test_init_rejects_bad_config_values(field, value):
+    lib = muon.load()
+    import ctypes
+    cfg = _lib.MuonConfig()
+    assert lib.muon_config_init(ctypes.byref(cfg)) == 0
+    setattr(cfg, field, value)
+    h = ctypes.c_void_p()
+    assert lib.muon_init(0, ctypes.byref(cfg), ctypes.byref(h)) == 1
+    assert field.encode() in lib.muon_last_error()
+
+
+@pytest.mark.parametrize("other", [("ns_precision", 1), ("cta_pair", 1)])
+def test_gram_form_needs_bf16_single_cta(other):
+    # Checked before any device is touched, so it runs without a GPU.
+    lib = muon.load()
+    import ctypes
+    cfg = _lib.MuonConfig()
+    lib.muon_config_init(ctypes.byref(cfg))
+    cfg.ns_algorithm = 1
+    setattr(cfg, other[0], other[1])
+    h = ctypes.c_void_p()
+    assert lib.muon_init(0, ctypes.byref(cfg), ctypes.byref(h)) == 1
+    assert b"Gram" in lib.muon_last_error()

@@ -1,0 +1,54 @@
+"""Host-side checks of the benchmark's FLOP and byte accounting (no GPU)."""
+
+import pytest
+
+import bench
+import workloads as W
+
+
+def test_nominal_flops_formula():
+    # 4 s^2 l + 2 s^3 per iteration, s = min, l = max; orientation-free.
+    assert W.ns_flops(256, 512, 1) == 4 * 256 ** 2 * 512 + 2 * 256 ** 3
+    assert W.ns_flops(512, 256, 5) == W.ns_flops(256, 512, 5) == 5 * (4 * 256 ** 2 * 512 + 2 * 256 ** 3)
+
+
+def test_gram_form_flops_formula():
+    # Two-step segment: Gram + final product (2 s^2 l each) + five s^3 products.
+    s, l = 1024, 4096
+    assert W.gram_ns_flops(s, l, 2) == 4 * s * s * l + 10 * s ** 3
+    assert W.gram_ns_flops(s, l, 1) == W.ns_flops(s, l, 1)
+    assert W.gram_ns_flops(l, s, 5) == 2 * (4 * s * s * l + 10 * s ** 3) + W.ns_flops(s, l, 1)
+
+
+def test_executed_flops_hand_count():
+    # 512 x 1024 (wide, s = 512, l = 1024): Gram upper tiles with 128-row and
+    # 256-column tiles are (ti, tj) with tj >= ti // 2: tj = 0 -> ti 0, 1;
+    # tj = 1 -> ti 0..3 (4 row tiles of 128): 6 tiles; the polynomial lists the
+    # same 6; the combine covers 512 x 1024 with 4 x 4 = 16 tiles.
+    per_tile = 2 * 128 * 256
+    gram = 6 * per_tile * 1024
+    poly = 6 * per_tile * 512
+    comb = 16 * per_tile * 512
+    assert bench.executed_flops([(512, 1024)], 1) == gram + poly + comb
+    assert bench.executed_flops([(512, 1024)], 5) == 5 * (gram + poly + comb)
+    # Gram form, two steps: Gram + 5 symmetric products + combine.
+    assert bench.executed_flops([(512, 1024)], 2, gram=True) == gram + 5 * poly + comb
+
+
+def test_executed_flops_small_path_counts_nominal():
+    # 128 x 128 runs on the on-chip path: counted at its nominal FLOPs.
+    assert bench.executed_flops([(128, 128)], 5) == W.ns_flops(128, 128, 5)
+
+
+@pytest.mark.parametrize("name", ["llama3", "gpt2", "moe"])
+def test_executed_below_nominal_for_tiled_sets(name):
+    shapes = {"llama3": W.llama3_8b_shapes(), "gpt2": W.gpt2_shapes(), "moe": W.moe_shapes()}[name]
+    ratio = bench.executed_flops(shapes, 5) / W.total_ns_flops(shapes, 5)
+    # Symmetric upper tiles save part of the Gram and polynomial work.
+    assert 0.6 < ratio < 0.9
+
+
+def test_elementwise_bytes():
+    # K1: g + m read, m + bf16 X written; K4: p + bf16 O read, p written.
+    assert W.step_bytes(10, 10, 2) == (100 * 12, 100 * 10)
+    assert W.step_bytes(10, 10, 4) == (100 * 14, 100 * 10)
