@@ -15,7 +15,7 @@ import pytest
 import torch
 import torch.multiprocessing as mp
 
-from muon_newton_schulz_03_b200.distributed import assign_owners, step_cost
+from muon_newton_schulz_03_b200.distributed import assign_owners, assign_rounds, step_cost
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 SHAPES = [(64, 96), (96, 64), (32, 32), (128, 40), (40, 128), (16, 200), (48, 48)]
@@ -47,7 +47,7 @@ def _oracle_step(params, grads, momenta, ns_steps=5, **kw):
         m.copy_(torch.from_numpy(m2))
 
 
-def _worker(rank, world, port, out):
+def _worker(rank, world, port, out, rounds=4):
     import torch.distributed as dist
     from muon_newton_schulz_03_b200.distributed import LayerwiseMuon
     os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
@@ -57,18 +57,18 @@ def _worker(rank, world, port, out):
         P = [torch.tensor(p) for p in ps]
         G = [torch.tensor(g) for g in gs]
         M = [torch.tensor(m) for m in ms]
-        lw = LayerwiseMuon(group=None, local_step=_oracle_step)
+        lw = LayerwiseMuon(group=None, local_step=_oracle_step, rounds=rounds)
         owners = lw.step(P, G, M, lr=0.01, beta=0.9, wd=0.1)
         out[rank] = ([p.numpy() for p in P], [m.numpy() for m in M], owners)
     finally:
         dist.destroy_process_group()
 
 
-@pytest.mark.parametrize("world", [2, 3])
-def test_layerwise_step_matches_single_process(world):
+@pytest.mark.parametrize("world,rounds", [(2, 1), (2, 4), (3, 2), (3, 9)])
+def test_layerwise_step_matches_single_process(world, rounds):
     port = _free_port()
     out = mp.Manager().dict()
-    mp.spawn(_worker, args=(world, port, out), nprocs=world, join=True)
+    mp.spawn(_worker, args=(world, port, out, rounds), nprocs=world, join=True)
     ps, gs, ms = _inputs()
     P = [torch.tensor(p) for p in ps]
     M = [torch.tensor(m) for m in ms]
@@ -100,3 +100,23 @@ def test_assignment_is_balanced_and_deterministic():
     assert assign_owners([(8, 8)], 4) == [0]
     with pytest.raises(ValueError):
         assign_owners(shapes, 0)
+
+
+def test_rounds_cover_each_owned_matrix_once():
+    import workloads as W
+    shapes = W.llama3_8b_shapes()
+    for world in (2, 4, 8):
+        owners = assign_owners(shapes, world)
+        for rounds in (1, 3, 4, 16):
+            rr = assign_rounds(shapes, owners, world, rounds)
+            assert rr == assign_rounds(shapes, owners, world, rounds)
+            for r in range(world):
+                flat = [i for g in rr[r] for i in g]
+                assert sorted(flat) == [i for i in range(len(shapes)) if owners[i] == r]
+                assert flat == sorted(flat)                     # consecutive, index order
+                costs = [sum(step_cost(*shapes[i]) for i in g) for g in rr[r]]
+                biggest = max(step_cost(*shapes[i]) for i in flat)
+                share = sum(costs) / rounds
+                assert all(abs(c - share) <= biggest for c in costs)   # within one matrix of even
+    with pytest.raises(ValueError):
+        assign_rounds(shapes, assign_owners(shapes, 2), 2, 0)
