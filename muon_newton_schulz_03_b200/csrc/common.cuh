@@ -5,11 +5,27 @@
 // instructions, all as inline PTX.
 #pragma once
 
+#include <atomic>
 #include <cstdint>
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
 
 namespace muon {
+
+// A kernel's dynamic shared-memory limit is a per-device setting: raise it
+// once on every device the process launches the kernel on.
+template <typename Kernel>
+inline cudaError_t ensure_dynamic_smem(Kernel kernel, int smem, std::atomic<unsigned long long>& done_mask) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  const unsigned long long bit = dev < 64 ? (1ull << dev) : 0ull;
+  if (bit != 0 && (done_mask.load(std::memory_order_acquire) & bit) != 0) return cudaSuccess;
+  e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e == cudaSuccess && bit != 0) done_mask.fetch_or(bit, std::memory_order_acq_rel);
+  return e;
+}
+
 
 // ---------------------------------------------------------------------------
 // Plan-level and call-level per-matrix records (device resident).

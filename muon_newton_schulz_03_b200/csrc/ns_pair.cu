@@ -454,12 +454,11 @@ int pair_clusters_resident(int smem) {
 cudaError_t launch_ns_phase_pair(const NsLaunch& L, int phase, int src_sel, int dst_sel, int first, float a,
                                  float b, float c, cudaStream_t st) {
   if (L.ntiles <= 0) return cudaSuccess;
-  static bool attr_set = false;
+  static std::atomic<unsigned long long> attr_done{0};
   const int smem = ns_pair_smem_bytes();
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(ns_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  {
+    const cudaError_t e = ensure_dynamic_smem(ns_pair_kernel, smem, attr_done);
     if (e != cudaSuccess) return e;
-    attr_set = true;
   }
   PairArgs args;
   args.L = L;

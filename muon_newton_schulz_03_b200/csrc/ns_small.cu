@@ -316,12 +316,11 @@ cudaError_t launch_ns_small(const NsSmallLaunch& L, int ns_steps, int src_sel, i
                             cudaStream_t st) {
   if (L.nmats <= 0 || ns_steps <= 0) return cudaSuccess;
   if (ns_steps > kMaxNsSteps) return cudaErrorInvalidValue;
-  static bool attr_set = false;
+  static std::atomic<unsigned long long> attr_done{0};
   const int smem = ns_small_smem_bytes();
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(ns_small_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  {
+    const cudaError_t e = ensure_dynamic_smem(ns_small_kernel, smem, attr_done);
     if (e != cudaSuccess) return e;
-    attr_set = true;
   }
   SmallArgs args;
   args.L = L;

@@ -524,12 +524,11 @@ int ns_bf16_smem_bytes() { return (int)sizeof(SmemLayout) + 1024; }
 cudaError_t launch_ns_phase_bf16(const NsLaunch& L, int phase, int src_sel, int dst_sel, int first, float a,
                                  float b, float c, cudaStream_t st, const PhaseSpec& spec) {
   if (L.ntiles <= 0) return cudaSuccess;
-  static bool attr_set = false;
+  static std::atomic<unsigned long long> attr_done{0};
   const int smem = ns_bf16_smem_bytes();
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(ns_phase_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  {
+    const cudaError_t e = ensure_dynamic_smem(ns_phase_kernel, smem, attr_done);
     if (e != cudaSuccess) return e;
-    attr_set = true;
   }
   NsArgs args;
   args.L = L;
