@@ -265,6 +265,16 @@ def executed_flops(shapes, steps, gram=False, pair=False):
     return per + small
 
 
+def all_ranks_ok(torch, dist, device, flag):
+    """True when `flag` holds on every rank (one all-reduce of the minimum),
+    so every rank takes the same branch on an error path."""
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return bool(flag)
+    t = torch.tensor([1 if flag else 0], dtype=torch.int32, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MIN)
+    return bool(t.item())
+
+
 def max_over_ranks(torch, dist, value, device):
     """Largest value over all ranks (timing is reported as the slowest rank)."""
     if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
@@ -332,8 +342,9 @@ def run_ours(args):
         stepper.step(params, grads, moms, lr=LR, beta=BETA, wd=WD, ns_steps=NS_STEPS)
     torch.cuda.synchronize()
     code, ew, nf = opt.status()
-    if code != 0:
-        raise RuntimeError(f"device status {code} after warm-up (error word {ew}, non-finite {nf})")
+    if not all_ranks_ok(torch, dist, device, code == 0):
+        raise RuntimeError(f"device status {code} after warm-up on this or another rank (error word {ew}, "
+                           f"non-finite {nf})")
     launches_per_step = opt.last_launch_count()
 
     opt.profile_enable(args.steps)
@@ -352,8 +363,9 @@ def run_ours(args):
     prof = opt.profile_read()
     opt.profile_enable(0)
     code, ew, nf = opt.status()
-    if code != 0:
-        raise RuntimeError(f"device status {code} after timing (error word {ew}, non-finite {nf})")
+    if not all_ranks_ok(torch, dist, device, code == 0):
+        raise RuntimeError(f"device status {code} after timing on this or another rank (error word {ew}, "
+                           f"non-finite {nf})")
 
     ms_step = max_over_ranks(torch, dist, elapsed_ms / args.steps, device)
 
@@ -383,8 +395,9 @@ def run_ours(args):
         graph_ms = max_over_ranks(torch, dist, start.elapsed_time(end) / args.steps, device)
         del graph
         code, ew, nf = opt.status()
-        if code != 0:
-            raise RuntimeError(f"device status {code} after graph replay (error word {ew}, non-finite {nf})")
+        if not all_ranks_ok(torch, dist, device, code == 0):
+            raise RuntimeError(f"device status {code} after graph replay on this or another rank (error word {ew}, "
+                               f"non-finite {nf})")
 
     by_kind = {}
     for kind, ms in prof:
@@ -492,12 +505,36 @@ def run_e2e(torch, muon, opt, shapes, params, grads, moms, args, device, world, 
         h.copy_(t)
         return h
 
+    def all_ok(flag):
+        # Every rank takes the same path: the decision is the minimum over ranks.
+        if world == 1:
+            return bool(flag)
+        t = torch.tensor([1 if flag else 0], dtype=torch.int32, device=device)
+        dist.all_reduce(t, op=dist.ReduceOp.MIN)
+        return bool(t.item())
+
+    # The host copies of every rank on this node must fit in host memory with
+    # room to spare; otherwise no rank runs this leg.
+    need = sum(t.numel() * t.element_size() for t in list(params) + list(grads) + list(moms))
+    local_ranks = int(os.environ.get("LOCAL_WORLD_SIZE", "1"))
+    try:
+        import psutil
+        avail = psutil.virtual_memory().available
+    except Exception:  # pragma: no cover - psutil missing
+        avail = 0
+    if not all_ok(need * local_ranks <= 0.8 * avail):
+        return {"value": None, "unit": "steps/s",
+                "error": f"host memory: {local_ranks} ranks x {need / 1e9:.1f} GB of pinned buffers would not fit"}
+    hp, hg, hm, err = [], [], [], None
     try:
         hp = [pinned_copy(p) for p in params]
         hg = [pinned_copy(g) for g in grads]
         hm = [pinned_copy(m) for m in moms]
     except Exception as e:  # pragma: no cover - host memory limits
-        return {"value": None, "unit": "steps/s", "error": f"pinned host buffers unavailable: {e}"}
+        err = str(e)
+    if not all_ok(err is None):
+        del hp, hg, hm
+        return {"value": None, "unit": "steps/s", "error": f"pinned host buffers unavailable: {err or 'on another rank'}"}
     h2d = sum(t.numel() * t.element_size() for t in hp + hg + hm)
     d2h = sum(t.numel() * t.element_size() for t in hp + hm)
     # Free the device-resident copies so the staging area fits.
@@ -520,8 +557,8 @@ def run_e2e(torch, muon, opt, shapes, params, grads, moms, args, device, world, 
     torch.cuda.synchronize()
     ms = max_over_ranks(torch, dist, start.elapsed_time(end) / steps, device)
     code, ew, _ = opt.status()
-    if code != 0:
-        return {"value": None, "unit": "steps/s", "error": f"device status {code}"}
+    if not all_ok(code == 0):
+        return {"value": None, "unit": "steps/s", "error": f"device status {code} on this or another rank"}
     return {"value": world * 1e3 / ms, "unit": "steps/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
             "ms_per_step": ms, "steps": steps,
             "path": "muon_step_host: params, grads, momenta in pinned host memory; 8 chunks pipelined over "

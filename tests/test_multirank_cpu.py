@@ -31,7 +31,10 @@ def _worker(rank, world, port, out):
     dist.init_process_group("gloo", rank=rank, world_size=world)
     try:
         got = bench.max_over_ranks(torch, dist, 10.0 * (rank + 1), torch.device("cpu"))
-        out[rank] = got
+        # An error on one rank is seen by all (every rank takes the same branch).
+        ok_all = bench.all_ranks_ok(torch, dist, torch.device("cpu"), True)
+        ok_one_bad = bench.all_ranks_ok(torch, dist, torch.device("cpu"), rank != 1)
+        out[rank] = (got, ok_all, ok_one_bad)
     finally:
         dist.destroy_process_group()
 
@@ -41,7 +44,7 @@ def test_max_over_ranks_gloo():
     port = _free_port()
     out = mp.Manager().dict()
     mp.spawn(_worker, args=(world, port, out), nprocs=world, join=True)
-    assert out[0] == 20.0 and out[1] == 20.0
+    assert out[0] == (20.0, True, False) and out[1] == (20.0, True, False)
 
 
 def test_max_over_ranks_single_process():
@@ -50,6 +53,7 @@ def test_max_over_ranks_single_process():
     sys.path.insert(0, ROOT)
     import bench
     assert bench.max_over_ranks(torch, dist, 3.5, torch.device("cpu")) == 3.5
+    assert bench.all_ranks_ok(torch, dist, torch.device("cpu"), False) is False
 
 
 def test_reference_arm_non_zero_rank_exits_quietly():
