@@ -103,7 +103,8 @@ enum muon_ns_algorithm {
                            Newton-Schulz"), in segments of two steps: a
                            fresh Gram every second step; equal in exact
                            arithmetic, fewer FLOPs when max(m,n) >> min(m,n).
-                           bf16 and single-CTA tiles only                  */
+                           bf16 and single-CTA tiles only; matrices on the
+                           on-chip small path keep the standard form       */
 };
 
 #define MUON_FLAG_GRAD_BF16 1
@@ -132,8 +133,9 @@ typedef struct muon_config {
                                  (default): one double atomic per block    */
   int cta_pair;               /* 1: tiled phases use 256 x 256 tiles on CTA
                                  pairs (tcgen05 cta_group::2); 0: 128 x 256
-                                 tiles on single CTAs. Default 0 (both
-                                 measure alike on B200 under its power cap) */
+                                 tiles on single CTAs. Default 0 (the
+                                 single-CTA tiles measured 2-4% faster on
+                                 the Llama-shaped set under the power cap) */
 } muon_config;
 
 /* plan_flags of muon_plan_query */
