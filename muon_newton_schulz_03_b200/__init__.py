@@ -81,6 +81,58 @@ def _check_2d(t, what, dtypes, device=None, contiguous=True):
     return torch
 
 
+def _bad_matrix(i, p, g, m, host):
+    """Raise the precise error for matrix i of a step's lists."""
+    import torch
+    dev = None if host else p.device
+    _check_2d(p, f"params[{i}]", (torch.float32,), dev)
+    _check_2d(m, f"momenta[{i}]", (torch.float32,), dev)
+    if m.shape != p.shape:
+        raise ValueError(f"momenta[{i}] shape {tuple(m.shape)} != params shape {tuple(p.shape)}")
+    if g is not None:
+        _check_2d(g, f"grads[{i}]", (torch.float32, torch.bfloat16), dev)
+        if g.shape != p.shape:
+            raise ValueError(f"grads[{i}] shape {tuple(g.shape)} != params shape {tuple(p.shape)}")
+    for t, what in ((p, "params"), (m, "momenta"), (g, "grads")):
+        if t is not None and (t.device.type == "cpu") != host:
+            where = "in host memory" if host else "on a CUDA device"
+            raise ValueError(f"{what}[{i}] must be {where}")
+    raise ValueError(f"matrix {i}: invalid tensors")   # not reached
+
+
+def _marshal_step(params, grads, momenta, host=False):
+    """Pointer arrays and shape table of a step's matrix lists.
+
+    Every tensor is 2D and contiguous; params and momenta are fp32, grads
+    fp32 or bf16 (None skips the matrix); the tensors of one matrix have one
+    shape and one device, which is host memory for ``host`` and a CUDA device
+    otherwise (the C side cannot see tensor sizes, so they are checked
+    here). Returns (params, grads, momenta, shapes, count) as ctypes arrays.
+    """
+    import torch
+    f32, bf16 = torch.float32, torch.bfloat16
+    pp, gp, mp, flat = [], [], [], []
+    for i, (p, g, m) in enumerate(zip(params, grads, momenta, strict=True)):
+        dev = p.device
+        ok = (p.dim() == 2 and p.dtype == f32 and p.is_contiguous() and (dev.type == "cpu") == host
+              and m.dtype == f32 and m.is_contiguous() and m.shape == p.shape and m.device == dev)
+        if ok and g is not None:
+            ok = (g.dtype == f32 or g.dtype == bf16) and g.is_contiguous() and g.shape == p.shape and g.device == dev
+        if not ok:
+            _bad_matrix(i, p, g, m, host)
+        pp.append(p.data_ptr())
+        mp.append(m.data_ptr())
+        if g is None:
+            gp.append(None)
+            flat += (p.shape[0], p.shape[1], 0)
+        else:
+            gp.append(g.data_ptr())
+            flat += (p.shape[0], p.shape[1], FLAG_GRAD_BF16 if g.dtype == bf16 else 0)
+    n = len(pp)
+    return ((ctypes.c_void_p * n)(*pp), (ctypes.c_void_p * n)(*gp), (ctypes.c_void_p * n)(*mp),
+            (ctypes.c_int32 * (3 * n))(*flat), n)
+
+
 def x_layout(m: int, n: int, dtype, device):
     """An empty X-layout buffer: row-major m x round_up(n, 8)."""
     import torch
@@ -210,26 +262,11 @@ class Muon:
         heights; every block is then a Muon matrix of its own (its rows are
         contiguous, so the blocks are passed as views, no copy).
         """
-        import torch
         if row_splits is not None:
             params, grads, momenta = split_rows(params, grads, momenta, row_splits)
-        shapes, pp, gp, mp = [], [], [], []
-        for i, (p, g, m) in enumerate(zip(params, grads, momenta, strict=True)):
-            _check_2d(p, f"params[{i}]", (torch.float32,))
-            _check_2d(m, f"momenta[{i}]", (torch.float32,), p.device)
-            flag = 0
-            if g is not None:
-                _check_2d(g, f"grads[{i}]", (torch.float32, torch.bfloat16), p.device)
-                if g.shape != p.shape:
-                    raise ValueError(f"grads[{i}] shape {tuple(g.shape)} != params shape {tuple(p.shape)}")
-                flag = FLAG_GRAD_BF16 if g.dtype == torch.bfloat16 else 0
-            if m.shape != p.shape:
-                raise ValueError(f"momenta[{i}] shape {tuple(m.shape)} != params shape {tuple(p.shape)}")
-            shapes.append((p.shape[0], p.shape[1], flag))
-            pp.append(p.data_ptr()); gp.append(_ptr(g)); mp.append(m.data_ptr())
-        check(self._lib.muon_step(self._h, _ptr_array(pp), _ptr_array(gp), _ptr_array(mp), _shapes_array(shapes),
-                                  len(shapes), float(lr), float(beta), int(bool(nesterov)), float(wd),
-                                  int(ns_steps), _coeffs(coeffs), _stream_handle(stream)))
+        pa, ga, ma, sa, n = _marshal_step(params, grads, momenta)
+        check(self._lib.muon_step(self._h, pa, ga, ma, sa, n, float(lr), float(beta), int(bool(nesterov)),
+                                  float(wd), int(ns_steps), _coeffs(coeffs), _stream_handle(stream)))
 
     def step_schedule(self, params, grads, momenta, coeff_table, lr, beta=0.95, nesterov=True, wd=0.1,
                       stream=None):
@@ -239,20 +276,9 @@ class Muon:
         if not rows or any(len(r) != 3 for r in rows):
             raise ValueError("coeff_table must be a non-empty list of (a, b, c)")
         table = (ctypes.c_float * (3 * len(rows)))(*[v for r in rows for v in r])
-        shapes, pp, gp, mp = [], [], [], []
-        for i, (p, g, m) in enumerate(zip(params, grads, momenta, strict=True)):
-            _check_2d(p, f"params[{i}]", (torch.float32,))
-            _check_2d(m, f"momenta[{i}]", (torch.float32,), p.device)
-            flag = 0
-            if g is not None:
-                _check_2d(g, f"grads[{i}]", (torch.float32, torch.bfloat16), p.device)
-                flag = FLAG_GRAD_BF16 if g.dtype == torch.bfloat16 else 0
-            shapes.append((p.shape[0], p.shape[1], flag))
-            pp.append(p.data_ptr()); gp.append(_ptr(g)); mp.append(m.data_ptr())
-        check(self._lib.muon_step_schedule(self._h, _ptr_array(pp), _ptr_array(gp), _ptr_array(mp),
-                                           _shapes_array(shapes), len(shapes), float(lr), float(beta),
-                                           int(bool(nesterov)), float(wd), len(rows), table, len(rows),
-                                           _stream_handle(stream)))
+        pa, ga, ma, sa, n = _marshal_step(params, grads, momenta)
+        check(self._lib.muon_step_schedule(self._h, pa, ga, ma, sa, n, float(lr), float(beta), int(bool(nesterov)),
+                                           float(wd), len(rows), table, len(rows), _stream_handle(stream)))
 
     def qk_clip(self, weights, s_max, head_rows, tau=100.0, stream=None):
         """QK-Clip in place on W_q / W_k weights (fp32 CUDA tensors).
@@ -280,24 +306,9 @@ class Muon:
         The copies and the kernels are enqueued on ``stream``; synchronise it
         before reading params / momenta.
         """
-        import torch
-        shapes, pp, gp, mp = [], [], [], []
-        for i, (p, g, m) in enumerate(zip(params, grads, momenta, strict=True)):
-            _check_2d(p, f"params[{i}]", (torch.float32,))
-            _check_2d(m, f"momenta[{i}]", (torch.float32,))
-            flag = 0
-            if g is not None:
-                _check_2d(g, f"grads[{i}]", (torch.float32, torch.bfloat16))
-                flag = FLAG_GRAD_BF16 if g.dtype == torch.bfloat16 else 0
-            for t, what in ((p, "params"), (m, "momenta"), (g, "grads")):
-                if t is not None and t.device.type != "cpu":
-                    raise ValueError(f"{what}[{i}] must be in host memory for step_host")
-            shapes.append((p.shape[0], p.shape[1], flag))
-            pp.append(p.data_ptr()); gp.append(_ptr(g)); mp.append(m.data_ptr())
-        check(self._lib.muon_step_host(self._h, _ptr_array(pp), _ptr_array(gp), _ptr_array(mp),
-                                       _shapes_array(shapes), len(shapes), float(lr), float(beta),
-                                       int(bool(nesterov)), float(wd), int(ns_steps), _coeffs(coeffs),
-                                       _stream_handle(stream)))
+        pa, ga, ma, sa, n = _marshal_step(params, grads, momenta, host=True)
+        check(self._lib.muon_step_host(self._h, pa, ga, ma, sa, n, float(lr), float(beta), int(bool(nesterov)),
+                                       float(wd), int(ns_steps), _coeffs(coeffs), _stream_handle(stream)))
 
     # -- stages -------------------------------------------------------------
     def momentum_norm(self, grads, momenta, ys, sumsq, beta=0.95, nesterov=True, stream=None):
