@@ -100,14 +100,15 @@ def _bad_matrix(i, p, g, m, host):
     raise ValueError(f"matrix {i}: invalid tensors")   # not reached
 
 
-def _marshal_step(params, grads, momenta, host=False):
+def _marshal_step(params, grads, momenta, host=False, device_index=None):
     """Pointer arrays and shape table of a step's matrix lists.
 
     Every tensor is 2D and contiguous; params and momenta are fp32, grads
     fp32 or bf16 (None skips the matrix); the tensors of one matrix have one
     shape and one device, which is host memory for ``host`` and a CUDA device
     otherwise (the C side cannot see tensor sizes, so they are checked
-    here). Returns (params, grads, momenta, shapes, count) as ctypes arrays.
+    here; with ``device_index`` the device must be that CUDA device). Returns
+    (params, grads, momenta, shapes, count) as ctypes arrays.
     """
     import torch
     f32, bf16 = torch.float32, torch.bfloat16
@@ -120,6 +121,8 @@ def _marshal_step(params, grads, momenta, host=False):
             ok = (g.dtype == f32 or g.dtype == bf16) and g.is_contiguous() and g.shape == p.shape and g.device == dev
         if not ok:
             _bad_matrix(i, p, g, m, host)
+        if device_index is not None and not host and dev.index != device_index:
+            raise ValueError(f"params[{i}] is on {dev}, the handle on cuda:{device_index}")
         pp.append(p.data_ptr())
         mp.append(m.data_ptr())
         if g is None:
@@ -264,7 +267,7 @@ class Muon:
         """
         if row_splits is not None:
             params, grads, momenta = split_rows(params, grads, momenta, row_splits)
-        pa, ga, ma, sa, n = _marshal_step(params, grads, momenta)
+        pa, ga, ma, sa, n = _marshal_step(params, grads, momenta, device_index=self.device)
         check(self._lib.muon_step(self._h, pa, ga, ma, sa, n, float(lr), float(beta), int(bool(nesterov)),
                                   float(wd), int(ns_steps), _coeffs(coeffs), _stream_handle(stream)))
 
@@ -276,7 +279,7 @@ class Muon:
         if not rows or any(len(r) != 3 for r in rows):
             raise ValueError("coeff_table must be a non-empty list of (a, b, c)")
         table = (ctypes.c_float * (3 * len(rows)))(*[v for r in rows for v in r])
-        pa, ga, ma, sa, n = _marshal_step(params, grads, momenta)
+        pa, ga, ma, sa, n = _marshal_step(params, grads, momenta, device_index=self.device)
         check(self._lib.muon_step_schedule(self._h, pa, ga, ma, sa, n, float(lr), float(beta), int(bool(nesterov)),
                                            float(wd), len(rows), table, len(rows), _stream_handle(stream)))
 
@@ -319,11 +322,13 @@ class Muon:
             _check_2d(m, f"momenta[{i}]", (torch.float32,))
             if g is not None:
                 _check_2d(g, f"grads[{i}]", (torch.float32, torch.bfloat16), m.device)
+                if g.shape != m.shape:
+                    raise ValueError(f"grads[{i}] shape {tuple(g.shape)} != momenta shape {tuple(m.shape)}")
+            self._check_on_device(m, f"momenta[{i}]")
             self._check_x(y, m.shape, f"y[{i}]")
             shapes.append((m.shape[0], m.shape[1],
                            FLAG_GRAD_BF16 if (g is not None and g.dtype == torch.bfloat16) else 0))
-        if sumsq.dtype != torch.float64 or sumsq.numel() < len(shapes) or not sumsq.is_contiguous():
-            raise ValueError("sumsq must be a contiguous float64 tensor with one entry per matrix")
+        self._check_sumsq(sumsq, len(shapes))
         check(self._lib.muon_momentum_norm(self._h, _ptr_array([_ptr(g) for g in grads]),
                                            _ptr_array([m.data_ptr() for m in momenta]),
                                            _ptr_array([y.data_ptr() for y in ys]), sumsq.data_ptr(),
@@ -336,6 +341,8 @@ class Muon:
         for i, ((m, n, _), xi, xo) in enumerate(zip(sh, x_in, x_out, strict=True)):
             self._check_x(xi, (m, n), f"x_in[{i}]")
             self._check_x(xo, (m, n), f"x_out[{i}]")
+        if sumsq is not None:
+            self._check_sumsq(sumsq, len(sh))
         check(self._lib.muon_newton_schulz(self._h, _ptr_array([x.data_ptr() for x in x_in]),
                                            _ptr_array([x.data_ptr() for x in x_out]),
                                            None if sumsq is None else sumsq.data_ptr(), _shapes_array(sh),
@@ -347,15 +354,29 @@ class Muon:
         shapes = []
         for i, (p, o) in enumerate(zip(params, os_, strict=True)):
             _check_2d(p, f"params[{i}]", (torch.float32,))
+            self._check_on_device(p, f"params[{i}]")
             if o is not None:
                 self._check_x(o, p.shape, f"o[{i}]")
             shapes.append((p.shape[0], p.shape[1], 0))
+        if sumsq is not None:
+            self._check_sumsq(sumsq, len(shapes))
         check(self._lib.muon_apply(self._h, _ptr_array([p.data_ptr() for p in params]),
                                    _ptr_array([_ptr(o) for o in os_]),
                                    None if sumsq is None else sumsq.data_ptr(), _shapes_array(shapes),
                                    len(shapes), float(lr), float(wd), _stream_handle(stream)))
 
+    def _check_on_device(self, t, what):
+        if t.device.type != "cuda" or t.device.index != self.device:
+            raise ValueError(f"{what} must be on cuda:{self.device}, got {t.device}")
+
+    def _check_sumsq(self, sumsq, count):
+        import torch
+        if sumsq.dtype != torch.float64 or sumsq.numel() < count or not sumsq.is_contiguous():
+            raise ValueError("sumsq must be a contiguous float64 tensor with one entry per matrix")
+        self._check_on_device(sumsq, "sumsq")
+
     def _check_x(self, x, shape, what):
+        self._check_on_device(x, what)
         m, n = int(shape[0]), int(shape[1])
         if x.dtype != self._xdtype():
             raise TypeError(f"{what} must be {self._xdtype()} in {self.ns_precision} mode")
