@@ -52,3 +52,11 @@ def test_elementwise_bytes():
     # K1: g + m read, m + bf16 X written; K4: p + bf16 O read, p written.
     assert W.step_bytes(10, 10, 2) == (100 * 12, 100 * 10)
     assert W.step_bytes(10, 10, 4) == (100 * 14, 100 * 10)
+
+
+def test_executed_flops_pair_tiles_hand_count():
+    # 256 x 256 tiles on CTA pairs, 512 x 1024: upper tiles (0,0), (0,1), (1,1)
+    # for the symmetric phases, 2 x 4 = 8 combine tiles.
+    per_tile = 2 * 256 * 256
+    want = 3 * per_tile * 1024 + 3 * per_tile * 512 + 8 * per_tile * 512
+    assert bench.executed_flops([(512, 1024)], 1, pair=True) == want
