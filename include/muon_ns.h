@@ -338,11 +338,11 @@ const char* muon_version(void);
 /* ---- Allocation-free Newton-Schulz stage ----
  *
  * The pages have no counterpart to this entry point; it exists for callers
- * that cannot allocate device memory when they run the stage: a stream being
- * captured in global capture mode (allocation calls are refused then), a
- * process whose device memory belongs to its own fixed-budget pool, or a
- * latency-critical path that cannot take the implicit synchronisation an
- * allocation may bring.
+ * that cannot allocate device memory when they run the stage: a process
+ * whose device memory belongs to its own fixed-budget pool allocator (a
+ * cudaMalloc from outside the pool fails or takes memory the pool counts
+ * on), or a serving process that reserved its memory at start-up and must
+ * keep its device footprint fixed while it runs.
  *
  * Same computation and the same tensor-core kernels as muon_newton_schulz,
  * in bf16, on the CURRENT device, with no handle. All scratch (X ping-pong
@@ -361,6 +361,11 @@ const char* muon_version(void);
  *   error_word  : device int32 or NULL; receives 0, or the code of a
  *                 device-side wait that ran out (results then invalid).
  *   stream      : cudaStream_t.
+ * Errors (MUON_ERR_INVALID_ARG, message in muon_last_error): NULL, unaligned
+ * or overlapping matrices, a matrix that is not device memory of the
+ * current device, non-finite coefficients, and a call on a stream that is
+ * being captured (each call writes its tables from host memory that lives
+ * only during the call).
  * A shape table whose scratch (tables plus the workspace muon_plan_query
  * reports) exceeds MUON_NOALLOC_SCRATCH_BYTES is rejected with
  * MUON_ERR_INVALID_ARG and a message giving both sizes.

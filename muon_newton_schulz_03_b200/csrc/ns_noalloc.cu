@@ -1,10 +1,10 @@
 // Newton-Schulz stage for callers that cannot allocate device memory.
 //
-// Some callers cannot call cudaMalloc when they need this stage: a stream
-// that is being captured in global capture mode (the runtime refuses
-// allocation calls then), a process whose device memory is entirely owned by
-// its own pool allocator with a fixed budget, or a latency-critical path that
-// cannot afford the implicit device synchronisation an allocation may bring.
+// Some callers cannot call cudaMalloc when they need this stage: a process
+// whose device memory is entirely owned by its own pool allocator with a
+// fixed budget (a cudaMalloc from outside the pool fails or steals from it),
+// or a serving process that reserved its memory at start-up and must keep
+// its device footprint fixed while it runs.
 // muon_newton_schulz_noalloc serves them: it runs the same tensor-core
 // Newton-Schulz kernels as muon_newton_schulz, but every byte of scratch it
 // needs (the X ping-pong buffers, the Gram and polynomial matrices, the tile
@@ -16,9 +16,15 @@
 // cudaGetSymbolAddress, looked up once per device (the array's host-side
 // name is a stand-in, not a device address). That set-up happens on the
 // first call on each device, with that device current.
+//
+// Each call writes its tables (plans, tile lists, tensor maps) from host
+// memory that lives only for the duration of the call, with a stream-ordered
+// copy; a call on a stream that is being captured is therefore refused
+// before anything is enqueued.
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <cmath>
 #include <cstring>
 #include <mutex>
 #include <string>
@@ -140,6 +146,18 @@ extern "C" int muon_newton_schulz_noalloc(const void* const* x_in, void* const* 
   if (ns_steps < 0 || ns_steps > 64) return noalloc_fail(MUON_ERR_INVALID_ARG, "ns_steps must be in [0, 64]");
   const float def[3] = {3.4445f, -4.7750f, 2.0315f};
   const float* abc = coeffs ? coeffs : def;
+  for (int k = 0; k < 3; ++k)
+    if (!std::isfinite(abc[k])) return noalloc_fail(MUON_ERR_INVALID_ARG, "coefficients must be finite");
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  {
+    cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+    cudaError_t e = cudaStreamIsCapturing(st, &cs);
+    if (e != cudaSuccess) return noalloc_fail(MUON_ERR_CUDA, std::string("cudaStreamIsCapturing: ") + cudaGetErrorString(e));
+    if (cs != cudaStreamCaptureStatusNone)
+      return noalloc_fail(MUON_ERR_INVALID_ARG,
+                          "muon_newton_schulz_noalloc uploads its tables from host memory that lives only during "
+                          "the call; it is refused while the stream is being captured");
+  }
   HostPlan hp;
   std::string why;
   if (!build_plan(shapes, count, 0, /*small_path=*/false, /*pair_tiles=*/false, hp, why)) return noalloc_fail(MUON_ERR_INVALID_ARG, why);
@@ -179,6 +197,24 @@ extern "C" int muon_newton_schulz_noalloc(const void* const* x_in, void* const* 
   DeviceScratch* ds = nullptr;
   int rc = scratch_for_current_device(&ds);
   if (rc) return rc;
+  // Every matrix must live on the current device: its address goes into a
+  // tensor map that this device's kernels read.
+  int cur = -1;
+  NOALLOC_CUDA_TRY(cudaGetDevice(&cur));
+  for (int i = 0; i < count; ++i) {
+    for (int k = 0; k < 2; ++k) {
+      const void* ptr = k == 0 ? x_in[i] : static_cast<const void*>(x_out[i]);
+      cudaPointerAttributes at;
+      cudaError_t e = cudaPointerGetAttributes(&at, ptr);
+      if (e != cudaSuccess) {
+        cudaGetLastError();
+        return noalloc_fail(MUON_ERR_INVALID_ARG, "matrix " + std::to_string(i) + ": pointer not known to CUDA");
+      }
+      if (at.type != cudaMemoryTypeDevice || at.device != cur)
+        return noalloc_fail(MUON_ERR_INVALID_ARG, "matrix " + std::to_string(i) +
+                                                      ": x_in and x_out must be device memory of the current device");
+    }
+  }
   unsigned char* base = ds->base;
   unsigned char* ws = base + o_ws;
 
@@ -214,7 +250,6 @@ extern "C" int muon_newton_schulz_noalloc(const void* const* x_in, void* const* 
       t[k] = make_int4(hp.tiles[p][k].mat, hp.tiles[p][k].ti, hp.tiles[p][k].tj, 0);
   }
 
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
   DevStatus* status = reinterpret_cast<DevStatus*>(base);
   // The status word must start at zero; the tables are rewritten in full.
   // Both are stream-ordered after earlier calls on the same stream.

@@ -7,10 +7,11 @@ Sources (web pages; cited by title and section):
 
 * "About Muon: Why Not Adam" -- the authority on the arithmetic.
   - section "The whole thing, in about forty lines": the step order
-    (momentum lerp, Nesterov lerp, bf16 cast, Frobenius normalisation with
-    eps = 1e-7, short-side transpose, the quintic loop, cast back, scale,
-    decoupled weight decay, write), default hyper-parameters and the
-    Moonlight scale used by that program.
+    (momentum lerp, Nesterov lerp, Frobenius normalisation with eps = 1e-7,
+    the quintic iteration on the short side, scale, decoupled weight decay,
+    write), default hyper-parameters, the Moonlight scale used by that
+    program, and the precision of its iteration (a bf16 tensor, so every
+    operation returns bf16).
   - section "The lemma that makes it possible": an odd polynomial in X and
     X^T X acts on the singular values only.
   - section "The iteration does not converge, and that is deliberate":
@@ -34,10 +35,14 @@ design notes):
 * Nesterov defaults to on; a flag turns it off (``u = m'``).
 * The norm is taken of the float64 ``u``; eps = 1e-7 is added to the norm,
   not to its square.
-* The short-side transpose is strict: only m > n is transposed.
-* No bf16 rounding in the exact mode. ``emulate_bf16=True`` rounds X, A, B
-  (round-to-nearest-even) at the points where the GPU rounds: the cast of
-  u, and every Gram / polynomial / combine output. Diagnostic only.
+* The short side is chosen by a strict test: only rows > columns works with
+  X^T X (from the right); a square matrix uses X X^T (from the left). No
+  transpose is formed: the two forms are the same matrix.
+* ``precision="exact"`` (the default) rounds nothing. ``precision="bf16"``
+  rounds to bf16 (round-to-nearest-even) wherever the pages' bf16 program
+  returns a bf16 tensor: the cast of the input, its norm, norm + eps, the
+  normalised matrix, and each of the eight operations of a step. It is the
+  yardstick for how far bf16 arithmetic itself lands from the exact result.
 * ``ns_steps = 0`` returns the normalised matrix.
 """
 
@@ -61,7 +66,7 @@ SCALE_NONE = 3        # 1
 
 
 # ---------------------------------------------------------------------------
-# bf16 rounding (used only by the emulating diagnostic mode)
+# bf16 rounding (the precision of the pages' bf16 program)
 # ---------------------------------------------------------------------------
 
 def bf16_round(x: np.ndarray) -> np.ndarray:
@@ -107,13 +112,26 @@ def ns_poly_iterate(s, steps=5, coeffs=DEFAULT_COEFFS):
 # ---------------------------------------------------------------------------
 # Matrix Newton-Schulz
 # ---------------------------------------------------------------------------
+#
+# The lemma ("About Muon: Why Not Adam", section "The lemma that makes it
+# possible"): for X = U S V^T, an odd polynomial written with the Gram of
+# either side, a X + b (X X^T) X + c (X X^T)^2 X = a X + b X (X^T X) +
+# c X (X^T X)^2, equals U p(S) V^T with p(s) = a s + b s^3 + c s^5. The
+# work is cheapest with the s x s Gram of the short side, s = min(rows, cols):
+# X X^T multiplied from the left when rows <= cols, X^T X from the right when
+# rows > cols. That choice is the pages' "run on the short side" rule (a
+# strict rows > cols test, so a square matrix takes the left form) written
+# without transposing the matrix: the two forms are the same matrix.
 
-def _matmul(P, Q, accum_fp32):
-    """P @ Q; with accum_fp32 the operands (bf16 values, exact in float32)
-    are multiplied with float32 accumulation, as tensor cores accumulate."""
-    if not accum_fp32:
-        return P @ Q
-    return (P.astype(np.float32) @ Q.astype(np.float32)).astype(np.float64)
+
+def _short_gram(X):
+    """The s x s Gram of the short side: X X^T (rows <= cols) or X^T X."""
+    return X @ X.T if X.shape[0] <= X.shape[1] else X.T @ X
+
+
+def _on_short_side(P, X):
+    """P (s x s) applied on the short side: P X (rows <= cols) or X P."""
+    return P @ X if X.shape[0] <= X.shape[1] else X @ P
 
 
 def coeff_rows(coeffs, steps):
@@ -131,153 +149,140 @@ def coeff_rows(coeffs, steps):
     return [tuple(r) for r in arr]
 
 
-def _ns_iterations(X, steps, coeffs, emulate_bf16, accum_fp32=False, start=0):
-    """Run the quintic iteration on a short-side-first matrix X (s x l).
+def quintic_map(X, a, b, c):
+    """p(X) = a X + b A X + c A^2 X in float64, A the short-side Gram.
 
-    Each step forms the Gram A = X X^T, the polynomial B = bA + cA^2 and the
-    combine X <- aX + BX. This equals aX + bX(X^T X) + cX(X^T X)^2 because
-    (X X^T)^k X = X (X^T X)^k ("About Muon: Why Not Adam", section "The lemma
-    that makes it possible"). ``coeffs`` holds one triple per step (see
-    coeff_rows); steps ``start..steps-1`` are run.
+    Evaluated in the pages' order: the Gram A, the polynomial part
+    B = b A + c A^2, then the combine a X + B X (B acting on the short
+    side).
     """
-    rnd = bf16_round if emulate_bf16 else (lambda v: v)
-    for k in range(start, steps):
-        a, b, c = coeffs[k]
-        A = rnd(_matmul(X, X.T, accum_fp32))
-        B = rnd(b * A + c * _matmul(A, A, accum_fp32))
-        X = rnd(a * X + _matmul(B, X, accum_fp32))
-    return X
+    A = _short_gram(X)
+    B = b * A + c * (A @ A)
+    return a * X + _on_short_side(B, X)
 
 
-def newton_schulz(G, steps=5, coeffs=DEFAULT_COEFFS, eps=EPS,
-                  emulate_bf16=False, accum_fp32=False):
-    """Approximate orthogonal polar factor of G (float64).
+def quintic_map_bf16(X, a, b, c):
+    """The same map at the precision of the pages' bf16 program.
 
     "About Muon: Why Not Adam", section "The whole thing, in about forty
-    lines": normalise by the Frobenius norm plus eps so every singular value
-    lies in (0, 1], work on the short side (transpose when rows > columns),
-    iterate the quintic ``steps`` times, undo the transpose.
+    lines", runs the iteration on a bfloat16 tensor with plain tensor
+    operations, so every operation returns a bf16 tensor: the Gram, the
+    product A A, the scalings b A, c A^2 and a X, the sum that forms B, the
+    product B X and the final sum. Each of those eight results is rounded to
+    bf16 here. Reading: a bf16 matrix product is its exact value rounded once
+    (accumulation in float32 on the devices that run such programs adds
+    error far below one bf16 rounding), and a scalar times a bf16 tensor is
+    the exact product rounded once.
+    """
+    r = bf16_round
+    A = r(_short_gram(X))
+    AA = r(A @ A)
+    B = r(r(b * A) + r(c * AA))
+    BX = r(_on_short_side(B, X))
+    return r(r(a * X) + BX)
 
-    With ``emulate_bf16`` the input is rounded to bf16 before normalising and
-    the normalisation factor is applied exactly where the GPU applies it
-    (inside the first Gram and first combine); otherwise no rounding happens.
-    ``accum_fp32`` (with ``emulate_bf16``) accumulates the products in
-    float32 instead of float64: a second, equally valid bf16 realization.
+
+def frobenius_normalise(G, eps=EPS):
+    """G / (||G||_F + eps): every singular value lands in [0, 1)."""
+    G = np.asarray(G, dtype=np.float64)
+    return G / (np.linalg.norm(G) + eps)
+
+
+def frobenius_normalise_bf16(G, eps=EPS):
+    """The normalisation of the pages' bf16 program: the matrix is cast to
+    bf16 first, its norm is a bf16 scalar, adding eps rounds again, and the
+    division returns a bf16 tensor."""
+    Y = bf16_round(G)
+    nrm = bf16_round(np.sqrt(np.sum(Y * Y)))
+    return bf16_round(Y / bf16_round(nrm + eps))
+
+
+PRECISIONS = ("exact", "bf16")
+
+
+def _check_precision(precision):
+    if precision not in PRECISIONS:
+        raise ValueError(f"precision must be one of {PRECISIONS}")
+
+
+def newton_schulz(G, steps=5, coeffs=DEFAULT_COEFFS, eps=EPS, precision="exact"):
+    """Approximate orthogonal polar factor of G.
+
+    Normalise by the Frobenius norm plus eps, then apply the quintic map
+    ``steps`` times with the short-side Gram ("About Muon: Why Not Adam",
+    sections "The whole thing, in about forty lines" and "The lemma that
+    makes it possible"). ``precision="exact"`` works in float64 without any
+    rounding; ``precision="bf16"`` rounds where the pages' bf16 program
+    rounds (``frobenius_normalise_bf16``, ``quintic_map_bf16``). Zero steps
+    return the normalised matrix.
     """
     G = np.asarray(G, dtype=np.float64)
     if G.ndim != 2:
         raise ValueError("Newton-Schulz is defined for 2D matrices only")
+    _check_precision(precision)
     rows = coeff_rows(coeffs, steps)
-    transposed = G.shape[0] > G.shape[1]
-    if not emulate_bf16:
-        X = G / (np.linalg.norm(G) + eps)
-        if transposed:
-            X = X.T
-        X = _ns_iterations(X, steps, rows, False)
-        return X.T if transposed else X
-
-    # bf16-emulating diagnostic: Y = bf16(G); alpha = 1/(||G|| + eps) is
-    # folded into the first Gram (alpha^2) and the first combine (alpha).
-    alpha = 1.0 / (np.linalg.norm(G) + eps)
-    Y = bf16_round(G)
-    if transposed:
-        Y = Y.T
-    if steps == 0:
-        X = alpha * Y
+    if precision == "exact":
+        X, step = frobenius_normalise(G, eps), quintic_map
     else:
-        a, b, c = rows[0]
-        A = bf16_round(alpha * alpha * _matmul(Y, Y.T, accum_fp32))
-        B = bf16_round(b * A + c * _matmul(A, A, accum_fp32))
-        X = bf16_round(alpha * (a * Y + _matmul(B, Y, accum_fp32)))
-        X = _ns_iterations(X, steps, rows, True, accum_fp32, start=1)
-    return X.T if transposed else X
+        X, step = frobenius_normalise_bf16(G, eps), quintic_map_bf16
+    for a, b, c in rows:
+        X = step(X, a, b, c)
+    return X
 
 
-def gram_newton_schulz(G, steps=5, coeffs=DEFAULT_COEFFS, eps=EPS, emulate_bf16=False, accum_fp32=False,
-                       segment=2):
+def gram_newton_schulz(G, steps=5, coeffs=DEFAULT_COEFFS, eps=EPS, segment=2):
     """Gram Newton-Schulz ("About Muon: Why Not Adam", section "Gram
     Newton-Schulz"): the same odd polynomial, iterated on the small Gram.
 
-    With X the normalised short-side-first matrix, a segment of L steps
-    forms A = X X^T once and then, for each step, B = bA + cA^2 (so the
-    plain step is X <- (aI + B) X); the segment's product
-    Q = (a_L I + B_L) ... (a_1 I + B_1) is applied to X at the end, and the
-    Gram is carried between the steps of a segment as A <- P A P (the Gram
-    of P X, P = aI + B commutes with A). In exact arithmetic every segment
-    length gives ``newton_schulz``. Reading: segments of 2 steps (a fresh
-    Gram every second step) keep bf16 rounding from accumulating in the
-    carried Gram; ``segment=None`` runs all steps in one segment (exact mode
-    only). The aI parts are never stored: with B0, B1 the two steps' B,
-      R = a0 A + B0 A,   A1 = a0 R + R B0,
-      Q - a0 a1 I = a1 B0 + a0 B1 + B1 B0,
-      X' = a0 a1 X + (Q - a0 a1 I) X.
-    With ``emulate_bf16`` each of A, B0, R, A1, B1, Q - a0 a1 I and X' is
-    rounded to bf16 (the normalisation folded into the first segment's Gram
-    as alpha^2 and its final product as alpha).
+    With X the normalised matrix and A its short-side Gram, one step is
+    X <- P X with P = a I + b A + c A^2 (P on the short side), and the Gram
+    of P X is P A P (P commutes with A). A segment of L steps forms A once,
+    then for each step builds P from the carried Gram, accumulates the
+    product Q = P_L ... P_1 and carries A <- P A P; the segment ends with
+    X <- Q X. In exact arithmetic every segment length gives
+    ``newton_schulz``. Reading: segments of 2 steps (a fresh Gram every
+    second step), which is what keeps bf16 rounding from building up in the
+    carried Gram; ``segment=None`` runs all steps in one segment.
     """
     G = np.asarray(G, dtype=np.float64)
     if G.ndim != 2:
         raise ValueError("Newton-Schulz is defined for 2D matrices only")
     rows = coeff_rows(coeffs, steps)
     seg = steps if segment is None else int(segment)
-    if emulate_bf16 and not 1 <= seg <= 2:
-        raise ValueError("the bf16 mode restates segments of 1 or 2 steps")
-    rnd = bf16_round if emulate_bf16 else (lambda v: v)
-    acc = accum_fp32 and emulate_bf16
-    transposed = G.shape[0] > G.shape[1]
-    alpha = 1.0 / (np.linalg.norm(G) + eps)
-    X = bf16_round(G) if emulate_bf16 else G
-    if transposed:
-        X = X.T
-    if steps == 0:
-        X = alpha * X
-        return X.T if transposed else X
-    k, sc = 0, alpha
+    if seg < 1 and steps > 0:
+        raise ValueError("segments hold at least one step")
+    X = frobenius_normalise(G, eps)
+    k = 0
     while k < steps:
-        L = min(max(seg, 1), steps - k)
-        A = rnd(sc * sc * _matmul(X, X.T, acc))
-        if emulate_bf16 or L <= 2:
-            a0, b0, c0 = rows[k]
-            B0 = rnd(b0 * A + c0 * _matmul(A, A, acc))
-            if L == 1:
-                X = rnd(sc * (a0 * X + _matmul(B0, X, acc)))
-            else:
-                a1, b1, c1 = rows[k + 1]
-                R = rnd(a0 * A + _matmul(B0, A, acc))
-                A1 = rnd(a0 * R + _matmul(R, B0, acc))
-                B1 = rnd(b1 * A1 + c1 * _matmul(A1, A1, acc))
-                Qd = rnd(a1 * B0 + a0 * B1 + _matmul(B1, B0, acc))
-                X = rnd(sc * (a0 * a1 * X + _matmul(Qd, X, acc)))
-        else:
-            eye = np.eye(A.shape[0])
-            Q = None
-            for j in range(L):
-                a, b, c = rows[k + j]
-                P = a * eye + b * A + c * (A @ A)
-                Q = P if Q is None else P @ Q
-                A = P @ A @ P
-            X = sc * (Q @ X)
-        k += L
-        sc = 1.0
-    return X.T if transposed else X
+        A = _short_gram(X)
+        eye = np.eye(A.shape[0])
+        Q = eye
+        for a, b, c in rows[k:k + seg]:
+            P = a * eye + b * A + c * (A @ A)
+            Q = P @ Q
+            A = P @ A @ P
+        X = _on_short_side(Q, X)
+        k += seg
+    return X
 
 
-def ns_only(X, steps=5, coeffs=DEFAULT_COEFFS, emulate_bf16=False, accum_fp32=False):
-    """The Newton-Schulz phases alone on an already-scaled X (no norm).
+def ns_only(X, steps=5, coeffs=DEFAULT_COEFFS, precision="exact"):
+    """The Newton-Schulz iterations alone on an already-scaled X (no norm).
 
-    Used for the NS-only sweep workload, whose inputs are generated with
-    singular values already in [1e-4, 1]. Same orientation rule as
-    ``newton_schulz``; with ``emulate_bf16`` the input and every Gram,
-    polynomial and combine output are rounded to bf16.
+    For the NS-only sweep, whose inputs are generated with singular values
+    already in [1e-4, 1]. With ``precision="bf16"`` the input is cast to
+    bf16 and each step rounds as the pages' bf16 program does.
     """
     X = np.asarray(X, dtype=np.float64)
-    if emulate_bf16:
+    if X.ndim != 2:
+        raise ValueError("Newton-Schulz is defined for 2D matrices only")
+    _check_precision(precision)
+    step = quintic_map if precision == "exact" else quintic_map_bf16
+    if precision == "bf16":
         X = bf16_round(X)
-    transposed = X.shape[0] > X.shape[1]
-    if transposed:
-        X = X.T
-    X = _ns_iterations(X, steps, coeff_rows(coeffs, steps), emulate_bf16, accum_fp32 and emulate_bf16)
-    return X.T if transposed else X
+    for a, b, c in coeff_rows(coeffs, steps):
+        X = step(X, a, b, c)
+    return X
 
 
 # ---------------------------------------------------------------------------
@@ -354,14 +359,16 @@ def apply_update(p, O, lr, wd, scale):
 def muon_step_matrix(p, g, m, *, lr, beta=0.95, nesterov=True, wd=0.1,
                      ns_steps=5, coeffs=DEFAULT_COEFFS,
                      scale_mode=SCALE_MOONLIGHT, extra_scale=1.0,
-                     emulate_bf16=False, accum_fp32=False, gram=False):
+                     precision="exact", gram=False):
     """One Muon step on one matrix. Returns (p', m', O, ||u||_F).
 
     ``gram`` selects the Gram form of Newton-Schulz (same result in exact
-    arithmetic).
+    arithmetic; exact precision only). ``precision`` is the Newton-Schulz
+    precision ("exact" or the pages' "bf16" program); the momentum, blend,
+    scale and write are float64 in both.
 
-    Order: momentum, Nesterov blend, Newton-Schulz (normalise, orient,
-    iterate, orient back), scale, decoupled weight decay, write.
+    Order: momentum, Nesterov blend, Newton-Schulz (normalise, iterate on
+    the short side), scale, decoupled weight decay, write.
     """
     p = np.asarray(p, dtype=np.float64)
     if p.ndim != 2:
@@ -370,9 +377,11 @@ def muon_step_matrix(p, g, m, *, lr, beta=0.95, nesterov=True, wd=0.1,
     u = nesterov_blend(g, m_new, beta, nesterov)
     nu = float(np.linalg.norm(u))
     if gram:
-        O = gram_newton_schulz(u, ns_steps, coeffs, EPS, emulate_bf16, accum_fp32)
+        if precision != "exact":
+            raise ValueError("the Gram form is restated in exact arithmetic only")
+        O = gram_newton_schulz(u, ns_steps, coeffs, EPS)
     else:
-        O = newton_schulz(u, ns_steps, coeffs, EPS, emulate_bf16, accum_fp32)
+        O = newton_schulz(u, ns_steps, coeffs, EPS, precision)
     scale = update_scale(p.shape[0], p.shape[1], scale_mode, extra_scale)
     p_new = apply_update(p, O, lr, wd, scale)
     return p_new, m_new, O, nu
@@ -425,7 +434,7 @@ def muon_step_matrix_split(p, g, m, row_blocks, **kw):
 def muon_step(params, grads, momenta, *, lr, beta=0.95, nesterov=True,
               wd=0.1, ns_steps=5, coeffs=DEFAULT_COEFFS,
               scale_mode=SCALE_MOONLIGHT, extra_scale=1.0,
-              emulate_bf16=False):
+              precision="exact"):
     """One Muon step over a list of matrices, one at a time.
 
     A ``None`` gradient skips its matrix (parameter and momentum unchanged).
@@ -443,7 +452,7 @@ def muon_step(params, grads, momenta, *, lr, beta=0.95, nesterov=True,
         r = muon_step_matrix(p, g, m, lr=lr, beta=beta, nesterov=nesterov,
                              wd=wd, ns_steps=ns_steps, coeffs=coeffs,
                              scale_mode=scale_mode, extra_scale=extra_scale,
-                             emulate_bf16=emulate_bf16)
+                             precision=precision)
         out_p.append(r[0])
         out_m.append(r[1])
         out_o.append(r[2])

@@ -1,10 +1,14 @@
 """Helpers shared by the GPU parity tests (inputs, comparisons)."""
 
+import json
+import os
+
 import numpy as np
 import torch
 
 import muon_newton_schulz_03_b200 as muon
 import workloads as W
+from oracle import muon_oracle as O
 
 DEV = torch.device("cuda:0")
 
@@ -12,40 +16,57 @@ DEV = torch.device("cuda:0")
 TOL_BF16_NS = 2e-2      # bf16 Newton-Schulz vs the float64 oracle
 TOL_FP32_NS = 1e-4      # fp32 debug Newton-Schulz vs the float64 oracle
 TOL_ELEM = 1e-6         # elementwise stages vs the float64 oracle
-TOL_BF16_EMU = 1e-2     # bf16 Newton-Schulz vs the oracle's bf16-rounding mode
+TOL_GPU_VS_GPU = 1e-2   # two GPU kernels with the same rounding points (small path vs tiled phases)
+
+_GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden", "bf16_program_errors.json")
+_PROGRAM_ERRORS = None
 
 
-def bf16_gate(got, exact, emulated, emulated32, what=""):
-    """Two-tier parity of a bf16 Newton-Schulz result.
+def bf16_program_error(x, steps=5, coeffs=O.DEFAULT_COEFFS, normalised=True):
+    """Frozen distance from exact of the pages' bf16 program on this input.
 
-    `emulated` and `emulated32` are the oracle at the pages' precision (bf16
-    rounding of the input and of every Gram / polynomial / combine output),
-    accumulating in float64 and in float32: two equally valid bf16
-    realizations. Their distance, `spread`, measures how strongly rounding
-    differences grow through the iteration at this input (tiny for
-    well-conditioned inputs, ~1e-2 and more when singular values reach down to
-    1e-4 without normalisation).
-    1. The GPU is a bf16 realization: its distance to the nearer of the two
-       is within max(TOL_BF16_EMU, 3 * spread, inherent / 2). The last term
-       only matters where bf16 arithmetic is far from exact (inherent above
-       the gate): there the tensor cores' accumulation makes a third
-       realization whose drift the float32 emulation does not bound.
-    2. The GPU is as accurate as bf16 arithmetic allows: its distance to the
-       exact float64 oracle is within TOL_BF16_NS, or, where bf16 arithmetic
-       itself cannot meet that (the emulations' own distance `inherent`
-       exceeds it), within 1.05 * inherent + 3 * spread.
-    Returns (err_vs_exact, err_vs_emulated, inherent, spread).
+    The values were written once by tests/golden/make_bf16_program_errors.py
+    (oracle only) and are looked up by a digest of the input's float64
+    bytes, the step count, the coefficients and the normalisation flag; an
+    input that is not in the file is an error, never a default.
     """
-    e_emu = min(rel(got, emulated), rel(got, emulated32))
-    e_exact = rel(got, exact)
-    inherent = max(rel(emulated, exact), rel(emulated32, exact))
-    spread = rel(emulated32, emulated)
-    bound1 = max(TOL_BF16_EMU, 3.0 * spread, 0.5 * inherent if inherent > TOL_BF16_NS else 0.0)
-    assert e_emu <= bound1, f"{what}: {e_emu:.3e} from the bf16-rounding oracle (spread {spread:.3e})"
-    bound2 = TOL_BF16_NS if inherent <= TOL_BF16_NS else 1.05 * inherent + 3.0 * spread
-    assert e_exact <= bound2, (f"{what}: {e_exact:.3e} from the exact oracle "
-                               f"(bf16 arithmetic alone: {inherent:.3e}, spread {spread:.3e})")
-    return e_exact, e_emu, inherent, spread
+    global _PROGRAM_ERRORS
+    if _PROGRAM_ERRORS is None:
+        with open(_GOLDEN) as f:
+            _PROGRAM_ERRORS = json.load(f)["cases"]
+    key = W.case_key(x, steps, coeffs, normalised)
+    if key not in _PROGRAM_ERRORS:
+        raise KeyError(f"no frozen bf16-program distance for input {key}: "
+                       "rerun tests/golden/make_bf16_program_errors.py")
+    return _PROGRAM_ERRORS[key]["err"]
+
+
+def bf16_ns_tolerance(x, steps=5, coeffs=O.DEFAULT_COEFFS, normalised=True):
+    """The bf16 gate on a Newton-Schulz output: 2e-2 from exact, or the
+    pages' own bf16 program's distance from exact where that is larger."""
+    return max(TOL_BF16_NS, bf16_program_error(x, steps, coeffs, normalised))
+
+
+def gate_bf16_ns(got, exact, x, steps=5, coeffs=O.DEFAULT_COEFFS, normalised=True, what=""):
+    """Assert the bf16 gate on O; returns (error, tolerance)."""
+    tol = bf16_ns_tolerance(x, steps, coeffs, normalised)
+    e = rel(got, exact)
+    assert e <= tol, f"{what}: {e:.3e} from the exact oracle (gate {tol:.3e})"
+    return e, tol
+
+
+def gate_bf16_update(p_gpu, p0, p_exact, o_exact, lr_scale, tol_o, what=""):
+    """The same gate carried to the update dp = p' - p.
+
+    p' = p (1 - lr wd) - lr scale O, so an error E in O moves dp by
+    lr scale E: the O tolerance becomes tol_o * lr scale ||O|| / ||dp||,
+    plus the float32 rounding of the written p' (2^-23 of ||p'||)."""
+    dp_exact = p_exact - p0
+    ndp = np.linalg.norm(dp_exact)
+    tol = (tol_o * abs(lr_scale) * np.linalg.norm(o_exact) + 2.0 ** -23 * np.linalg.norm(p_exact)) / ndp
+    e = rel(p_gpu - p0, dp_exact)
+    assert e <= tol, f"{what}: update {e:.3e} from the exact oracle (gate {tol:.3e})"
+    return e
 
 
 def rel(a, b):
@@ -83,18 +104,28 @@ def bf16_ulp(x):
 
 
 def make_set(config, shapes, grad_dtype, seed_base=0):
-    """CPU-generated inputs: list of (p, g, m) float64 arrays and torch CUDA tensors."""
+    """Inputs of a shape set (workloads.set_values): list of (p, g, m)
+    float64 arrays holding the device's values, and the CUDA tensors."""
+    vals = W.set_values(config, shapes, grad_dtype == torch.bfloat16, seed_base)
     cpu, dev = [], []
-    for i, (m, n) in enumerate(shapes):
-        seed = W.seed_for(config, i // 7, i % 7) + seed_base
-        g = W.gradient_cpu(config, m, n, seed)
-        p = W.param_cpu(m, n, seed)
-        mom = np.zeros((m, n))
+    for i in range(len(shapes)):
+        p, g, mom = vals[i]
         gt = (cuda_bf16(g) if grad_dtype == torch.bfloat16 else cuda_f32(g))
         pt, mt = cuda_f32(p), cuda_f32(mom)
         cpu.append((to64(pt), to64(gt), to64(mt)))
+        assert np.array_equal(cpu[-1][1], g)
         dev.append((pt, gt, mt))
     return cpu, dev
+
+
+def gaussian_buffers(shapes, seed, scale=1.0, dtype=torch.bfloat16):
+    """workloads.gaussian_set in the library's X layout: (buffers, float64 values)."""
+    xs = W.gaussian_set(shapes, seed, scale)
+    bufs = [x_buffer(m, n, dtype, fill=x) for (m, n), x in zip(shapes, xs)]
+    vals = [to64(b[:, :n]) for b, (m, n) in zip(bufs, shapes)]
+    for a, b in zip(vals, xs):
+        assert np.array_equal(a, b)
+    return bufs, vals
 
 
 def workspace_matrix(opt, shapes, index, region, dtype=torch.bfloat16):

@@ -60,3 +60,26 @@ def test_executed_flops_pair_tiles_hand_count():
     per_tile = 2 * 256 * 256
     want = 3 * per_tile * 1024 + 3 * per_tile * 512 + 8 * per_tile * 512
     assert bench.executed_flops([(512, 1024)], 1, pair=True) == want
+
+
+def test_symmetric_flops_formula():
+    # Upper triangles of the Gram (s^2 l) and polynomial (s^3), full combine
+    # (2 s^2 l): 3 s^2 l + s^3 per iteration, between the executed tile count
+    # and the nominal dense count on the tiled sets.
+    s, l = 256, 512
+    assert W.ns_flops_symmetric(s, l, 1) == 3 * s * s * l + s ** 3
+    assert W.ns_flops_symmetric(l, s, 5) == 5 * (3 * s * s * l + s ** 3)
+    assert W.gram_ns_flops_symmetric(s, l, 2) == 3 * s * s * l + 5 * s ** 3
+    assert W.gram_ns_flops_symmetric(s, l, 5) == 2 * (3 * s * s * l + 5 * s ** 3) + W.ns_flops_symmetric(s, l, 1)
+    shapes = W.llama3_8b_shapes()
+    alg = W.total_ns_flops_symmetric(shapes)
+    assert alg < bench.executed_flops(shapes, 5) < W.total_ns_flops(shapes)
+    assert abs(alg / 1e12 - 471.8) < 0.5     # TFLOP per Muon step on the Llama-3-8B set
+
+
+def test_shape_classes_and_set_extrapolation():
+    classes = W.shape_classes(W.llama3_8b_shapes())
+    assert classes == {(4096, 4096): (64, 0), (1024, 4096): (64, 1), (14336, 4096): (64, 4), (4096, 14336): (32, 6)}
+    secs = {(4096, 4096): 1.0, (1024, 4096): 0.5, (14336, 4096): 2.0, (4096, 14336): 3.0}
+    assert bench.set_seconds("llama3", secs) == 64 * 1.0 + 64 * 0.5 + 64 * 2.0 + 32 * 3.0
+    assert W.shape_classes(W.moe_shapes()) == {(2048, 7168): (256, 0), (7168, 2048): (128, 2)}

@@ -12,13 +12,15 @@ import torch
 import muon_newton_schulz_03_b200 as muon
 from oracle import muon_oracle as O
 
-from gpu_helpers import (DEV, TOL_BF16_EMU, TOL_BF16_NS, TOL_ELEM, TOL_FP32_NS, bf16_gate, bf16_ulp, cuda_bf16,
+from gpu_helpers import (DEV, TOL_BF16_NS, TOL_ELEM, TOL_FP32_NS, TOL_GPU_VS_GPU, bf16_ulp, cuda_bf16, gate_bf16_ns,
+                         gaussian_buffers,
                          cuda_f32, rel, to64, x_buffer)
 
 pytestmark = pytest.mark.gpu
 
-RAGGED = [(1, 1), (3, 5), (5, 3), (1, 300), (300, 1), (127, 129), (129, 127), (64, 64), (256, 512), (512, 256),
-          (384, 384), (200, 1000), (1000, 200), (520, 520), (768, 2304)]
+import workloads as W  # noqa: E402
+
+RAGGED = W.PARITY_SHAPES["ragged"]
 
 
 @pytest.fixture(scope="module")
@@ -160,14 +162,7 @@ def test_apply_with_norm_scale(opt_bf16):
 # ---------------------------------------------------------------------------
 
 def _ns_inputs(shapes, seed, scale=1.0):
-    rng = np.random.default_rng(seed)
-    xin, x64 = [], []
-    for (m, n) in shapes:
-        x = rng.standard_normal((m, n)) * scale
-        buf = x_buffer(m, n, fill=x)
-        xin.append(buf)
-        x64.append(to64(buf[:, :n]))
-    return xin, x64
+    return gaussian_buffers(shapes, seed, scale)
 
 
 @pytest.mark.parametrize("kind", ["pair", "single"])
@@ -199,10 +194,8 @@ def test_ns_single_step_phases(opts, kind, coeffs):
     torch.cuda.synchronize()
     for i, (m, n) in enumerate(shapes):
         ref = O.ns_only(x64[i], 1, coeffs)
-        emu = O.ns_only(x64[i], 1, coeffs, emulate_bf16=True)
-        emu32 = O.ns_only(x64[i], 1, coeffs, emulate_bf16=True, accum_fp32=True)
         got = to64(xout[i][:, :n])
-        bf16_gate(got, ref, emu, emu32, f"matrix {i} {m}x{n}")
+        gate_bf16_ns(got, ref, x64[i], 1, coeffs, normalised=False, what=f"matrix {i} {m}x{n}")
     _assert_status_clean(opt_bf16)
 
 
@@ -218,10 +211,8 @@ def test_ns_bf16_matches_oracle(opts, kind, steps):
     torch.cuda.synchronize()
     for i, (m, n) in enumerate(shapes):
         ref = O.newton_schulz(x64[i], steps)
-        emu = O.newton_schulz(x64[i], steps, emulate_bf16=True)
-        emu32 = O.newton_schulz(x64[i], steps, emulate_bf16=True, accum_fp32=True)
         got = to64(xout[i][:, :n])
-        bf16_gate(got, ref, emu, emu32, f"matrix {i} {m}x{n}")
+        gate_bf16_ns(got, ref, x64[i], steps, what=f"matrix {i} {m}x{n}")
     # Inputs were not modified.
     for i, (m, n) in enumerate(shapes):
         assert np.array_equal(to64(xin[i][:, :n]), x64[i])
@@ -279,36 +270,35 @@ def test_ns_gram_is_symmetric_in_workspace(opts, kind):
         assert rel(A, ref) <= 4e-3
 
 
-SWEEP_POINTS = [(128, 128, 4), (128, 512, 2), (512, 128, 2), (256, 256, 3), (256, 2048, 1), (2048, 256, 1),
-                (1024, 1024, 1), (512, 4096, 1)]
+SWEEP_POINTS = W.PARITY_SHAPES["sweep"]
 
 
 @pytest.mark.parametrize("point", SWEEP_POINTS, ids=lambda p: f"{p[0]}x{p[1]}x{p[2]}")
 def test_ns_only_sweep_inputs(opt_bf16, point):
     # NS-only workload: bf16 X with log-uniform singular values in [1e-4, 1],
-    # no normalisation; five steps.
-    import workloads as W
+    # no normalisation; five steps. The pages' own bf16 program lands far
+    # above 2e-2 from exact on these inputs (small singular values grow by
+    # the polynomial's slope a = 3.4445 per step, rounding noise with them):
+    # its frozen distance is the gate.
     m, n, batch = point
     shapes = [(m, n)] * batch
     xin, x64 = [], []
     for b in range(batch):
-        x = W.gradient_cpu(W.CONFIG_SWEEP, m, n, W.seed_for(W.CONFIG_SWEEP, m // 128, n // 128, b))
+        x = W.sweep_matrix(m, n, b)
         buf = x_buffer(m, n, fill=x)
         xin.append(buf)
         x64.append(to64(buf[:, :n]))
+        assert np.array_equal(x64[-1], x)
     xout = [x_buffer(m, n) for _ in shapes]
     opt_bf16.newton_schulz(xin, xout, shapes, None, ns_steps=5)
     torch.cuda.synchronize()
     for b in range(batch):
         ref = O.ns_only(x64[b], 5)
-        emu = O.ns_only(x64[b], 5, emulate_bf16=True)
-        emu32 = O.ns_only(x64[b], 5, emulate_bf16=True, accum_fp32=True)
-        bf16_gate(to64(xout[b][:, :n]), ref, emu, emu32, f"{m}x{n} #{b}")
+        gate_bf16_ns(to64(xout[b][:, :n]), ref, x64[b], 5, normalised=False, what=f"{m}x{n} #{b}")
     _assert_status_clean(opt_bf16)
 
 
-SMALL_SHAPES = [(1, 1), (3, 5), (5, 3), (64, 64), (100, 300), (300, 100), (128, 128), (128, 512), (512, 128),
-                (127, 129), (1, 300), (300, 1), (16, 512), (512, 16), (96, 200), (65, 65)]
+SMALL_SHAPES = W.PARITY_SHAPES["small"]
 
 
 @pytest.mark.parametrize("steps", [1, 5])
@@ -329,10 +319,8 @@ def test_small_path_matches_oracle_and_tiled_path(opt_bf16, steps):
     for i, (m, n) in enumerate(shapes):
         got = to64(out_small[i][:, :n])
         ref = O.newton_schulz(x64[i], steps)
-        emu = O.newton_schulz(x64[i], steps, emulate_bf16=True)
-        emu32 = O.newton_schulz(x64[i], steps, emulate_bf16=True, accum_fp32=True)
-        bf16_gate(got, ref, emu, emu32, f"small path {m}x{n}")
-        assert rel(got, to64(out_tiled[i][:, :n])) <= TOL_BF16_EMU, f"small vs tiled {m}x{n}"
+        gate_bf16_ns(got, ref, x64[i], steps, what=f"small path {m}x{n}")
+        assert rel(got, to64(out_tiled[i][:, :n])) <= TOL_GPU_VS_GPU, f"small vs tiled {m}x{n}"
     _assert_status_clean(opt_bf16)
     assert tiled.status() == (0, 0, 0)
     tiled.close()

@@ -337,7 +337,7 @@ def test_full_step_against_composed_closed_form():
 
 
 # ---------------------------------------------------------------------------
-# bf16 rounding (diagnostic mode) against torch's float32 -> bfloat16 cast.
+# bf16 rounding and the pages' bf16 program, against torch's bfloat16 tensors.
 # ---------------------------------------------------------------------------
 
 def test_bf16_round_matches_torch_on_float32_values():
@@ -362,56 +362,91 @@ def test_bf16_ties_to_even():
     assert O.bf16_round(np.array([one + ulp / 2 + 1e-12]))[0] == one + ulp
 
 
-def test_emulated_bf16_close_to_exact():
+def test_bf16_program_close_to_exact_but_rounded():
+    # The pages' bf16 program on a well-conditioned input: a few bf16
+    # roundings per operation, amplified by the polynomial's slopes, land a
+    # few 1e-2 from exact; never zero and never order one.
     rng = np.random.default_rng(17)
     m, n = 48, 80
     G = (_haar(rng, m, m) * np.linspace(1, 0.05, m)) @ _haar(rng, n, m).T
     exact = O.newton_schulz(G)
-    emu = O.newton_schulz(G, emulate_bf16=True)
-    rel = np.linalg.norm(emu - exact) / np.linalg.norm(exact)
-    assert 1e-5 < rel < 2e-2
+    prog = O.newton_schulz(G, precision="bf16")
+    assert np.array_equal(O.bf16_round(prog), prog)          # a bf16 tensor
+    rel = np.linalg.norm(prog - exact) / np.linalg.norm(exact)
+    assert 1e-3 < rel < 1e-1
 
 
 @pytest.mark.parametrize("shape", [(6, 10), (10, 6), (9, 9)])
 @pytest.mark.parametrize("steps", [0, 1, 5])
-def test_bf16_mode_is_exact_mode_plus_rounding(monkeypatch, shape, steps):
-    # The bf16-rounding mode differs from the exact mode only by the rounding
-    # it inserts (and by applying 1/(||G||+eps) inside the first Gram and
-    # combine, which is the same product). With rounding made the identity,
-    # both modes agree to float64 accuracy.
+def test_bf16_program_is_exact_mode_plus_rounding(monkeypatch, shape, steps):
+    # With rounding made the identity, the bf16 program is the exact
+    # iteration to float64 accuracy: it adds roundings and nothing else.
     rng = np.random.default_rng(18)
     G = rng.standard_normal(shape)
     monkeypatch.setattr(O, "bf16_round", lambda v: np.asarray(v, dtype=np.float64))
-    a = O.newton_schulz(G, steps, emulate_bf16=True)
+    a = O.newton_schulz(G, steps, precision="bf16")
+    b = O.ns_only(G * 0.1, steps, precision="bf16")
     monkeypatch.undo()
-    b = O.newton_schulz(G, steps)
-    assert np.max(np.abs(a - b)) < 1e-12
+    assert np.max(np.abs(a - O.newton_schulz(G, steps))) < 1e-12
+    assert np.max(np.abs(b - O.ns_only(G * 0.1, steps))) < 1e-12
 
 
-def test_ns_only_bf16_mode_structure(monkeypatch):
-    rng = np.random.default_rng(19)
-    X = rng.standard_normal((7, 12)) * 0.1
-    monkeypatch.setattr(O, "bf16_round", lambda v: np.asarray(v, dtype=np.float64))
-    a = O.ns_only(X, 5, emulate_bf16=True)
-    monkeypatch.undo()
-    assert np.max(np.abs(a - O.ns_only(X, 5))) < 1e-13
+def _torch_bf16_iteration(G, steps, normalise):
+    """The iteration run by torch on a CPU bfloat16 tensor, one eager
+    operation at a time (each returns bf16): the precision the oracle's
+    bf16 mode restates."""
+    torch = pytest.importorskip("torch")
+    a, b, c = O.DEFAULT_COEFFS
+    t = torch.from_numpy(G).to(torch.bfloat16)
+    if normalise:
+        t = t / (torch.linalg.vector_norm(t) + O.EPS)
+    left = t.shape[0] <= t.shape[1]
+    for _ in range(steps):
+        gram = t @ t.mT if left else t.mT @ t
+        poly = b * gram + c * (gram @ gram)
+        t = a * t + (poly @ t if left else t @ poly)
+    return t.to(torch.float64).numpy()
 
 
-def test_bf16_mode_fp32_accumulation_is_a_nearby_realization():
-    # On a well-conditioned input the two bf16 realizations (float64 and
-    # float32 accumulation) agree far below the bf16 gate, and with rounding
-    # made the identity the float32-accumulated mode stays within float32
-    # accuracy of the exact mode.
-    rng = np.random.default_rng(20)
-    G = (_haar(rng, 40, 40) * np.linspace(1, 0.1, 40)) @ _haar(rng, 90, 40).T
-    a = O.newton_schulz(G, emulate_bf16=True)
-    b = O.newton_schulz(G, emulate_bf16=True, accum_fp32=True)
-    assert np.linalg.norm(a - b) / np.linalg.norm(a) < 5e-3
-    monkey = pytest.MonkeyPatch()
-    monkey.setattr(O, "bf16_round", lambda v: np.asarray(v, dtype=np.float64))
-    c = O.newton_schulz(G, emulate_bf16=True, accum_fp32=True)
-    monkey.undo()
-    assert np.max(np.abs(c - O.newton_schulz(G))) < 1e-5
+@pytest.mark.parametrize("shape", [(12, 20), (20, 12), (16, 16)])
+def test_bf16_program_matches_torch_bf16_tensors(shape):
+    # One step: every element equal to torch's, except where torch's float32
+    # accumulation lands on the other side of a bf16 rounding boundary (rare,
+    # one bf16 step at most). Five steps: the two stay far closer to each
+    # other than to the exact result.
+    rng = np.random.default_rng(40)
+    G = O.bf16_round(rng.standard_normal(shape))
+    one = O.newton_schulz(G, 1, precision="bf16")
+    ref = _torch_bf16_iteration(G, 1, True)
+    same = np.mean(one == ref)
+    assert same >= 0.97, f"only {same:.3f} of the elements agree"
+    assert np.all(np.abs(one - ref) <= 2.0 ** -7 * np.maximum(np.abs(ref), 2.0 ** -20))
+    five = O.newton_schulz(G, 5, precision="bf16")
+    ref5 = _torch_bf16_iteration(G, 5, True)
+    exact = O.newton_schulz(G, 5)
+    assert np.linalg.norm(five - ref5) < 0.5 * np.linalg.norm(five - exact)
+    # Without the norm (NS-only inputs).
+    X = O.bf16_round(G * 0.05)
+    assert np.mean(O.ns_only(X, 1, precision="bf16") == _torch_bf16_iteration(X, 1, False)) >= 0.97
+
+
+def test_bf16_program_norm_is_a_bf16_scalar():
+    # The program divides by the bf16 norm of the bf16 copy plus eps (a bf16
+    # scalar): the normalised matrix equals torch's bf16 division.
+    torch = pytest.importorskip("torch")
+    rng = np.random.default_rng(41)
+    G = rng.standard_normal((33, 17)) * 3.0
+    t = torch.from_numpy(G).to(torch.bfloat16)
+    want = (t / (torch.linalg.vector_norm(t) + O.EPS)).to(torch.float64).numpy()
+    got = O.newton_schulz(G, 0, precision="bf16")
+    assert np.array_equal(got, want)
+
+
+def test_precision_names_are_checked():
+    with pytest.raises(ValueError):
+        O.newton_schulz(np.eye(3), 1, precision="fp16")
+    with pytest.raises(ValueError):
+        O.muon_step_matrix(np.eye(3), np.eye(3), np.zeros((3, 3)), lr=0.1, gram=True, precision="bf16")
 
 
 # ---------------------------------------------------------------------------
@@ -476,9 +511,9 @@ def test_schedule_follows_composed_scalar_polynomials():
     for a, b, c in table:
         x = a * x + b * x ** 3 + c * x ** 5
     assert np.max(np.abs(O.newton_schulz(G, 4, table) - (U * x) @ Vt)) < 1e-12
-    for mode in (False, True):
+    for precision in ("exact", "bf16"):
         with pytest.raises(ValueError):
-            O.newton_schulz(G, 3, table, emulate_bf16=mode)
+            O.newton_schulz(G, 3, table, precision=precision)
 
 
 def test_alternating_convergent_schedule_gives_polar_factor():
@@ -532,22 +567,11 @@ def test_gram_ns_equals_standard_ns(shape, steps, segment):
     assert np.max(np.abs(got - O.newton_schulz(G, steps))) < 1e-11
 
 
-def test_gram_ns_segment_one_is_the_standard_bf16_iteration():
-    rng = np.random.default_rng(29)
-    G = rng.standard_normal((24, 56))
-    assert np.array_equal(O.gram_newton_schulz(G, 5, emulate_bf16=True, segment=1),
-                          O.newton_schulz(G, 5, emulate_bf16=True))
-
-
-def test_gram_ns_with_schedule_and_bf16_structure(monkeypatch):
+def test_gram_ns_with_schedule_and_steps():
     rng = np.random.default_rng(27)
     G = rng.standard_normal((12, 30))
     table = [(3.4445, -4.7750, 2.0315), (1.875, -1.25, 0.375), (1.5, -0.5, 0.0)]
     assert np.max(np.abs(O.gram_newton_schulz(G, 3, table) - O.newton_schulz(G, 3, table))) < 1e-11
-    monkeypatch.setattr(O, "bf16_round", lambda v: np.asarray(v, dtype=np.float64))
-    a = O.gram_newton_schulz(G, 5, emulate_bf16=True)
-    monkeypatch.undo()
-    assert np.max(np.abs(a - O.newton_schulz(G, 5))) < 1e-11
     rng = np.random.default_rng(28)
     p, g = rng.standard_normal((10, 40)), rng.standard_normal((10, 40))
     r1 = O.muon_step_matrix(p, g, np.zeros_like(p), lr=0.1, gram=True)

@@ -203,6 +203,93 @@ def param_gpu(m: int, n: int, seed: int, device, std: float = 0.02):
     return std * torch.randn(m, n, generator=gen, device=device, dtype=torch.float32)
 
 
+# ---------------------------------------------------------------------------
+# Values as the device holds them, and the input recipes of the parity tests
+# ---------------------------------------------------------------------------
+
+def as_float32_values(x):
+    """float64 array holding the float32 values the device receives."""
+    return np.asarray(x, dtype=np.float32).astype(np.float64)
+
+
+def as_bf16_values(x):
+    """float64 array holding the bf16 values the device receives (a float32
+    cast, then torch's cast to bfloat16, as the tests upload them)."""
+    import torch
+    t = torch.from_numpy(np.ascontiguousarray(np.asarray(x, dtype=np.float32)))
+    return t.to(torch.bfloat16).to(torch.float64).numpy()
+
+
+def set_values(config: int, shapes, grad_bf16: bool, seed_base: int = 0, indices=None):
+    """The parity tests' inputs for a shape set: {index: (p, g, m0)} with the
+    values the device holds (float32 p, float32 or bf16 g, zero m0). Matrix
+    i uses seed_for(config, i // 7, i % 7) + seed_base."""
+    out = {}
+    for i, (m, n) in enumerate(shapes):
+        if indices is not None and i not in indices:
+            continue
+        seed = seed_for(config, i // 7, i % 7) + seed_base
+        g = gradient_cpu(config, m, n, seed)
+        g = as_bf16_values(g) if grad_bf16 else as_float32_values(g)
+        out[i] = (as_float32_values(param_cpu(m, n, seed)), g, np.zeros((m, n)))
+    return out
+
+
+def gaussian_set(shapes, seed: int, scale: float = 1.0):
+    """Standard-normal matrices (times scale) from one generator, in order,
+    as bf16 values: the stage tests' inputs."""
+    rng = np.random.default_rng(seed)
+    return [as_bf16_values(rng.standard_normal((m, n)) * scale) for (m, n) in shapes]
+
+
+def sweep_matrix(m: int, n: int, index: int):
+    """bf16 values of NS-only sweep input `index` of an m x n point."""
+    return as_bf16_values(gradient_cpu(CONFIG_SWEEP, m, n, seed_for(CONFIG_SWEEP, m // 128, n // 128, index)))
+
+
+# Shape lists of the parity tests (one definition for the tests and for the
+# script that freezes the bf16 program's errors on the same inputs).
+PARITY_SHAPES = {
+    # ragged tiles: 1 x 1, thin rows and columns, tails of 1, tall and wide
+    "ragged": [(1, 1), (3, 5), (5, 3), (1, 300), (300, 1), (127, 129), (129, 127), (64, 64), (256, 512),
+               (512, 256), (384, 384), (200, 1000), (1000, 200), (520, 520), (768, 2304)],
+    # every matrix on the on-chip small path (s <= 128, l <= 512)
+    "small": [(1, 1), (3, 5), (5, 3), (64, 64), (100, 300), (300, 100), (128, 128), (128, 512), (512, 128),
+              (127, 129), (1, 300), (300, 1), (16, 512), (512, 16), (96, 200), (65, 65)],
+    # NS-only sweep points (m, n, batch) small enough for the oracle
+    "sweep": [(128, 128, 4), (128, 512, 2), (512, 128, 2), (256, 256, 3), (256, 2048, 1), (2048, 256, 1),
+              (1024, 1024, 1), (512, 4096, 1)],
+    "mixed": [(128, 512), (512, 128), (64, 64), (768, 768), (300, 100), (1024, 256), (2, 2)],
+    "gram": [(256, 1024), (1024, 256), (384, 384), (300, 1000), (1000, 300), (600, 257), (128, 512), (64, 96)],
+    "deterministic": [(2304, 768), (768, 3072), (300, 1000), (64, 96), (4096, 1024)],
+    "split": [(2304, 768), (768, 768), (768, 3072)],
+    "schedule": [(256, 768), (768, 256), (100, 300), (512, 512)],
+    "wait": [(512, 1024), (1024, 512)],
+    "layerwise": [(256, 768), (768, 256), (64, 64), (1024, 512), (512, 1024), (300, 700)],
+    "noalloc": [(300, 700), (700, 300), (256, 256), (5, 3), (1024, 1024)],
+}
+
+# Row blocks of the split-Muon test (None: the matrix stays whole).
+SPLIT_ROWS = [768, 64, None]
+
+# The varying coefficient table of the schedule test.
+SCHEDULE_TABLE = [(3.4445, -4.7750, 2.0315), (3.0, -3.2, 1.2), (2.5, -2.0, 0.6), (1.875, -1.25, 0.375)]
+
+# Sampled matrices of the full-size sets: Llama layer 0 q (square), k (wide,
+# small), gate (tall) and layer 31 down (wide); three MoE experts' matrices.
+LLAMA_SAMPLE = [0, 1, 4, 223]
+MOE_SAMPLE = [0, 5, 382]
+
+
+def case_key(x, steps: int, coeffs, normalised: bool) -> str:
+    """Identity of one Newton-Schulz input: a digest of its float64 bytes,
+    the iteration count, the coefficients and whether it is normalised."""
+    import hashlib
+    h = hashlib.sha256(np.ascontiguousarray(np.asarray(x, dtype=np.float64)).tobytes())
+    h.update(repr((int(steps), [float(v) for v in np.ravel(coeffs)], bool(normalised))).encode())
+    return h.hexdigest()[:20]
+
+
 def ns_flops(m: int, n: int, steps: int = 5) -> float:
     """Nominal FLOPs of the Newton-Schulz phases: steps * (4 s^2 l + 2 s^3)."""
     s, l = min(m, n), max(m, n)
@@ -216,6 +303,38 @@ def gram_ns_flops(m: int, n: int, steps: int = 5) -> float:
     s, l = min(m, n), max(m, n)
     two, one = steps // 2, steps % 2
     return two * (4.0 * s * s * l + 10.0 * s ** 3) + one * (4.0 * s * s * l + 2.0 * s ** 3)
+
+
+def ns_flops_symmetric(m: int, n: int, steps: int = 5) -> float:
+    """The method's own work per matrix: the Gram and the polynomial are
+    symmetric, so only their upper triangles are computed (s^2 l + s^3),
+    plus the combine (2 s^2 l): steps * (3 s^2 l + s^3)."""
+    s, l = min(m, n), max(m, n)
+    return steps * (3.0 * s * s * l + 1.0 * s ** 3)
+
+
+def gram_ns_flops_symmetric(m: int, n: int, steps: int = 5) -> float:
+    """The Gram form's own work: per two-step segment one symmetric Gram
+    (s^2 l), five symmetric s x s products (s^3 each) and the final product
+    (2 s^2 l); a one-step segment is the plain step."""
+    s, l = min(m, n), max(m, n)
+    two, one = steps // 2, steps % 2
+    return two * (3.0 * s * s * l + 5.0 * s ** 3) + one * (3.0 * s * s * l + 1.0 * s ** 3)
+
+
+def total_ns_flops_symmetric(shapes, steps: int = 5, gram: bool = False) -> float:
+    f = gram_ns_flops_symmetric if gram else ns_flops_symmetric
+    return float(sum(f(m, n, steps) for m, n in shapes))
+
+
+def shape_classes(shapes):
+    """{(m, n): (count, first index)} of a shape set, in first-seen order."""
+    out = {}
+    for i, s in enumerate(shapes):
+        s = (int(s[0]), int(s[1]))
+        c, first = out.get(s, (0, i))
+        out[s] = (c + 1, first)
+    return out
 
 
 def step_bytes(m: int, n: int, grad_bytes: int) -> tuple:
