@@ -117,7 +117,14 @@ typedef struct muon_config {
   int check_nonfinite;        /* 1: count non-finite u entries; read back
                                  with muon_get_status. Default 0           */
   int num_sms;                /* persistent-grid width; 0 = all SMs        */
-  size_t workspace_cap_bytes; /* 0 = no cap                                */
+  size_t workspace_cap_bytes; /* 0 = no cap. With a cap below the
+                                 workspace of a shape table, consecutive
+                                 matrices are packed into groups whose
+                                 workspace fits and the step runs the groups
+                                 one after another through one shared
+                                 workspace (muon_plan_groups gives the
+                                 partition); a matrix that alone exceeds the
+                                 cap fails with MUON_ERR_OOM               */
   double wait_timeout_s;      /* limit of every device-side wait; a wait
                                  that runs out sets the error word and the
                                  kernel returns. Default 2.0 seconds       */
@@ -220,8 +227,11 @@ int muon_qk_clip(muon_handle* h, float* const* weights, const int32_t* shapes,
  * copy-out. Pinned host memory is needed for the copies to overlap. Only
  * matrices with a gradient are copied. The host buffers must stay valid and
  * untouched until `stream` reaches that point, and calls on one handle must
- * be ordered by the caller (one stream). Staging (three chunk slots) is
- * allocated on first use per shape table and counts against the cap. */
+ * be ordered by the caller (one stream). Staging (three chunk slots, 12
+ * bytes per element of the largest chunk) is allocated on first use per
+ * shape table, in addition to the workspace: the workspace cap does not
+ * bound it. Under a cap that splits the set into groups, the chunks are
+ * those groups. */
 int muon_step_host(muon_handle* h, float* const* params,
                    const void* const* grads, float* const* momenta,
                    const int32_t* shapes, int count, float lr, float beta,
@@ -282,8 +292,27 @@ int muon_plan_query(const int32_t* shapes, int count, int ns_precision,
                     int plan_flags, int64_t* ws_bytes, int64_t* region_offsets,
                     int32_t* ntiles, int32_t* tiles, int64_t* chunk_prefix);
 
+/* Matrix groups of a shape table under a workspace cap (needs no GPU). The
+ * workspace holds one double per matrix, then per group the X0, X1, A and B
+ * regions of its matrices; groups run one after another and share it. With
+ * cap = 0, or when everything fits under the cap, there is one group.
+ *   ngroups       : number of groups.
+ *   group_bounds  : int32[count + 1]; group g is matrices
+ *                   group_bounds[g] .. group_bounds[g+1]-1 (entries past
+ *                   ngroups are not written).
+ *   region_offsets: int64[count][4], byte offsets of X0, X1, A, B.
+ *   ws_bytes      : workspace bytes (sum-of-squares block + largest group).
+ * plan_flags as for muon_plan_query. A matrix whose regions alone exceed the
+ * cap is MUON_ERR_OOM; bad shapes are MUON_ERR_INVALID_ARG. Any output
+ * pointer may be NULL. */
+int muon_plan_groups(const int32_t* shapes, int count, int ns_precision,
+                     int plan_flags, size_t cap, int32_t* ngroups,
+                     int32_t* group_bounds, int64_t* region_offsets,
+                     int64_t* ws_bytes);
+
 /* Workspace bytes the handle would allocate for this shape table
- * (excluding muon_step_host staging). */
+ * (excluding muon_step_host staging; under the handle's cap, the grouped
+ * workspace). */
 int muon_workspace_size(muon_handle* h, const int32_t* shapes, int count,
                         size_t* bytes);
 

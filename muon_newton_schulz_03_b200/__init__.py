@@ -202,6 +202,26 @@ def plan_query(shapes, ns_precision: str = "bf16", small_path: bool = True, cta_
     }
 
 
+def plan_groups(shapes, cap_bytes: int, ns_precision: str = "bf16", small_path: bool = True,
+                cta_pair: bool = False):
+    """Matrix groups under a workspace cap. Returns dict(bounds (group g is
+    matrices bounds[g]..bounds[g+1]-1), region_offsets [count][4],
+    ws_bytes). Needs no GPU."""
+    lib = load()
+    sh = [(int(s[0]), int(s[1]), int(s[2]) if len(s) > 2 else 0) for s in shapes]
+    count = len(sh)
+    arr = _shapes_array(sh)
+    sp = (1 if small_path else 0) | (2 if cta_pair else 0)
+    ng = ctypes.c_int32()
+    bounds = (ctypes.c_int32 * (count + 1))()
+    offs = (ctypes.c_int64 * (4 * count))()
+    ws = ctypes.c_int64()
+    check(lib.muon_plan_groups(arr, count, PRECISIONS[ns_precision], sp, int(cap_bytes), ctypes.byref(ng), bounds,
+                               offs, ctypes.byref(ws)))
+    return {"bounds": list(bounds[:ng.value + 1]), "region_offsets": [list(offs[4 * i:4 * i + 4]) for i in range(count)],
+            "ws_bytes": ws.value}
+
+
 class Muon:
     """A handle of the Muon library on one CUDA device."""
 

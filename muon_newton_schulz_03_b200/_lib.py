@@ -61,6 +61,8 @@ _SIGNATURES = {
                            c_float, c_float, c_void_p]),
     "muon_plan_query": (c_int, [P(ctypes.c_int32), c_int, c_int, c_int, P(ctypes.c_int64), P(ctypes.c_int64),
                                 P(ctypes.c_int32), P(ctypes.c_int32), P(ctypes.c_int64)]),
+    "muon_plan_groups": (c_int, [P(ctypes.c_int32), c_int, c_int, c_int, c_size_t, P(ctypes.c_int32),
+                                 P(ctypes.c_int32), P(ctypes.c_int64), P(ctypes.c_int64)]),
     "muon_workspace_size": (c_int, [c_void_p, P(ctypes.c_int32), c_int, P(c_size_t)]),
     "muon_workspace_ptr": (c_int, [c_void_p, P(c_void_p), P(c_size_t)]),
     "muon_get_status": (c_int, [c_void_p, c_void_p, P(ctypes.c_int32), P(ctypes.c_uint64)]),

@@ -11,12 +11,12 @@ namespace muon {
 
 // Grouped elementwise launch: one block per chunk of kElemChunk elements.
 struct ElemLaunch {
-  const MatPlan* plans;     // device
-  const MatBind* binds;     // device
-  const long long* prefix;  // device, count + 1 entries
-  int count;
-  long long block_base;     // first chunk of the launch (0 for a whole set)
-  long long nblocks;        // chunks in the launch (prefix[count] for a whole set)
+  const MatPlan* plans = nullptr;     // device
+  const MatBind* binds = nullptr;     // device
+  const long long* prefix = nullptr;  // device, count + 1 entries
+  int count = 0;
+  long long block_base = 0;           // first chunk of the launch (0 for a whole set)
+  long long nblocks = 0;              // chunks in the launch (prefix[count] for a whole set)
 };
 
 // partials == nullptr: one double atomic per block into sumsq; else each
@@ -83,16 +83,16 @@ enum MapIdx : int {
 };
 
 struct NsLaunch {
-  const MatPlan* plans;      // device
-  const MatBind* binds;      // device
-  const TmapBlob* maps;      // device, kMapsPerMat per matrix (workspace)
-  const TmapBlob* in_maps;   // device, kInMapsPerMat per matrix (caller input) or NULL
-  const int4* tiles;         // device tile list of the phase
-  int ntiles;
-  const double* sumsq;       // device or NULL
-  DevStatus* status;         // device
-  int grid;                  // persistent CTAs
-  unsigned long long timeout_ns;
+  const MatPlan* plans = nullptr;     // device
+  const MatBind* binds = nullptr;     // device
+  const TmapBlob* maps = nullptr;     // device, kMapsPerMat per matrix (workspace)
+  const TmapBlob* in_maps = nullptr;  // device, kInMapsPerMat per matrix (caller input) or NULL
+  const int4* tiles = nullptr;        // device tile list of the phase
+  int ntiles = 0;
+  const double* sumsq = nullptr;      // device or NULL
+  DevStatus* status = nullptr;        // device
+  int grid = 0;                       // persistent CTAs
+  unsigned long long timeout_ns = 0;
   const TmapBlob* gmaps = nullptr;   // device, kGramMapsPerMat per matrix (Gram form only)
   int tma_store = 0;                 // 1: the *_ST store maps are present, stage outputs
                                      //    in shared memory and write them with bulk stores
@@ -110,6 +110,7 @@ struct NsSmallLaunch {
   const double* sumsq;       // device or NULL
   DevStatus* status;         // device
   unsigned long long timeout_ns;
+  int max_l = 1 << 30;       // largest max(m, n) of the listed matrices (<= 128: compact kernel)
 };
 
 // abc: ns_steps rows of (a, b, c).

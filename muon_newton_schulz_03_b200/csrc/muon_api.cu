@@ -55,32 +55,92 @@ struct DeviceGuard {
   }
 };
 
-// Device copy of a host byte blob, uploaded once and kept while in the cache.
-struct DevBlob {
-  std::vector<unsigned char> key;
-  void* dptr = nullptr;
-};
-
 // Builds the bytes of a table on a cache miss.
 typedef int (*BlobBuilder)(const void* ctx, std::vector<unsigned char>& out);
 
-class BlobCache {
+// Device copies of the per-call pointer tables (matrix bindings, tensor maps
+// of caller buffers), in a fixed ring of slots made once per plan.
+//
+// A call whose table bytes match a slot reuses it (nothing is uploaded). A
+// call with new bytes takes the least recently used slot: it writes the bytes
+// into that slot's pinned host staging (after that staging's previous upload
+// has executed), makes the stream wait for the last work that read the slot
+// (an event, so no host synchronisation), and uploads with one
+// cudaMemcpyAsync on the call's stream. After a call's kernels are enqueued,
+// every slot it used records a "used" event on the stream.
+// Slots used while a stream is being captured are pinned: a graph keeps
+// pointing at them, so they are never overwritten until the plan changes.
+// A miss during capture is an error (the upload and the waits cannot be
+// captured): run the call once uncaptured with the same pointers first.
+class TableRing {
  public:
-  ~BlobCache() { clear(); }
-  // Returns the device copy of `bytes`, uploading it (synchronously) on a miss.
-  int get(const void* bytes, size_t n, void** out) { return get_keyed(bytes, n, nullptr, nullptr, out); }
+  ~TableRing() { release(); }
 
-  // Device table identified by `key`; on a miss its bytes come from
-  // build(ctx) (or are the key itself when build is NULL).
-  int get_keyed(const void* key, size_t nkey, BlobBuilder build, const void* ctx, void** out) {
+  // Frees everything (callers make sure no queued work uses the slots).
+  void release() {
+    for (Slot& s : slots_) {
+      if (s.dev) cudaFree(s.dev);
+      if (s.host) cudaFreeHost(s.host);
+      if (s.copied) cudaEventDestroy(s.copied);
+      if (s.used) cudaEventDestroy(s.used);
+    }
+    slots_.clear();
+    cap_ = 0;
+    tick_ = 0;
+    in_call_.clear();
+  }
+
+  // Makes kSlots slots of at least `bytes` each (outside any capture).
+  int reserve(size_t bytes) {
+    bytes = std::max<size_t>(bytes, 256);
+    if (!slots_.empty() && cap_ >= bytes) return MUON_OK;
+    if (!slots_.empty()) {
+      for (const Slot& s : slots_)
+        if (s.pinned)
+          return fail(MUON_ERR_INVALID_ARG, "pointer tables grew while a captured graph holds the old ones");
+      // Growing: queued work may still read the old slots.
+      cudaError_t e = cudaDeviceSynchronize();
+      if (e != cudaSuccess) return fail(MUON_ERR_CUDA, std::string("table ring: ") + cudaGetErrorString(e));
+      release();
+    }
+    slots_.resize(kSlots);
+    for (Slot& s : slots_) {
+      cudaError_t e = cudaMalloc(&s.dev, bytes);
+      if (e == cudaSuccess) e = cudaHostAlloc(&s.host, bytes, cudaHostAllocDefault);
+      if (e == cudaSuccess) e = cudaEventCreateWithFlags(&s.copied, cudaEventDisableTiming);
+      if (e == cudaSuccess) e = cudaEventCreateWithFlags(&s.used, cudaEventDisableTiming);
+      if (e != cudaSuccess) {
+        cudaGetLastError();
+        release();
+        return fail(e == cudaErrorMemoryAllocation ? MUON_ERR_OOM : MUON_ERR_CUDA,
+                    std::string("table ring allocation: ") + cudaGetErrorString(e));
+      }
+    }
+    cap_ = bytes;
+    return MUON_OK;
+  }
+
+  // Device table for `key`; on a miss its bytes come from build(ctx) (or are
+  // the key itself when build is NULL). Stream-ordered on `st`.
+  int get(const void* key, size_t nkey, BlobBuilder build, const void* ctx, cudaStream_t st, void** out) {
+    cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+    cudaError_t e = cudaStreamIsCapturing(st, &cs);
+    if (e != cudaSuccess) return fail(MUON_ERR_CUDA, std::string("cudaStreamIsCapturing: ") + cudaGetErrorString(e));
+    const bool capturing = cs != cudaStreamCaptureStatusNone;
     const unsigned char* k = static_cast<const unsigned char*>(key);
-    for (auto it = entries_.begin(); it != entries_.end(); ++it) {
-      if (it->key.size() == nkey && std::memcmp(it->key.data(), k, nkey) == 0) {
-        entries_.splice(entries_.begin(), entries_, it);
-        *out = entries_.front().dptr;
+    for (size_t i = 0; i < slots_.size(); ++i) {
+      Slot& s = slots_[i];
+      if (s.filled && s.key.size() == nkey && std::memcmp(s.key.data(), k, nkey) == 0) {
+        s.last = ++tick_;
+        if (capturing) s.pinned = true;
+        note_use(i);
+        *out = s.dev;
         return MUON_OK;
       }
     }
+    if (capturing)
+      return fail(MUON_ERR_INVALID_ARG, "these pointers have no device tables yet and tables cannot be uploaded "
+                                        "during stream capture: run the same call once before capturing it");
     std::vector<unsigned char> content;
     const unsigned char* src = k;
     size_t n = nkey;
@@ -90,32 +150,74 @@ class BlobCache {
       src = content.data();
       n = content.size();
     }
-    if (entries_.size() >= kMax) {
-      // The evicted table may still be read by queued work: wait for it.
-      MUON_CUDA_TRY(cudaDeviceSynchronize());
-      cudaFree(entries_.back().dptr);
-      entries_.pop_back();
+    int rc = reserve(n);
+    if (rc) return rc;
+    size_t victim = slots_.size();
+    for (size_t i = 0; i < slots_.size(); ++i) {
+      if (slots_[i].pinned || is_in_call(i)) continue;
+      if (victim == slots_.size() || slots_[i].last < slots_[victim].last) victim = i;
     }
-    DevBlob e;
-    e.key.assign(k, k + nkey);
-    MUON_CUDA_TRY(cudaMalloc(&e.dptr, std::max<size_t>(n, 16)));
-    cudaError_t err = cudaMemcpy(e.dptr, src, n, cudaMemcpyHostToDevice);
-    if (err != cudaSuccess) {
-      cudaFree(e.dptr);
-      return fail(MUON_ERR_CUDA, std::string("table upload: ") + cudaGetErrorString(err));
+    if (victim == slots_.size())
+      return fail(MUON_ERR_INVALID_ARG, "every pointer-table slot is pinned by a captured graph or used by this "
+                                        "call; release the graphs (or change the plan) to free them");
+    Slot& s = slots_[victim];
+    if (s.filled) {
+      // The staging's previous upload must have executed before it is
+      // rewritten; the device copy waits for the slot's last readers.
+      e = cudaEventSynchronize(s.copied);
+      if (e == cudaSuccess) e = cudaStreamWaitEvent(st, s.used, 0);
+      if (e != cudaSuccess) return fail(MUON_ERR_CUDA, std::string("table ring: ") + cudaGetErrorString(e));
     }
-    entries_.push_front(std::move(e));
-    *out = entries_.front().dptr;
+    std::memcpy(s.host, src, n);
+    e = cudaMemcpyAsync(s.dev, s.host, n, cudaMemcpyHostToDevice, st);
+    if (e == cudaSuccess) e = cudaEventRecord(s.copied, st);
+    if (e != cudaSuccess) return fail(MUON_ERR_CUDA, std::string("table upload: ") + cudaGetErrorString(e));
+    s.key.assign(k, k + nkey);
+    s.filled = true;
+    s.last = ++tick_;
+    note_use(victim);
+    *out = s.dev;
     return MUON_OK;
   }
-  void clear() {
-    for (auto& e : entries_) cudaFree(e.dptr);
-    entries_.clear();
+
+  // After a call's kernels are enqueued: the slots it used record that
+  // point of the stream (skipped while capturing: those slots are pinned).
+  int end_call(cudaStream_t st) {
+    cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+    cudaStreamIsCapturing(st, &cs);
+    int rc = MUON_OK;
+    if (cs == cudaStreamCaptureStatusNone)
+      for (size_t i : in_call_) {
+        cudaError_t e = cudaEventRecord(slots_[i].used, st);
+        if (e != cudaSuccess && rc == MUON_OK) rc = fail(MUON_ERR_CUDA, std::string("table ring: ") + cudaGetErrorString(e));
+      }
+    in_call_.clear();
+    return rc;
   }
 
+  void abandon_call() { in_call_.clear(); }
+  size_t slot_bytes() const { return cap_; }
+
  private:
-  static constexpr size_t kMax = 8;
-  std::list<DevBlob> entries_;
+  struct Slot {
+    std::vector<unsigned char> key;
+    void* dev = nullptr;
+    void* host = nullptr;        // pinned staging of the upload
+    cudaEvent_t copied = nullptr;
+    cudaEvent_t used = nullptr;
+    unsigned long long last = 0;
+    bool filled = false;
+    bool pinned = false;
+  };
+  static constexpr int kSlots = 8;
+  void note_use(size_t i) {
+    if (!is_in_call(i)) in_call_.push_back(i);
+  }
+  bool is_in_call(size_t i) const { return std::find(in_call_.begin(), in_call_.end(), i) != in_call_.end(); }
+  std::vector<Slot> slots_;
+  size_t cap_ = 0;
+  unsigned long long tick_ = 0;
+  std::vector<size_t> in_call_;
 };
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
@@ -206,6 +308,9 @@ struct DevPlan {
   size_t staging_size = 0;
   size_t slot_bytes = 0;
   std::vector<int64_t> staging_off;              // count * 3: param, grad, momentum (within the slot)
+  bool grouped = false;                          // chunks are the workspace cap's groups
+  std::vector<TileRec> chunk_tiles_host[3];      // host copies of the per-chunk tile lists
+  std::vector<int> chunk_small_host;
 };
 
 // Work of one enqueue: matrices [m0, m1), elementwise chunks [blk0, blk1),
@@ -228,8 +333,9 @@ struct muon_handle {
   int num_sms = 0;
   DevStatus* status = nullptr;
   std::unique_ptr<DevPlan> plan;
-  BlobCache binds;
-  BlobCache in_maps;
+  TableRing binds;     // MatBind tables of the calls
+  TableRing in_maps;   // tensor maps of the callers' X inputs (stage call)
+  TableRing subsets;   // tile lists restricted to the matrices with a gradient
   int last_launches = 0;
   // Per-launch timing (muon_profile_enable / muon_profile_read).
   std::vector<cudaEvent_t> prof_ev;   // 2 per slot
@@ -268,12 +374,19 @@ int ensure_gram_buffers(DevPlan& P) {
   for (int i : P.hp.small) tiled[(size_t)i] = 0;
   std::vector<int64_t> off((size_t)count * 2, -1);
   int64_t total = 0;
-  for (int i = 0; i < count; ++i)
-    if (tiled[(size_t)i])
-      for (int k = 0; k < 2; ++k) {
-        off[(size_t)i * 2 + k] = total;
-        total = align_up(total + (int64_t)P.mats[i].s * P.mats[i].lds * 2, kRegionAlign);
-      }
+  // Groups of a capped plan run one after another: each lays out its own
+  // buffers from offset 0.
+  const std::vector<int>& groups = P.hp.groups;
+  for (size_t gi = 0; gi + 1 < groups.size(); ++gi) {
+    int64_t goff = 0;
+    for (int i = groups[gi]; i < groups[gi + 1]; ++i)
+      if (tiled[(size_t)i])
+        for (int k = 0; k < 2; ++k) {
+          off[(size_t)i * 2 + k] = goff;
+          goff = align_up(goff + (int64_t)P.mats[i].s * P.mats[i].lds * 2, kRegionAlign);
+        }
+    total = std::max(total, goff);
+  }
   if (total > 0) {
     cudaError_t e = cudaMalloc(&P.gram_ws, (size_t)total);
     if (e != cudaSuccess) {
@@ -354,17 +467,21 @@ int ensure_plan(muon_handle* h, const int32_t* shapes, int count) {
   std::string why;
   if (!build_plan(shapes, count, h->cfg.ns_precision, h->cfg.small_path != 0, h->cfg.cta_pair != 0, np->hp, why))
     return fail(MUON_ERR_INVALID_ARG, why);
+  // Under a workspace cap the matrices run in groups that share one
+  // workspace (consecutive matrices, each group as large as fits).
+  if (h->cfg.workspace_cap_bytes &&
+      !build_plan(shapes, count, h->cfg.ns_precision, h->cfg.small_path != 0, h->cfg.cta_pair != 0, np->hp, why,
+                  (int64_t)h->cfg.workspace_cap_bytes))
+    return fail(MUON_ERR_OOM, why);
   np->key = key;
   const HostPlan& hp = np->hp;
-  if (h->cfg.workspace_cap_bytes && (size_t)hp.ws_bytes > h->cfg.workspace_cap_bytes)
-    return fail(MUON_ERR_OOM, "workspace of " + std::to_string(hp.ws_bytes) + " bytes exceeds the cap of " +
-                                  std::to_string(h->cfg.workspace_cap_bytes));
 
   // Drop the previous plan first (queued work may still use it).
   if (h->plan) {
     MUON_CUDA_TRY(cudaDeviceSynchronize());
-    h->binds.clear();
-    h->in_maps.clear();
+    h->binds.release();
+    h->in_maps.release();
+    h->subsets.release();
     free_plan(h->plan.get());
     h->plan.reset();
   }
@@ -398,8 +515,14 @@ int ensure_plan(muon_handle* h, const int32_t* shapes, int count) {
   }
   const int64_t o_small = off;
   off = align_up(off + (int64_t)sizeof(int) * std::max<size_t>(hp.small.size(), 1), 256);
-  // Chunk partition and per-chunk slices of the tile lists.
-  {
+  // Chunk partition and per-chunk slices of the tile lists: the cap's
+  // groups when there are several (muon_step and muon_newton_schulz run them
+  // one after another), else up to kHostChunks chunks of about equal element
+  // counts for the pipelined host-buffer step.
+  np->grouped = hp.groups.size() > 2;
+  if (np->grouped) {
+    np->chunk_bounds = hp.groups;
+  } else {
     const int nch = std::min(count, kHostChunks);
     long long total = 0;
     for (int i = 0; i < count; ++i) total += np->mats[i].numel;
@@ -459,6 +582,8 @@ int ensure_plan(muon_handle* h, const int32_t* shapes, int count) {
   }
   if (!chunk_small.empty())
     std::memcpy(host.data() + o_csmall, chunk_small.data(), sizeof(int) * chunk_small.size());
+  for (int p = 0; p < 3; ++p) np->chunk_tiles_host[p] = chunk_tiles[p];
+  np->chunk_small_host = chunk_small;
   if (bf16) {
     TmapBlob* maps = reinterpret_cast<TmapBlob*>(host.data() + o_maps);
     for (int i = 0; i < count; ++i) {
@@ -632,6 +757,8 @@ int enqueue_ns(muon_handle* h, const MatBind* d_binds, const std::vector<MatBind
     S.sumsq = sumsq;
     S.status = h->status;
     S.timeout_ns = (unsigned long long)(h->cfg.wait_timeout_s * 1e9);
+    S.max_l = 0;
+    for (int i : hp.small) S.max_l = std::max(S.max_l, P.mats[i].l);
     const int flips = h->cfg.ns_algorithm == MUON_NS_GRAM ? (ns_steps + 1) / 2 : ns_steps;
     const int final_sel = last_dst >= 0 ? last_dst : (flips % 2 == 1 ? BUF_X1 : BUF_X0);
     const int slot = prof_before(h, MUON_KERNEL_NS_SMALL, st);
@@ -789,7 +916,7 @@ int check_scalars(float lr, float beta, float wd) {
 
 // Device pointer table of a step (cached by content).
 int step_binds(muon_handle* h, float* const* params, const void* const* grads, float* const* momenta,
-               const int32_t* shapes, int count, std::vector<MatBind>& hb, const MatBind** db) {
+               const int32_t* shapes, int count, cudaStream_t st, std::vector<MatBind>& hb, const MatBind** db) {
   hb.assign((size_t)count, MatBind());
   for (int i = 0; i < count; ++i) {
     MatBind& b = hb[i];
@@ -802,8 +929,95 @@ int step_binds(muon_handle* h, float* const* params, const void* const* grads, f
   }
   void* d_binds = nullptr;
   int rc;
-  if ((rc = h->binds.get(hb.data(), sizeof(MatBind) * count, &d_binds))) return rc;
+  if ((rc = h->binds.get(hb.data(), sizeof(MatBind) * count, nullptr, nullptr, st, &d_binds))) return rc;
   *db = static_cast<const MatBind*>(d_binds);
+  return MUON_OK;
+}
+
+// Ends a call for the pointer-table rings on scope exit: every slot the call
+// used records the point of `st` after its kernels.
+struct CallTables {
+  muon_handle* h;
+  cudaStream_t st;
+  ~CallTables() {
+    h->binds.end_call(st);
+    h->in_maps.end_call(st);
+    h->subsets.end_call(st);
+  }
+};
+
+// Work ranges of a step: one per group of the plan (one group without a
+// workspace cap). When some matrices have no gradient, the Newton-Schulz
+// tile lists and the small-path list are restricted to the active matrices:
+// the lists of every group, filtered, are one device table (kept in a ring
+// keyed by the active mask), so a step over a few owned matrices (a round
+// of layer-wise Muon) launches over their tiles only.
+int step_ranges(muon_handle* h, const std::vector<MatBind>& hb, cudaStream_t st, std::vector<WorkRange>& out) {
+  DevPlan& P = *h->plan;
+  const int count = P.hp.count;
+  const int nch = P.grouped ? (int)P.chunk_bounds.size() - 1 : 1;
+  out.clear();
+  for (int c = 0; c < nch; ++c) out.push_back(P.grouped ? chunk_range(P, c) : full_range(P));
+  std::vector<unsigned char> mask((size_t)count);
+  bool all = true;
+  for (int i = 0; i < count; ++i) {
+    mask[i] = hb[i].active ? 1 : 0;
+    all = all && hb[i].active;
+  }
+  if (all) return MUON_OK;
+  // Filtered lists, chunk by chunk: 3 tile lists (int4) then the small list
+  // (int), each section 16-byte aligned.
+  std::vector<size_t> sec_off((size_t)nch * 4 + 1, 0);
+  std::vector<int> sec_n((size_t)nch * 4, 0);
+  std::vector<unsigned char> bytes;
+  auto put = [&](const void* src, size_t n) {
+    const size_t at = bytes.size();
+    bytes.resize(at + ((n + 15) / 16) * 16, 0);
+    if (n) std::memcpy(bytes.data() + at, src, n);
+  };
+  for (int c = 0; c < nch; ++c) {
+    for (int p = 0; p < 3; ++p) {
+      const std::vector<TileRec>& src = P.grouped ? P.chunk_tiles_host[p] : P.hp.tiles[p];
+      const int t0 = P.grouped ? P.chunk_tile_off[p][c] : 0;
+      const int t1 = P.grouped ? P.chunk_tile_off[p][c + 1] : (int)src.size();
+      std::vector<int4> f;
+      for (int t = t0; t < t1; ++t)
+        if (mask[src[t].mat]) f.push_back(make_int4(src[t].mat, src[t].ti, src[t].tj, 0));
+      sec_off[(size_t)c * 4 + p] = bytes.size();
+      sec_n[(size_t)c * 4 + p] = (int)f.size();
+      put(f.data(), sizeof(int4) * f.size());
+    }
+    const std::vector<int>& ssrc = P.grouped ? P.chunk_small_host : P.hp.small;
+    const int s0 = P.grouped ? P.chunk_small_off[c] : 0;
+    const int s1 = P.grouped ? P.chunk_small_off[c + 1] : (int)ssrc.size();
+    std::vector<int> f;
+    for (int k = s0; k < s1; ++k)
+      if (mask[ssrc[k]]) f.push_back(ssrc[k]);
+    sec_off[(size_t)c * 4 + 3] = bytes.size();
+    sec_n[(size_t)c * 4 + 3] = (int)f.size();
+    put(f.data(), sizeof(int) * f.size());
+  }
+  if (bytes.empty()) bytes.resize(16, 0);
+  struct Ctx {
+    const std::vector<unsigned char>* b;
+  } ctx{&bytes};
+  auto build = [](const void* c, std::vector<unsigned char>& o) -> int {
+    o = *static_cast<const Ctx*>(c)->b;
+    return MUON_OK;
+  };
+  void* d = nullptr;
+  int rc;
+  if ((rc = h->subsets.get(mask.data(), mask.size(), build, &ctx, st, &d))) return rc;
+  char* base = static_cast<char*>(d);
+  for (int c = 0; c < nch; ++c) {
+    WorkRange& R = out[c];
+    for (int p = 0; p < 3; ++p) {
+      R.tiles[p] = reinterpret_cast<const int4*>(base + sec_off[(size_t)c * 4 + p]);
+      R.ntiles[p] = sec_n[(size_t)c * 4 + p];
+    }
+    R.small = reinterpret_cast<const int*>(base + sec_off[(size_t)c * 4 + 3]);
+    R.nsmall = sec_n[(size_t)c * 4 + 3];
+  }
   return MUON_OK;
 }
 
@@ -843,14 +1057,19 @@ int step_impl(muon_handle* h, float* const* params, const void* const* grads, fl
               const float* abc, cudaStream_t st) {
   int rc;
   if ((rc = ensure_plan(h, shapes, count))) return rc;
+  CallTables ct{h, st};
   std::vector<MatBind> hb;
   const MatBind* db = nullptr;
-  if ((rc = step_binds(h, params, grads, momenta, shapes, count, hb, &db))) return rc;
+  if ((rc = step_binds(h, params, grads, momenta, shapes, count, st, hb, &db))) return rc;
   int launches = 0;
   prof_call_begin(h);
-  if ((rc = enqueue_step_range(h, db, hb, full_range(*h->plan), lr, beta, nesterov, wd, ns_steps, abc, st,
-                               &launches)))
-    return rc;
+  DevPlan& P = *h->plan;
+  std::vector<WorkRange> ranges;
+  if ((rc = step_ranges(h, hb, st, ranges))) return rc;
+  // Groups under the workspace cap run one after another on the stream.
+  for (const WorkRange& R : ranges)
+    if ((rc = enqueue_step_range(h, db, hb, R, lr, beta, nesterov, wd, ns_steps, abc, st, &launches))) return rc;
+  (void)P;
   h->last_launches = launches;
   return MUON_OK;
 }
@@ -927,8 +1146,9 @@ int muon_destroy(muon_handle* h) {
   {
     DeviceGuard g(h->device);
     cudaDeviceSynchronize();
-    h->binds.clear();
-    h->in_maps.clear();
+    h->binds.release();
+    h->in_maps.release();
+    h->subsets.release();
     if (h->plan) free_plan(h->plan.get());
     prof_free(h);
     for (cudaEvent_t e : h->hev) cudaEventDestroy(e);
@@ -1032,8 +1252,6 @@ int muon_step_host(muon_handle* h, float* const* params, const void* const* grad
     }
     const int slots = std::min(nch, kStagingSlots);
     const size_t total = slot * (size_t)slots;
-    if (h->cfg.workspace_cap_bytes && total + (size_t)P.hp.ws_bytes > h->cfg.workspace_cap_bytes)
-      return fail(MUON_ERR_OOM, "staging plus workspace exceed the cap");
     cudaError_t e = cudaMalloc(&P.staging, total);
     if (e != cudaSuccess) {
       cudaGetLastError();
@@ -1067,9 +1285,10 @@ int muon_step_host(muon_handle* h, float* const* params, const void* const* grad
       dm[i] = reinterpret_cast<float*>(slot + P.staging_off[(size_t)i * 3 + 2]);
     }
   }
+  CallTables ct{h, st};
   std::vector<MatBind> hb;
   const MatBind* db = nullptr;
-  if ((rc = step_binds(h, dp.data(), dg.data(), dm.data(), shapes, count, hb, &db))) return rc;
+  if ((rc = step_binds(h, dp.data(), dg.data(), dm.data(), shapes, count, st, hb, &db))) return rc;
 
   cudaStream_t s_in = h->hs[0], s_comp = h->hs[1], s_out = h->hs[2];
   MUON_CUDA_TRY(cudaEventRecord(ev_begin, st));
@@ -1137,9 +1356,10 @@ int muon_momentum_norm(muon_handle* h, const void* const* grads, float* const* m
     hb[i].flags = shapes[3 * i + 2];
     hb[i].active = grads[i] != nullptr;
   }
-  void* d_binds = nullptr;
-  if ((rc = h->binds.get(hb.data(), sizeof(MatBind) * count, &d_binds))) return rc;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
+  CallTables ct{h, st};
+  void* d_binds = nullptr;
+  if ((rc = h->binds.get(hb.data(), sizeof(MatBind) * count, nullptr, nullptr, st, &d_binds))) return rc;
   MUON_CUDA_TRY(cudaMemsetAsync(sumsq, 0, sizeof(double) * count, st));
   prof_call_begin(h);
   const ElemLaunch EL = elem_launch(P, static_cast<const MatBind*>(d_binds));
@@ -1183,10 +1403,11 @@ int muon_newton_schulz(muon_handle* h, const void* const* x_in, void* const* x_o
     hb[i].xout = x_out[i];
     hb[i].active = 1;
   }
-  void* d_binds = nullptr;
-  if ((rc = h->binds.get(hb.data(), sizeof(MatBind) * count, &d_binds))) return rc;
-  const MatBind* db = static_cast<const MatBind*>(d_binds);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
+  CallTables ct{h, st};
+  void* d_binds = nullptr;
+  if ((rc = h->binds.get(hb.data(), sizeof(MatBind) * count, nullptr, nullptr, st, &d_binds))) return rc;
+  const MatBind* db = static_cast<const MatBind*>(d_binds);
   int launches = 0;
   prof_call_begin(h);
   if (ns_steps == 0) {
@@ -1216,12 +1437,19 @@ int muon_newton_schulz(muon_handle* h, const void* const* x_in, void* const* x_o
       return MUON_OK;
     };
     void* dm = nullptr;
-    if ((rc = h->in_maps.get_keyed(x_in, sizeof(void*) * (size_t)count, build, &ctx, &dm))) return rc;
+    if ((rc = h->in_maps.get(x_in, sizeof(void*) * (size_t)count, build, &ctx, st, &dm))) return rc;
     d_in = static_cast<const TmapBlob*>(dm);
   }
   int res = BUF_IN;
-  if ((rc = enqueue_ns(h, db, hb, full_range(P), d_in, sumsq, ns_steps, abc, BUF_IN, BUF_OUT, st, &launches, &res)))
+  if (P.grouped) {
+    for (int c = 0; c + 1 < (int)P.chunk_bounds.size(); ++c)
+      if ((rc = enqueue_ns(h, db, hb, chunk_range(P, c), d_in, sumsq, ns_steps, abc, BUF_IN, BUF_OUT, st, &launches,
+                           &res)))
+        return rc;
+  } else if ((rc = enqueue_ns(h, db, hb, full_range(P), d_in, sumsq, ns_steps, abc, BUF_IN, BUF_OUT, st, &launches,
+                              &res))) {
     return rc;
+  }
   h->last_launches = launches;
   return MUON_OK;
 }
@@ -1248,9 +1476,10 @@ int muon_apply(muon_handle* h, float* const* params, const void* const* o, const
     hb[i].xin = o[i];
     hb[i].active = o[i] != nullptr;
   }
-  void* d_binds = nullptr;
-  if ((rc = h->binds.get(hb.data(), sizeof(MatBind) * count, &d_binds))) return rc;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
+  CallTables ct{h, st};
+  void* d_binds = nullptr;
+  if ((rc = h->binds.get(hb.data(), sizeof(MatBind) * count, nullptr, nullptr, st, &d_binds))) return rc;
   prof_call_begin(h);
   const int slot = prof_before(h, MUON_KERNEL_APPLY, st);
   MUON_CUDA_TRY(launch_apply(elem_launch(P, static_cast<const MatBind*>(d_binds)), BUF_IN, lr, wd,
@@ -1303,7 +1532,30 @@ int muon_workspace_size(muon_handle* h, const int32_t* shapes, int count, size_t
   std::string why;
   if (!build_plan(shapes, count, h->cfg.ns_precision, h->cfg.small_path != 0, h->cfg.cta_pair != 0, hp, why))
     return fail(MUON_ERR_INVALID_ARG, why);
+  if (h->cfg.workspace_cap_bytes &&
+      !build_plan(shapes, count, h->cfg.ns_precision, h->cfg.small_path != 0, h->cfg.cta_pair != 0, hp, why,
+                  (int64_t)h->cfg.workspace_cap_bytes))
+    return fail(MUON_ERR_OOM, why);
   *bytes = (size_t)hp.ws_bytes;
+  return MUON_OK;
+}
+
+int muon_plan_groups(const int32_t* shapes, int count, int ns_precision, int plan_flags, size_t cap,
+                     int32_t* ngroups, int32_t* group_bounds, int64_t* region_offsets, int64_t* ws_bytes) {
+  g_last_error.clear();
+  if (plan_flags & ~(MUON_PLAN_SMALL_PATH | MUON_PLAN_CTA_PAIR)) return fail(MUON_ERR_INVALID_ARG, "unknown plan flags");
+  HostPlan hp;
+  std::string why;
+  const bool small = (plan_flags & MUON_PLAN_SMALL_PATH) != 0, pair = (plan_flags & MUON_PLAN_CTA_PAIR) != 0;
+  if (!build_plan(shapes, count, ns_precision, small, pair, hp, why)) return fail(MUON_ERR_INVALID_ARG, why);
+  if (cap && !build_plan(shapes, count, ns_precision, small, pair, hp, why, (int64_t)cap))
+    return fail(MUON_ERR_OOM, why);
+  const int ng = (int)hp.groups.size() - 1;
+  if (ngroups) *ngroups = ng;
+  if (group_bounds)
+    for (int g = 0; g <= ng; ++g) group_bounds[g] = hp.groups[g];
+  if (region_offsets) std::memcpy(region_offsets, hp.region_off.data(), sizeof(int64_t) * hp.region_off.size());
+  if (ws_bytes) *ws_bytes = hp.ws_bytes;
   return MUON_OK;
 }
 

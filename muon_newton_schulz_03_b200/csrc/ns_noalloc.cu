@@ -264,6 +264,7 @@ extern "C" int muon_newton_schulz_noalloc(const void* const* x_in, void* const* 
     EL.binds = d_binds;
     EL.prefix = reinterpret_cast<const long long*>(base + o_pref);
     EL.count = count;
+    EL.block_base = 0;
     EL.nblocks = hp.prefix[count];
     NOALLOC_CUDA_TRY(launch_scale_copy(EL, BUF_IN, BUF_OUT, sumsq, false, st));
   } else {

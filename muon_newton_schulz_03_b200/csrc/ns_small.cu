@@ -24,6 +24,14 @@
 // w reads tensor-memory lanes 32w..32w+31, i.e. output rows). Every wait is
 // bounded; on expiry the error word is set, the outstanding copy or MMA is
 // drained, tensor memory is freed and the CTA returns.
+//
+// Two sizes of the kernel: the general one (X up to 128 x 512 or 512 x 128:
+// 192 KiB of shared memory and all 512 tensor-memory columns, one CTA per
+// SM), and a compact one for calls whose small matrices all have
+// max(m, n) <= 128 (X image 32 KiB, 96 KiB in all, 256 columns: the Gram
+// accumulator in columns 0..127 is dead once the polynomial's epilogue has
+// read it, and the combine reuses them), so two CTAs share an SM and hide
+// each other's phase latencies.
 #include "common.cuh"
 #include "kernels.h"
 
@@ -32,11 +40,11 @@ namespace muon {
 namespace {
 
 constexpr int kThreads = 128;
-constexpr int kXBytes = 128 * 1024;     // X image
 constexpr int kABytes = 128 * 128 * 2;  // A image (two 16 KiB chunks)
 constexpr int kChunk = 128 * 128;       // one 64-column chunk of a 128-row image
-constexpr int kTmemCols = 512;
 
+// kXBytes: X image capacity; kTmemCols: tensor-memory columns of the CTA.
+template <int kXBytes>
 struct __align__(1024) SmallSmem {
   uint8_t x[kXBytes];
   uint8_t a[kABytes];
@@ -46,6 +54,9 @@ struct __align__(1024) SmallSmem {
   uint32_t tmem_base;
   int abort_flag;
 };
+
+constexpr int kXFull = 128 * 1024, kTmemFull = 512;      // X up to 128 x 512 / 512 x 128
+constexpr int kXCompact = 32 * 1024, kTmemCompact = 256;  // X up to 128 x 128
 
 struct SmallArgs {
   NsSmallLaunch L;
@@ -85,9 +96,11 @@ __device__ __forceinline__ void sts_row32(uint8_t* img, int r, int c0, int cs, c
 
 __device__ __forceinline__ float bf16r(float v) { return __bfloat162float(__float2bfloat16_rn(v)); }
 
-__global__ void __launch_bounds__(kThreads, 1) ns_small_kernel(const __grid_constant__ SmallArgs args) {
+template <int kXBytes, int kTmemCols, int kMinBlocks>
+__global__ void __launch_bounds__(kThreads, kMinBlocks) ns_small_kernel(const __grid_constant__ SmallArgs args) {
   extern __shared__ uint8_t smem_raw[];
-  SmallSmem& sm = *reinterpret_cast<SmallSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  SmallSmem<kXBytes>& sm =
+      *reinterpret_cast<SmallSmem<kXBytes>*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const NsSmallLaunch& L = args.L;
   const int mat = L.mats[blockIdx.x];
   const MatPlan mp = L.plans[mat];
@@ -310,18 +323,12 @@ __global__ void __launch_bounds__(kThreads, 1) ns_small_kernel(const __grid_cons
 
 }  // namespace
 
-int ns_small_smem_bytes() { return (int)sizeof(SmallSmem) + 1024; }
+int ns_small_smem_bytes() { return (int)sizeof(SmallSmem<kXFull>) + 1024; }
 
 cudaError_t launch_ns_small(const NsSmallLaunch& L, int ns_steps, int src_sel, int final_sel, const float* abc,
                             cudaStream_t st) {
   if (L.nmats <= 0 || ns_steps <= 0) return cudaSuccess;
   if (ns_steps > kMaxNsSteps) return cudaErrorInvalidValue;
-  static std::atomic<unsigned long long> attr_done{0};
-  const int smem = ns_small_smem_bytes();
-  {
-    const cudaError_t e = ensure_dynamic_smem(ns_small_kernel, smem, attr_done);
-    if (e != cudaSuccess) return e;
-  }
   SmallArgs args;
   args.L = L;
   args.ns_steps = ns_steps;
@@ -329,7 +336,21 @@ cudaError_t launch_ns_small(const NsSmallLaunch& L, int ns_steps, int src_sel, i
   args.final_sel = final_sel;
   for (int t = 0; t < ns_steps; ++t)
     for (int k = 0; k < 3; ++k) args.coef[t][k] = abc[3 * t + k];
-  ns_small_kernel<<<L.nmats, kThreads, smem, st>>>(args);
+  if (L.max_l <= 128) {
+    static std::atomic<unsigned long long> attr_done{0};
+    const int smem = (int)sizeof(SmallSmem<kXCompact>) + 1024;
+    auto kern = ns_small_kernel<kXCompact, kTmemCompact, 2>;
+    const cudaError_t e = ensure_dynamic_smem(kern, smem, attr_done);
+    if (e != cudaSuccess) return e;
+    kern<<<L.nmats, kThreads, smem, st>>>(args);
+  } else {
+    static std::atomic<unsigned long long> attr_done{0};
+    const int smem = ns_small_smem_bytes();
+    auto kern = ns_small_kernel<kXFull, kTmemFull, 1>;
+    const cudaError_t e = ensure_dynamic_smem(kern, smem, attr_done);
+    if (e != cudaSuccess) return e;
+    kern<<<L.nmats, kThreads, smem, st>>>(args);
+  }
   return cudaGetLastError();
 }
 

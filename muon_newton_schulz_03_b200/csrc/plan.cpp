@@ -17,7 +17,12 @@
 //  * small path (when enabled): matrices with s <= 128 and l <= 512 are left
 //    out of the tile lists and listed, in index order, for the on-chip
 //    kernel that runs the whole iteration in one CTA;
-//  * elementwise: kElemChunk elements per block, prefix over matrices.
+//  * elementwise: kElemChunk elements per block, prefix over matrices;
+//  * workspace cap: when the layout above exceeds a cap, consecutive
+//    matrices are packed into groups (each as large as fits, in index
+//    order); each group's X0, X1, A and B regions are laid out as above
+//    starting right after the sum-of-squares block, so the workspace is that
+//    block plus the largest group.
 #include "plan.h"
 
 #include <algorithm>
@@ -50,7 +55,7 @@ void comb_tiles(int mat, int m, int n, int bm, std::vector<TileRec>& out) {
 }  // namespace
 
 bool build_plan(const int32_t* shapes, int count, int prec, bool small_path, bool pair_tiles, HostPlan& P,
-                std::string& why) {
+                std::string& why, int64_t ws_cap) {
   if (shapes == nullptr) { why = "shapes is NULL"; return false; }
   if (count < 1) { why = "count must be >= 1"; return false; }
   if (prec != 0 && prec != 1) { why = "ns_precision must be 0 (bf16) or 1 (fp32)"; return false; }
@@ -85,17 +90,46 @@ bool build_plan(const int32_t* shapes, int count, int prec, bool small_path, boo
   }
   const int64_t elem = prec == 0 ? 2 : 4;
   P.head_bytes = round_up64(8 * (int64_t)count, kRegionAlign);
-  int64_t off = P.head_bytes;
-  P.region_off.assign((size_t)count * 4, 0);
-  for (int which = 0; which < 4; ++which) {
+  auto region_bytes = [&](int i, int which) {
+    const MatPlan& mp = P.mats[i];
+    return round_up64((which < 2 ? (int64_t)mp.m * mp.ldx : (int64_t)mp.s * mp.lds) * elem, kRegionAlign);
+  };
+  auto matrix_bytes = [&](int i) {
+    int64_t b = 0;
+    for (int which = 0; which < 4; ++which) b += region_bytes(i, which);
+    return b;
+  };
+  int64_t all = 0;
+  for (int i = 0; i < count; ++i) all += matrix_bytes(i);
+  P.groups.assign(1, 0);
+  if (ws_cap > 0 && P.head_bytes + all > ws_cap) {
+    int64_t in_group = 0;
     for (int i = 0; i < count; ++i) {
-      const MatPlan& mp = P.mats[i];
-      const int64_t bytes = (which < 2 ? (int64_t)mp.m * mp.ldx : (int64_t)mp.s * mp.lds) * elem;
-      P.region_off[(size_t)i * 4 + which] = off;
-      off = round_up64(off + bytes, kRegionAlign);
+      const int64_t b = matrix_bytes(i);
+      if (P.head_bytes + b > ws_cap) {
+        why = "matrix " + std::to_string(i) + " alone needs " + std::to_string(P.head_bytes + b) +
+              " bytes of workspace, above the cap of " + std::to_string(ws_cap);
+        return false;
+      }
+      if (P.head_bytes + in_group + b > ws_cap) {
+        P.groups.push_back(i);
+        in_group = 0;
+      }
+      in_group += b;
     }
   }
-  P.ws_bytes = off;
+  P.groups.push_back(count);
+  P.region_off.assign((size_t)count * 4, 0);
+  P.ws_bytes = P.head_bytes;
+  for (size_t g = 0; g + 1 < P.groups.size(); ++g) {
+    int64_t off = P.head_bytes;
+    for (int which = 0; which < 4; ++which)
+      for (int i = P.groups[g]; i < P.groups[g + 1]; ++i) {
+        P.region_off[(size_t)i * 4 + which] = off;
+        off += region_bytes(i, which);
+      }
+    P.ws_bytes = std::max(P.ws_bytes, off);
+  }
 
   std::vector<char> is_small((size_t)count, 0);
   if (small_path)

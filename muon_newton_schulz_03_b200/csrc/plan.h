@@ -35,6 +35,11 @@ struct HostPlan {
   std::vector<int> small;             // matrices on the on-chip small path
   int tile_m = kTileM;                // 128 (single CTA) or 256 (CTA pair)
   std::vector<long long> prefix;      // count + 1
+  // Matrix groups under a workspace cap: group g is matrices
+  // [groups[g], groups[g + 1]); every group's regions start after the
+  // sum-of-squares block, so groups share the workspace and run one after
+  // another. Without a cap (or when everything fits) there is one group.
+  std::vector<int> groups;
 };
 
 // Validates the shape table (m, n in [1, kMaxDim], flags in {0, 1}) and
@@ -42,7 +47,10 @@ struct HostPlan {
 // l <= kSmallMaxL go to the on-chip small path instead of the tile lists.
 // With pair_tiles the tiles are 256 x 256 (one per CTA pair), else
 // 128 x 256. Returns false with a message on invalid input.
+// With ws_cap > 0 and a workspace above it, consecutive matrices are packed
+// into groups whose workspace fits (each group as large as the cap allows,
+// in index order); a matrix that alone exceeds the cap is an error.
 bool build_plan(const int32_t* shapes, int count, int prec, bool small_path, bool pair_tiles, HostPlan& out,
-                std::string& why);
+                std::string& why, int64_t ws_cap = 0);
 
 }  // namespace muon

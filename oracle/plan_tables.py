@@ -20,6 +20,13 @@ The workspace begins with one float64 sum-of-squares accumulator per
 matrix, padded to 1024 bytes; then all X0 regions, all X1
 regions, all A regions, all B regions, each region aligned to 1024 bytes.
 
+Workspace cap. When that layout is larger than a cap, consecutive matrices
+are packed into groups in index order, each group as large as fits under
+the cap; every group lays out its own X0, X1, A and B regions (same order,
+same alignment) starting right after the sum-of-squares block, so the
+groups share one workspace and run one after another. A matrix whose
+regions alone exceed the cap is rejected.
+
 Tiles. Output tiles are BM rows by BN = 256 columns: BM = 128 on single
 CTAs, BM = 256 on CTA pairs.
   * Gram and polynomial (both symmetric s x s): tile (ti, tj) is listed iff
@@ -69,19 +76,39 @@ def matrix_geometry(m: int, n: int):
     return tall, s, l, round_up(n, 8), round_up(s, 8)
 
 
-def workspace_layout(shapes, elem_bytes: int = 2):
-    """Byte offsets (X0, X1, A, B) per matrix and the total workspace size."""
+def workspace_layout(shapes, elem_bytes: int = 2, cap: int = 0):
+    """Byte offsets (X0, X1, A, B) per matrix, the workspace size and the
+    group bounds (a list starting with 0 and ending with len(shapes))."""
     count = len(shapes)
     head = round_up(8 * count, ALIGN)
-    off = head
+
+    def region(i, which):
+        m, n = shapes[i]
+        _, s, _, ldx, lds = matrix_geometry(m, n)
+        return round_up((m * ldx if which < 2 else s * lds) * elem_bytes, ALIGN)
+
+    sizes = [sum(region(i, w) for w in range(4)) for i in range(count)]
+    bounds = [0]
+    if cap and head + sum(sizes) > cap:
+        used = 0
+        for i, b in enumerate(sizes):
+            if head + b > cap:
+                raise ValueError(f"matrix {i} alone needs {head + b} bytes, above the cap {cap}")
+            if head + used + b > cap:
+                bounds.append(i)
+                used = 0
+            used += b
+    bounds.append(count)
     regions = [[0, 0, 0, 0] for _ in range(count)]
-    for which in range(4):
-        for i, (m, n) in enumerate(shapes):
-            _, s, _, ldx, lds = matrix_geometry(m, n)
-            nbytes = (m * ldx if which < 2 else s * lds) * elem_bytes
-            regions[i][which] = off
-            off = round_up(off + nbytes, ALIGN)
-    return regions, off
+    total = head
+    for g0, g1 in zip(bounds[:-1], bounds[1:]):
+        off = head
+        for which in range(4):
+            for i in range(g0, g1):
+                regions[i][which] = off
+                off += region(i, which)
+        total = max(total, off)
+    return regions, total, bounds
 
 
 BM_PAIR = 256

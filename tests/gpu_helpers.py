@@ -47,10 +47,18 @@ def bf16_ns_tolerance(x, steps=5, coeffs=O.DEFAULT_COEFFS, normalised=True):
     return max(TOL_BF16_NS, bf16_program_error(x, steps, coeffs, normalised))
 
 
+def report(what, err, tol, program=None):
+    """One line per gated comparison (shown with pytest -s)."""
+    extra = "" if program is None else f" program={program:.3e}"
+    print(f"PARITY {what}: gpu={err:.3e} gate={tol:.3e}{extra}")
+
+
 def gate_bf16_ns(got, exact, x, steps=5, coeffs=O.DEFAULT_COEFFS, normalised=True, what=""):
     """Assert the bf16 gate on O; returns (error, tolerance)."""
-    tol = bf16_ns_tolerance(x, steps, coeffs, normalised)
+    prog = bf16_program_error(x, steps, coeffs, normalised)
+    tol = max(TOL_BF16_NS, prog)
     e = rel(got, exact)
+    report(f"O {what}", e, tol, prog)
     assert e <= tol, f"{what}: {e:.3e} from the exact oracle (gate {tol:.3e})"
     return e, tol
 
@@ -65,6 +73,7 @@ def gate_bf16_update(p_gpu, p0, p_exact, o_exact, lr_scale, tol_o, what=""):
     ndp = np.linalg.norm(dp_exact)
     tol = (tol_o * abs(lr_scale) * np.linalg.norm(o_exact) + 2.0 ** -23 * np.linalg.norm(p_exact)) / ndp
     e = rel(p_gpu - p0, dp_exact)
+    report(f"dp {what}", e, tol)
     assert e <= tol, f"{what}: update {e:.3e} from the exact oracle (gate {tol:.3e})"
     return e
 

@@ -61,7 +61,7 @@ SHAPE_SETS = {
 def test_plan_tables_bit_exact(name, prec, small_path, pair):
     shapes = SHAPE_SETS[name]
     got = muon.plan_query(shapes, prec, small_path, pair)
-    regions, ws = PT.workspace_layout(shapes, 2 if prec == "bf16" else 4)
+    regions, ws, _ = PT.workspace_layout(shapes, 2 if prec == "bf16" else 4)
     assert got["ws_bytes"] == ws
     assert got["region_offsets"] == regions
     gram, poly, comb, small = PT.tile_lists(shapes, small_path, pair)
@@ -183,3 +183,42 @@ def test_gram_form_needs_bf16_single_cta(other):
     h = ctypes.c_void_p()
     assert lib.muon_init(0, ctypes.byref(cfg), ctypes.byref(h)) == 1
     assert b"Gram" in lib.muon_last_error()
+
+
+@pytest.mark.parametrize("name", ["gpt2", "llama3", "moe", "ragged"])
+@pytest.mark.parametrize("frac", [1.0, 0.5, 0.23, 0.05])
+def test_capped_plan_groups_bit_exact(name, frac):
+    # Under a workspace cap the matrices are packed into consecutive groups
+    # that share one workspace; the C++ plan and the restatement agree.
+    shapes = SHAPE_SETS[name]
+    _, full, _ = PT.workspace_layout(shapes)
+    cap = int(full * frac)
+    try:
+        regions, ws, bounds = PT.workspace_layout(shapes, 2, cap)
+    except ValueError:
+        with pytest.raises(muon.MuonError) as e:
+            muon.plan_groups(shapes, cap)
+        assert e.value.code == 3
+        return
+    got = muon.plan_groups(shapes, cap)
+    assert got["bounds"] == bounds and got["region_offsets"] == regions and got["ws_bytes"] == ws
+    assert ws <= cap
+    if frac == 1.0:
+        assert bounds == [0, len(shapes)] and got["region_offsets"] == muon.plan_query(shapes)["region_offsets"]
+    # Regions of one group are aligned and disjoint.
+    for g0, g1 in zip(bounds[:-1], bounds[1:]):
+        spans = []
+        for i in range(g0, g1):
+            m, n = shapes[i]
+            s = min(m, n)
+            sizes = [m * muon.round_up(n, 8) * 2] * 2 + [s * muon.round_up(s, 8) * 2] * 2
+            spans += [(o, o + z) for o, z in zip(got["region_offsets"][i], sizes)]
+        spans.sort()
+        assert all(a1 <= b0 for (_, a1), (b0, _) in zip(spans, spans[1:]))
+        assert spans[-1][1] <= ws
+
+
+def test_capped_plan_rejects_a_matrix_above_the_cap():
+    with pytest.raises(muon.MuonError) as e:
+        muon.plan_groups([(4096, 4096), (64, 64)], 1 << 20)
+    assert e.value.code == 3 and "matrix 0" in str(e.value)

@@ -16,7 +16,7 @@ import workloads as W
 from oracle import muon_oracle as O
 
 from gpu_helpers import (DEV, TOL_BF16_NS, TOL_ELEM, TOL_FP32_NS, bf16_ns_tolerance, cuda_bf16, cuda_f32,
-                         gate_bf16_update, make_set, rel, to64, workspace_matrix, x_buffer)
+                         gate_bf16_update, make_set, rel, report, to64, workspace_matrix, x_buffer)
 
 pytestmark = pytest.mark.gpu
 
@@ -54,6 +54,7 @@ def _check_step(cpu, dev, shapes, opt, *, lr, beta, wd, nesterov=True, ns_steps=
             flips = (ns_steps + 1) // 2 if gram_mats else ns_steps
             o_gpu = to64(workspace_matrix(opt, shapes, i, flips % 2, dtype)[:, :n])
             eo = rel(o_gpu, o_ref)
+            report(f"O matrix {i} {m}x{n}", eo, tol_o)
             assert eo <= tol_o, f"matrix {i} {m}x{n}: O off by {eo:.3e} (gate {tol_o:.3e})"
             # p' itself at the elementwise gate, with the oracle fed the GPU's O.
             p_from_o = O.apply_update(p0, o_gpu, F32(lr), F32(wd), scale)
@@ -253,7 +254,7 @@ def test_bounded_wait_expiry_reports_timeout_and_recovers():
     opt = muon.Muon(device=0, wait_timeout_s=1e-9)
     opt.step([d[0].clone() for d in dev], [d[1] for d in dev], [d[2].clone() for d in dev], lr=2e-4)
     code, ew, nf = opt.status()
-    assert code == 4 and ew in (1, 2, 3, 4)
+    assert code == 4 and ew in (1, 2, 3, 4, 6)
     opt.close()
     ok = muon.Muon(device=0)
     ok.step([d[0] for d in dev], [d[1] for d in dev], [d[2] for d in dev], lr=2e-4)
@@ -502,3 +503,143 @@ def test_layerwise_single_rank_matches_oracle():
         opt.close()
     finally:
         dist.destroy_process_group()
+
+
+def _group_launches(plan, bounds, deterministic=True):
+    """Launches of a grouped step: per group K1 (+ fixed-order sum), the
+    small path if the group has small matrices, 15 phases if it has tiled
+    ones, and the apply kernel."""
+    small = set(plan["small"])
+    total = 0
+    for g0, g1 in zip(bounds[:-1], bounds[1:]):
+        mats = range(g0, g1)
+        total += 2 + (1 if deterministic else 0)
+        total += 1 if any(i in small for i in mats) else 0
+        total += 15 if any(i not in small for i in mats) else 0
+    return total
+
+
+def test_workspace_cap_runs_groups_and_matches_uncapped():
+    # A cap of a third of the workspace packs the matrices into groups that
+    # share one workspace and run one after another. In the fixed-order norm
+    # mode the result is bitwise the uncapped step's (every tile computes the
+    # same products), and it meets the oracle's gates; the stage call and
+    # the host-buffer step run the same groups.
+    shapes = W.PARITY_SHAPES["layerwise"]
+    full = muon.plan_query(shapes)["ws_bytes"]
+    cap = full // 3
+    bounds = muon.plan_groups(shapes, cap)["bounds"]
+    assert len(bounds) - 1 >= 3
+    cpu, dev = make_set(W.CONFIG_GPT2, shapes, torch.float32)
+    twin = [(p.clone(), g.clone(), m.clone()) for (p, g, m) in dev]
+    capped = muon.Muon(device=0, workspace_cap_bytes=cap, deterministic=True)
+    plain = muon.Muon(device=0, deterministic=True)
+    capped.step([d[0] for d in dev], [d[1] for d in dev], [d[2] for d in dev], lr=2e-4, beta=0.95, wd=0.1)
+    plain.step([t[0] for t in twin], [t[1] for t in twin], [t[2] for t in twin], lr=2e-4, beta=0.95, wd=0.1)
+    torch.cuda.synchronize()
+    assert capped.workspace()[1] <= cap
+    assert capped.last_launch_count() == _group_launches(muon.plan_query(shapes), bounds)
+    for (p, _, m), (p2, _, m2) in zip(dev, twin):
+        assert torch.equal(p, p2) and torch.equal(m, m2)
+    _check_step(cpu, dev, shapes, capped, lr=2e-4, beta=0.95, wd=0.1, check_o=False)
+    assert capped.status() == (0, 0, 0)
+    # The stage call under the cap.
+    xin = [x_buffer(m, n, fill=W.gaussian_set([(m, n)], 50 + i)[0]) for i, (m, n) in enumerate(shapes)]
+    sumsq = torch.tensor([float(torch.sum(x[:, :n].double() ** 2)) for x, (m, n) in zip(xin, shapes)],
+                         dtype=torch.float64, device=DEV)
+    outs = [[x_buffer(m, n) for (m, n) in shapes] for _ in range(2)]
+    capped.newton_schulz(xin, outs[0], shapes, sumsq, ns_steps=5)
+    plain.newton_schulz(xin, outs[1], shapes, sumsq, ns_steps=5)
+    torch.cuda.synchronize()
+    for a, b, (m, n) in zip(outs[0], outs[1], shapes):
+        assert torch.equal(a[:, :n], b[:, :n])
+    # The host-buffer step under the cap: the same groups, bitwise the device step.
+    hp = [t[0].cpu().pin_memory() for t in twin]
+    hg = [t[1].cpu().pin_memory() for t in twin]
+    hm = [t[2].cpu().pin_memory() for t in twin]
+    capped.step_host(hp, hg, hm, lr=2e-4)
+    capped.step([d[0] for d in dev], [d[1] for d in dev], [d[2] for d in dev], lr=2e-4)
+    torch.cuda.synchronize()
+    for a, d in zip(hp, dev):
+        assert torch.equal(a, d[0].cpu())
+    assert capped.status() == (0, 0, 0)
+    capped.close()
+    plain.close()
+    tight = muon.Muon(device=0, workspace_cap_bytes=1 << 20)
+    with pytest.raises(muon.MuonError) as e:    # a matrix above the cap on its own
+        tight.step([d[0] for d in dev], [d[1] for d in dev], [d[2] for d in dev], lr=2e-4)
+    assert e.value.code == 3
+    tight.close()
+
+
+def test_fresh_pointers_every_step_match_fixed_pointers():
+    # A training loop that hands over new gradient and momentum tensors each
+    # step (a fresh allocation per step): the pointer tables go through the
+    # handle's ring of device slots with stream-ordered uploads, more steps
+    # than slots. The parameters and momenta match the fixed-pointer run
+    # bitwise (fixed-order norm), and the step time stays close to it.
+    shapes = W.gpt2_shapes()[:8] + [(64, 64), (300, 700)]
+    steps = 20
+    grads = [[cuda_f32(W.gradient_cpu(W.CONFIG_GPT2, m, n, 900 + 31 * k + i)) for i, (m, n) in enumerate(shapes)]
+             for k in range(4)]
+    p0 = [cuda_f32(W.param_cpu(m, n, i)) for i, (m, n) in enumerate(shapes)]
+    opt = muon.Muon(device=0, deterministic=True)
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+
+    def run(fresh):
+        p = [t.clone() for t in p0]
+        mo = [torch.zeros_like(t) for t in p0]
+        g = [torch.empty_like(t) for t in p0]
+        total = 0.0
+        for k in range(steps):
+            if fresh:
+                g = [t.clone() for t in grads[k % 4]]
+                mo = [t.clone() for t in mo]
+            else:
+                for dst, src in zip(g, grads[k % 4]):
+                    dst.copy_(src)
+            ev[0].record()
+            opt.step(p, g, mo, lr=2e-4)
+            ev[1].record()
+            torch.cuda.synchronize()
+            if k >= 2:
+                total += ev[0].elapsed_time(ev[1])
+        return p, mo, total
+
+    p_fix, m_fix, t_fix = run(False)
+    p_new, m_new, t_new = run(True)
+    for a, b in zip(p_fix, p_new):
+        assert torch.equal(a, b)
+    for a, b in zip(m_fix, m_new):
+        assert torch.equal(a, b)
+    assert opt.status() == (0, 0, 0)
+    print(f"fixed pointers {t_fix / (steps - 2):.3f} ms/step, fresh pointers {t_new / (steps - 2):.3f} ms/step")
+    assert t_new <= 1.25 * t_fix + 0.05 * (steps - 2)
+    opt.close()
+
+
+def test_steps_over_a_subset_launch_only_its_tiles():
+    # Matrices without a gradient drop out of the tile lists: a step over a
+    # subset (one round of layer-wise Muon) launches over the active
+    # matrices' tiles only, and matches the oracle on them while the others
+    # stay untouched.
+    shapes = W.PARITY_SHAPES["layerwise"]
+    cpu, dev = make_set(W.CONFIG_GPT2, shapes, torch.float32)
+    before = [(d[0].clone(), d[2].clone()) for d in dev]
+    opt = muon.Muon(device=0)
+    opt.profile_enable(1)
+    active = {1, 4}                 # two tiled matrices
+    g = [d[1] if i in active else None for i, d in enumerate(dev)]
+    opt.step([d[0] for d in dev], g, [d[2] for d in dev], lr=2e-4)
+    torch.cuda.synchronize()
+    prof = opt.profile_read()
+    opt.profile_enable(0)
+    kinds = [k for k, _ in prof]
+    assert kinds.count("ns_gram") == kinds.count("ns_poly") == kinds.count("ns_comb") == 5
+    assert "ns_small" not in kinds          # the small matrix (64 x 64) has no gradient
+    for i, d in enumerate(dev):
+        if i not in active:
+            assert torch.equal(d[0], before[i][0]) and torch.equal(d[2], before[i][1])
+    _check_step(cpu, dev, shapes, opt, lr=2e-4, beta=0.95, wd=0.1, indices=sorted(active))
+    assert opt.status() == (0, 0, 0)
+    opt.close()
