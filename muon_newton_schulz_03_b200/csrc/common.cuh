@@ -69,11 +69,6 @@ struct DevStatus {
   int error_word;                   // first expired wait's code, 0 = none
   int pad_;
   unsigned long long nonfinite;     // non-finite u entries seen
-  // Dynamic tile scheduler of the Newton-Schulz phase kernel: the next tile
-  // to hand out and the number of CTAs that have finished; the last CTA of a
-  // launch resets both to zero, so every launch starts from zero.
-  unsigned int sched_next;
-  unsigned int sched_done;
 };
 
 // Codes written to the error word.
@@ -83,8 +78,7 @@ enum WaitCode : int {
   WAIT_TMA_FULL = 2,      // MMA issuer waiting for loaded operands
   WAIT_ACC_EMPTY = 3,     // MMA issuer waiting for a drained accumulator
   WAIT_ACC_FULL = 4,      // epilogue waiting for a finished accumulator
-  WAIT_DRAIN = 5,         // clean-up wait after an abort
-  WAIT_TILE_QUEUE = 6     // a role waiting for the next tile index (or a free queue slot)
+  WAIT_DRAIN = 5          // clean-up wait after an abort
 };
 
 constexpr int kElemChunk = 8192;  // elements per block in the elementwise kernels

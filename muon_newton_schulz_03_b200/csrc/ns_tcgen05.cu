@@ -44,6 +44,7 @@ constexpr int kThreads = 192;
 constexpr int kTmemCols = 2 * BN;               // two fp32 accumulators
 constexpr int kOutBox = 32;                     // bulk-store box: 32 rows x 32 columns
 constexpr int kOutStageBytes = kOutBox * kOutBox * 2;
+constexpr int kAuxTmaMinK = 2048;               // combine tiles with K >= this read X by bulk loads
 
 struct __align__(1024) SmemLayout {
   uint8_t stage[kStages][kStageBytes];
@@ -55,6 +56,7 @@ struct __align__(1024) SmemLayout {
   uint64_t acc_full[2];
   uint64_t acc_empty[2];
   uint64_t drain;
+  uint64_t aux_full[4][2];   // per epilogue warp: bulk loads of the combine's X blocks
   uint32_t tmem_base;
 };
 
@@ -230,6 +232,8 @@ __global__ void __launch_bounds__(kThreads, 1) ns_phase_kernel(const __grid_cons
       mbar_init(&sm.acc_empty[b], 4);
     }
     mbar_init(&sm.drain, 1);
+    for (int w = 0; w < 4; ++w)
+      for (int b = 0; b < 2; ++b) mbar_init(&sm.aux_full[w][b], 1);
     fence_barrier_init();
   }
   if (warp == 1) {
@@ -343,6 +347,16 @@ __global__ void __launch_bounds__(kThreads, 1) ns_phase_kernel(const __grid_cons
     uint32_t acc_phase = 0;
     int obuf = 0;   // staging block pair used by this warp's next chunk
     const bool tma_out = L.tma_store != 0 && !(args.phase == PHASE_COMB && args.dst_sel == BUF_OUT);
+    // The combine's auxiliary X comes through bulk-tensor loads of 32 x 32
+    // blocks into this warp's two transposed-staging buffers (the combine
+    // never writes transposed blocks) when X is a workspace buffer with a
+    // 32 x 32 map and the tile's main loop is long (K = s >= kAuxTmaMinK); a
+    // per-lane row load touches 32 cache lines per instruction, but on short
+    // tiles the bulk loads wait behind the producer's operand loads in the
+    // same copy engine and the epilogue, then on the critical path, slows.
+    const bool aux_tma_phase = L.tma_store != 0 && args.phase == PHASE_COMB && args.src_sel != BUF_IN;
+    uint32_t aux_parity = 0;    // bit b: parity of the next wait on aux_full[quarter][b]
+    uint32_t aux_pending = 0;   // bit b: a load into buffer b has not been waited for
     for (int t = blockIdx.x; t < L.ntiles; t += gridDim.x) {
       const int4 tile = L.tiles[t];
       const MatBind mb = L.binds[tile.x];
@@ -392,21 +406,54 @@ __global__ void __launch_bounds__(kThreads, 1) ns_phase_kernel(const __grid_cons
       const float ca = args.a, cb = args.b, cc = args.c;
       const __nv_bfloat16* aux_row = aux != nullptr ? aux + (size_t)row * aux_ld : nullptr;
       uint4 xa[4], xb[4];   // packed bf16 auxiliary values of the current and the next chunk
-      if (aux_row != nullptr) load_aux_chunk(aux_row, tj * BN, cols, row_ok, xa);
+      const bool aux_tma = aux_tma_phase && mp.s >= kAuxTmaMinK;
+      const TmapBlob* aux_map =
+          aux_tma ? L.maps + (size_t)tile.x * kMapsPerMat + (args.src_sel == BUF_X0 ? MAP_X0_ST : MAP_X1_ST) : nullptr;
+      // Bulk load of the auxiliary block of chunk `c` into buffer c & 1
+      // (issued by lane 0 after every lane has finished reading that buffer).
+      auto aux_issue = [&](int c) {
+        const int b = c & 1;
+        __syncwarp();   // every lane has read the buffer's previous block
+        if (lane == 0) {
+          fence_proxy_async_smem();
+          mbar_arrive_expect_tx(&sm.aux_full[quarter][b], kOutStageBytes);
+          tma_load_2d(sm.ostage[quarter][2 + b], aux_map, &sm.aux_full[quarter][b], tj * BN + c * 32, warp_row0);
+        }
+        aux_pending |= 1u << b;
+      };
+      if (aux_tma) {
+        aux_issue(0);
+      } else if (aux_row != nullptr) {
+        load_aux_chunk(aux_row, tj * BN, cols, row_ok, xa);
+      }
 
       if (!mbar_wait_bounded(&sm.acc_full[acc], acc_phase, err, tmo, WAIT_ACC_FULL)) break;
       tc_fence_after();
 
       // One 32-column chunk: returns false past the last column.
-      auto chunk = [&](int ch, const uint4 (&cur)[4], uint4 (&nxt)[4]) -> bool {
+      auto chunk = [&](int ch, uint4 (&cur)[4], uint4 (&nxt)[4]) -> bool {
         const int col0 = tj * BN + ch * 32;
         if (col0 >= cols) return false;                // warp-uniform
-        if (aux_row != nullptr && ch + 1 < BN / 32 && col0 + 32 < cols)
+        if (aux_tma) {
+          if (ch + 1 < BN / 32 && col0 + 32 < cols) aux_issue(ch + 1);
+        } else if (aux_row != nullptr && ch + 1 < BN / 32 && col0 + 32 < cols) {
           load_aux_chunk(aux_row, col0 + 32, cols, row_ok, nxt);
+        }
         float v[32];
         tmem_ld_32x32b_x32(t_base + (uint32_t)(ch * 32), v);
         const bool full_chunk = col0 + 32 <= cols;
         float o[32];
+        if (aux_tma) {
+          // This lane's row of the block, from the swizzled shared copy.
+          const int b = ch & 1;
+          if (!mbar_wait_bounded(&sm.aux_full[quarter][b], (aux_parity >> b) & 1u, err, tmo, WAIT_ACC_FULL))
+            return false;
+          aux_parity ^= 1u << b;
+          aux_pending &= ~(1u << b);
+          const uint8_t* ab = sm.ostage[quarter][2 + b];
+#pragma unroll
+          for (int q = 0; q < 4; ++q) cur[q] = *reinterpret_cast<const uint4*>(ab + sw64_offset(lane, q));
+        }
         if (aux_row == nullptr) {
 #pragma unroll
           for (int i = 0; i < 32; ++i) o[i] = v[i] * sc;
@@ -505,8 +552,12 @@ __global__ void __launch_bounds__(kThreads, 1) ns_phase_kernel(const __grid_cons
       if (lane == 0) mbar_arrive(&sm.acc_empty[acc]);
       if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
     }
-    // Bulk stores read this CTA's shared memory: let them finish.
+    // Bulk stores read this CTA's shared memory: let them finish; loads that
+    // were issued but not waited for (after an abort) must land too.
     if (tma_out && lane == 0) bulk_wait_group_all();
+    if (lane == 0)
+      for (int b = 0; b < 2; ++b)
+        if (aux_pending & (1u << b)) mbar_wait_drain(&sm.aux_full[quarter][b], (aux_parity >> b) & 1u, drain_tmo);
   }
 
   tc_fence_before();

@@ -294,7 +294,7 @@ def test_ns_only_sweep_inputs(opt_bf16, point):
     torch.cuda.synchronize()
     for b in range(batch):
         ref = O.ns_only(x64[b], 5)
-        gate_bf16_ns(to64(xout[b][:, :n]), ref, x64[b], 5, normalised=False, what=f"{m}x{n} #{b}")
+        gate_bf16_ns(to64(xout[b][:, :n]), ref, x64[b], 5, normalised=False, what=f"config sweep {m}x{n} #{b}")
     _assert_status_clean(opt_bf16)
 
 
