@@ -50,7 +50,9 @@ struct GramBufs {
 };
 // T (K-major 128- and 256-row boxes), B1 (same), then the 32 x 32 store
 // boxes of T and B1.
-constexpr int kGramMapsPerMat = 6;
+// Gram-form maps per matrix: T K128, T K256, B1 K128, B1 K256, T store,
+// B1 store, T 64 x 64 (M/N-major loads), B1 64 x 64.
+constexpr int kGramMapsPerMat = 8;
 
 // Operands and epilogue of one launch beyond the phase itself.
 struct PhaseSpec {
@@ -78,7 +80,11 @@ enum MapIdx : int {
   MAP_B_K128 = 8, MAP_B_K256 = 9,
   // 32 x 32 boxes with 64-byte swizzle for the epilogue's bulk stores
   MAP_X0_ST = 10, MAP_X1_ST = 11, MAP_A_ST = 12, MAP_B_ST = 13,
-  kMapsPerMat = 14,
+  // 64 x 64 boxes of A and B for M/N-major loads: the single-CTA kernel
+  // writes only the upper 256-block triangle of a symmetric buffer and reads
+  // the blocks below it transposed from there
+  MAP_A_MN = 14, MAP_B_MN = 15,
+  kMapsPerMat = 16,
   kInMapsPerMat = 3
 };
 

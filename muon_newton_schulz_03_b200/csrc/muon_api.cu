@@ -413,7 +413,9 @@ int ensure_gram_buffers(DevPlan& P) {
         (rc = encode_map(m + 2, gb[i].b1, mp.s, mp.s, mp.lds, 64, 128)) ||
         (rc = encode_map(m + 3, gb[i].b1, mp.s, mp.s, mp.lds, 64, 256)) ||
         (rc = encode_store_map(m + 4, gb[i].t, mp.s, mp.s, mp.lds)) ||
-        (rc = encode_store_map(m + 5, gb[i].b1, mp.s, mp.s, mp.lds)))
+        (rc = encode_store_map(m + 5, gb[i].b1, mp.s, mp.s, mp.lds)) ||
+        (rc = encode_map(m + 6, gb[i].t, mp.s, mp.s, mp.lds, 64, 64)) ||
+        (rc = encode_map(m + 7, gb[i].b1, mp.s, mp.s, mp.lds, 64, 64)))
       return rc;
   }
   void* d = nullptr;
@@ -596,6 +598,8 @@ int ensure_plan(muon_handle* h, const int32_t* shapes, int count) {
       if ((rc = encode_map(mm + MAP_A_K256, mp.a, mp.s, mp.s, mp.lds, 64, 256))) { free_plan(np.get()); return rc; }
       if ((rc = encode_map(mm + MAP_B_K128, mp.b, mp.s, mp.s, mp.lds, 64, 128))) { free_plan(np.get()); return rc; }
       if ((rc = encode_map(mm + MAP_B_K256, mp.b, mp.s, mp.s, mp.lds, 64, 256))) { free_plan(np.get()); return rc; }
+      if ((rc = encode_map(mm + MAP_A_MN, mp.a, mp.s, mp.s, mp.lds, 64, 64))) { free_plan(np.get()); return rc; }
+      if ((rc = encode_map(mm + MAP_B_MN, mp.b, mp.s, mp.s, mp.lds, 64, 64))) { free_plan(np.get()); return rc; }
       if ((rc = encode_store_map(mm + MAP_X0_ST, mp.x0, mp.m, mp.n, mp.ldx)) ||
           (rc = encode_store_map(mm + MAP_X1_ST, mp.x1, mp.m, mp.n, mp.ldx)) ||
           (rc = encode_store_map(mm + MAP_A_ST, mp.a, mp.s, mp.s, mp.lds)) ||

@@ -240,7 +240,9 @@ extern "C" int muon_newton_schulz_noalloc(const void* const* x_in, void* const* 
         (rc = encode(mm + MAP_A_K128, mp.a, mp.s, mp.s, mp.lds, 64, 128)) ||
         (rc = encode(mm + MAP_A_K256, mp.a, mp.s, mp.s, mp.lds, 64, 256)) ||
         (rc = encode(mm + MAP_B_K128, mp.b, mp.s, mp.s, mp.lds, 64, 128)) ||
-        (rc = encode(mm + MAP_B_K256, mp.b, mp.s, mp.s, mp.lds, 64, 256)) || (rc = encode_x(im, x_in[i], mp)))
+        (rc = encode(mm + MAP_B_K256, mp.b, mp.s, mp.s, mp.lds, 64, 256)) ||
+        (rc = encode(mm + MAP_A_MN, mp.a, mp.s, mp.s, mp.lds, 64, 64)) ||
+        (rc = encode(mm + MAP_B_MN, mp.b, mp.s, mp.s, mp.lds, 64, 64)) || (rc = encode_x(im, x_in[i], mp)))
       return rc;
   }
   std::memcpy(host.data() + o_pref, hp.prefix.data(), sizeof(long long) * (count + 1));

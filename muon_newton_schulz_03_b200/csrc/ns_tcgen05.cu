@@ -8,10 +8,14 @@
 //   COMB : X' = a X + B X       (wide)               or  a X + X B  (tall;
 //                                                         B is symmetric)
 // Gram and polynomial outputs are symmetric: only tiles on or right of the
-// 256-block diagonal are computed; off-diagonal tiles are written twice,
-// directly and transposed. Tall matrices (m > n) are never transposed in
-// memory: the Gram reads X with M/N-major operand tiles, and the combine
-// computes X B instead of B X^T.
+// 256-block diagonal are computed and stored, so a symmetric buffer holds its
+// upper 256-block triangle (diagonal blocks whole). Its lower part is the
+// mirror image of the upper, taken at load time: a consumer that needs a
+// K-block below the diagonal block of its operand rows loads it transposed
+// (M/N-major boxes) from the stored block above the diagonal, and the MMA
+// takes that K-block with M/N-major operand layout. Tall matrices (m > n) are
+// never transposed in memory: the Gram reads X with M/N-major operand tiles,
+// and the combine computes X B instead of B X^T.
 // The Frobenius normalisation X0 = Y/(||u|| + eps) of the first step is
 // folded into its epilogues: A0 = alpha^2 Y Y^T and X1 = alpha (a Y + B0 Y).
 //
@@ -48,8 +52,9 @@ constexpr int kAuxTmaMinK = 2048;               // combine tiles with K >= this 
 
 struct __align__(1024) SmemLayout {
   uint8_t stage[kStages][kStageBytes];
-  // Epilogue staging for bulk stores: per epilogue warp two direct and two
-  // transposed 32 x 32 bf16 blocks (64-byte rows, 64-byte swizzle).
+  // Epilogue staging: per epilogue warp two 32 x 32 bf16 output blocks for
+  // bulk stores and two for bulk loads of the auxiliary operand (64-byte
+  // rows, 64-byte swizzle).
   uint8_t ostage[4][4][kOutStageBytes];
   uint64_t full[kStages];
   uint64_t empty[kStages];
@@ -75,7 +80,17 @@ struct TileJob {
   const void* map_b;
   int a_mn, b_mn;      // operand majorness: 0 = K-major, 1 = M/N-major
   int a_coord, b_coord;  // K-major: first row; M/N-major: first M/N index
+  // Operand rows from a symmetric buffer (upper 256-block triangle stored):
+  // K-blocks left of the rows' diagonal block come transposed through the
+  // 64 x 64 map.
+  int a_sym, b_sym;
+  const void* map_a_mn;
+  const void* map_b_mn;
 };
+
+// K-block kb of operand rows starting at r0 of a symmetric buffer is below
+// the stored triangle (its 256-column block lies left of the rows' 256-block).
+__device__ __forceinline__ bool below_stored(int r0, int kb) { return (kb * BK) / 256 < r0 / 256; }
 
 __device__ __forceinline__ const TmapBlob* src_maps(const NsLaunch& L, int mat, int src_sel) {
   if (src_sel == BUF_IN) return L.in_maps + (size_t)mat * kInMapsPerMat;
@@ -87,6 +102,13 @@ __device__ __forceinline__ const TmapBlob* sym_map(const NsLaunch& L, int mat, i
   if (id == SB_A) return L.maps + (size_t)mat * kMapsPerMat + (rows256 ? MAP_A_K256 : MAP_A_K128);
   if (id == SB_B) return L.maps + (size_t)mat * kMapsPerMat + (rows256 ? MAP_B_K256 : MAP_B_K128);
   return L.gmaps + (size_t)mat * kGramMapsPerMat + (id == SB_T ? 0 : 2) + (rows256 ? 1 : 0);
+}
+
+// 64 x 64 map of an s x s buffer (transposed loads of the missing triangle).
+__device__ __forceinline__ const TmapBlob* sym_map_mn(const NsLaunch& L, int mat, int id) {
+  if (id == SB_A) return L.maps + (size_t)mat * kMapsPerMat + MAP_A_MN;
+  if (id == SB_B) return L.maps + (size_t)mat * kMapsPerMat + MAP_B_MN;
+  return L.gmaps + (size_t)mat * kGramMapsPerMat + (id == SB_T ? 6 : 7);
 }
 
 __device__ __forceinline__ __nv_bfloat16* sym_ptr(const NsLaunch& L, const MatPlan& mp, int mat, int id) {
@@ -116,6 +138,8 @@ __device__ __forceinline__ TileJob decode(const NsArgs& A, const int4 t, const M
   j.mat = t.x;
   j.ti = t.y;
   j.tj = t.z;
+  j.a_sym = j.b_sym = 0;
+  j.map_a_mn = j.map_b_mn = nullptr;
   const TmapBlob* own = A.L.maps + (size_t)j.mat * kMapsPerMat;
   if (A.phase == PHASE_GRAM) {
     const TmapBlob* xs = src_maps(A.L, j.mat, A.src_sel);
@@ -131,19 +155,28 @@ __device__ __forceinline__ TileJob decode(const NsArgs& A, const int4 t, const M
     j.kblocks = (mp.s + BK - 1) / BK;
     j.map_a = own + MAP_A_K128; j.a_mn = 0; j.a_coord = j.ti * BM;
     j.map_b = own + MAP_A_K256; j.b_mn = 0; j.b_coord = j.tj * BN;
+    j.a_sym = j.b_sym = 1;
+    j.map_a_mn = j.map_b_mn = own + MAP_A_MN;
   } else if (A.phase == PHASE_SYM) {   // (L R)[i][j] = sum_k L[i][k] R[j][k], R symmetric
     j.kblocks = (mp.s + BK - 1) / BK;
     j.map_a = sym_map(A.L, j.mat, A.spec.sym_l, false); j.a_mn = 0; j.a_coord = j.ti * BM;
     j.map_b = sym_map(A.L, j.mat, A.spec.sym_r, true);  j.b_mn = 0; j.b_coord = j.tj * BN;
+    j.a_sym = j.b_sym = 1;
+    j.map_a_mn = sym_map_mn(A.L, j.mat, A.spec.sym_l);
+    j.map_b_mn = sym_map_mn(A.L, j.mat, A.spec.sym_r);
   } else {
     const TmapBlob* xs = src_maps(A.L, j.mat, A.src_sel);
     j.kblocks = (mp.s + BK - 1) / BK;
     if (!mp.tall) {  // (B X)[r][c] = sum_k B[r][k] X[k][c]
       j.map_a = sym_map(A.L, j.mat, A.spec.comb_b, false); j.a_mn = 0; j.a_coord = j.ti * BM;
       j.map_b = xs + MAP_MN;      j.b_mn = 1; j.b_coord = j.tj * BN;
+      j.a_sym = 1;
+      j.map_a_mn = sym_map_mn(A.L, j.mat, A.spec.comb_b);
     } else {         // (X B)[r][c] = sum_k X[r][k] B[c][k]
       j.map_a = xs + MAP_K128;    j.a_mn = 0; j.a_coord = j.ti * BM;
       j.map_b = sym_map(A.L, j.mat, A.spec.comb_b, true); j.b_mn = 0; j.b_coord = j.tj * BN;
+      j.b_sym = 1;
+      j.map_b_mn = sym_map_mn(A.L, j.mat, A.spec.comb_b);
     }
   }
   return j;
@@ -266,19 +299,23 @@ __global__ void __launch_bounds__(kThreads, 1) ns_phase_kernel(const __grid_cons
           uint8_t* sa = sm.stage[stage];
           uint8_t* sb = sa + kABytes;
           const int k0 = kb * BK;
-          if (!j.a_mn) {
+          const bool ta = j.a_sym && below_stored(j.a_coord, kb);   // mirrored K-block
+          const bool tb = j.b_sym && below_stored(j.b_coord, kb);
+          if (!j.a_mn && !ta) {
             tma_load_2d(sa, j.map_a, &sm.full[stage], k0, j.a_coord);
           } else {
+            const void* ma = ta ? j.map_a_mn : j.map_a;
 #pragma unroll
             for (int c = 0; c < BM / 64; ++c)
-              tma_load_2d(sa + c * kMnChunkBytes, j.map_a, &sm.full[stage], j.a_coord + 64 * c, k0);
+              tma_load_2d(sa + c * kMnChunkBytes, ma, &sm.full[stage], j.a_coord + 64 * c, k0);
           }
-          if (!j.b_mn) {
+          if (!j.b_mn && !tb) {
             tma_load_2d(sb, j.map_b, &sm.full[stage], k0, j.b_coord);
           } else {
+            const void* mb = tb ? j.map_b_mn : j.map_b;
 #pragma unroll
             for (int c = 0; c < BN / 64; ++c)
-              tma_load_2d(sb + c * kMnChunkBytes, j.map_b, &sm.full[stage], j.b_coord + 64 * c, k0);
+              tma_load_2d(sb + c * kMnChunkBytes, mb, &sm.full[stage], j.b_coord + 64 * c, k0);
           }
           armed |= 1u << stage;
           last_parity = (last_parity & ~(1u << stage)) | (phase << stage);
@@ -310,18 +347,22 @@ __global__ void __launch_bounds__(kThreads, 1) ns_phase_kernel(const __grid_cons
         if (!mbar_wait_bounded(&sm.acc_empty[acc], acc_phase ^ 1u, err, tmo, WAIT_ACC_EMPTY)) { ok = false; break; }
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BN);
-        const uint32_t idesc = umma_idesc_bf16(BM, BN, j.a_mn, j.b_mn);
         for (int kb = 0; kb < j.kblocks; ++kb) {
           if (!mbar_wait_bounded(&sm.full[stage], phase, err, tmo, WAIT_TMA_FULL)) { ok = false; break; }
           tc_fence_after();
+          // Majorness of this K-block's operands (mirrored K-blocks of a
+          // symmetric buffer arrive M/N-major, as the producer loaded them).
+          const int amn = j.a_mn | (j.a_sym && below_stored(j.a_coord, kb) ? 1 : 0);
+          const int bmn = j.b_mn | (j.b_sym && below_stored(j.b_coord, kb) ? 1 : 0);
+          const uint32_t idesc = umma_idesc_bf16(BM, BN, amn, bmn);
           const uint32_t sa = smem_u32(sm.stage[stage]);
           const uint32_t sb = sa + kABytes;
 #pragma unroll
           for (int k16 = 0; k16 < BK / 16; ++k16) {
-            const uint64_t da = j.a_mn ? umma_desc_sw128(sa + k16 * 2048, kMnChunkBytes, 1024)
-                                       : umma_desc_sw128(sa + k16 * 32, 16, 1024);
-            const uint64_t db = j.b_mn ? umma_desc_sw128(sb + k16 * 2048, kMnChunkBytes, 1024)
-                                       : umma_desc_sw128(sb + k16 * 32, 16, 1024);
+            const uint64_t da = amn ? umma_desc_sw128(sa + k16 * 2048, kMnChunkBytes, 1024)
+                                    : umma_desc_sw128(sa + k16 * 32, 16, 1024);
+            const uint64_t db = bmn ? umma_desc_sw128(sb + k16 * 2048, kMnChunkBytes, 1024)
+                                    : umma_desc_sw128(sb + k16 * 32, 16, 1024);
             tc_mma_bf16(d_tmem, da, db, idesc, (kb | k16) != 0);
           }
           issued = true;
@@ -347,14 +388,15 @@ __global__ void __launch_bounds__(kThreads, 1) ns_phase_kernel(const __grid_cons
     uint32_t acc_phase = 0;
     int obuf = 0;   // staging block pair used by this warp's next chunk
     const bool tma_out = L.tma_store != 0 && !(args.phase == PHASE_COMB && args.dst_sel == BUF_OUT);
-    // The combine's auxiliary X comes through bulk-tensor loads of 32 x 32
-    // blocks into this warp's two transposed-staging buffers (the combine
-    // never writes transposed blocks) when X is a workspace buffer with a
-    // 32 x 32 map and the tile's main loop is long (K = s >= kAuxTmaMinK); a
-    // per-lane row load touches 32 cache lines per instruction, but on short
-    // tiles the bulk loads wait behind the producer's operand loads in the
-    // same copy engine and the epilogue, then on the critical path, slows.
-    const bool aux_tma_phase = L.tma_store != 0 && args.phase == PHASE_COMB && args.src_sel != BUF_IN;
+    // The auxiliary operand of the polynomial (A) and of the combine (X)
+    // comes through bulk-tensor loads of 32 x 32 blocks into this warp's two
+    // auxiliary buffers when it is a workspace buffer with a 32 x 32 map and
+    // the tile's main loop is long (K = s >= kAuxTmaMinK); a per-lane row
+    // load touches 32 cache lines per instruction, but on short tiles the
+    // bulk loads wait behind the producer's operand loads in the same copy
+    // engine and the epilogue, then on the critical path, slows.
+    const bool aux_tma_phase = L.tma_store != 0 &&
+                               (args.phase == PHASE_POLY || (args.phase == PHASE_COMB && args.src_sel != BUF_IN));
     uint32_t aux_parity = 0;    // bit b: parity of the next wait on aux_full[quarter][b]
     uint32_t aux_pending = 0;   // bit b: a load into buffer b has not been waited for
     for (int t = blockIdx.x; t < L.ntiles; t += gridDim.x) {
@@ -390,7 +432,8 @@ __global__ void __launch_bounds__(kThreads, 1) ns_phase_kernel(const __grid_cons
         aux = static_cast<const __nv_bfloat16*>(sel_buf(mp, mb, args.src_sel)); aux_ld = mp.ldx;
         if (args.first) sc = (float)inv_norm(L.sumsq, tile.x);
       }
-      const bool mirror = (phase != PHASE_COMB) && (tj > (ti >> 1));
+      // Symmetric outputs are stored as computed (upper 256-block triangle);
+      // their consumers read the blocks below it transposed.
       const TmapBlob* st_map = nullptr;
       if (tma_out) {
         if (phase == PHASE_GRAM) st_map = sym_store_map(L, tile.x, SB_A);
@@ -408,7 +451,9 @@ __global__ void __launch_bounds__(kThreads, 1) ns_phase_kernel(const __grid_cons
       uint4 xa[4], xb[4];   // packed bf16 auxiliary values of the current and the next chunk
       const bool aux_tma = aux_tma_phase && mp.s >= kAuxTmaMinK;
       const TmapBlob* aux_map =
-          aux_tma ? L.maps + (size_t)tile.x * kMapsPerMat + (args.src_sel == BUF_X0 ? MAP_X0_ST : MAP_X1_ST) : nullptr;
+          !aux_tma ? nullptr
+          : L.maps + (size_t)tile.x * kMapsPerMat +
+                (phase == PHASE_POLY ? MAP_A_ST : (args.src_sel == BUF_X0 ? MAP_X0_ST : MAP_X1_ST));
       // Bulk load of the auxiliary block of chunk `c` into buffer c & 1
       // (issued by lane 0 after every lane has finished reading that buffer).
       auto aux_issue = [&](int c) {
@@ -486,12 +531,10 @@ __global__ void __launch_bounds__(kThreads, 1) ns_phase_kernel(const __grid_cons
           }
         }
         if (tma_out) {
-          // Stage the 32 x 32 block (and its transpose) in shared memory and
-          // write it with bulk stores; the tensor map clips rows and columns
-          // beyond the matrix.
+          // Stage the 32 x 32 block in shared memory and write it with a bulk
+          // store; the tensor map clips rows and columns beyond the matrix.
           uint8_t* dbuf = sm.ostage[quarter][obuf];
-          uint8_t* mbuf = sm.ostage[quarter][2 + obuf];
-          if (lane == 0) bulk_wait_group_read<1>();   // the pair used two chunks ago is free
+          if (lane == 0) bulk_wait_group_read<1>();   // the block used two chunks ago is free
           __syncwarp();
 #pragma unroll
           for (int q = 0; q < 4; ++q) {
@@ -501,22 +544,10 @@ __global__ void __launch_bounds__(kThreads, 1) ns_phase_kernel(const __grid_cons
             for (int i = 0; i < 4; ++i) h[i] = __floats2bfloat162_rn(o[8 * q + 2 * i], o[8 * q + 2 * i + 1]);
             *reinterpret_cast<uint4*>(dbuf + sw64_offset(lane, q)) = raw;
           }
-          if (mirror) {
-            // Element (j, lane) of the transposed block: for a fixed j the
-            // warp writes one 64-byte row.
-            const uint32_t in_group = (uint32_t)(lane & 7) * 2;
-#pragma unroll
-            for (int j = 0; j < 32; ++j)
-              *reinterpret_cast<__nv_bfloat16*>(mbuf + sw64_offset(j, lane >> 3) + in_group) =
-                  __float2bfloat16_rn(o[j]);
-          }
           fence_proxy_async_smem();
           __syncwarp();
           if (lane == 0) {
-            if (warp_row0 < rows) {
-              tma_store_2d(st_map, dbuf, col0, warp_row0);
-              if (mirror) tma_store_2d(st_map, mbuf, warp_row0, col0);
-            }
+            if (warp_row0 < rows) tma_store_2d(st_map, dbuf, col0, warp_row0);
             bulk_commit_group();
           }
           obuf ^= 1;
@@ -531,13 +562,6 @@ __global__ void __launch_bounds__(kThreads, 1) ns_phase_kernel(const __grid_cons
             for (int i = 0; i < 32; ++i)
               if (col0 + i < cols) dst[i] = __float2bfloat16_rn(o[i]);
           }
-        }
-        if (mirror && row_ok) {
-          // Transposed copy: for a fixed column the 32 lanes write 32
-          // consecutive elements of one output row.
-#pragma unroll
-          for (int i = 0; i < 32; ++i)
-            if (col0 + i < cols) out[(size_t)(col0 + i) * ld + row] = __float2bfloat16_rn(o[i]);
         }
         return true;
       };

@@ -31,9 +31,10 @@ Tiles. Output tiles are BM rows by BN = 256 columns: BM = 128 on single
 CTAs, BM = 256 on CTA pairs.
   * Gram and polynomial (both symmetric s x s): tile (ti, tj) is listed iff
     tj >= ti * BM // 256, i.e. its 256-wide column block is on or right of
-    the 256-block diagonal. Tiles whose column block starts at or after the
-    end of their row block are also written transposed, so each entry is
-    produced once.
+    the 256-block diagonal. The entries of tiles whose column block starts
+    at or after the end of their row block also stand for their mirror
+    image (written transposed, or read transposed by the consumers), so each
+    entry of the symmetric matrix is produced once.
   * Combine (output in the original m x n layout): every tile of the
     ceil(m/BM) x ceil(n/256) grid. For wide matrices (m <= n) the column
     block is the outer loop, for tall ones the row block.
@@ -123,7 +124,7 @@ def _sym_tiles(s: int, bm: int):
 
 
 def mirrored(ti: int, tj: int, bm: int) -> bool:
-    """Whether a symmetric tile is also written transposed."""
+    """Whether a symmetric tile also stands for its mirror image."""
     return tj * BN >= (ti + 1) * bm
 
 

@@ -251,9 +251,12 @@ def test_ns_fp32_matches_oracle(opt_fp32, steps):
 
 
 @pytest.mark.parametrize("kind", ["pair", "single"])
-def test_ns_gram_is_symmetric_in_workspace(opts, kind):
-    # The Gram tiles right of the diagonal are mirrored: A must be exactly
-    # symmetric, and equal to the float64 Gram of the bf16 input at bf16 level.
+def test_ns_gram_upper_triangle_in_workspace(opts, kind):
+    # The Gram tiles on and right of the 256-block diagonal hold the Gram of
+    # the bf16 input at bf16 level; the diagonal blocks are exactly
+    # symmetric. The single-CTA kernel stores only that upper 256-block
+    # triangle (its consumers read the blocks below it transposed), the
+    # CTA-pair kernel also writes the mirror image.
     from gpu_helpers import workspace_matrix
     opt_bf16 = opts[kind]
     shapes = [(600, 900), (900, 600), (513, 513), (1100, 300)]
@@ -264,10 +267,17 @@ def test_ns_gram_is_symmetric_in_workspace(opts, kind):
     for i, (m, n) in enumerate(shapes):
         s = min(m, n)
         A = to64(workspace_matrix(opt_bf16, shapes, i, 2)[:, :s])
-        assert np.array_equal(A, A.T)
+        blk = np.arange(s) // 256
+        upper = blk[None, :] >= blk[:, None]          # stored: column block at or right of the row block
+        full = np.where(upper, A, A.T)                 # the mirror image of the stored part
         X = x64[i] if m <= n else x64[i].T
         ref = X @ X.T
-        assert rel(A, ref) <= 4e-3
+        assert rel(full, ref) <= 4e-3
+        for b in range(0, s, 256):
+            d = A[b:b + 256, b:b + 256]
+            assert np.array_equal(d, d.T)
+        if kind == "pair":
+            assert np.array_equal(A, A.T)
 
 
 SWEEP_POINTS = W.PARITY_SHAPES["sweep"]
