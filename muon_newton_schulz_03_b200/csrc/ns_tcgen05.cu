@@ -277,6 +277,11 @@ __global__ void __launch_bounds__(kThreads, 1) ns_phase_kernel(const __grid_cons
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = sm.tmem_base;
+  // Launched as a programmatic dependent of the previous kernel on the
+  // stream: everything above may overlap that kernel's last CTAs; nothing it
+  // wrote is read before this wait (which returns once it has completed and
+  // its memory operations are visible).
+  asm volatile("griddepcontrol.wait;" ::: "memory");
 
   if (warp == 0) {
     // ------------------------------------------------------------------
@@ -616,8 +621,20 @@ cudaError_t launch_ns_phase_bf16(const NsLaunch& L, int phase, int src_sel, int 
   args.c = c;
   args.spec = spec;
   const int grid = L.grid < L.ntiles ? L.grid : L.ntiles;
-  ns_phase_kernel<<<grid, kThreads, smem, st>>>(args);
-  return cudaGetLastError();
+  // Programmatic stream serialization: this launch may begin while the
+  // previous kernel's last CTAs finish; the kernel waits for it before its
+  // first dependent read (griddepcontrol.wait).
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)grid, 1, 1);
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = (size_t)smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, ns_phase_kernel, args);
 }
 
 }  // namespace muon
