@@ -186,8 +186,18 @@ int muon_destroy(muon_handle* h);
  * Scale mode, extra scale and precision come from the handle's config.
  * The first call for a shape table builds the plan and the workspace
  * (device allocation and a host-to-device copy of the tables; do it before
- * any stream capture); later calls with the same shape table and pointers
- * only enqueue kernels and are safe to capture in a CUDA graph. */
+ * any stream capture). The per-call pointer tables live in a ring of eight
+ * device slots made with the plan: a call with pointers seen recently reuses
+ * its slot; a call with new pointers (fresh tensors every step are fine)
+ * takes the least recently used slot and uploads with one cudaMemcpyAsync on
+ * `stream` from pinned staging, without allocating or synchronising the
+ * device. Calls with the same shape table and pointers as an earlier
+ * uncaptured call only enqueue kernels and may be captured in a CUDA graph;
+ * the slots such a capture uses are kept for the graph (never overwritten)
+ * until the shape table changes or the handle is destroyed. A call with new
+ * pointers on a stream being captured fails with MUON_ERR_INVALID_ARG (the
+ * upload cannot be captured). Matrices with a NULL gradient drop out of the
+ * Newton-Schulz launches (their tiles are not listed). */
 int muon_step(muon_handle* h, float* const* params, const void* const* grads,
               float* const* momenta, const int32_t* shapes, int count,
               float lr, float beta, int nesterov, float wd, int ns_steps,

@@ -89,6 +89,9 @@ def main():
     for steps in (1, 5):
         for (m, n), x in zip(P["small"], W.gaussian_set(P["small"], 30 + steps)):
             record(f"small path {m}x{n} steps {steps}", x, steps)
+    # Extreme aspect ratios, normalised, five steps.
+    for (m, n), x in zip(P["extreme"], W.gaussian_set(P["extreme"], 60)):
+        record(f"extreme {m}x{n}", x, 5)
     # Allocation-free stage: two calls with fresh inputs.
     for call in range(2):
         for (m, n), x in zip(P["noalloc"], W.gaussian_set(P["noalloc"], call)):

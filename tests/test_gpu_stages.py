@@ -308,6 +308,23 @@ def test_ns_only_sweep_inputs(opt_bf16, point):
     _assert_status_clean(opt_bf16)
 
 
+@pytest.mark.parametrize("kind", ["pair", "single"])
+def test_ns_extreme_aspect_ratios(opts, kind):
+    # Rows of a million elements (one K-block polynomial, a Gram over 16384
+    # K-blocks), million-row combines, a ragged 70001-long row: five
+    # normalised steps on the tiled phases against the oracle.
+    opt_bf16 = opts[kind]
+    shapes = W.PARITY_SHAPES["extreme"]
+    xin, x64 = _ns_inputs(shapes, 60)
+    sumsq = torch.tensor([np.sum(x ** 2) for x in x64], dtype=torch.float64, device=DEV)
+    xout = [x_buffer(m, n) for (m, n) in shapes]
+    opt_bf16.newton_schulz(xin, xout, shapes, sumsq, ns_steps=5)
+    torch.cuda.synchronize()
+    for i, (m, n) in enumerate(shapes):
+        gate_bf16_ns(to64(xout[i][:, :n]), O.newton_schulz(x64[i], 5), x64[i], 5, what=f"{kind} {m}x{n}")
+    _assert_status_clean(opt_bf16)
+
+
 SMALL_SHAPES = W.PARITY_SHAPES["small"]
 
 

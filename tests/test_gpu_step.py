@@ -652,3 +652,58 @@ def test_steps_over_a_subset_launch_only_its_tiles():
     _check_step(cpu, dev, shapes, opt, lr=2e-4, beta=0.95, wd=0.1, indices=sorted(active))
     assert opt.status() == (0, 0, 0)
     opt.close()
+
+
+def test_captured_graph_keeps_its_tables_while_pointers_churn():
+    # A step captured in a CUDA graph keeps pointing at the device tables of
+    # its pointer set: those ring slots are pinned, so ten uncaptured steps
+    # with fresh tensors (more than the ring's eight slots) do not overwrite
+    # them, and a replay afterwards still updates the captured tensors exactly
+    # as an uncaptured step does. A new pointer set during capture is refused.
+    shapes = W.gpt2_shapes()[:4]
+    cpu, dev = make_set(W.CONFIG_GPT2, shapes, torch.float32)
+    base_p = [d[0].clone() for d in dev]
+    opt = muon.Muon(device=0, deterministic=True)
+    p = [t.clone() for t in base_p]
+    mo = [torch.zeros_like(t) for t in base_p]
+    g = [d[1] for d in dev]
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        opt.step(p, g, mo, lr=2e-4)                      # tables for these pointers exist
+    torch.cuda.current_stream().wait_stream(side)
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        opt.step(p, g, mo, lr=2e-4)
+    # Churn: ten steps on fresh tensors each time.
+    for k in range(10):
+        fp = [t.clone() for t in base_p]
+        fm = [torch.zeros_like(t) for t in base_p]
+        fg = [t.clone() for t in g]
+        opt.step(fp, fg, fm, lr=2e-4)
+    torch.cuda.synchronize()
+    want_p = [t.clone() for t in base_p]
+    want_m = [torch.zeros_like(t) for t in base_p]
+    opt.step(want_p, g, want_m, lr=2e-4)
+    for t, b in zip(p, base_p):
+        t.copy_(b)
+    for t in mo:
+        t.zero_()
+    graph.replay()
+    torch.cuda.synchronize()
+    for a, b in zip(p, want_p):
+        assert torch.equal(a, b)
+    for a, b in zip(mo, want_m):
+        assert torch.equal(a, b)
+    # New pointers while capturing: refused (the upload cannot be captured).
+    other = [t.clone() for t in base_p]
+    s2 = torch.cuda.Stream()
+    s2.wait_stream(torch.cuda.current_stream())
+    g2 = torch.cuda.CUDAGraph()
+    with pytest.raises(muon.MuonError):
+        with torch.cuda.graph(g2, stream=s2):
+            opt.step(other, g, [torch.zeros_like(t) for t in base_p], lr=2e-4)
+    del graph
+    assert opt.status() == (0, 0, 0)
+    opt.close()

@@ -267,6 +267,9 @@ PARITY_SHAPES = {
     "wait": [(512, 1024), (1024, 512)],
     "layerwise": [(256, 768), (768, 256), (64, 64), (1024, 512), (512, 1024), (300, 700)],
     "noalloc": [(300, 700), (700, 300), (256, 256), (5, 3), (1024, 1024)],
+    # extreme aspect ratios on the tiled phases: one K-block Grams of a
+    # million-long row, million-row combines, a ragged 70001-long row
+    "extreme": [(1, 1 << 20), (1 << 20, 1), (8, 131072), (131072, 8), (3, 70001)],
 }
 
 # Row blocks of the split-Muon test (None: the matrix stays whole).
