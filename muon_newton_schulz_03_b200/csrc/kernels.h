@@ -103,6 +103,8 @@ struct NsLaunch {
   int tma_store = 0;                 // 1: the *_ST store maps are present, stage outputs
                                      //    in shared memory and write them with bulk stores
   const GramBufs* gbufs = nullptr;   // device, one per matrix (Gram form only)
+  int max_s = 1 << 30;               // largest s = min(m, n) of the listed matrices, or an
+                                     // upper bound (the polynomial's identity form needs < 2048)
 };
 
 // Small-matrix path: one CTA per listed matrix runs every iteration on chip.

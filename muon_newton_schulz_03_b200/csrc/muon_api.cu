@@ -195,9 +195,6 @@ class TableRing {
     return rc;
   }
 
-  void abandon_call() { in_call_.clear(); }
-  size_t slot_bytes() const { return cap_; }
-
  private:
   struct Slot {
     std::vector<unsigned char> key;
@@ -701,6 +698,13 @@ ElemLaunch elem_launch(const DevPlan& P, const MatBind* d_binds) {
   return L;
 }
 
+// Largest s of the matrices a range covers (an upper bound for its tile lists).
+int range_max_s(const DevPlan& P, const WorkRange& R) {
+  int s = 0;
+  for (int i = R.m0; i < R.m1; ++i) s = std::max(s, P.mats[i].s);
+  return s;
+}
+
 ElemLaunch elem_launch(const DevPlan& P, const MatBind* d_binds, const WorkRange& R) {
   ElemLaunch L = elem_launch(P, d_binds);
   L.block_base = R.blk0;
@@ -791,6 +795,7 @@ int enqueue_ns(muon_handle* h, const MatBind* d_binds, const std::vector<MatBind
     L.gmaps = P.d_gmaps;
     L.gbufs = P.d_gbufs;
     L.tma_store = 1;
+    L.max_s = range_max_s(P, R);
     auto run = [&](int phase, int src_sel, int dst_sel, int first, float a, float b, float c,
                    const PhaseSpec& spec) -> int {
       const int list = phase == PHASE_SYM ? PHASE_POLY : phase;
@@ -861,15 +866,18 @@ int enqueue_ns(muon_handle* h, const MatBind* d_binds, const std::vector<MatBind
       L.grid = h->num_sms;
       L.timeout_ns = (unsigned long long)(h->cfg.wait_timeout_s * 1e9);
       L.tma_store = 1;
+      L.max_s = range_max_s(P, R);
       for (int ph = 0; ph < 3; ++ph) {
         L.tiles = R.tiles[ph];
         L.ntiles = R.ntiles[ph];
         if (L.ntiles == 0) continue;
         const int slot = prof_before(h, MUON_KERNEL_NS_GRAM + ph, st);
+        // a goes on the diagonal of B (POLY), so the combine adds no a X.
+        const float a = ph == PHASE_COMB ? 0.0f : c3[0];
         if (hp.tile_m == kTileMPair)
-          MUON_CUDA_TRY(launch_ns_phase_pair(L, ph, src, dst, first, c3[0], c3[1], c3[2], st));
+          MUON_CUDA_TRY(launch_ns_phase_pair(L, ph, src, dst, first, a, c3[1], c3[2], st));
         else
-          MUON_CUDA_TRY(launch_ns_phase_bf16(L, ph, src, dst, first, c3[0], c3[1], c3[2], st));
+          MUON_CUDA_TRY(launch_ns_phase_bf16(L, ph, src, dst, first, a, c3[1], c3[2], st));
         prof_after(h, slot, st);
         ++*launches;
       }

@@ -279,13 +279,17 @@ extern "C" int muon_newton_schulz_noalloc(const void* const* x_in, void* const* 
     L.status = status;
     L.grid = ds->num_sms;
     L.timeout_ns = (unsigned long long)(kNoallocWaitSeconds * 1e9);
+    L.max_s = 0;
+    for (int i = 0; i < count; ++i) L.max_s = std::max(L.max_s, hp.mats[i].s);
     int src = BUF_IN;
     for (int t = 1; t <= ns_steps; ++t) {
       const int dst = t == ns_steps ? BUF_OUT : (t % 2 == 1 ? BUF_X1 : BUF_X0);
       for (int ph = 0; ph < 3; ++ph) {
         L.tiles = reinterpret_cast<const int4*>(base + o_tiles[ph]);
         L.ntiles = (int)hp.tiles[ph].size();
-        NOALLOC_CUDA_TRY(launch_ns_phase_bf16(L, ph, src, dst, t == 1 ? 1 : 0, abc[0], abc[1], abc[2], st));
+        // a goes on the diagonal of B (POLY), so the combine adds no a X.
+        const float a = ph == PHASE_COMB ? 0.0f : abc[0];
+        NOALLOC_CUDA_TRY(launch_ns_phase_bf16(L, ph, src, dst, t == 1 ? 1 : 0, a, abc[1], abc[2], st));
       }
       src = dst;
     }

@@ -2,8 +2,8 @@
 //
 // Same three phases as ns_tcgen05.cu ("About Muon: Why Not Adam", sections
 // "The lemma that makes it possible" and "The whole thing, in about forty
-// lines"): GRAM A = X X^T (or X^T X), POLY B = bA + cA^2, COMB X' = aX + BX
-// (or aX + XB), with the normalisation folded into the first step's
+// lines"): GRAM A = X X^T (or X^T X), POLY B = aI + bA + cA^2, COMB X' = BX
+// (or XB), with the normalisation folded into the first step's
 // epilogues. Here each output tile is 256 x 256 and belongs to a cluster of
 // two CTAs on neighbouring SMs: CTA r holds rows 128r..128r+127 of the
 // tile's A operand and N-rows 128r..128r+127 of its B operand in its own
@@ -315,7 +315,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       } else {
         rows = mp.m; cols = mp.n; ld = mp.ldx;
         out = static_cast<__nv_bfloat16*>(const_cast<void*>(sel_buf(mp, mb, args.dst_sel)));
-        aux = static_cast<const __nv_bfloat16*>(sel_buf(mp, mb, args.src_sel)); aux_ld = mp.ldx;
+        // a X only when a is not already on the diagonal of B
+        if (args.a != 0.0f) { aux = static_cast<const __nv_bfloat16*>(sel_buf(mp, mb, args.src_sel)); aux_ld = mp.ldx; }
         if (args.first) sc = (float)inv_norm(L.sumsq, tile.x);
       }
       const bool mirror = (phase != PHASE_COMB) && (tj > ti);
@@ -337,7 +338,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         tmem_ld_32x32b_x32(t_base + (uint32_t)(ch * 32), v);
         const bool full_chunk = col0 + 32 <= cols;
         float o[32];
-        if (phase == PHASE_GRAM) {
+        if (aux == nullptr) {
 #pragma unroll
           for (int i = 0; i < 32; ++i) o[i] = v[i] * sc;
         } else {
@@ -350,8 +351,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
               x[i] = (row_ok && col0 + i < cols) ? __bfloat162float(aux[(size_t)row * aux_ld + col0 + i]) : 0.0f;
           }
           if (phase == PHASE_POLY) {
+            const int dcol = col0 == warp_row0 ? lane : -1;   // B + a I: this warp's diagonal chunk
 #pragma unroll
-            for (int i = 0; i < 32; ++i) o[i] = fmaf(cb, x[i], cc * v[i]);
+            for (int i = 0; i < 32; ++i) o[i] = fmaf(cb, x[i], cc * v[i]) + (i == dcol ? ca : 0.0f);
           } else {
 #pragma unroll
             for (int i = 0; i < 32; ++i) o[i] = sc * fmaf(ca, x[i], v[i]);

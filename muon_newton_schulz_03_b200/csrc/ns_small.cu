@@ -1,8 +1,9 @@
 // Small-matrix Newton-Schulz path: the whole iteration on chip.
 //
 // For a matrix with s = min(m, n) <= 128 and l = max(m, n) <= 512 one CTA
-// keeps X in shared memory, forms A = X X^T (or X^T X), B = bA + cA^2 and
-// X <- aX + BX (or aX + XB) on the tensor cores with the accumulators in
+// keeps X in shared memory, forms A = X X^T (or X^T X), B = aI + bA + cA^2
+// (a added to the diagonal in fp32 before B's rounding, as the tiled
+// kernels do) and X <- BX (or XB) on the tensor cores with the accumulators in
 // tensor memory, and runs all ns_steps iterations in one launch ("About
 // Muon: Why Not Adam", sections "The lemma that makes it possible" and "The
 // whole thing, in about forty lines"). Only the input and the final result
@@ -66,21 +67,6 @@ struct SmallArgs {
 
 __device__ __forceinline__ uint32_t swz(int r, int c, int chunk_stride) {
   return (uint32_t)((c >> 6) * chunk_stride + r * 128 + ((((c & 63) >> 3) ^ (r & 7)) << 4) + ((c & 7) << 1));
-}
-
-// 32 bf16 from an image row (r, c0..c0+31), c0 a multiple of 32.
-__device__ __forceinline__ void lds_row32(const uint8_t* img, int r, int c0, int cs, float (&o)[32]) {
-#pragma unroll
-  for (int q = 0; q < 4; ++q) {
-    const uint4 raw = *reinterpret_cast<const uint4*>(img + swz(r, c0 + 8 * q, cs));
-    const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&raw);
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const float2 f = __bfloat1622float2(h[i]);
-      o[8 * q + 2 * i] = f.x;
-      o[8 * q + 2 * i + 1] = f.y;
-    }
-  }
 }
 
 __device__ __forceinline__ void sts_row32(uint8_t* img, int r, int c0, int cs, const float (&o)[32]) {
@@ -232,8 +218,11 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) ns_small_kernel(const __
       float av[32], pv[32];
       tmem_ld_32x32b_x32(lane_base + (uint32_t)c0, av);          // A (fp32, before rounding)
       tmem_ld_32x32b_x32(lane_base + 128u + (uint32_t)c0, pv);   // A A
+      // B + a I: the chunk whose columns are this warp's rows holds the
+      // diagonal, lane i at column i.
+      const int dcol = (c0 == warp * 32 && row < mp.s) ? lane : -1;
 #pragma unroll
-      for (int i = 0; i < 32; ++i) pv[i] = fmaf(cb, bf16r(av[i] * sc_gram), cc * pv[i]);
+      for (int i = 0; i < 32; ++i) pv[i] = fmaf(cb, bf16r(av[i] * sc_gram), cc * pv[i]) + (i == dcol ? ca : 0.0f);
       sts_row32(sm.b, row, c0, kChunk, pv);
     }
     fence_proxy_async_smem();
@@ -284,11 +273,10 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) ns_small_kernel(const __
       const int r = blk * 128 + row;        // row of X
 #pragma unroll 1
       for (int c0 = 0; c0 < cols; c0 += 32) {
-        float v[32], x[32];
+        float v[32];
         tmem_ld_32x32b_x32(lane_base + (uint32_t)(blk * 128 + c0), v);
-        lds_row32(sm.x, r, c0, x_cs, x);
 #pragma unroll
-        for (int i = 0; i < 32; ++i) v[i] = sc * fmaf(ca, x[i], v[i]);
+        for (int i = 0; i < 32; ++i) v[i] *= sc;
         if (!last) {
           sts_row32(sm.x, r, c0, x_cs, v);
         } else if (r < mp.m && c0 < mp.n) {

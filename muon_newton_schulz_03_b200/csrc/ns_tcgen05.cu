@@ -4,9 +4,13 @@
 // makes it possible" and "The whole thing, in about forty lines") is three
 // grouped launches of this persistent kernel over all matrices of a call:
 //   GRAM : A = X X^T            (wide, X is s x l)   or  X^T X  (tall)
-//   POLY : B = b A + c A A      (A symmetric)
-//   COMB : X' = a X + B X       (wide)               or  a X + X B  (tall;
+//   POLY : B = a I + b A + c A A   (A symmetric)
+//   COMB : X' = B X             (wide)               or  X B  (tall;
 //                                                         B is symmetric)
+// so that X' = a X + (b A + c A^2) X: a sits on B's diagonal, added in fp32
+// before B's one bf16 rounding, and the combine is a bare product whose
+// epilogue reads nothing but the accumulator. (The Gram form, which runs the
+// polynomial with a = 0, asks the combine for a X itself: a != 0 there.)
 // Gram and polynomial outputs are symmetric: only tiles on or right of the
 // 256-block diagonal are computed and stored, so a symmetric buffer holds its
 // upper 256-block triangle (diagonal blocks whole). Its lower part is the
@@ -17,19 +21,21 @@
 // never transposed in memory: the Gram reads X with M/N-major operand tiles,
 // and the combine computes X B instead of B X^T.
 // The Frobenius normalisation X0 = Y/(||u|| + eps) of the first step is
-// folded into its epilogues: A0 = alpha^2 Y Y^T and X1 = alpha (a Y + B0 Y).
+// folded into its epilogues: A0 = alpha^2 Y Y^T and X1 = alpha B0 Y.
 //
 // Structure of one CTA (192 threads, one CTA per SM, persistent over a
 // static round-robin tile list):
 //   warp 0     : bulk-tensor (TMA) producer, 4-stage shared-memory ring
 //   warp 1     : tensor-memory allocator and single-thread tcgen05.mma issuer
 //   warps 2..5 : epilogue; tcgen05.ld of a 128 x 256 fp32 accumulator,
-//                fused combine, bf16 round-to-nearest-even stores
+//                fused polynomial, bf16 round-to-nearest-even stores
 // Two accumulators in tensor memory (2 x 256 columns) let the epilogue of
 // one tile overlap the main loop of the next.
 // Every wait is bounded: on expiry the error word is set, every role stops,
 // in-flight copies and MMAs are drained and tensor memory is freed.
+#include <cmath>
 #include <cstdio>
+#include <cstring>
 
 #include "common.cuh"
 #include "kernels.h"
@@ -49,13 +55,20 @@ constexpr int kTmemCols = 2 * BN;               // two fp32 accumulators
 constexpr int kOutBox = 32;                     // bulk-store box: 32 rows x 32 columns
 constexpr int kOutStageBytes = kOutBox * kOutBox * 2;
 constexpr int kAuxTmaMinK = 2048;               // combine tiles with K >= this read X by bulk loads
+// A polynomial launch whose matrices all have s below this takes b A on the
+// tensor cores (short tiles: the epilogue, not the MMA, is the critical
+// path); longer ones read A through bulk loads in the epilogue.
+constexpr int kIdentMaxS = 2048;
 
 struct __align__(1024) SmemLayout {
   uint8_t stage[kStages][kStageBytes];
-  // Epilogue staging: per epilogue warp two 32 x 32 bf16 output blocks for
-  // bulk stores and two for bulk loads of the auxiliary operand (64-byte
-  // rows, 64-byte swizzle).
-  uint8_t ostage[4][4][kOutStageBytes];
+  // Epilogue staging, per epilogue warp: two 32 x 32 bf16 output blocks for
+  // bulk stores and two blocks for bulk loads of the auxiliary operand
+  // (64-byte rows, 64-byte swizzle). A polynomial launch that takes b A on
+  // the tensor cores holds its two scaled 64 x 64 identities in the 16 KiB
+  // of auxiliary blocks instead (128-byte swizzle; 1024-byte aligned).
+  uint8_t ostage[4][2][kOutStageBytes];
+  uint8_t auxstage[4][2][kOutStageBytes];
   uint64_t full[kStages];
   uint64_t empty[kStages];
   uint64_t acc_full[2];
@@ -70,7 +83,15 @@ struct NsArgs {
   int phase, src_sel, dst_sel, first;
   float a, b, c;
   PhaseSpec spec;
+  // Polynomial launches with c != 0 over short matrices (s < kIdentMaxS):
+  // B = c (A A + q A) + a I, q = b / c split into two bf16 values (hi + lo)
+  // whose scaled identities the MMA multiplies A by.
+  int poly_ident;
+  uint32_t ident_bits;   // bf16 bits of hi (low half) and lo (high half)
+  int ident_parts;       // identities to apply: 0 when b == 0, 1 when lo == 0, else 2
 };
+
+constexpr int kIdentBytes = 64 * BK * 2;   // one 64 x 64 bf16 identity, 8 KiB
 
 // Everything a role needs to know about one tile.
 struct TileJob {
@@ -273,6 +294,25 @@ __global__ void __launch_bounds__(kThreads, 1) ns_phase_kernel(const __grid_cons
     tmem_alloc(&sm.tmem_base, kTmemCols);
     tmem_relinquish();
   }
+  const bool ident = args.phase == PHASE_POLY && args.poly_ident != 0;
+  if (ident && warp >= 2) {
+    // hi I and lo I as 64 x 64 K-major tiles in the 128-byte swizzle of the
+    // operand loads: thread e writes row e % 64 of tile e / 64 (element
+    // (r, k) sits in 16-byte unit (k / 8) ^ (r % 8) of row r).
+    const int e = (int)threadIdx.x - 64;
+    const int r = e & 63;
+    const uint32_t bits = (e >> 6) ? (args.ident_bits >> 16) : (args.ident_bits & 0xffffu);
+    uint8_t* rowp = &sm.auxstage[0][0][0] + (e >> 6) * kIdentBytes + r * 128;
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      uint32_t w[4];
+#pragma unroll
+      for (int h = 0; h < 4; ++h)
+        w[h] = ((q ^ (r & 7)) == (r >> 3) && ((r & 7) >> 1) == h) ? bits << (16 * (r & 1)) : 0u;
+      *reinterpret_cast<uint4*>(rowp + q * 16) = make_uint4(w[0], w[1], w[2], w[3]);
+    }
+    fence_proxy_async_smem();
+  }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -344,6 +384,7 @@ __global__ void __launch_bounds__(kThreads, 1) ns_phase_kernel(const __grid_cons
       uint32_t acc_phase = 0;
       bool ok = true;
       bool issued = false;
+      const uint32_t ident_base = smem_u32(&sm.auxstage[0][0][0]);
       for (int t = blockIdx.x; t < L.ntiles && ok; t += gridDim.x) {
         const int4 tile = L.tiles[t];
         if (!L.binds[tile.x].active) continue;
@@ -370,6 +411,21 @@ __global__ void __launch_bounds__(kThreads, 1) ns_phase_kernel(const __grid_cons
                                     : umma_desc_sw128(sb + k16 * 32, 16, 1024);
             tc_mma_bf16(d_tmem, da, db, idesc, (kb | k16) != 0);
           }
+          if (ident && (kb * BK) / BN == j.tj) {
+            // q A on the 64 output columns equal to this K-block's indices:
+            // D[:, k - tj*256] += A[:, k] (hi + lo), N = 64.
+            const uint32_t d_sub = d_tmem + (uint32_t)(kb * BK - j.tj * BN);
+            const uint32_t idesc64 = umma_idesc_bf16(BM, 64, amn, 0);
+            for (int part = 0; part < args.ident_parts; ++part) {
+#pragma unroll
+              for (int k16 = 0; k16 < BK / 16; ++k16) {
+                const uint64_t da = amn ? umma_desc_sw128(sa + k16 * 2048, kMnChunkBytes, 1024)
+                                        : umma_desc_sw128(sa + k16 * 32, 16, 1024);
+                const uint64_t di = umma_desc_sw128(ident_base + (uint32_t)(part * kIdentBytes + k16 * 32), 16, 1024);
+                tc_mma_bf16(d_sub, da, di, idesc64, 1);
+              }
+            }
+          }
           issued = true;
           tc_commit(&sm.empty[stage]);      // frees the stage once these MMAs finish
           if (++stage == kStages) { stage = 0; phase ^= 1u; }
@@ -393,15 +449,20 @@ __global__ void __launch_bounds__(kThreads, 1) ns_phase_kernel(const __grid_cons
     uint32_t acc_phase = 0;
     int obuf = 0;   // staging block pair used by this warp's next chunk
     const bool tma_out = L.tma_store != 0 && !(args.phase == PHASE_COMB && args.dst_sel == BUF_OUT);
-    // The auxiliary operand of the polynomial (A) and of the combine (X)
-    // comes through bulk-tensor loads of 32 x 32 blocks into this warp's two
-    // auxiliary buffers when it is a workspace buffer with a 32 x 32 map and
-    // the tile's main loop is long (K = s >= kAuxTmaMinK); a per-lane row
-    // load touches 32 cache lines per instruction, but on short tiles the
-    // bulk loads wait behind the producer's operand loads in the same copy
-    // engine and the epilogue, then on the critical path, slows.
+    // The combine reads X a second time only when it adds a X itself
+    // (a != 0, the Gram form); the plain iteration puts a on the diagonal of
+    // B in the polynomial's epilogue, so its combine is the bare product.
+    const bool comb_ax = args.phase == PHASE_COMB && args.a != 0.0f;
+    // The auxiliary operand of the polynomial (A, when it does not take b A
+    // on the tensor cores) and of the combine (X) comes through bulk-tensor
+    // loads of 32 x 32 blocks into this warp's two auxiliary buffers when it
+    // is a workspace buffer with a 32 x 32 map: always for the polynomial,
+    // and for the combine when its main loop is long (K = s >= kAuxTmaMinK).
+    // A per-lane row load touches 32 cache lines per instruction; on short
+    // combine tiles the bulk loads wait behind the producer's operand loads
+    // in the same copy engine instead.
     const bool aux_tma_phase = L.tma_store != 0 &&
-                               (args.phase == PHASE_POLY || (args.phase == PHASE_COMB && args.src_sel != BUF_IN));
+                               ((args.phase == PHASE_POLY && !ident) || (comb_ax && args.src_sel != BUF_IN));
     uint32_t aux_parity = 0;    // bit b: parity of the next wait on aux_full[quarter][b]
     uint32_t aux_pending = 0;   // bit b: a load into buffer b has not been waited for
     for (int t = blockIdx.x; t < L.ntiles; t += gridDim.x) {
@@ -426,7 +487,8 @@ __global__ void __launch_bounds__(kThreads, 1) ns_phase_kernel(const __grid_cons
         if (args.first) { const double al = inv_norm(L.sumsq, tile.x); sc = (float)(al * al); }
       } else if (phase == PHASE_POLY) {
         rows = cols = mp.s; ld = mp.lds; out = sym_ptr(L, mp, tile.x, args.spec.poly_out);
-        aux = static_cast<const __nv_bfloat16*>(mp.a); aux_ld = mp.lds;
+        if (ident) sc = args.c;   // the accumulator holds A A + q A
+        else { aux = static_cast<const __nv_bfloat16*>(mp.a); aux_ld = mp.lds; }
       } else if (phase == PHASE_SYM) {
         rows = cols = mp.s; ld = mp.lds; out = sym_ptr(L, mp, tile.x, args.spec.sym_out);
         aux = sym_ptr(L, mp, tile.x, args.spec.aux1); aux2 = sym_ptr(L, mp, tile.x, args.spec.aux2);
@@ -434,7 +496,7 @@ __global__ void __launch_bounds__(kThreads, 1) ns_phase_kernel(const __grid_cons
       } else {
         rows = mp.m; cols = mp.n; ld = mp.ldx;
         out = static_cast<__nv_bfloat16*>(const_cast<void*>(sel_buf(mp, mb, args.dst_sel)));
-        aux = static_cast<const __nv_bfloat16*>(sel_buf(mp, mb, args.src_sel)); aux_ld = mp.ldx;
+        if (comb_ax) { aux = static_cast<const __nv_bfloat16*>(sel_buf(mp, mb, args.src_sel)); aux_ld = mp.ldx; }
         if (args.first) sc = (float)inv_norm(L.sumsq, tile.x);
       }
       // Symmetric outputs are stored as computed (upper 256-block triangle);
@@ -454,7 +516,7 @@ __global__ void __launch_bounds__(kThreads, 1) ns_phase_kernel(const __grid_cons
       const float ca = args.a, cb = args.b, cc = args.c;
       const __nv_bfloat16* aux_row = aux != nullptr ? aux + (size_t)row * aux_ld : nullptr;
       uint4 xa[4], xb[4];   // packed bf16 auxiliary values of the current and the next chunk
-      const bool aux_tma = aux_tma_phase && mp.s >= kAuxTmaMinK;
+      const bool aux_tma = aux_tma_phase && (phase == PHASE_POLY || mp.s >= kAuxTmaMinK);
       const TmapBlob* aux_map =
           !aux_tma ? nullptr
           : L.maps + (size_t)tile.x * kMapsPerMat +
@@ -467,7 +529,7 @@ __global__ void __launch_bounds__(kThreads, 1) ns_phase_kernel(const __grid_cons
         if (lane == 0) {
           fence_proxy_async_smem();
           mbar_arrive_expect_tx(&sm.aux_full[quarter][b], kOutStageBytes);
-          tma_load_2d(sm.ostage[quarter][2 + b], aux_map, &sm.aux_full[quarter][b], tj * BN + c * 32, warp_row0);
+          tma_load_2d(sm.auxstage[quarter][b], aux_map, &sm.aux_full[quarter][b], tj * BN + c * 32, warp_row0);
         }
         aux_pending |= 1u << b;
       };
@@ -500,7 +562,7 @@ __global__ void __launch_bounds__(kThreads, 1) ns_phase_kernel(const __grid_cons
             return false;
           aux_parity ^= 1u << b;
           aux_pending &= ~(1u << b);
-          const uint8_t* ab = sm.ostage[quarter][2 + b];
+          const uint8_t* ab = sm.auxstage[quarter][b];
 #pragma unroll
           for (int q = 0; q < 4; ++q) cur[q] = *reinterpret_cast<const uint4*>(ab + sw64_offset(lane, q));
         }
@@ -534,6 +596,13 @@ __global__ void __launch_bounds__(kThreads, 1) ns_phase_kernel(const __grid_cons
 #pragma unroll
             for (int i = 0; i < 32; ++i) o[i] = sc * fmaf(ca, x[i], v[i]);
           }
+        }
+        if (phase == PHASE_POLY) {
+          // B + a I: the chunk whose columns are this warp's rows holds the
+          // diagonal, lane i at column i.
+          const int dcol = col0 == warp_row0 ? lane : -1;
+#pragma unroll
+          for (int i = 0; i < 32; ++i) o[i] += i == dcol ? ca : 0.0f;
         }
         if (tma_out) {
           // Stage the 32 x 32 block in shared memory and write it with a bulk
@@ -601,6 +670,30 @@ __global__ void __launch_bounds__(kThreads, 1) ns_phase_kernel(const __grid_cons
 
 int ns_bf16_smem_bytes() { return (int)sizeof(SmemLayout) + 1024; }
 
+namespace {
+
+// Round-to-nearest-even bf16 bits of a finite float.
+uint32_t bf16_bits_rne(float f) {
+  uint32_t u;
+  std::memcpy(&u, &f, sizeof(u));
+  u += 0x7fffu + ((u >> 16) & 1u);
+  return u >> 16;
+}
+
+float bf16_bits_value(uint32_t h) {
+  const uint32_t u = h << 16;
+  float f;
+  std::memcpy(&f, &u, sizeof(f));
+  return f;
+}
+
+// The polynomial takes q A = (b / c) A on the tensor cores while |q| stays
+// this small: the accumulator then holds A A + q A with entries a few times
+// those of A A, so its fp32 rounding stays far below the bf16 rounding of B.
+constexpr double kIdentMaxRatio = 64.0;
+
+}  // namespace
+
 cudaError_t launch_ns_phase_bf16(const NsLaunch& L, int phase, int src_sel, int dst_sel, int first, float a,
                                  float b, float c, cudaStream_t st, const PhaseSpec& spec) {
   if (L.ntiles <= 0) return cudaSuccess;
@@ -620,6 +713,19 @@ cudaError_t launch_ns_phase_bf16(const NsLaunch& L, int phase, int src_sel, int 
   args.b = b;
   args.c = c;
   args.spec = spec;
+  args.poly_ident = 0;
+  args.ident_bits = 0;
+  args.ident_parts = 1;
+  if (phase == PHASE_POLY && c != 0.0f && L.max_s < kIdentMaxS) {
+    const double q = (double)b / (double)c;
+    if (std::isfinite(q) && std::fabs(q) <= kIdentMaxRatio) {
+      const uint32_t hi = bf16_bits_rne((float)q);
+      const uint32_t lo = bf16_bits_rne((float)(q - (double)bf16_bits_value(hi)));
+      args.poly_ident = 1;
+      args.ident_bits = hi | (lo << 16);
+      args.ident_parts = (hi & 0x7fffu) == 0 ? 0 : (lo & 0x7fffu) != 0 ? 2 : 1;   // b = 0: A A alone
+    }
+  }
   const int grid = L.grid < L.ntiles ? L.grid : L.ntiles;
   // Programmatic stream serialization: this launch may begin while the
   // previous kernel's last CTAs finish; the kernel waits for it before its

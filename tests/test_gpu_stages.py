@@ -167,8 +167,9 @@ def _ns_inputs(shapes, seed, scale=1.0):
 
 @pytest.mark.parametrize("kind", ["pair", "single"])
 def test_ns_identity_combine_is_exact(opts, kind):
-    # (a, b, c) = (1, 0, 0): B = 0, so X1 = 1 * X + 0 * X exactly. Exercises
-    # every tile's combine epilogue addressing (direct, ragged tails, tall).
+    # (a, b, c) = (1, 0, 0): B = a I + 0 = I, so X1 = I X = X exactly.
+    # Exercises every tile's combine epilogue addressing (direct, ragged
+    # tails, tall) and the diagonal of the polynomial's tiles.
     opt_bf16 = opts[kind]
     shapes = RAGGED
     xin, x64 = _ns_inputs(shapes, 5)
