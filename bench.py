@@ -455,7 +455,8 @@ def run_ours(args):
 
     if rank == 0:
         value = (1 if args.layerwise else world) * 1e3 / ms_step
-        traffic = None if gram else profiled_traffic(args.workload)
+        # The committed captures are of the single-CTA kernel, standard form.
+        traffic = None if (gram or args.cta_pair) else profiled_traffic(args.workload)
         line = {
             "metric": METRIC,
             "value": value,
