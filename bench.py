@@ -648,16 +648,20 @@ def run_sweep(args):
             opt.newton_schulz(xin, xout, shapes, None, ns_steps=NS_STEPS)
         graph.replay()
         torch.cuda.synchronize()
+        # About 100 ms of replays (3 to 50): a short point's replays then
+        # queue back to back, and the first one's launch latency does not
+        # weigh on its mean.
+        greps = max(3, min(50, int(100.0 / max(ms_eager, 1e-3))))
         start.record()
-        for _ in range(reps):
+        for _ in range(greps):
             graph.replay()
         end.record()
         torch.cuda.synchronize()
-        ms = start.elapsed_time(end) / reps
+        ms = start.elapsed_time(end) / greps
         del graph
         flops = batch * W.ns_flops(m, n, NS_STEPS)
         tf = flops / (ms * 1e-3) / 1e12
-        points.append({"m": m, "n": n, "batch": batch, "ms": ms, "ms_eager": ms_eager, "tflops_nominal": tf,
+        points.append({"m": m, "n": n, "batch": batch, "ms": ms, "ms_eager": ms_eager, "replays": greps, "tflops_nominal": tf,
                        "frac_datasheet": tf / DATASHEET_BF16_TFLOPS, "frac_measured": tf / peaks["bf16_tflops"]})
         del xin, xout
         torch.cuda.empty_cache()
