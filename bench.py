@@ -457,6 +457,14 @@ def run_ours(args):
         value = (1 if args.layerwise else world) * 1e3 / ms_step
         # The committed captures are of the single-CTA kernel, standard form.
         traffic = None if (gram or args.cta_pair) else profiled_traffic(args.workload)
+        # The sustained peak (a seconds-long loop under the power cap) for a
+        # timed region of a second or more; the burst peak for a shorter one.
+        long_region = ms_step * args.steps >= 1000.0
+        peak_key = "bf16_tflops_sustained" if long_region else "bf16_tflops"
+        peak_note = (f"{peak_src} sustained dense bf16 (timed region of {ms_step * args.steps / 1e3:.1f} s, "
+                     "inside a long run)" if long_region else
+                     f"{peak_src} burst dense bf16 (timed region of {ms_step * args.steps:.0f} ms)")
+        peak_tf = peaks[peak_key]
         line = {
             "metric": METRIC,
             "value": value,
@@ -486,7 +494,7 @@ def run_ours(args):
             },
             "ns_tflops_nominal": ns_tflops,
             "ns_frac_of_datasheet_bf16": (ns_tflops / DATASHEET_BF16_TFLOPS) if ns_tflops else None,
-            "ns_frac_of_measured_bf16": (ns_tflops / peaks["bf16_tflops_sustained"]) if ns_tflops else None,
+            "ns_frac_of_measured_bf16": (ns_tflops / peak_tf) if ns_tflops else None,
             "matrices_per_s": count * value,
             "ns_ms_per_step": ns_ms,
             "elementwise": {
@@ -498,15 +506,15 @@ def run_ours(args):
                 "kernel": "ns_phase_kernel (tcgen05 Newton-Schulz phases, all matrices per launch)",
                 "bound": "tensor",
                 "achieved": ns_tflops_alg,
-                "peak": peaks["bf16_tflops_sustained"],
+                "peak": peak_tf,
                 "unit": "TFLOP/s",
-                "frac": (ns_tflops_alg / peaks["bf16_tflops_sustained"]) if ns_tflops_alg else None,
+                "frac": (ns_tflops_alg / peak_tf) if ns_tflops_alg else None,
                 "traffic": traffic,
-                "peak_source": f"{peak_src} sustained dense bf16 (kernel timed inside a long step)",
+                "peak_source": peak_note,
                 "flops_per_launch": per_launch_flops,
                 "achieved_nominal": ns_tflops,
                 "achieved_executed": ns_tflops_exec,
-                "frac_executed": (ns_tflops_exec / peaks["bf16_tflops_sustained"]) if ns_tflops_exec else None,
+                "frac_executed": (ns_tflops_exec / peak_tf) if ns_tflops_exec else None,
                 "executed_definition": "tile FLOPs the tensor cores run: listed tiles x BM x 256 x K (K padded "
                                        "to 64); symmetric phases list upper tiles only",
                 "avg_launch_ms": avg_ns_launch_ms,
@@ -594,7 +602,7 @@ def run_e2e(torch, muon, opt, shapes, params, grads, moms, args, device, world, 
         return {"value": None, "unit": "steps/s", "error": f"device status {code} on this or another rank"}
     return {"value": world * 1e3 / ms, "unit": "steps/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
             "ms_per_step": ms, "steps": steps,
-            "path": "muon_step_host: params, grads, momenta in pinned host memory; 8 chunks pipelined over "
+            "path": "muon_step_host: params, grads, momenta in pinned host memory; up to 32 chunks pipelined over "
                     "copy-in, compute and copy-out streams; the caller's stream waits for the last copy-out"}
 
 

@@ -230,7 +230,7 @@ int muon_qk_clip(muon_handle* h, float* const* weights, const int32_t* shapes,
                  const float* const* s_max, int count, float tau, void* stream);
 
 /* Same step with every tensor in HOST memory. The matrices are split into
- * up to 8 chunks of consecutive matrices with about equal element counts;
+ * up to 32 chunks of consecutive matrices with about equal element counts;
  * while chunk c is computed, chunk c+1 is copied in and chunk c-1 copied
  * out, on three library streams (copy-in, compute, copy-out) that start
  * after the work already queued on `stream`; `stream` waits for the last

@@ -321,7 +321,10 @@ struct WorkRange {
   int nsmall = 0;
 };
 
-constexpr int kHostChunks = 8;      // chunks of the pipelined host-buffer step
+// Chunks of the pipelined host-buffer step: enough that the last chunk's
+// compute and copy-out, which nothing overlaps, are a few percent of a step
+// whose copies both ways keep PCIe busy.
+constexpr int kHostChunks = 32;
 constexpr int kStagingSlots = 3;    // staging slots in flight (H2D, compute, D2H)
 
 struct muon_handle {
