@@ -220,6 +220,32 @@ def test_ns_bf16_matches_oracle(opts, kind, steps):
     _assert_status_clean(opt_bf16)
 
 
+def test_polynomial_identity_form_matches_bulk_load_form():
+    # A polynomial launch whose matrices all have s < 2048 takes b A on the
+    # tensor cores (scaled identities); a launch that also holds a larger
+    # matrix reads A in the epilogue instead. The same short matrices (the
+    # ragged inputs of the five-step test) through both forms: each within
+    # its oracle gate, and the two within fp32 summation order of each other.
+    h = muon.Muon(device=0, small_path=False)
+    shapes, big = RAGGED, [(2048, 2048)]
+    xin, x64 = _ns_inputs(shapes + big, 12)
+    sumsq = torch.tensor([np.sum(x ** 2) for x in x64], dtype=torch.float64, device=DEV)
+    short = len(shapes)
+    out_ident = [x_buffer(m, n) for (m, n) in shapes]
+    out_bulk = [x_buffer(m, n) for (m, n) in shapes + big]
+    h.newton_schulz(xin[:short], out_ident, shapes, sumsq[:short].contiguous(), ns_steps=5)
+    h.newton_schulz(xin, out_bulk, shapes + big, sumsq, ns_steps=5)
+    torch.cuda.synchronize()
+    for i, (m, n) in enumerate(shapes):
+        a, b = to64(out_ident[i][:, :n]), to64(out_bulk[i][:, :n])
+        ref = O.newton_schulz(x64[i], 5)
+        gate_bf16_ns(a, ref, x64[i], 5, what=f"identity form {m}x{n}")
+        gate_bf16_ns(b, ref, x64[i], 5, what=f"bulk-load form {m}x{n}")
+        assert rel(a, b) <= TOL_GPU_VS_GPU, f"identity vs bulk-load form {m}x{n}: {rel(a, b):.3e}"
+    assert h.status() == (0, 0, 0)
+    h.close()
+
+
 def test_ns_zero_steps_scales(opt_bf16):
     shapes = [(10, 20), (20, 10)]
     xin, x64 = _ns_inputs(shapes, 9)
