@@ -7,7 +7,9 @@
  *      per-matrix sum of squares of u and the bf16 cast of u (one kernel);
  *   2. the quintic Newton-Schulz iteration on the short side,
  *      A = X X^T, B = bA + cA^2, X <- aX + BX, with X = u / (||u||_F + 1e-7)
- *      (tensor-core GEMMs, one launch per phase for all matrices);
+ *      (tensor-core GEMMs, one launch per phase for all matrices; in bf16
+ *      the polynomial's epilogue forms aI + bA + cA^2, rounded once, and the
+ *      combine is the product of that with X);
  *   3. p' = p*(1 - lr*wd) - lr*scale(m, n)*O (one kernel).
  *
  * Sources (web pages, cited by title and section):

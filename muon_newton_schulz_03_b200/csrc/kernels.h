@@ -56,7 +56,7 @@ constexpr int kGramMapsPerMat = 8;
 
 // Operands and epilogue of one launch beyond the phase itself.
 struct PhaseSpec {
-  int poly_out = SB_B;                 // POLY: where B = bA + cA^2 goes
+  int poly_out = SB_B;                 // POLY: where B = aI + bA + cA^2 goes (a = 0 in the Gram form)
   int sym_l = SB_A, sym_r = SB_A;      // SYM: D = L R (both symmetric)
   int sym_out = SB_T;
   int aux1 = SB_NONE, aux2 = SB_NONE;  // SYM: out = D + e1 aux1 + e2 aux2

@@ -1,7 +1,7 @@
-// fp32 debug Newton-Schulz: plain FFMA tiled GEMMs with the same fused
-// epilogues as the tensor-core path (Gram with the alpha^2 fold, bA + cA^2,
-// alpha (aX + BX)), launched once per matrix and phase. Full (not
-// symmetric) outputs. Performance is not a goal; the arithmetic is fp32 with
+// fp32 debug Newton-Schulz: plain FFMA tiled GEMMs with fused epilogues
+// (Gram with the alpha^2 fold, bA + cA^2, alpha (aX + BX): the program's own
+// grouping, where the bf16 kernels put a on the diagonal of B instead),
+// launched once per matrix and phase. Full (not symmetric) outputs. Performance is not a goal; the arithmetic is fp32 with
 // fp32 accumulation so the result can be held to a tight tolerance against
 // the float64 oracle.
 #include "common.cuh"
