@@ -500,6 +500,8 @@ def run_ours(args):
             "elementwise": {
                 "momentum_norm_ms": k1_ms, "momentum_norm_gbs": (k1_bytes / (k1_ms * 1e-3) / 1e9) if k1_ms else None,
                 "apply_ms": k4_ms, "apply_gbs": (k4_bytes / (k4_ms * 1e-3) / 1e9) if k4_ms else None,
+                # no apply kernel ran: the last combine wrote p' itself
+                "apply_fused": k4_ms is None,
                 "hbm_peak_gbs": peaks["hbm_gbs"], "peak_source": peak_src,
             },
             "roofline": {

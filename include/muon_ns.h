@@ -143,8 +143,22 @@ typedef struct muon_config {
   int cta_pair;               /* 1: tiled phases use 256 x 256 tiles on CTA
                                  pairs (tcgen05 cta_group::2); 0: 128 x 256
                                  tiles on single CTAs. Default 0 (the
-                                 single-CTA tiles measured 2-4% faster on
+                                 single-CTA tiles measured 2-10% faster on
                                  the Llama-shaped set under the power cap) */
+  int fused_apply;            /* 1 (default): in muon_step and
+                                 muon_step_host, with bf16 Newton-Schulz in
+                                 the standard form on single-CTA tiles,
+                                 ns_steps >= 1, no active matrix on the
+                                 small path and every parameter's rows
+                                 16-byte aligned (n % 4 == 0, aligned base),
+                                 the last combine's epilogue writes
+                                 p' = p (1 - lr wd) - lr scale O itself
+                                 (O rounded to bf16 first, so p' is bitwise
+                                 the same as with 0; p moved by bulk copies)
+                                 and O is not stored. 0, or any other step:
+                                 O is stored in the workspace buffer
+                                 muon_plan_query names and a separate pass
+                                 applies it                                 */
 } muon_config;
 
 /* plan_flags of muon_plan_query */

@@ -228,7 +228,8 @@ class Muon:
     def __init__(self, device: int = 0, scale_mode: str = "moonlight", extra_scale: float = 1.0,
                  ns_precision: str = "bf16", check_nonfinite: bool = False, num_sms: int = 0,
                  workspace_cap_bytes: int = 0, wait_timeout_s: float = 2.0, small_path: bool = True,
-                 cta_pair: bool = False, ns_algorithm: str = "standard", deterministic: bool = False):
+                 cta_pair: bool = False, ns_algorithm: str = "standard", deterministic: bool = False,
+                 fused_apply: bool = True):
         self._lib = load()
         cfg = MuonConfig()
         check(self._lib.muon_config_init(ctypes.byref(cfg)))
@@ -243,6 +244,7 @@ class Muon:
         cfg.cta_pair = int(bool(cta_pair))
         cfg.ns_algorithm = ALGORITHMS[ns_algorithm]
         cfg.deterministic = int(bool(deterministic))
+        cfg.fused_apply = int(bool(fused_apply))
         h = ctypes.c_void_p()
         check(self._lib.muon_init(int(device), ctypes.byref(cfg), ctypes.byref(h)))
         self._h = h
@@ -251,6 +253,11 @@ class Muon:
         self.small_path = bool(small_path)
         self.cta_pair = bool(cta_pair)
         self.ns_algorithm = ns_algorithm
+        # True when this handle's steps may write p' in their last combine and
+        # store no O (muon_config.fused_apply); a step does so when no active
+        # matrix is on the small path and every row is 16-byte aligned.
+        self.fused_apply = (bool(fused_apply) and ns_precision == "bf16" and ns_algorithm == "standard"
+                            and not cta_pair)
 
     # -- lifetime -----------------------------------------------------------
     def close(self):

@@ -38,6 +38,7 @@ class MuonConfig(ctypes.Structure):
         ("ns_algorithm", c_int),
         ("deterministic", c_int),
         ("cta_pair", c_int),
+        ("fused_apply", c_int),
     ]
 
 

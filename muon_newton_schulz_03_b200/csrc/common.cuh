@@ -110,6 +110,37 @@ __device__ __forceinline__ double inv_norm(const double* sumsq, int mat) {
   return 1.0 / (sqrt(sumsq[mat]) + kNormEps);
 }
 
+// Shape-dependent update scale of an m x n matrix ("Why Muon Works",
+// configuration block; "About Muon: Why Not Adam", the program's
+// 0.2 sqrt(max(m, n))) times the caller's extra factor.
+__device__ __forceinline__ float update_scale_dev(int m, int n, int mode, float extra) {
+  double s;
+  const double dm = m, dn = n;
+  switch (mode) {
+    case 0: s = 0.2 * sqrt(dm > dn ? dm : dn); break;          // Moonlight
+    case 1: s = sqrt((dm / dn) > 1.0 ? (dm / dn) : 1.0); break; // Jordan
+    case 2: s = sqrt(dm / dn); break;                          // Bernstein
+    default: s = 1.0; break;
+  }
+  return (float)(s * (double)extra);
+}
+
+// 1 - lr wd, rounded the same way wherever the update is applied.
+__device__ __forceinline__ float apply_decay(float lr, float wd) { return __fsub_rn(1.0f, __fmul_rn(lr, wd)); }
+
+// Multiplier of O in p' = p (1 - lr wd) - step O: lr times the update scale,
+// times inv = 1/(||u|| + eps) when O was not normalised (zero iterations).
+__device__ __forceinline__ float apply_step(float lr, int m, int n, int mode, float extra, double inv) {
+  return (float)((double)lr * (double)update_scale_dev(m, n, mode, extra) * inv);
+}
+
+// One entry of the update from an fp32 O value: O is rounded to bf16 first,
+// so the result is bitwise that of the separate apply pass, which reads the
+// stored bf16 O.
+__device__ __forceinline__ float apply_one(float p, float o, float decay, float step) {
+  return fmaf(p, decay, -step * __bfloat162float(__float2bfloat16_rn(o)));
+}
+
 // ---------------------------------------------------------------------------
 // mbarrier (shared::cta) with bounded waits
 // ---------------------------------------------------------------------------

@@ -218,18 +218,6 @@ __global__ void __launch_bounds__(kThreads) k1b_reduce_partials(const MatBind* _
   if (lane == 0) sumsq[mat] = v;
 }
 
-__device__ __forceinline__ float update_scale_dev(int m, int n, int mode, float extra) {
-  double s;
-  const double dm = m, dn = n;
-  switch (mode) {
-    case 0: s = 0.2 * sqrt(dm > dn ? dm : dn); break;          // Moonlight
-    case 1: s = sqrt((dm / dn) > 1.0 ? (dm / dn) : 1.0); break; // Jordan
-    case 2: s = sqrt(dm / dn); break;                          // Bernstein
-    default: s = 1.0; break;
-  }
-  return (float)(s * (double)extra);
-}
-
 template <bool kFp32In>
 __global__ void __launch_bounds__(kThreads) k4_apply(const MatPlan* __restrict__ plans,
                                                      const MatBind* __restrict__ binds,
@@ -246,9 +234,8 @@ __global__ void __launch_bounds__(kThreads) k4_apply(const MatPlan* __restrict__
   if (obase == nullptr) return;
   const long long e0 = (blk - prefix[mat]) * (long long)kElemChunk;
   const long long e1 = min(e0 + (long long)kElemChunk, mp.numel);
-  const float decay = 1.0f - lr * wd;
-  const float step = (float)((double)lr * (double)update_scale_dev(mp.m, mp.n, scale_mode, extra_scale) *
-                             inv_norm(sumsq, mat));
+  const float decay = apply_decay(lr, wd);
+  const float step = apply_step(lr, mp.m, mp.n, scale_mode, extra_scale, inv_norm(sumsq, mat));
   if ((mp.n % kVec) == 0 && e1 - e0 == kElemChunk) {
     // Whole chunk: two vector steps in flight per thread, as in K1.
     const long long eb = e0 + (long long)threadIdx.x * kVec;

@@ -88,6 +88,17 @@ enum MapIdx : int {
   kInMapsPerMat = 3
 };
 
+// The parameter update p' = p (1 - lr wd) - lr scale O taken into the last
+// combine's epilogue: O (rounded to bf16, as the separate apply pass reads
+// it) is not stored; 32 x 32 blocks of p are bulk-loaded into shared memory,
+// updated there and bulk-stored back through `p_maps` of the launch.
+struct ApplyArgs {
+  int on = 0;
+  float lr = 0.0f, wd = 0.0f;
+  int scale_mode = 0;
+  float extra_scale = 1.0f;
+};
+
 struct NsLaunch {
   const MatPlan* plans = nullptr;     // device
   const MatBind* binds = nullptr;     // device
@@ -105,6 +116,8 @@ struct NsLaunch {
   const GramBufs* gbufs = nullptr;   // device, one per matrix (Gram form only)
   int max_s = 1 << 30;               // largest s = min(m, n) of the listed matrices, or an
                                      // upper bound (the polynomial's identity form needs < 2048)
+  ApplyArgs apply;                   // COMB only: update p instead of storing O
+  const TmapBlob* p_maps = nullptr;  // device, one fp32 32 x 32 map of p per matrix (apply only)
 };
 
 // Small-matrix path: one CTA per listed matrix runs every iteration on chip.

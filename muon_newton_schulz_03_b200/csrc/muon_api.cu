@@ -268,6 +268,22 @@ int encode_store_map(TmapBlob* out, const void* base, int rows, int cols, int ld
   return encode_map(out, base, rows, cols, ld, 32, 32, CU_TENSOR_MAP_SWIZZLE_64B);
 }
 
+// A caller's fp32 parameter (dense rows x cols, cols % 4 == 0, 16-byte
+// aligned): 32 x 32 boxes, 128-byte swizzle (a box row is 128 bytes).
+int encode_p_map(TmapBlob* out, const float* base, int rows, int cols) {
+  EncodeTiledFn enc = get_encode_fn();
+  if (!enc) return fail(MUON_ERR_CUDA, "cuTensorMapEncodeTiled is not available");
+  cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)cols * 4};
+  cuuint32_t box[2] = {32, 32};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = enc(reinterpret_cast<CUtensorMap*>(out), CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<float*>(base),
+                   dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(MUON_ERR_CUDA, "cuTensorMapEncodeTiled failed: " + std::to_string((int)r));
+  return MUON_OK;
+}
+
 }  // namespace
 
 namespace muon {
@@ -336,6 +352,7 @@ struct muon_handle {
   TableRing binds;     // MatBind tables of the calls
   TableRing in_maps;   // tensor maps of the callers' X inputs (stage call)
   TableRing subsets;   // tile lists restricted to the matrices with a gradient
+  TableRing p_maps;    // tensor maps of the callers' parameters (update in the last combine)
   int last_launches = 0;
   // Per-launch timing (muon_profile_enable / muon_profile_read).
   std::vector<cudaEvent_t> prof_ev;   // 2 per slot
@@ -484,6 +501,7 @@ int ensure_plan(muon_handle* h, const int32_t* shapes, int count) {
     h->binds.release();
     h->in_maps.release();
     h->subsets.release();
+    h->p_maps.release();
     free_plan(h->plan.get());
     h->plan.reset();
   }
@@ -751,7 +769,8 @@ WorkRange chunk_range(const DevPlan& P, int c) {
 // last_dst < 0). *result receives the selector of the result buffer.
 int enqueue_ns(muon_handle* h, const MatBind* d_binds, const std::vector<MatBind>& hbinds, const WorkRange& R,
                const TmapBlob* d_in_maps, const double* sumsq, int ns_steps, const float* abc, int first_src,
-               int last_dst, cudaStream_t st, int* launches, int* result) {
+               int last_dst, cudaStream_t st, int* launches, int* result, const ApplyArgs* apply = nullptr,
+               const TmapBlob* d_p_maps = nullptr) {
   DevPlan& P = *h->plan;
   const HostPlan& hp = P.hp;
   const bool bf16 = h->cfg.ns_precision == MUON_NS_BF16;
@@ -874,6 +893,11 @@ int enqueue_ns(muon_handle* h, const MatBind* d_binds, const std::vector<MatBind
         L.tiles = R.tiles[ph];
         L.ntiles = R.ntiles[ph];
         if (L.ntiles == 0) continue;
+        // The step's last combine may carry the parameter update.
+        if (apply && ph == PHASE_COMB && t == ns_steps) {
+          L.apply = *apply;
+          L.p_maps = d_p_maps;
+        }
         const int slot = prof_before(h, MUON_KERNEL_NS_GRAM + ph, st);
         // a goes on the diagonal of B (POLY), so the combine adds no a X.
         const float a = ph == PHASE_COMB ? 0.0f : c3[0];
@@ -958,6 +982,7 @@ struct CallTables {
     h->binds.end_call(st);
     h->in_maps.end_call(st);
     h->subsets.end_call(st);
+    h->p_maps.end_call(st);
   }
 };
 
@@ -1037,9 +1062,52 @@ int step_ranges(muon_handle* h, const std::vector<MatBind>& hb, cudaStream_t st,
 }
 
 // Momentum/norm/cast, Newton-Schulz and apply for the matrices of R.
+// Tensor maps of the parameters for the update in the last combine, or
+// NULL when the step applies O in a separate pass: other forms of the
+// iteration, zero iterations, fused_apply off, an active matrix on the small
+// path, or a parameter whose rows are not 16-byte aligned (n % 4 != 0 or an
+// unaligned base) for the bulk copies.
+int step_p_maps(muon_handle* h, float* const* params, const std::vector<MatBind>& hb, int ns_steps, cudaStream_t st,
+                const TmapBlob** out) {
+  *out = nullptr;
+  const DevPlan& P = *h->plan;
+  if (!h->cfg.fused_apply || h->cfg.ns_precision != MUON_NS_BF16 || h->cfg.ns_algorithm != MUON_NS_STANDARD ||
+      P.hp.tile_m == kTileMPair || ns_steps <= 0)
+    return MUON_OK;
+  const int count = P.hp.count;
+  std::vector<char> small((size_t)count, 0);
+  for (int i : P.hp.small) small[i] = 1;
+  for (int i = 0; i < count; ++i) {
+    if (!hb[i].active) continue;
+    if (small[i] || P.mats[i].n % 4 != 0 || (reinterpret_cast<uintptr_t>(params[i]) & 15u) != 0) return MUON_OK;
+  }
+  struct PCtx {
+    float* const* p;
+    const DevPlan* plan;
+  } ctx{params, &P};
+  auto build = [](const void* c, std::vector<unsigned char>& bytes) -> int {
+    const PCtx& pc = *static_cast<const PCtx*>(c);
+    const int n = pc.plan->hp.count;
+    bytes.assign(sizeof(TmapBlob) * (size_t)n, 0);
+    TmapBlob* maps = reinterpret_cast<TmapBlob*>(bytes.data());
+    for (int i = 0; i < n; ++i) {
+      const MatPlan& mp = pc.plan->mats[i];
+      if (mp.n % 4 != 0 || (reinterpret_cast<uintptr_t>(pc.p[i]) & 15u) != 0) continue;   // never applied here
+      const int rc = encode_p_map(maps + i, pc.p[i], mp.m, mp.n);
+      if (rc) return rc;
+    }
+    return MUON_OK;
+  };
+  void* d = nullptr;
+  int rc;
+  if ((rc = h->p_maps.get(params, sizeof(float*) * (size_t)count, build, &ctx, st, &d))) return rc;
+  *out = static_cast<const TmapBlob*>(d);
+  return MUON_OK;
+}
+
 int enqueue_step_range(muon_handle* h, const MatBind* db, const std::vector<MatBind>& hb, const WorkRange& R,
                        float lr, float beta, int nesterov, float wd, int ns_steps, const float* abc, cudaStream_t st,
-                       int* launches) {
+                       int* launches, const TmapBlob* d_p_maps) {
   DevPlan& P = *h->plan;
   double* sumsq = static_cast<double*>(P.ws);
   const bool fp32 = h->cfg.ns_precision == MUON_NS_FP32;
@@ -1058,7 +1126,18 @@ int enqueue_step_range(muon_handle* h, const MatBind* db, const std::vector<MatB
     ++*launches;
   }
   int res = BUF_X0;
-  if ((rc = enqueue_ns(h, db, hb, R, nullptr, sumsq, ns_steps, abc, BUF_X0, -1, st, launches, &res))) return rc;
+  // With parameter maps the last combine writes p' itself (step_p_maps says
+  // when); otherwise O is stored and applied by a separate pass.
+  ApplyArgs ap;
+  ap.on = 1;
+  ap.lr = lr;
+  ap.wd = wd;
+  ap.scale_mode = h->cfg.scale_mode;
+  ap.extra_scale = h->cfg.extra_scale;
+  if ((rc = enqueue_ns(h, db, hb, R, nullptr, sumsq, ns_steps, abc, BUF_X0, -1, st, launches, &res,
+                       d_p_maps ? &ap : nullptr, d_p_maps)))
+    return rc;
+  if (d_p_maps) return MUON_OK;
   slot = prof_before(h, MUON_KERNEL_APPLY, st);
   MUON_CUDA_TRY(launch_apply(EL, res, lr, wd, h->cfg.scale_mode, h->cfg.extra_scale, ns_steps == 0 ? sumsq : nullptr,
                              fp32, st));
@@ -1081,9 +1160,12 @@ int step_impl(muon_handle* h, float* const* params, const void* const* grads, fl
   DevPlan& P = *h->plan;
   std::vector<WorkRange> ranges;
   if ((rc = step_ranges(h, hb, st, ranges))) return rc;
+  const TmapBlob* d_p_maps = nullptr;
+  if ((rc = step_p_maps(h, params, hb, ns_steps, st, &d_p_maps))) return rc;
   // Groups under the workspace cap run one after another on the stream.
   for (const WorkRange& R : ranges)
-    if ((rc = enqueue_step_range(h, db, hb, R, lr, beta, nesterov, wd, ns_steps, abc, st, &launches))) return rc;
+    if ((rc = enqueue_step_range(h, db, hb, R, lr, beta, nesterov, wd, ns_steps, abc, st, &launches, d_p_maps)))
+      return rc;
   (void)P;
   h->last_launches = launches;
   return MUON_OK;
@@ -1114,6 +1196,7 @@ int muon_config_init(muon_config* cfg) {
   cfg->cta_pair = 0;
   cfg->ns_algorithm = MUON_NS_STANDARD;
   cfg->deterministic = 0;
+  cfg->fused_apply = 1;
   return MUON_OK;
 }
 
@@ -1129,6 +1212,7 @@ int muon_init(int device, const muon_config* cfg, muon_handle** out) {
     return fail(MUON_ERR_INVALID_ARG, "wait_timeout_s must be in (0, 600]");
   if (c.num_sms < 0) return fail(MUON_ERR_INVALID_ARG, "num_sms must be >= 0");
   if (c.deterministic != 0 && c.deterministic != 1) return fail(MUON_ERR_INVALID_ARG, "deterministic must be 0 or 1");
+  if (c.fused_apply != 0 && c.fused_apply != 1) return fail(MUON_ERR_INVALID_ARG, "fused_apply must be 0 or 1");
   if (c.ns_algorithm != MUON_NS_STANDARD && c.ns_algorithm != MUON_NS_GRAM)
     return fail(MUON_ERR_INVALID_ARG, "unknown ns_algorithm");
   if (c.ns_algorithm == MUON_NS_GRAM && (c.ns_precision != MUON_NS_BF16 || c.cta_pair))
@@ -1164,6 +1248,7 @@ int muon_destroy(muon_handle* h) {
     h->binds.release();
     h->in_maps.release();
     h->subsets.release();
+    h->p_maps.release();
     if (h->plan) free_plan(h->plan.get());
     prof_free(h);
     for (cudaEvent_t e : h->hev) cudaEventDestroy(e);
@@ -1304,6 +1389,8 @@ int muon_step_host(muon_handle* h, float* const* params, const void* const* grad
   std::vector<MatBind> hb;
   const MatBind* db = nullptr;
   if ((rc = step_binds(h, dp.data(), dg.data(), dm.data(), shapes, count, st, hb, &db))) return rc;
+  const TmapBlob* d_p_maps = nullptr;
+  if ((rc = step_p_maps(h, dp.data(), hb, ns_steps, st, &d_p_maps))) return rc;
 
   cudaStream_t s_in = h->hs[0], s_comp = h->hs[1], s_out = h->hs[2];
   MUON_CUDA_TRY(cudaEventRecord(ev_begin, st));
@@ -1325,7 +1412,7 @@ int muon_step_host(muon_handle* h, float* const* params, const void* const* grad
     // Compute.
     MUON_CUDA_TRY(cudaStreamWaitEvent(s_comp, ev_in(c), 0));
     if ((rc = enqueue_step_range(h, db, hb, chunk_range(P, c), lr, beta, nesterov, wd, ns_steps, abc, s_comp,
-                                 &launches)))
+                                 &launches, d_p_maps)))
       return rc;
     MUON_CUDA_TRY(cudaEventRecord(ev_comp(c), s_comp));
     // Copy-out.

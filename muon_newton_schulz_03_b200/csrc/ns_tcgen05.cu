@@ -448,7 +448,14 @@ __global__ void __launch_bounds__(kThreads, 1) ns_phase_kernel(const __grid_cons
     int acc = 0;
     uint32_t acc_phase = 0;
     int obuf = 0;   // staging block pair used by this warp's next chunk
-    const bool tma_out = L.tma_store != 0 && !(args.phase == PHASE_COMB && args.dst_sel == BUF_OUT);
+    // The last combine of a step may update the parameters in place of
+    // storing O (ApplyArgs): p' = p (1 - lr wd) - lr scale O, O rounded to
+    // bf16 first, p moved in 32 x 32 fp32 blocks by bulk copies through this
+    // warp's two staging regions (the output blocks and the auxiliary
+    // blocks, 4 KiB each, both unused by that launch otherwise).
+    const bool apply = args.phase == PHASE_COMB && L.apply.on != 0;
+    const float decay = apply ? apply_decay(L.apply.lr, L.apply.wd) : 1.0f;
+    const bool tma_out = L.tma_store != 0 && !(args.phase == PHASE_COMB && args.dst_sel == BUF_OUT) && !apply;
     // The combine reads X a second time only when it adds a X itself
     // (a != 0, the Gram form); the plain iteration puts a on the diagonal of
     // B in the polynomial's epilogue, so its combine is the bare product.
@@ -533,6 +540,67 @@ __global__ void __launch_bounds__(kThreads, 1) ns_phase_kernel(const __grid_cons
         }
         aux_pending |= 1u << b;
       };
+      if (apply) {
+        const TmapBlob* pm = L.p_maps + tile.x;
+        const float step = apply_step(L.apply.lr, mp.m, mp.n, L.apply.scale_mode, L.apply.extra_scale, 1.0);
+        const int nch = min(BN / 32, (cols - tj * BN + 31) / 32);   // chunks holding a column of the matrix
+        uint8_t* const pbuf[2] = {&sm.ostage[quarter][0][0], &sm.auxstage[quarter][0][0]};
+        // Bulk load of p's block for chunk c into buffer c & 1, once that
+        // buffer's previous block has been stored (read by the copy engine)
+        // and read by every lane.
+        auto p_load = [&](int c) {
+          const int b = c & 1;
+          if (lane == 0) bulk_wait_group_read<0>();
+          __syncwarp();
+          if (lane == 0) {
+            fence_proxy_async_smem();
+            mbar_arrive_expect_tx(&sm.aux_full[quarter][b], 32 * 32 * 4);
+            tma_load_2d(pbuf[b], pm, &sm.aux_full[quarter][b], tj * BN + c * 32, warp_row0);
+          }
+          aux_pending |= 1u << b;
+        };
+        p_load(0);
+        if (!mbar_wait_bounded(&sm.acc_full[acc], acc_phase, err, tmo, WAIT_ACC_FULL)) break;
+        tc_fence_after();
+        bool ok = true;
+        for (int c = 0; c < nch; ++c) {
+          if (c + 1 < nch) p_load(c + 1);
+          float v[32];
+          tmem_ld_32x32b_x32(t_base + (uint32_t)(c * 32), v);
+          const int b = c & 1;
+          if (!mbar_wait_bounded(&sm.aux_full[quarter][b], (aux_parity >> b) & 1u, err, tmo, WAIT_ACC_FULL)) {
+            ok = false;
+            break;
+          }
+          aux_parity ^= 1u << b;
+          aux_pending &= ~(1u << b);
+          // This lane's row of the block: 128 bytes, 16-byte unit u at unit
+          // u ^ (row % 8) (128-byte swizzle of the copy engine).
+          uint8_t* rowp = pbuf[b] + lane * 128;
+#pragma unroll
+          for (int u = 0; u < 8; ++u) {
+            float4* q = reinterpret_cast<float4*>(rowp + ((u ^ (lane & 7)) << 4));
+            float4 pv = *q;
+            pv.x = apply_one(pv.x, v[4 * u + 0] * sc, decay, step);
+            pv.y = apply_one(pv.y, v[4 * u + 1] * sc, decay, step);
+            pv.z = apply_one(pv.z, v[4 * u + 2] * sc, decay, step);
+            pv.w = apply_one(pv.w, v[4 * u + 3] * sc, decay, step);
+            *q = pv;
+          }
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            if (warp_row0 < rows) tma_store_2d(pm, pbuf[b], tj * BN + c * 32, warp_row0);
+            bulk_commit_group();
+          }
+        }
+        if (!ok) break;
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sm.acc_empty[acc]);
+        if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
+        continue;
+      }
       if (aux_tma) {
         aux_issue(0);
       } else if (aux_row != nullptr) {
@@ -652,7 +720,7 @@ __global__ void __launch_bounds__(kThreads, 1) ns_phase_kernel(const __grid_cons
     }
     // Bulk stores read this CTA's shared memory: let them finish; loads that
     // were issued but not waited for (after an abort) must land too.
-    if (tma_out && lane == 0) bulk_wait_group_all();
+    if ((tma_out || apply) && lane == 0) bulk_wait_group_all();
     if (lane == 0)
       for (int b = 0; b < 2; ++b)
         if (aux_pending & (1u << b)) mbar_wait_drain(&sm.aux_full[quarter][b], (aux_parity >> b) & 1u, drain_tmo);

@@ -23,13 +23,27 @@ pytestmark = pytest.mark.gpu
 F32 = lambda v: float(np.float32(v))  # noqa: E731  (scalars as the kernels see them)
 
 
+def _step_fused(opt, shapes, active=None):
+    """Whether a step of `opt` on these shapes writes p' in its last combine
+    and stores no O (muon_config.fused_apply): the handle allows it, and no
+    active matrix is on the small path or has rows whose length is not a
+    multiple of four."""
+    if not opt.fused_apply:
+        return False
+    small = set(muon.plan_query(shapes, opt.ns_precision, opt.small_path, opt.cta_pair)["small"])
+    idx = range(len(shapes)) if active is None else active
+    return not any(i in small for i in idx) and all(shapes[i][1] % 4 == 0 for i in idx)
+
+
 def _check_step(cpu, dev, shapes, opt, *, lr, beta, wd, nesterov=True, ns_steps=5, scale_mode=O.SCALE_MOONLIGHT,
                 tol=TOL_BF16_NS, check_o=True, indices=None, gram_mats=(), coeffs=O.DEFAULT_COEFFS, tag=""):
     """Every checked matrix against the exact oracle: momentum at 1e-6; O and
     the update at the bf16 gate (bf16 mode: 2e-2, or the pages' own bf16
     program's frozen distance where that is larger; ``tol`` for zero
     iterations) or at ``tol`` (fp32 debug mode); p' at 1e-6 with the oracle
-    fed the GPU's own O."""
+    fed the GPU's own O. A handle whose last iteration writes p' itself
+    (``fused_apply``) leaves no O in the workspace: there the update alone is
+    checked (its gate carries O's tolerance)."""
     indices = range(len(shapes)) if indices is None else indices
     worst = 0.0
     bf16 = opt.ns_precision == "bf16"
@@ -49,7 +63,7 @@ def _check_step(cpu, dev, shapes, opt, *, lr, beta, wd, nesterov=True, ns_steps=
             tol_o = tol
         e = gate_bf16_update(p_gpu, p0, p_ref, o_ref, F32(lr) * scale, tol_o, f"{tag} matrix {i} {m}x{n}")
         worst = max(worst, e)
-        if check_o and ns_steps > 0:
+        if check_o and ns_steps > 0 and not _step_fused(opt, shapes, indices):
             dtype = torch.bfloat16 if bf16 else torch.float32
             flips = (ns_steps + 1) // 2 if gram_mats else ns_steps
             o_gpu = to64(workspace_matrix(opt, shapes, i, flips % 2, dtype)[:, :n])
@@ -69,7 +83,8 @@ def test_single_matrix_workload(prec, tol):
     # lr 0.02, wd 0, Jordan scale (the lr 0.02 pairing).
     shapes = W.single_shapes()
     cpu, dev = make_set(W.CONFIG_SINGLE, shapes, torch.float32)
-    opt = muon.Muon(device=0, scale_mode="jordan", ns_precision=prec)
+    # O stored (fused_apply off), so that it is checked as well as p'.
+    opt = muon.Muon(device=0, scale_mode="jordan", ns_precision=prec, fused_apply=False)
     opt.step([d[0] for d in dev], [d[1] for d in dev], [d[2] for d in dev], lr=0.02, beta=0.95, wd=0.0)
     torch.cuda.synchronize()
     _check_step(cpu, dev, shapes, opt, lr=0.02, beta=0.95, wd=0.0, scale_mode=O.SCALE_JORDAN, tol=tol,
@@ -84,7 +99,7 @@ def test_single_matrix_workload(prec, tol):
 def test_gpt2_small_set(prec, tol, pair):
     shapes = W.gpt2_shapes()
     cpu, dev = make_set(W.CONFIG_GPT2, shapes, torch.float32)
-    opt = muon.Muon(device=0, ns_precision=prec, cta_pair=pair)
+    opt = muon.Muon(device=0, ns_precision=prec, cta_pair=pair, fused_apply=False)   # O stored and checked
     opt.step([d[0] for d in dev], [d[1] for d in dev], [d[2] for d in dev], lr=2e-4, beta=0.95, wd=0.1)
     torch.cuda.synchronize()
     idx = range(len(shapes)) if prec == "bf16" else range(4)
@@ -317,11 +332,9 @@ def _full_set_sampled(config, shapes, grad_dtype, sample, lr=2e-4, wd=0.1, tag="
         tol_o = bf16_ns_tolerance(u)
         errs.append((gate_bf16_update(p_gpu, p0, p_ref, o_ref, F32(lr) * O.update_scale(m, n), tol_o,
                                       f"config {tag} matrix {i} {m}x{n}"), tol_o))
-        # O itself (five steps end in the X1 buffer).
-        o_gpu = to64(workspace_matrix(opt, shapes, i, 1)[:, :n])
-        eo = rel(o_gpu, o_ref)
-        report(f"O config {tag} matrix {i} {m}x{n}", eo, tol_o, bf16_program_error(u))
-        assert eo <= tol_o
+    # The bench's configuration: the last iteration writes p' itself, so the
+    # update's gate (which carries O's tolerance) is the check; no O is stored.
+    assert opt.fused_apply and opt.last_launch_count() == 1 + 15
     opt.close()
     return errs
 
@@ -353,7 +366,7 @@ def test_mixed_small_and_tiled_matrices_in_one_step():
     opt.step([d[0] for d in dev], [d[1] for d in dev], [d[2] for d in dev], lr=2e-4, beta=0.95, wd=0.1)
     torch.cuda.synchronize()
     _check_step(cpu, dev, shapes, opt, lr=2e-4, beta=0.95, wd=0.1)
-    assert opt.last_launch_count() == 1 + 1 + 15 + 1
+    assert opt.last_launch_count() == 1 + 1 + 15 + 1   # K1, small path, phases, apply (a small matrix)
     assert opt.status() == (0, 0, 0)
     opt.close()
 
@@ -376,6 +389,45 @@ def test_gram_form_step(ns_steps):
     assert opt.last_launch_count() == 1 + 1 + 7 * segs2 + 3 * segs1 + 1
     assert opt.status() == (0, 0, 0)
     opt.close()
+
+
+FUSED_CASES = {
+    "single": (W.CONFIG_SINGLE, W.single_shapes(), torch.float32, None),
+    "gpt2": (W.CONFIG_GPT2, W.gpt2_shapes()[:8], torch.bfloat16, None),
+    # ragged edges: the bulk copies of p clip rows and columns past the matrix
+    "ragged": (W.CONFIG_GPT2, [(300, 700), (1000, 200), (520, 520), (768, 2304), (2304, 768), (200, 1000)],
+               torch.float32, None),
+    "split": (W.CONFIG_GPT2, W.PARITY_SHAPES["split"], torch.float32, W.SPLIT_ROWS),
+    # not fused (a small-path matrix; rows whose length is not a multiple of 4)
+    "mixed": (W.CONFIG_GPT2, W.PARITY_SHAPES["mixed"], torch.float32, None),
+    "odd_rows": (W.CONFIG_GPT2, [(300, 701), (1000, 201)], torch.float32, None),
+}
+
+
+@pytest.mark.parametrize("case", sorted(FUSED_CASES))
+def test_fused_apply_is_bitwise_the_separate_pass(case):
+    # Where a step qualifies, its last combine writes p' = p (1 - lr wd) -
+    # lr scale O itself (O rounded to bf16 first; p moved by bulk copies):
+    # p' and m' are bitwise those of the separate apply pass on the same
+    # inputs (fixed-order norm), with one launch fewer. Where it does not, the
+    # separate pass runs in both handles.
+    config, shapes, gdtype, splits = FUSED_CASES[case]
+    cpu, dev = make_set(config, shapes, gdtype)
+    twin = [(p.clone(), g.clone(), m.clone()) for (p, g, m) in dev]
+    fused = muon.Muon(device=0, deterministic=True)
+    separate = muon.Muon(device=0, deterministic=True, fused_apply=False)
+    kw = dict(lr=2e-4, beta=0.95, wd=0.1, row_splits=splits)
+    fused.step([d[0] for d in dev], [d[1] for d in dev], [d[2] for d in dev], **kw)
+    separate.step([t[0] for t in twin], [t[1] for t in twin], [t[2] for t in twin], **kw)
+    torch.cuda.synchronize()
+    for i, ((p, _, m), (p2, _, m2)) in enumerate(zip(dev, twin)):
+        assert torch.equal(m, m2), f"momentum of matrix {i}"
+        assert torch.equal(p, p2), f"p' of matrix {i}: {float(torch.max(torch.abs(p - p2))):.3e} apart"
+    expect_fused = case not in ("mixed", "odd_rows")
+    assert separate.last_launch_count() == fused.last_launch_count() + (1 if expect_fused else 0)
+    assert fused.status() == (0, 0, 0) and separate.status() == (0, 0, 0)
+    fused.close()
+    separate.close()
 
 
 def test_deterministic_norm_is_bitwise_repeatable():
@@ -425,7 +477,7 @@ def test_split_muon_qkv_and_per_head():
     opt.step([d[0] for d in dev], [d[1] for d in dev], [d[2] for d in dev], lr=2e-4, wd=0.1, row_splits=splits)
     torch.cuda.synchronize()
     assert opt.status() == (0, 0, 0)
-    assert opt.last_launch_count() >= 17
+    assert opt.last_launch_count() >= 16
     for i, (m, n) in enumerate(shapes):
         p0, g, m0 = cpu[i]
         rows = m if splits[i] is None else splits[i]
@@ -514,15 +566,15 @@ def test_layerwise_single_rank_matches_oracle():
         dist.destroy_process_group()
 
 
-def _group_launches(plan, bounds, deterministic=True):
+def _group_launches(plan, bounds, deterministic=True, fused=False):
     """Launches of a grouped step: per group K1 (+ fixed-order sum), the
     small path if the group has small matrices, 15 phases if it has tiled
-    ones, and the apply kernel."""
+    ones, and the apply kernel unless the last phases write p' themselves."""
     small = set(plan["small"])
     total = 0
     for g0, g1 in zip(bounds[:-1], bounds[1:]):
         mats = range(g0, g1)
-        total += 2 + (1 if deterministic else 0)
+        total += 1 + (0 if fused else 1) + (1 if deterministic else 0)
         total += 1 if any(i in small for i in mats) else 0
         total += 15 if any(i not in small for i in mats) else 0
     return total
