@@ -10,7 +10,9 @@
  *      (tensor-core GEMMs, one launch per phase for all matrices; in bf16
  *      the polynomial's epilogue forms aI + bA + cA^2, rounded once, and the
  *      combine is the product of that with X);
- *   3. p' = p*(1 - lr*wd) - lr*scale(m, n)*O (one kernel).
+ *   3. p' = p*(1 - lr*wd) - lr*scale(m, n)*O: in the last combine's epilogue
+ *      (blocks of p moved by bulk copies; see muon_config.fused_apply), or
+ *      one separate kernel.
  *
  * Sources (web pages, cited by title and section):
  *   "About Muon: Why Not Adam": "The whole thing, in about forty lines"
