@@ -235,6 +235,9 @@ def test_repeat_runs_agree_and_graph_replay():
     # matrix without a gradient
     [(256, 768), (768, 256), (64, 64), (1024, 512), (300, 700), (512, 1024), (128, 128), (640, 320),
      (256, 256), (200, 600), (900, 300), (384, 384)],
+    # no small-path matrix: the last combine of each chunk writes p' into
+    # the staging slot through the parameter maps of the staging pointers
+    [(256, 768), (768, 256), (1024, 512), (512, 1024), (300, 700), (700, 300)],
 ])
 def test_step_host_matches_device_step(shapes):
     cpu, dev = make_set(W.CONFIG_GPT2, shapes, torch.bfloat16)
@@ -631,6 +634,31 @@ def test_workspace_cap_runs_groups_and_matches_uncapped():
         tight.step([d[0] for d in dev], [d[1] for d in dev], [d[2] for d in dev], lr=2e-4)
     assert e.value.code == 3
     tight.close()
+
+
+def test_workspace_cap_with_the_update_in_the_last_combine():
+    # Groups under a workspace cap on a set without small-path matrices: each
+    # group's last combine writes p' (no apply launch), bitwise the uncapped
+    # step's in the fixed-order norm mode (whose update is gated against the
+    # oracle by the other step tests).
+    shapes = [(256, 768), (768, 256), (1024, 512), (512, 1024), (300, 700), (700, 300)]
+    cap = muon.plan_query(shapes)["ws_bytes"] // 3
+    bounds = muon.plan_groups(shapes, cap)["bounds"]
+    assert len(bounds) - 1 >= 3
+    cpu, dev = make_set(W.CONFIG_GPT2, shapes, torch.float32)
+    twin = [(p.clone(), g.clone(), m.clone()) for (p, g, m) in dev]
+    capped = muon.Muon(device=0, workspace_cap_bytes=cap, deterministic=True)
+    plain = muon.Muon(device=0, deterministic=True)
+    capped.step([d[0] for d in dev], [d[1] for d in dev], [d[2] for d in dev], lr=2e-4, beta=0.95, wd=0.1)
+    plain.step([t[0] for t in twin], [t[1] for t in twin], [t[2] for t in twin], lr=2e-4, beta=0.95, wd=0.1)
+    torch.cuda.synchronize()
+    assert _step_fused(capped, shapes)
+    assert capped.last_launch_count() == _group_launches(muon.plan_query(shapes), bounds, fused=True)
+    for (p, _, m), (p2, _, m2) in zip(dev, twin):
+        assert torch.equal(p, p2) and torch.equal(m, m2)
+    assert capped.status() == (0, 0, 0) and plain.status() == (0, 0, 0)
+    capped.close()
+    plain.close()
 
 
 def test_fresh_pointers_every_step_match_fixed_pointers():
