@@ -75,6 +75,16 @@ def kernel_source_hash():
     return h.hexdigest()[:16]
 
 
+def tensor_peak(peaks, peak_src, timed_ms):
+    """The dense bf16 peak a timed region is held to: the sustained figure (a
+    seconds-long loop under the power cap) for a region of a second or more,
+    the burst figure for a shorter one. Returns (TFLOP/s, description)."""
+    if timed_ms >= 1000.0:
+        return (peaks["bf16_tflops_sustained"],
+                f"{peak_src} sustained dense bf16 (timed region of {timed_ms / 1e3:.1f} s, inside a long run)")
+    return peaks["bf16_tflops"], f"{peak_src} burst dense bf16 (timed region of {timed_ms:.0f} ms)"
+
+
 def profiled_traffic(workload):
     """DRAM bytes per launch of the Newton-Schulz kernel from a committed ncu
     summary, if it was taken on the current kernel source; else None."""
@@ -457,14 +467,7 @@ def run_ours(args):
         value = (1 if args.layerwise else world) * 1e3 / ms_step
         # The committed captures are of the single-CTA kernel, standard form.
         traffic = None if (gram or args.cta_pair) else profiled_traffic(args.workload)
-        # The sustained peak (a seconds-long loop under the power cap) for a
-        # timed region of a second or more; the burst peak for a shorter one.
-        long_region = ms_step * args.steps >= 1000.0
-        peak_key = "bf16_tflops_sustained" if long_region else "bf16_tflops"
-        peak_note = (f"{peak_src} sustained dense bf16 (timed region of {ms_step * args.steps / 1e3:.1f} s, "
-                     "inside a long run)" if long_region else
-                     f"{peak_src} burst dense bf16 (timed region of {ms_step * args.steps:.0f} ms)")
-        peak_tf = peaks[peak_key]
+        peak_tf, peak_note = tensor_peak(peaks, peak_src, ms_step * args.steps)
         line = {
             "metric": METRIC,
             "value": value,

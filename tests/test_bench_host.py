@@ -83,3 +83,14 @@ def test_shape_classes_and_set_extrapolation():
     secs = {(4096, 4096): 1.0, (1024, 4096): 0.5, (14336, 4096): 2.0, (4096, 14336): 3.0}
     assert bench.set_seconds("llama3", secs) == 64 * 1.0 + 64 * 0.5 + 64 * 2.0 + 32 * 3.0
     assert W.shape_classes(W.moe_shapes()) == {(2048, 7168): (256, 0), (7168, 2048): (128, 2)}
+
+
+def test_tensor_peak_follows_the_length_of_the_timed_region():
+    # A timed region of a second or more runs at the power cap: the sustained
+    # figure; a shorter one at full clock: the burst figure.
+    peaks = dict(bench.FALLBACK)
+    tf, note = bench.tensor_peak(peaks, "fallback", 4300.0)
+    assert tf == peaks["bf16_tflops_sustained"] and "sustained" in note and "4.3 s" in note
+    tf, note = bench.tensor_peak(peaks, "fallback", 15.0)
+    assert tf == peaks["bf16_tflops"] and "burst" in note and "15 ms" in note
+    assert bench.tensor_peak(peaks, "measured", 1000.0)[0] == peaks["bf16_tflops_sustained"]
